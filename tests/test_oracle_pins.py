@@ -1,0 +1,296 @@
+"""Pins of the float64 oracle against facts fixed by the pages and by mathematics.
+
+Each test checks the oracle against something other than itself: a hand-worked
+example, a closed form, an invariant, or an independent formulation (complex
+multiplication for RoPE, the block-masked quadratic form for the carry).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+D = 32
+
+
+def _rand(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+def _qkv(B, N, H, seed, Nk=None):
+    Nk = N if Nk is None else Nk
+    return (_rand((B, N, H, D), seed), _rand((B, Nk, H, D), seed + 1),
+            _rand((B, Nk, H, D), seed + 2))
+
+
+def _vec(spec):
+    x = np.zeros(D)
+    for k, val in spec.items():
+        x[int(k)] = val
+    return x
+
+
+# --------------------------------------------------------------------------
+# Hand-worked examples (tests/golden)
+
+
+def test_worked_example_relu_attention():
+    g = json.load(open(os.path.join(GOLDEN, "worked_example_relu.json")))
+    Q = _vec(g["q"]).reshape(1, 1, 1, D)
+    K = np.stack([_vec(s) for s in g["k"]]).reshape(1, 2, 1, D)
+    V = np.stack([_vec(s) for s in g["v"]]).reshape(1, 2, 1, D)
+    want = _vec(g["expected_o"])
+    for out in (orc.attention(Q, K, V, g["eps"]),
+                orc.attention_bruteforce(Q, K, V, g["eps"])):
+        np.testing.assert_allclose(out[0, 0, 0], want, rtol=1e-15, atol=1e-15)
+
+
+def test_rope_convention_hand_worked():
+    g = json.load(open(os.path.join(GOLDEN, "rope_convention.json")))
+    T, Hh, W, t0 = (g["grid"][k] for k in ("T", "Hh", "W", "t_offset"))
+    theta = orc.rope_angles(T, Hh, W, t0)
+    N = T * Hh * W
+    for case in g["cases"]:
+        t, h, w = case["token"]
+        n = (t * Hh + h) * W + w
+        d = case["dim"]
+        ang = eval(case["angle"], {"__builtins__": {}}, {})  # arithmetic only
+        for which, want in ((d, (math.cos(ang), math.sin(ang))),
+                            (d + 1, (-math.sin(ang), math.cos(ang)))):
+            x = np.zeros((1, N, 1, D))
+            x[0, n, 0, which] = 1.0
+            y = orc.rope_rotate(x, theta)[0, n, 0]
+            np.testing.assert_allclose(y[d:d + 2], want, rtol=0, atol=1e-14,
+                                       err_msg=case["note"])
+            others = np.delete(y, [d, d + 1])
+            assert np.all(others == 0.0), case["note"]
+
+
+# --------------------------------------------------------------------------
+# RoPE against an independent formulation and its invariants
+
+
+def test_rope_equals_complex_multiplication():
+    theta = orc.rope_angles(3, 4, 5, t_offset=7)
+    x = _rand((2, 60, 3, D), 11)
+    y = orc.rope_rotate(x, theta)
+    zc = (x[..., 0::2] + 1j * x[..., 1::2]) * np.exp(1j * theta)[None, :, None, :]
+    np.testing.assert_allclose(y[..., 0::2], zc.real, atol=1e-13)
+    np.testing.assert_allclose(y[..., 1::2], zc.imag, atol=1e-13)
+
+
+def test_rope_zero_positions_is_identity_and_norm_preserving():
+    x = _rand((1, 1, 2, D), 3)
+    th0 = orc.rope_angles(1, 1, 1, t_offset=0)
+    np.testing.assert_array_equal(orc.feature_map(x, th0), orc.relu(x))
+    th = orc.rope_angles(4, 3, 5, t_offset=2)
+    x = _rand((1, 60, 2, D), 4)
+    np.testing.assert_allclose(np.linalg.norm(orc.feature_map(x, th), axis=-1),
+                               np.linalg.norm(orc.relu(x), axis=-1), rtol=1e-13)
+
+
+@pytest.mark.parametrize("axis", ["t", "h", "w"])
+def test_rope_relative_shift_invariance(axis):
+    # phi(q_i).phi(k_j) depends only on p_i - p_j, so shifting every query and
+    # key position along one axis by the same amount leaves O unchanged.
+    T, Hh, W = 2, 3, 4
+    N = T * Hh * W
+    Q, K, V = _qkv(1, N, 2, 21)
+    t, h, w = orc.rope_positions(T, Hh, W, 0)
+    pos = {"t": t, "h": h, "w": w}
+
+    def angles(shift):
+        p = dict(pos)
+        p[axis] = p[axis] + shift
+        cols = []
+        for ax, _f, width in orc.ROPE_SEGMENTS:
+            for k in range(width // 2):
+                cols.append(p[ax] * 10000.0 ** (-2.0 * k / width))
+        return np.stack(cols, 1)
+
+    np.testing.assert_allclose(angles(0), orc.rope_angles(T, Hh, W, 0), rtol=0, atol=0)
+    th0, th9 = angles(0), angles(9)
+    o0 = orc.attention_bruteforce(Q, K, V, 1e-6, th0, th0)
+    o9 = orc.attention_bruteforce(Q, K, V, 1e-6, th9, th9)
+    np.testing.assert_allclose(o9, o0, rtol=1e-10, atol=1e-12)
+    # ...whereas shifting the queries alone changes it (the shift is not a no-op)
+    o_q = orc.attention_bruteforce(Q, K, V, 1e-6, th9, th0)
+    assert np.max(np.abs(o_q - o0)) > 1e-3
+
+
+def test_block_t_offset_is_global_frame_index():
+    th_a = orc.rope_angles(4, 2, 3, t_offset=0)
+    th_b = orc.rope_angles(2, 2, 3, t_offset=2)
+    np.testing.assert_array_equal(th_a[12:], th_b)
+
+
+# --------------------------------------------------------------------------
+# The quadratic form: closed forms and invariants
+
+
+def test_one_hot_keys_give_group_means():
+    # With one-hot keys and a one-hot query, ReLU(q).ReLU(k_j) is 1 for keys in
+    # the query's group and 0 elsewhere, so O is the mean of that group's values.
+    rng = np.random.default_rng(5)
+    N = 40
+    groups = rng.integers(0, D, N)
+    K = np.zeros((1, N, 1, D))
+    K[0, np.arange(N), 0, groups] = 1.0
+    V = _rand((1, N, 1, D), 6)
+    for a in np.unique(groups)[:5]:
+        Q = np.zeros((1, 1, 1, D))
+        Q[0, 0, 0, a] = 1.0
+        want = V[0, groups == a, 0].mean(axis=0)
+        for out in (orc.attention_bruteforce(Q, K, V, 0.0), orc.attention(Q, K, V, 0.0)):
+            np.testing.assert_allclose(out[0, 0, 0], want, rtol=1e-13, atol=1e-14)
+
+
+def test_single_key_closed_form():
+    Q, K, V = _qkv(1, 3, 1, 8, Nk=1)
+    Q, K = np.abs(Q), np.abs(K)
+    eps = 0.25
+    w = (Q[0, :, 0] @ K[0, 0, 0])
+    want = w[:, None] * V[0, 0, 0][None, :] / (w[:, None] + eps)
+    np.testing.assert_allclose(orc.attention(Q, K, V, eps)[0, :, 0], want, rtol=1e-13)
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_factorised_equals_bruteforce(rope):
+    T, Hh, W = 3, 4, 5
+    N = T * Hh * W
+    Q, K, V = _qkv(2, N, 3, 31)
+    th = orc.rope_angles(T, Hh, W, 4) if rope else None
+    fact = orc.attention(Q, K, V, 1e-6, th)
+    brute = orc.attention_bruteforce(Q, K, V, 1e-6, th, th)
+    np.testing.assert_allclose(fact, brute, rtol=1e-12, atol=1e-14)
+
+
+def test_constant_values_closed_form():
+    # v_j = c for every j gives O_i = c * x_i / (x_i + eps), x_i = ReLU(q_i).z.
+    B, N, H = 1, 50, 2
+    Q, K, _ = _qkv(B, N, H, 41)
+    Q = Q * 1e-6  # make eps matter
+    c = _rand((D,), 42)
+    V = np.broadcast_to(c, (B, N, H, D)).copy()
+    eps = 1e-6
+    z = orc.relu(K).sum(axis=1)
+    x = np.einsum("bnhd,bhd->bnh", orc.relu(Q), z)
+    want = c[None, None, None, :] * (x / (x + eps))[..., None]
+    np.testing.assert_allclose(orc.attention(Q, K, V, eps), want, rtol=1e-12)
+    np.testing.assert_allclose(orc.attention_bruteforce(Q, K, V, eps), want, rtol=1e-12)
+
+
+def test_convex_bound_and_degenerate_rows():
+    Q, K, V = _qkv(1, 64, 2, 51)
+    Q[0, :8] = -np.abs(Q[0, :8])  # ReLU(q) = 0 rows
+    O = orc.attention(Q, K, V, 1e-6)
+    assert np.all(O[0, :8] == 0.0)
+    vmax = np.abs(V).max(axis=(1, 3))  # per (b, h)
+    assert np.all(np.abs(O).max(axis=(1, 3)) <= vmax + 1e-12)
+
+
+def test_key_permutation_linearity_and_scale():
+    Q, K, V = _qkv(1, 40, 2, 61)
+    O = orc.attention(Q, K, V, 0.0)
+    perm = np.random.default_rng(1).permutation(40)
+    np.testing.assert_allclose(orc.attention(Q, K[:, perm], V[:, perm], 0.0), O, rtol=1e-12, atol=1e-14)
+    V2 = _rand(V.shape, 62)
+    np.testing.assert_allclose(orc.attention(Q, K, 2 * V - 3 * V2, 0.0),
+                               2 * O - 3 * orc.attention(Q, K, V2, 0.0), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(orc.attention(3.5 * Q, 0.25 * K, V, 0.0), O, rtol=1e-12, atol=1e-14)
+    # an all-negative key is cut by ReLU and changes nothing
+    Kx = np.concatenate([K, -np.abs(_rand((1, 1, 2, D), 63))], axis=1)
+    Vx = np.concatenate([V, _rand((1, 1, 2, D), 64)], axis=1)
+    np.testing.assert_allclose(orc.attention(Q, Kx, Vx, 0.0), O, rtol=1e-12, atol=1e-14)
+
+
+def test_state_additivity():
+    T, Hh, W = 4, 3, 5
+    N = T * Hh * W
+    _, K, V = _qkv(1, N, 2, 71)
+    th = orc.rope_angles(T, Hh, W, 0)
+    S, z = orc.state_reduce(K, V, th)
+    S1, z1 = orc.state_reduce(K[:, :17], V[:, :17], th[:17])
+    S2, z2 = orc.state_reduce(K[:, 17:], V[:, 17:], th[17:])
+    np.testing.assert_allclose(S, S1 + S2, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(z, z1 + z2, rtol=1e-13)
+    assert S.shape == (1, 2, D, D) and z.shape == (1, 2, D)
+    # constant-size state: D x D plus D, whatever N is
+    Sb, zb = orc.state_reduce(K[:, :3], V[:, :3], th[:3])
+    assert Sb.shape == S.shape and zb.shape == z.shape
+
+
+def test_denominator_is_unrotated():
+    # Rotating the keys changes S but not z; rotating the queries changes the
+    # numerator only.
+    T, Hh, W = 2, 2, 3
+    N = T * Hh * W
+    Q, K, V = _qkv(1, N, 1, 81)
+    th = orc.rope_angles(T, Hh, W, 1)
+    _, z_plain = orc.state_reduce(K, V)
+    _, z_rope = orc.state_reduce(K, V, th)
+    np.testing.assert_array_equal(z_plain, z_rope)
+    # the denominator of the brute force equals the plain ReLU one
+    ones = np.ones_like(V)
+    S_r, z_r = orc.state_reduce(K, ones, th)
+    x = np.einsum("bnhd,bhd->bnh", orc.relu(Q), z_r)
+    assert np.all(x > 0)
+
+
+# --------------------------------------------------------------------------
+# Block-causal state carry
+
+
+def _blocks(M, steps, T, Hh, W, H, seed, rope=True):
+    N = T * Hh * W
+    blocks = []
+    for m in range(M):
+        th = orc.rope_angles(T, Hh, W, m * T) if rope else None
+        passes = []
+        for s in range(steps):
+            passes.append(_qkv(1, N, H, seed + 1000 * m + 10 * s) + (th,))
+        _, Ku, Vu = _qkv(1, N, H, seed + 1000 * m + 10 * steps)
+        blocks.append({"passes": passes, "update": (Ku, Vu, th)})
+    return blocks
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_block_carry_equals_block_masked_quadratic(rope):
+    M, steps, T, Hh, W, H = 3, 2, 2, 2, 3, 2
+    eps = 1e-6
+    blocks = _blocks(M, steps, T, Hh, W, H, 100, rope)
+    want = orc.block_causal_bruteforce(blocks, eps)
+    S = np.zeros((1, H, D, D))
+    z = np.zeros((1, H, D))
+    for m, blk in enumerate(blocks):
+        for s, (Q, K, V, th) in enumerate(blk["passes"]):
+            O, S2, z2 = orc.block_causal_step(Q, K, V, S, z, 0, eps, th)
+            np.testing.assert_array_equal(S2, S)
+            np.testing.assert_allclose(O, want[m][s], rtol=1e-11, atol=1e-13)
+        Ku, Vu, th = blk["update"]
+        none, S, z = orc.block_causal_step(None, Ku, Vu, S, z, 2, eps, th)
+        assert none is None
+    # the final carry is the state of all update passes together
+    Kall = np.concatenate([b["update"][0] for b in blocks], axis=1)
+    Vall = np.concatenate([b["update"][1] for b in blocks], axis=1)
+    thall = None if not rope else np.concatenate([b["update"][2] for b in blocks], 0)
+    S_all, z_all = orc.state_reduce(Kall, Vall, thall)
+    np.testing.assert_allclose(S, S_all, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(z, z_all, rtol=1e-13)
+
+
+def test_single_block_is_noncausal_and_update1_matches():
+    Q, K, V = _qkv(1, 30, 2, 130)
+    S0 = np.zeros((1, 2, D, D))
+    z0 = np.zeros((1, 2, D))
+    O0, _, _ = orc.block_causal_step(Q, K, V, S0, z0, 0, 1e-6)
+    np.testing.assert_allclose(O0, orc.attention(Q, K, V, 1e-6), rtol=1e-13)
+    O1, S1, z1 = orc.block_causal_step(Q, K, V, S0, z0, 1, 1e-6)
+    np.testing.assert_array_equal(O1, O0)
+    S_own, z_own = orc.state_reduce(K, V)
+    np.testing.assert_array_equal(S1, S_own)
+    np.testing.assert_array_equal(z1, z_own)
