@@ -1,0 +1,590 @@
+#!/usr/bin/env python
+"""Benchmark of one ReLU linear-attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl la|reference]
+                    [--workload NAME]
+
+A step is one pass of the layer's hot path over one batch of synthetic input:
+the state reduce (S = sum phi(K)^T V, z = sum ReLU(K)) and the apply
+(O = phi(Q) S / (ReLU(Q).z + eps)) of the default workload, or a whole
+block-causal video (reset, 12 blocks x 5 calls) for the LongSANA workload.
+Rank 0 prints one JSON line. Multi-GPU runs are weak-scaled: every rank runs
+its own copy of the workload (heads and batches are independent), with no
+collective on the data path; the time is the max over ranks.
+
+--impl reference times the float64 CPU oracle (the only other program on the
+path) on this host's cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "linear-attn tokens/s per layer at 1 B200; achieved HBM GB/s vs peak"
+DEFAULT_WORKLOAD = "sana1.6b_1024px"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+D = 32
+
+
+# ---------------------------------------------------------------------------
+# helpers
+
+
+def env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def layer_bytes(w, io_bytes=2):
+    """Algorithmic HBM bytes of one layer: read Q, K, V, write O, write/read the state."""
+    th = w.B * w.N * w.H
+    state = w.B * w.H * (D * D + D) * 4
+    return {"state_reduce": 2 * th * D * io_bytes + state,   # read K, V; write S, z
+            "apply": 2 * th * D * io_bytes + state}          # read Q, S, z; write O
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, burst copy)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
+
+
+def sources_sha():
+    h = hashlib.sha256()
+    pat = os.path.join(ROOT, "linear_attention_diffusion_b200", "csrc", "*")
+    for fn in sorted(glob.glob(pat)):
+        with open(fn, "rb") as f:
+            h.update(os.path.basename(fn).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload, kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
+    when there is none or the kernel sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    sha = sources_sha()
+    for line in open(path):
+        if line.startswith("#") or "=" not in line:
+            continue
+        kv = dict(tok.split("=", 1) for tok in line.split())
+        if kv.get("kernel") == kernel and kv.get("sources_sha") == sha:
+            return int(float(kv["dram_bytes_per_launch"]))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 100 ms) of the GPU this process uses."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = (uuid or "").lower()
+        self.samples = []
+        self.proc = None
+        self.error = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception as e:  # no nvidia-smi
+            self.error = str(e)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            if self.uuid and self.uuid not in parts[0].lower():
+                continue
+            try:
+                self.samples.append((time.time(), float(parts[1]), float(parts[2]),
+                                     float(parts[3]) if parts[3] not in ("[N/A]", "") else None,
+                                     parts[5:9]))
+            except ValueError:
+                pass
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "note": f"no nvidia-smi samples ({self.error or 'none parsed'})"}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = "samples taken during the timed region"
+        if not inside:
+            mid = 0.5 * (t0 + t1)
+            inside = sorted(self.samples, key=lambda s: abs(s[0] - mid))[:3]
+            note = "timed region shorter than the 100 ms sampling period: nearest samples"
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in inside for i, v in enumerate(s[4])
+                          if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(s[1] for s in inside),
+                "sm_max_mhz": max(s[2] for s in inside), "reasons": reasons,
+                "samples": len(inside), "note": note}
+
+
+def cpu_cores_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, seconds, max_reps=None):
+    """Time the float64 oracle on a bounded sample of workload `w`.
+
+    One call covers a subset of heads sized so that it takes at most about
+    `seconds`/3; calls repeat until `seconds` have passed. Returns
+    (tokens per second for the whole workload, description, cores)."""
+    import numpy as np
+    import oracle as orc
+
+    def run(h_sub, Q, K, V, th):
+        if w.block_causal:
+            Sc = np.zeros((w.B, h_sub, D, D))
+            zc = np.zeros((w.B, h_sub, D))
+            orc.block_causal_step(Q, K, V, Sc, zc, 1, w.eps, th)
+        else:
+            orc.attention(Q, K, V, w.eps, th)
+
+    th = orc.rope_angles(w.T, w.Hh, w.W, 0, w.rope_base) if w.rope else None
+    Qa, Ka, Va = wl.make_qkv(w, 0)
+    h_sub = min(w.H, 2)
+    t = time.perf_counter()
+    run(h_sub, Qa[:, :, :h_sub], Ka[:, :, :h_sub], Va[:, :, :h_sub], th)
+    per_head = (time.perf_counter() - t) / h_sub
+    h_sub = max(1, min(w.H, int((seconds / 3) / max(per_head, 1e-9))))
+    Q, K, V = (x[:, :, :h_sub].contiguous() for x in (Qa, Ka, Va))
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        run(h_sub, Q, K, V, th)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_reps and reps >= max_reps):
+            break
+    per_call = el / reps
+    full_call = per_call * w.H / h_sub
+    if w.block_causal:
+        calls = w.M * (w.steps + 1)
+        tokens_per_s = w.M * w.N * w.B / (full_call * calls)
+        desc = (f"oracle block_causal_step on {h_sub} of {w.H} heads of one {w.N}-token block, "
+                f"{reps} calls in {el:.1f} s, scaled to {w.H} heads x {calls} calls per video")
+    else:
+        tokens_per_s = w.B * w.N / full_call
+        desc = (f"oracle attention on {h_sub} of {w.H} heads (B={w.B}, N={w.N}), {reps} calls "
+                f"in {el:.1f} s, scaled to {w.H} heads")
+    return tokens_per_s, desc, cpu_cores_used(), per_call, h_sub
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+
+
+def run_la(args, w, rank, world, local_rank):
+    import torch
+    import linear_attention_diffusion_b200 as la
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    props = torch.cuda.get_device_properties(dev)
+    uuid = str(getattr(props, "uuid", "") or "")
+    sampler = ClockSampler(uuid)
+    stream = torch.cuda.Stream(dev)
+    lib = la._lib
+    sp = stream.cuda_stream
+
+    per_set = 3 * w.B * w.N * w.H * D * 2
+    n_sets = max(1, min(8, math.ceil(2 * L2_BYTES / per_set)))
+    if w.block_causal:
+        n_sets = 5  # one set per call of a block; each set is far above L2
+    sets = []
+    for i in range(n_sets):
+        if w.block_causal:
+            q, k, v = wl.make_qkv(w, 1000 * rank, block=0, step=i)
+        else:
+            q, k, v = wl.make_qkv(w, 1000 * rank + 10 * i)
+        q, k, v = (x.to(dev) for x in (q, k, v))
+        sets.append((q, k, v, torch.empty_like(q)))
+    S = torch.zeros((w.B, w.H, D, D), device=dev)
+    z = torch.zeros((w.B, w.H, D), device=dev)
+
+    def shape_at(t_offset=0):
+        return la.make_shape(w.B, w.N, w.H, D, "bf16", w.rope, w.T, w.Hh, w.W, t_offset,
+                             w.rope_base, w.eps)
+
+    shape0 = shape_at(0)
+    ws = la.workspace(shape0, dev)
+    ws_p, ws_n = ws.data_ptr(), ws.numel()
+    S_p, z_p = S.data_ptr(), z.data_ptr()
+    ptrs = [tuple(t.data_ptr() for t in s) for s in sets]
+    keep = [shape_at(m * w.T) for m in range(max(1, w.M))]
+    shapes = [ctypes.byref(s) for s in keep]
+    status = []
+
+    if w.block_causal:
+        calls_per_step = w.M * (w.steps + 1)
+        launches_per_step = 2 * calls_per_step  # reduce + apply per call; reset is memsets
+
+        def step(i, evs=None):
+            status.append(lib.la_state_reset(S_p, z_p, w.B, w.H, D, sp))
+            c = 0
+            for m in range(w.M):
+                for s in range(w.steps + 1):
+                    q, k, v, o = ptrs[s % n_sets]
+                    upd = 1 if s == w.steps else 0
+                    if evs is not None and upd == 0 and m == w.M - 1 and s == 0:
+                        evs[0].record(stream)
+                    status.append(lib.la_block_causal_step(shapes[m], q, k, v, S_p, z_p, o, upd,
+                                                           ws_p, ws_n, sp))
+                    if evs is not None and upd == 0 and m == w.M - 1 and s == 0:
+                        evs[1].record(stream)
+                    c += 1
+        kernel_names = ("la_block_causal_step",)
+    else:
+        launches_per_step = 2
+
+        def step(i, evs=None):
+            q, k, v, o = ptrs[i % n_sets]
+            if evs is not None:
+                evs[0].record(stream)
+            status.append(lib.la_state_reduce(shapes[0], k, v, S_p, z_p, ws_p, ws_n, sp))
+            if evs is not None:
+                evs[1].record(stream)
+            status.append(lib.la_apply(shapes[0], q, S_p, z_p, o, sp))
+            if evs is not None:
+                evs[2].record(stream)
+        kernel_names = ("state_reduce", "apply")
+
+    def check_status():
+        bad = [s for s in status if s != 0]
+        status.clear()
+        if bad:
+            raise RuntimeError(f"library call failed: {la.la_status_string(bad[0])} "
+                               f"{la.la_last_error()}")
+
+    # warm-up, eager
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    torch.cuda.synchronize(dev)
+    check_status()
+
+    # chunk graph: C steps, with an event after every launch
+    n_ev = 3 if not w.block_causal else 2
+    chunk = n_sets * max(1, 100 // n_sets) if not w.block_causal else 1
+    chunk = min(chunk, args.steps) if args.steps > 0 else chunk
+    chunk = max(1, chunk - chunk % n_sets) if chunk >= n_sets else chunk
+
+    def capture(nsteps):
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
+               for _ in range(nsteps)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(nsteps):
+                step(i, evs[i])
+        check_status()
+        return g, evs
+
+    g_chunk, ev_chunk = capture(chunk)
+    full, rem = divmod(args.steps, chunk)
+    g_rem, ev_rem = capture(rem) if rem else (None, None)
+
+    # soak: the same graph, untimed, for about a second, so that clocks settle
+    torch.cuda.synchronize(dev)
+    t_soak = time.time()
+    with torch.cuda.stream(stream):
+        while time.time() - t_soak < args.soak:
+            g_chunk.replay()
+            torch.cuda.synchronize(dev)
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(full):
+            g_chunk.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        end.record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end)
+
+    # per-launch durations from the last replay of the chunk graph
+    evs = ev_chunk if full > 0 else ev_rem
+    seg = [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(n_ev - 1)]
+    seg_us = [1000.0 * statistics.mean(s) for s in seg]
+
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t.item())
+
+    # end-to-end through the public API with host buffers
+    e2e = run_e2e(args, w, dev, stream, la, rank)
+    clocks = sampler.summary(t0, t1)
+    sampler.stop()
+    del g_chunk, g_rem
+    return {"ms": ms_max, "seg_us": seg_us, "kernel_names": kernel_names, "e2e": e2e,
+            "clocks": clocks, "launches_per_step": launches_per_step, "n_sets": n_sets,
+            "chunk": chunk, "per_set_bytes": per_set}
+
+
+def run_e2e(args, w, dev, stream, la, rank):
+    """Same metric through la_attention / la_block_causal_step with pinned host
+    inputs copied in and the output copied out inside the timed region."""
+    import torch
+    steps = max(1, min(args.steps, args.e2e_steps))
+    if w.block_causal:
+        q, k, v = wl.make_qkv(w, 1000 * rank, block=0, step=0)
+    else:
+        q, k, v = wl.make_qkv(w, 1000 * rank + 7)
+    hq, hk, hv = (x.pin_memory() for x in (q, k, v))
+    ho = torch.empty_like(hq).pin_memory()
+    dq, dk, dv, do = (torch.empty_like(hq, device=dev) for _ in range(4))
+    S = torch.zeros((w.B, w.H, D, D), device=dev)
+    z = torch.zeros((w.B, w.H, D), device=dev)
+    shapes = [la.make_shape(w.B, w.N, w.H, D, "bf16", w.rope, w.T, w.Hh, w.W, m * w.T,
+                            w.rope_base, w.eps) for m in range(max(1, w.M))]
+    ws = la.workspace(shapes[0], dev)
+
+    def one_pass(shape, update):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        if w.block_causal:
+            la.la_block_causal_step(shape, dq, dk, dv, S, z, do, update, ws, stream)
+        else:
+            la.la_attention(shape, dq, dk, dv, S, z, do, ws, stream)
+        ho.copy_(do, non_blocking=True)
+
+    def one_step():
+        if w.block_causal:
+            la.la_state_reset(S, z, w.B, w.H, D, stream)
+            for m in range(w.M):
+                for s in range(w.steps + 1):
+                    one_pass(shapes[m], 1 if s == w.steps else 0)
+        else:
+            one_pass(shapes[0], 0)
+
+    with torch.cuda.stream(stream):
+        one_step()
+        torch.cuda.synchronize(dev)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            one_step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / steps
+    passes = w.M * (w.steps + 1) if w.block_causal else 1
+    tokens = (w.M if w.block_causal else 1) * w.B * w.N
+    nb = hq.numel() * hq.element_size()
+    return {"ms_per_step": ms, "tokens_per_step": tokens, "steps": steps,
+            "h2d_bytes_per_step": 3 * nb * passes, "d2h_bytes_per_step": nb * passes}
+
+
+# ---------------------------------------------------------------------------
+
+
+def config_of(w, world, n_sets=None, per_set=None):
+    c = {"workload": w.name, "model": "Sana-1.6B" if w.H == 70 else "Sana-0.6B",
+         "global_batch": w.B * world, "seq_len": w.N, "heads": w.H, "head_dim": D,
+         "rope": "3d 8/12/12 base 1e4" if w.rope else "none", "eps": w.eps,
+         "parallelism": f"dp{world} (independent replicas)", "io": "bf16",
+         "accumulate": "f32"}
+    if w.outlier_frac:
+        c["k_outliers"] = f"{w.outlier_frac:.0%} of K entries x{w.outlier_scale:g}"
+    if w.block_causal:
+        c.update({"blocks": w.M, "block_tokens": w.N, "passes_per_block": w.steps + 1,
+                  "video_tokens": w.M * w.N})
+    if n_sets is not None:
+        c["l2"] = (f"inputs larger than L2: {n_sets} rotating input sets of "
+                   f"{per_set / 1e6:.0f} MB ({n_sets * per_set / 1e6:.0f} MB > 126 MB L2)")
+    return c
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["la", "reference"], default="la")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--soak", type=float, default=1.0)
+    args = ap.parse_args()
+    w = wl.WORKLOADS[args.workload]
+    if args.steps is None:
+        per_step_us = {"sana0.6b_512px": 10, "sana1.6b_1024px": 30, "sana1.6b_4k": 120,
+                       "sanavideo_480p": 250, "longsana_block_causal": 12000}[w.name]
+        args.steps = max(10, int(0.5e6 / per_step_us))
+    args.warmup = max(args.warmup, 3)
+
+    world = env_int("WORLD_SIZE", 1)
+    rank = env_int("RANK", 0)
+    local_rank = env_int("LOCAL_RANK", 0)
+
+    if args.impl == "reference":
+        return main_reference(args, w, rank, world)
+
+    import torch
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    r = run_la(args, w, rank, world, local_rank)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+
+    ms_step = r["ms"] / args.steps
+    tokens_step = (w.M * w.N * w.B) if w.block_causal else w.B * w.N
+    value = world * tokens_step * args.steps / (r["ms"] / 1e3)
+    peak, peak_src = peaks()
+    lb = layer_bytes(w)
+    if w.block_causal:
+        name = "la_block_causal_step(update=0)"
+        alg = 4 * w.B * w.N * w.H * D * 2 + 2 * w.B * w.H * (D * D + D) * 4
+        dur_us = r["seg_us"][0]
+        kernels = {name: {"avg_us": dur_us, "algorithmic_bytes": alg,
+                          "gbs": alg / (dur_us * 1e-6) / 1e9, "launches": 2}}
+        dom = name
+        traffic = None
+    else:
+        kernels = {}
+        for nm, us in zip(r["kernel_names"], r["seg_us"]):
+            kernels[nm] = {"avg_us": us, "algorithmic_bytes": lb[nm],
+                           "gbs": lb[nm] / (us * 1e-6) / 1e9, "launches": 1}
+        dom = max(kernels, key=lambda k: kernels[k]["avg_us"])
+        traffic = profiled_traffic(w.name, dom)
+    kd = kernels[dom]
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(kd["gbs"], 1),
+                "peak": peak, "unit": "GB/s", "frac": round(kd["gbs"] / peak, 4),
+                "traffic": traffic, "algorithmic_bytes": kd["algorithmic_bytes"],
+                "avg_launch_us": round(kd["avg_us"], 3), "peak_source": peak_src,
+                "per_kernel": {k: {"avg_us": round(v["avg_us"], 3), "gbs": round(v["gbs"], 1),
+                                   "frac": round(v["gbs"] / peak, 4)}
+                               for k, v in kernels.items()}}
+    e = r["e2e"]
+    e2e = {"value": world * e["tokens_per_step"] / (e["ms_per_step"] / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": e["h2d_bytes_per_step"],
+           "d2h_bytes_per_step": e["d2h_bytes_per_step"], "steps": e["steps"],
+           "ms_per_step": round(e["ms_per_step"], 4),
+           "api": "la_block_causal_step" if w.block_causal else "la_attention"}
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+           "latency_us": ms_step * 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), bf16)",
+           "config": config_of(w, world, r["n_sets"], r["per_set_bytes"]),
+           "roofline": roofline, "e2e": e2e,
+           "gpu_launches": r["launches_per_step"] * args.steps,
+           "clocks": r["clocks"], "graph_chunk_steps": r["chunk"], "soak_s": args.soak}
+    if world == 1:
+        tps, desc, cores, _, _ = oracle_sample(w, args.cpu_seconds)
+        out["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores,
+                               "kind": "oracle", "sample": desc}
+    print(json.dumps(out), flush=True)
+
+
+def main_reference(args, w, rank, world):
+    """The float64 oracle, timed as it stands on the host's cores."""
+    if rank != 0:
+        return
+    budget = 150.0  # seconds for warm-up + timed steps together
+    per = budget / (args.steps + args.warmup)
+    _, _, cores, per_call, h_sub = oracle_sample(w, min(per, 3.0), max_reps=1)
+    # each step: one oracle call on h_sub heads (at most `per` seconds)
+    import oracle as orc
+    import numpy as np
+    th = orc.rope_angles(w.T, w.Hh, w.W, 0, w.rope_base) if w.rope else None
+    Q, K, V = (x[:, :, :h_sub].contiguous() for x in wl.make_qkv(w, 0))
+
+    def call():
+        if w.block_causal:
+            orc.block_causal_step(Q, K, V, np.zeros((w.B, h_sub, D, D)),
+                                  np.zeros((w.B, h_sub, D)), 1, w.eps, th)
+        else:
+            orc.attention(Q, K, V, w.eps, th)
+
+    for _ in range(args.warmup):
+        call()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        call()
+    el = time.perf_counter() - t0
+    per_call = el / args.steps
+    full_call = per_call * w.H / h_sub
+    if w.block_causal:
+        calls = w.M * (w.steps + 1)
+        value = w.M * w.N * w.B / (full_call * calls)
+        ms_step = full_call * calls * 1e3
+        sample = (f"each step: oracle block_causal_step on {h_sub} of {w.H} heads of one block; "
+                  f"scaled to {w.H} heads x {calls} calls per video")
+    else:
+        value = w.B * w.N / full_call
+        ms_step = full_call * 1e3
+        sample = f"each step: oracle attention on {h_sub} of {w.H} heads; scaled to {w.H} heads"
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded N(0,1), bf16 inputs read exactly)",
+           "config": config_of(w, world),
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

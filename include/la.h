@@ -1,0 +1,166 @@
+/*
+ * la.h -- C ABI of the B200 (sm_100a) ReLU linear-attention library.
+ *
+ * What the library computes, per batch element b and head h, with head
+ * width D = 32 and eps >= 0:
+ *
+ *   k+ = ReLU(k),  q+ = ReLU(q)
+ *   phi(x) = ReLU(x)                     (rope = 0)
+ *   phi(x) = R(t, h, w) ReLU(x)          (rope = 1: 3D RoPE after ReLU)
+ *   S = sum_n phi(k_n)^T v_n             (D x D, float32)
+ *   z = sum_n k+_n                       (D, float32; never rotated)
+ *   O_n = phi(q_n) S / (q+_n . z + eps)
+ *
+ * Sources (page title, section):
+ *   "Sana: Efficient High-Resolution Image Synthesis with Linear Diffusion
+ *   Transformers", section 模型架构 item 2: ReLU linear attention whose shared
+ *   terms sum ReLU(K_j)^T V_j and sum ReLU(K_j)^T are computed once and reused
+ *   by every query.
+ *   "SANA-Video: Efficient Video Generation with Block Linear Diffusion
+ *   Transformer", section 2.1 (state computed in advance, O(D^2) per token),
+ *   section 2.2 (RoPE after ReLU; the denominator stays unrotated), section
+ *   2.3 (causal state kept in D x D + D memory), section 4 (block inference
+ *   loop: the KV cache starts empty and folds in each block once, after its
+ *   last denoising step), "Stage 2" (3D RoPE over time, height and width).
+ *
+ * The formula of section 2.1 is lost on the pages. This library reads it as
+ * above: no 1/sqrt(D) scale and eps added to the denominator.
+ *
+ * 3D RoPE convention (not fixed by the pages): dims [0,8) turn with the frame
+ * index t, [8,20) with the row h, [20,32) with the column w; pairs (2i, 2i+1)
+ * are interleaved; pair k of a segment of width d turns by
+ * p * rope_base^(-2k/d); (x0, x1) -> (x0 cos - x1 sin, x0 sin + x1 cos).
+ * Tokens are in raster order n = (t_local*Hh + h)*W + w and
+ * t = t_offset + t_local is the global frame index.
+ *
+ * Conventions shared by every entry point:
+ *   - Layout: Q, K, V, O are dense row-major [B, N, H, D] tensors of
+ *     io_dtype (bf16 or float32). S is float32 [B, H, D, D] (row d, column
+ *     e) and z is float32 [B, H, D].
+ *   - Memory: every tensor pointer is a DEVICE pointer owned by the caller,
+ *     16-byte aligned. The library allocates nothing and keeps no state
+ *     between calls. Scratch memory ("workspace") is passed in by the
+ *     caller; its size comes from la_workspace_bytes(). A workspace must be
+ *     zero-filled once before its first use (cudaMemsetAsync(ws, 0, bytes));
+ *     every call leaves it zero-filled where it matters again, so it is
+ *     reused without clearing. One workspace serves one call at a time:
+ *     calls that share a workspace must be ordered (same stream or events).
+ *     After a call that failed with LA_ERR_CUDA, zero-fill it again.
+ *   - Execution: every call is asynchronous on `stream` (NULL = the legacy
+ *     default stream). A call returns after enqueuing its kernels; faults
+ *     inside kernels surface at the caller's next synchronisation.
+ *   - Errors: arguments are checked on the host before any launch; a bad
+ *     argument returns LA_ERR_INVALID_ARG / LA_ERR_UNSUPPORTED /
+ *     LA_ERR_WORKSPACE and launches nothing. A launch failure returns
+ *     LA_ERR_CUDA. Nothing throws across the ABI. la_last_error() gives a
+ *     one-line description of the last failure on the calling thread.
+ *   - Determinism: for a given shape the reduction order is fixed (split
+ *     count and combine order depend on the shape only), so S, z and O are
+ *     bitwise identical from run to run.
+ *   - Aliasing: O must not overlap Q, K or V; S and z must not overlap the
+ *     inputs or the workspace.
+ */
+#ifndef LA_H_
+#define LA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so that this header needs no
+ * CUDA header. */
+typedef struct CUstream_st* la_stream;
+
+typedef enum {
+  LA_OK = 0,
+  LA_ERR_INVALID_ARG = 1, /* null / misaligned pointer, negative size, bad flag */
+  LA_ERR_UNSUPPORTED = 2, /* a valid request this build does not handle (D != 32) */
+  LA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than la_workspace_bytes() */
+  LA_ERR_CUDA = 4         /* a CUDA runtime call or kernel launch failed */
+} la_status;
+
+typedef enum { LA_IO_BF16 = 0, LA_IO_F32 = 1 } la_io_dtype;
+
+typedef struct {
+  int B;            /* batch elements, >= 0 */
+  int N;            /* tokens per batch element (per block in block-causal mode), >= 0 */
+  int H;            /* heads, >= 0 */
+  int D;            /* head width; must be 32 */
+  int io_dtype;     /* la_io_dtype of Q, K, V and O */
+  int rope;         /* 0: phi = ReLU; 1: phi = 3D RoPE after ReLU */
+  int T, Hh, W;     /* RoPE latent grid; N == T*Hh*W when rope = 1 */
+  int t_offset;     /* global frame index of this block's first frame, >= 0 */
+  double rope_base; /* RoPE base (10000), > 1 */
+  float eps;        /* denominator guard, >= 0 and finite */
+} la_shape;
+
+/* Bytes of scratch memory that la_state_reduce, la_attention and
+ * la_block_causal_step need for `shape`. Returns 0 iff `shape` is invalid.
+ * Pure host function; it does not touch the GPU. */
+size_t la_workspace_bytes(const la_shape* shape);
+
+/* State reduce (the shared terms of the Sana Linear DiT, section 模型架构
+ * item 2; SANA-Video section 2.1):
+ *   S[b,h] = sum_n phi(k_n)^T v_n,  z[b,h] = sum_n ReLU(k_n).
+ * K, V: [B,N,H,D] io_dtype (device, read only). S: [B,H,D,D] float32, z:
+ * [B,H,D] float32 (device, written). ws: device workspace of at least
+ * la_workspace_bytes(shape) bytes (see the workspace rule above).
+ * One launch: the token axis is cut into splits that depend on the shape
+ * only; each CTA writes its split's partial state to the workspace and the
+ * last CTA to finish for a head sums the partials in split order.
+ * N == 0 gives S = 0, z = 0. */
+la_status la_state_reduce(const la_shape* shape, const void* K, const void* V,
+                          float* S, float* z, void* ws, size_t ws_bytes,
+                          la_stream stream);
+
+/* Apply (SANA-Video sections 2.1 and 2.2):
+ *   O_n = phi(q_n) S / (ReLU(q_n) . z + eps).
+ * Q: [B,N,H,D] io_dtype (read), S: [B,H,D,D] float32 and z: [B,H,D] float32
+ * (read), O: [B,N,H,D] io_dtype (written; bf16 output is rounded to
+ * nearest-even). A row with ReLU(q) = 0 gives O = 0. Needs no workspace. */
+la_status la_apply(const la_shape* shape, const void* Q, const float* S,
+                   const float* z, void* O, la_stream stream);
+
+/* Non-causal attention in one call: la_state_reduce followed by la_apply.
+ * S and z receive the state (they may be NULL, in which case the state is
+ * kept in the workspace only). */
+la_status la_attention(const la_shape* shape, const void* Q, const void* K,
+                       const void* V, float* S, float* z, void* O, void* ws,
+                       size_t ws_bytes, la_stream stream);
+
+/* One call of the block-causal mode with the constant-memory KV cache
+ * (SANA-Video sections 2.3 and 4; SANA-Video article, section 设计细节):
+ * the block's own state (S_own, z_own) is reduced from (K, V), then
+ *   update = 0: O = apply(Q, S_carry + S_own, z_carry + z_own); carry unchanged.
+ *   update = 1: the same O; then S_carry += S_own, z_carry += z_own.
+ *   update = 2: the carry update only; Q and O are not used (may be NULL).
+ * Earlier blocks reach this block only through the carry; attention within
+ * the block is global. S_carry [B,H,D,D], z_carry [B,H,D] float32 (device,
+ * read and, for update >= 1, written in place). shape->t_offset is the global
+ * frame index of the block's first frame. The sum carry + own is formed once,
+ * in a fixed order, and the apply uses exactly the value stored in the carry
+ * for update = 1. */
+la_status la_block_causal_step(const la_shape* shape, const void* Q,
+                               const void* K, const void* V, float* S_carry,
+                               float* z_carry, void* O, int update, void* ws,
+                               size_t ws_bytes, la_stream stream);
+
+/* Reset of the KV cache at the start of a video (SANA-Video section 4: the
+ * cache starts empty): S[B,H,D,D] = 0, z[B,H,D] = 0 on `stream`. */
+la_status la_state_reset(float* S, float* z, int B, int H, int D,
+                         la_stream stream);
+
+/* Static description of a status code. Never NULL. */
+const char* la_status_string(la_status status);
+
+/* One-line description of the last failure on the calling thread (empty
+ * string if none). The pointer stays valid until the thread's next call. */
+const char* la_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_H_ */

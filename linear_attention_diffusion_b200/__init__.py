@@ -1,0 +1,189 @@
+"""ReLU linear attention on B200 (sm_100a): a thin ctypes binding of ``libla_b200.so``.
+
+The functions below carry the names of the C ABI in ``include/la.h`` and only
+marshal arguments (tensor pointers, sizes, the stream) into it; every step of
+the computation runs in the library's CUDA kernels. There is no CPU path:
+importing this package fails if the library has not been built
+(``python linear_attention_diffusion_b200/build.py``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libla_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python linear_attention_diffusion_b200/build.py`"
+        " (this package has no CPU fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+LA_OK = 0
+LA_ERR_INVALID_ARG = 1
+LA_ERR_UNSUPPORTED = 2
+LA_ERR_WORKSPACE = 3
+LA_ERR_CUDA = 4
+LA_IO_BF16 = 0
+LA_IO_F32 = 1
+HEAD_DIM = 32
+
+
+class LaShape(ctypes.Structure):
+    """Mirror of ``la_shape`` in include/la.h."""
+
+    _fields_ = [
+        ("B", ctypes.c_int), ("N", ctypes.c_int), ("H", ctypes.c_int), ("D", ctypes.c_int),
+        ("io_dtype", ctypes.c_int), ("rope", ctypes.c_int),
+        ("T", ctypes.c_int), ("Hh", ctypes.c_int), ("W", ctypes.c_int),
+        ("t_offset", ctypes.c_int), ("rope_base", ctypes.c_double), ("eps", ctypes.c_float),
+    ]
+
+
+class LaError(RuntimeError):
+    def __init__(self, status: int, func: str):
+        self.status = status
+        detail = la_last_error()
+        super().__init__(f"{func}: {la_status_string(status)}" + (f" -- {detail}" if detail else ""))
+
+
+_vp = ctypes.c_void_p
+_sz = ctypes.c_size_t
+_i = ctypes.c_int
+_shape_p = ctypes.POINTER(LaShape)
+
+_lib.la_workspace_bytes.argtypes = [_shape_p]
+_lib.la_workspace_bytes.restype = _sz
+_lib.la_state_reduce.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.la_state_reduce.restype = _i
+_lib.la_apply.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp]
+_lib.la_apply.restype = _i
+_lib.la_attention.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.la_attention.restype = _i
+_lib.la_block_causal_step.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]
+_lib.la_block_causal_step.restype = _i
+_lib.la_state_reset.argtypes = [_vp, _vp, _i, _i, _i, _vp]
+_lib.la_state_reset.restype = _i
+_lib.la_status_string.argtypes = [_i]
+_lib.la_status_string.restype = ctypes.c_char_p
+_lib.la_last_error.argtypes = []
+_lib.la_last_error.restype = ctypes.c_char_p
+
+
+def make_shape(B: int, N: int, H: int, D: int = HEAD_DIM, io_dtype: str = "bf16",
+               rope: bool = False, T: int = 0, Hh: int = 0, W: int = 0,
+               t_offset: int = 0, rope_base: float = 10000.0, eps: float = 1e-6) -> LaShape:
+    io = {"bf16": LA_IO_BF16, "f32": LA_IO_F32, "float32": LA_IO_F32}[io_dtype]
+    return LaShape(int(B), int(N), int(H), int(D), io, int(bool(rope)), int(T), int(Hh),
+                   int(W), int(t_offset), float(rope_base), float(eps))
+
+
+def _ptr(x) -> Optional[int]:
+    """Device address of a tensor (or an int address); None for NULL."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if not x.is_cuda:
+        raise ValueError("tensor arguments must live on a CUDA device")
+    if not x.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous")
+    return x.data_ptr()
+
+
+def _nbytes(x) -> int:
+    return 0 if x is None else x.numel() * x.element_size()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, func: str) -> None:
+    if status != LA_OK:
+        raise LaError(status, func)
+
+
+def la_workspace_bytes(shape: LaShape) -> int:
+    return int(_lib.la_workspace_bytes(ctypes.byref(shape)))
+
+
+def la_state_reduce(shape: LaShape, K, V, S, z, ws, stream=None) -> None:
+    _check(_lib.la_state_reduce(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(S), _ptr(z),
+                                _ptr(ws), _nbytes(ws), _stream(stream)), "la_state_reduce")
+
+
+def la_apply(shape: LaShape, Q, S, z, O, stream=None) -> None:
+    _check(_lib.la_apply(ctypes.byref(shape), _ptr(Q), _ptr(S), _ptr(z), _ptr(O),
+                         _stream(stream)), "la_apply")
+
+
+def la_attention(shape: LaShape, Q, K, V, S, z, O, ws, stream=None) -> None:
+    _check(_lib.la_attention(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(z),
+                             _ptr(O), _ptr(ws), _nbytes(ws), _stream(stream)), "la_attention")
+
+
+def la_block_causal_step(shape: LaShape, Q, K, V, S_carry, z_carry, O, update: int, ws,
+                         stream=None) -> None:
+    _check(_lib.la_block_causal_step(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V),
+                                     _ptr(S_carry), _ptr(z_carry), _ptr(O), int(update),
+                                     _ptr(ws), _nbytes(ws), _stream(stream)),
+           "la_block_causal_step")
+
+
+def la_state_reset(S, z, B: int, H: int, D: int = HEAD_DIM, stream=None) -> None:
+    _check(_lib.la_state_reset(_ptr(S), _ptr(z), int(B), int(H), int(D), _stream(stream)),
+           "la_state_reset")
+
+
+def la_status_string(status: int) -> str:
+    return _lib.la_status_string(int(status)).decode()
+
+
+def la_last_error() -> str:
+    return _lib.la_last_error().decode()
+
+
+# ---------------------------------------------------------------------------
+# Convenience wrappers that allocate outputs with torch (device memory only).
+
+def shape_for(Q, eps: float = 1e-6, rope_grid=None, t_offset: int = 0,
+              rope_base: float = 10000.0) -> LaShape:
+    """la_shape for a [B, N, H, D] tensor; ``rope_grid`` = (T, Hh, W) turns on RoPE."""
+    import torch
+    B, N, H, D = Q.shape
+    io = "bf16" if Q.dtype == torch.bfloat16 else "f32"
+    if rope_grid is None:
+        return make_shape(B, N, H, D, io, False, eps=eps)
+    T, Hh, W = rope_grid
+    return make_shape(B, N, H, D, io, True, T, Hh, W, t_offset, rope_base, eps)
+
+
+def workspace(shape: LaShape, device="cuda"):
+    """A zero-filled workspace of la_workspace_bytes(shape) bytes."""
+    import torch
+    n = la_workspace_bytes(shape)
+    if n == 0:
+        raise LaError(LA_ERR_INVALID_ARG, "la_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def attention(Q, K, V, eps: float = 1e-6, rope_grid=None, t_offset: int = 0,
+              rope_base: float = 10000.0, stream=None):
+    """O, S, z of non-causal ReLU linear attention for [B, N, H, 32] CUDA tensors."""
+    import torch
+    shape = shape_for(Q, eps, rope_grid, t_offset, rope_base)
+    B, N, H, D = Q.shape
+    S = torch.empty((B, H, D, D), dtype=torch.float32, device=Q.device)
+    z = torch.empty((B, H, D), dtype=torch.float32, device=Q.device)
+    O = torch.empty_like(Q)
+    la_attention(shape, Q, K, V, S, z, O, workspace(shape, Q.device), stream)
+    return O, S, z

@@ -1,0 +1,316 @@
+// C-ABI layer: argument checks on the host, workspace layout, and the order
+// of the kernel launches for each entry point of include/la.h.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "la.h"
+#include "la_internal.h"
+
+namespace la {
+namespace {
+
+thread_local std::string g_last_error;
+
+la_status fail(la_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+la_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(LA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Token splits of the state reduce: a function of (B, N, H) only, so that
+// the reduction order, and with it every bit of S and z, is fixed per shape.
+// About two CTAs of four heads per SM, at least one 128-token tile per split.
+void choose_splits(Problem& p) {
+  const int groups = ceil_div(p.H, 4);
+  const long long units = static_cast<long long>(p.B) * groups;
+  int splits = units > 0 ? static_cast<int>((2LL * kNumSMs) / units) : 1;
+  const int max_splits = p.N > 0 ? ceil_div(p.N, kTileTokens) : 1;
+  if (splits > max_splits) splits = max_splits;
+  if (splits > 64) splits = 64;
+  if (splits < 1) splits = 1;
+  int chunk = p.N > 0 ? ceil_div(ceil_div(p.N, splits), kTileTokens) * kTileTokens : kTileTokens;
+  p.chunk = chunk;
+  p.splits = p.N > 0 ? ceil_div(p.N, chunk) : 1;
+}
+
+la_status make_problem(const la_shape* s, Problem& p) {
+  if (s == nullptr) return fail(LA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->B < 0 || s->N < 0 || s->H < 0)
+    return fail(LA_ERR_INVALID_ARG, "negative size B=%d N=%d H=%d", s->B, s->N, s->H);
+  if (s->D != kD) return fail(LA_ERR_UNSUPPORTED, "head width D=%d (only 32 is built)", s->D);
+  if (s->io_dtype != LA_IO_BF16 && s->io_dtype != LA_IO_F32)
+    return fail(LA_ERR_INVALID_ARG, "io_dtype=%d", s->io_dtype);
+  if (s->rope != 0 && s->rope != 1) return fail(LA_ERR_INVALID_ARG, "rope=%d", s->rope);
+  if (!(std::isfinite(s->eps) && s->eps >= 0.0f))
+    return fail(LA_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  const long long elems = 1LL * s->B * s->N * s->H * kD;
+  if (elems >= (1LL << 40)) return fail(LA_ERR_UNSUPPORTED, "tensor too large");
+  if (1LL * s->B * s->H * 65536LL >= (1LL << 40) || s->B > 65535 || s->H > 65535)
+    return fail(LA_ERR_UNSUPPORTED, "B or H above 65535");
+  std::memset(&p, 0, sizeof(p));
+  p.B = s->B;
+  p.N = s->N;
+  p.H = s->H;
+  p.io = s->io_dtype;
+  p.eps = s->eps;
+  if (s->rope) {
+    if (s->T < 1 || s->Hh < 1 || s->W < 1)
+      return fail(LA_ERR_INVALID_ARG, "RoPE grid T=%d Hh=%d W=%d", s->T, s->Hh, s->W);
+    if (1LL * s->T * s->Hh * s->W != s->N)
+      return fail(LA_ERR_INVALID_ARG, "N=%d != T*Hh*W=%lld", s->N, 1LL * s->T * s->Hh * s->W);
+    if (s->t_offset < 0 || 1LL * s->t_offset + s->T > (1LL << 30))
+      return fail(LA_ERR_INVALID_ARG, "t_offset=%d", s->t_offset);
+    if (!(std::isfinite(s->rope_base) && s->rope_base > 1.0))
+      return fail(LA_ERR_INVALID_ARG, "rope_base must be finite and > 1");
+    p.rope.enabled = 1;
+    p.rope.T = s->T;
+    p.rope.Hh = s->Hh;
+    p.rope.W = s->W;
+    p.rope.t_offset = s->t_offset;
+    // Segments of the head: 8 dims (4 pairs) time, 12 (6) height, 12 (6) width.
+    const int seg_pairs[3] = {4, 6, 6};
+    int j = 0;
+    for (int a = 0; a < 3; ++a) {
+      const int width = 2 * seg_pairs[a];
+      for (int k = 0; k < seg_pairs[a]; ++k, ++j) {
+        p.rope.axis[j] = a;
+        p.rope.inv_freq[j] = std::pow(s->rope_base, -2.0 * k / width);
+      }
+    }
+  }
+  choose_splits(p);
+  return LA_OK;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+la_status check_ptr(const void* ptr, const char* name, bool needed) {
+  if (!needed) return LA_OK;
+  if (ptr == nullptr) return fail(LA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(ptr)) return fail(LA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return LA_OK;
+}
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (a == nullptr || b == nullptr || na == 0 || nb == 0) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+size_t io_bytes(const Problem& p) {
+  return static_cast<size_t>(p.B) * p.N * p.H * kD * (p.io == 0 ? 2 : 4);
+}
+size_t s_bytes(const Problem& p) { return static_cast<size_t>(p.B) * p.H * kD * kD * 4; }
+size_t z_bytes(const Problem& p) { return static_cast<size_t>(p.B) * p.H * kD * 4; }
+
+#define LA_TRY(expr)                 \
+  do {                               \
+    const la_status st_ = (expr);    \
+    if (st_ != LA_OK) return st_;    \
+  } while (0)
+
+la_status check_ws(const Problem& p, const void* ws, size_t ws_bytes) {
+  const size_t need = workspace_layout(p).total;
+  if (ws == nullptr) return fail(LA_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", need);
+  if (!aligned16(ws)) return fail(LA_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+  if (ws_bytes < need)
+    return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", ws_bytes, need);
+  return LA_OK;
+}
+
+// State reduce of (K, V) into `out`, using the workspace's partials and
+// counters.
+la_status run_reduce(const Problem& p, const void* K, const void* V, char* ws,
+                     const StateOut& out, cudaStream_t st) {
+  const WsLayout L = workspace_layout(p);
+  const cudaError_t e = launch_reduce(p, K, V, reinterpret_cast<float*>(ws + L.partials),
+                                      reinterpret_cast<unsigned*>(ws + L.counters), out, st);
+  if (e != cudaSuccess) return cuda_fail(e, "state reduce");
+  return LA_OK;
+}
+
+}  // namespace
+
+WsLayout workspace_layout(const Problem& p) {
+  WsLayout L;
+  const size_t bh = static_cast<size_t>(p.B) * p.H;
+  L.counters = 0;
+  L.partials = align256(bh * sizeof(unsigned));
+  L.state_S = align256(L.partials + bh * p.splits * kStateFloats * sizeof(float));
+  L.state_z = align256(L.state_S + bh * kD * kD * sizeof(float));
+  L.total = align256(L.state_z + bh * kD * sizeof(float));
+  if (L.total == 0) L.total = 256;
+  return L;
+}
+
+}  // namespace la
+
+using namespace la;
+
+extern "C" {
+
+size_t la_workspace_bytes(const la_shape* shape) {
+  Problem p;
+  if (make_problem(shape, p) != LA_OK) return 0;
+  return workspace_layout(p).total;
+}
+
+la_status la_state_reduce(const la_shape* shape, const void* K, const void* V, float* S,
+                          float* z, void* ws, size_t ws_bytes, la_stream stream) {
+  Problem p;
+  LA_TRY(make_problem(shape, p));
+  const bool any_state = p.B > 0 && p.H > 0;
+  const bool any_input = any_state && p.N > 0;
+  LA_TRY(check_ptr(K, "K", any_input));
+  LA_TRY(check_ptr(V, "V", any_input));
+  LA_TRY(check_ptr(S, "S", any_state));
+  LA_TRY(check_ptr(z, "z", any_state));
+  LA_TRY(check_ws(p, ws, ws_bytes));
+  if (overlap(S, s_bytes(p), ws, ws_bytes) || overlap(z, z_bytes(p), ws, ws_bytes) ||
+      overlap(S, s_bytes(p), z, z_bytes(p)))
+    return fail(LA_ERR_INVALID_ARG, "S, z and the workspace must not overlap");
+  if (!any_state) return LA_OK;
+  const StateOut out = {nullptr, nullptr, S, z, nullptr, nullptr};
+  return run_reduce(p, K, V, static_cast<char*>(ws), out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status la_apply(const la_shape* shape, const void* Q, const float* S, const float* z,
+                   void* O, la_stream stream) {
+  Problem p;
+  LA_TRY(make_problem(shape, p));
+  const bool any = p.B > 0 && p.H > 0 && p.N > 0;
+  LA_TRY(check_ptr(Q, "Q", any));
+  LA_TRY(check_ptr(S, "S", any));
+  LA_TRY(check_ptr(z, "z", any));
+  LA_TRY(check_ptr(O, "O", any));
+  if (overlap(O, io_bytes(p), Q, io_bytes(p)) || overlap(O, io_bytes(p), S, s_bytes(p)) ||
+      overlap(O, io_bytes(p), z, z_bytes(p)))
+    return fail(LA_ERR_INVALID_ARG, "O must not overlap Q, S or z");
+  if (!any) return LA_OK;
+  const cudaError_t e = launch_apply(p, Q, S, z, O, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "apply");
+  return LA_OK;
+}
+
+la_status la_attention(const la_shape* shape, const void* Q, const void* K, const void* V,
+                       float* S, float* z, void* O, void* ws, size_t ws_bytes,
+                       la_stream stream) {
+  Problem p;
+  LA_TRY(make_problem(shape, p));
+  const bool any_state = p.B > 0 && p.H > 0;
+  const bool any_input = any_state && p.N > 0;
+  LA_TRY(check_ptr(Q, "Q", any_input));
+  LA_TRY(check_ptr(K, "K", any_input));
+  LA_TRY(check_ptr(V, "V", any_input));
+  LA_TRY(check_ptr(O, "O", any_input));
+  if ((S == nullptr) != (z == nullptr))
+    return fail(LA_ERR_INVALID_ARG, "S and z must both be given or both be NULL");
+  LA_TRY(check_ptr(S, "S", any_state && S != nullptr));
+  LA_TRY(check_ptr(z, "z", any_state && z != nullptr));
+  LA_TRY(check_ws(p, ws, ws_bytes));
+  const size_t nb = io_bytes(p);
+  if (overlap(O, nb, Q, nb) || overlap(O, nb, K, nb) || overlap(O, nb, V, nb) ||
+      overlap(O, nb, ws, ws_bytes) || overlap(S, s_bytes(p), ws, ws_bytes) ||
+      overlap(z, z_bytes(p), ws, ws_bytes) || overlap(O, nb, S, s_bytes(p)) ||
+      overlap(O, nb, z, z_bytes(p)))
+    return fail(LA_ERR_INVALID_ARG, "O, S, z and the workspace must not overlap each other or the inputs");
+  if (!any_state) return LA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const WsLayout L = workspace_layout(p);
+  float* Sw = reinterpret_cast<float*>(w + L.state_S);
+  float* zw = reinterpret_cast<float*>(w + L.state_z);
+  const StateOut out = {nullptr, nullptr, Sw, zw, S, z};
+  LA_TRY(run_reduce(p, K, V, w, out, st));
+  if (!any_input) return LA_OK;
+  const cudaError_t e = launch_apply(p, Q, Sw, zw, O, st);
+  if (e != cudaSuccess) return cuda_fail(e, "apply");
+  return LA_OK;
+}
+
+la_status la_block_causal_step(const la_shape* shape, const void* Q, const void* K,
+                               const void* V, float* S_carry, float* z_carry, void* O,
+                               int update, void* ws, size_t ws_bytes, la_stream stream) {
+  Problem p;
+  LA_TRY(make_problem(shape, p));
+  if (update < 0 || update > 2) return fail(LA_ERR_INVALID_ARG, "update=%d (0, 1 or 2)", update);
+  const bool any_state = p.B > 0 && p.H > 0;
+  const bool any_input = any_state && p.N > 0;
+  const bool uses_q = update != 2;
+  LA_TRY(check_ptr(Q, "Q", any_input && uses_q));
+  LA_TRY(check_ptr(O, "O", any_input && uses_q));
+  LA_TRY(check_ptr(K, "K", any_input));
+  LA_TRY(check_ptr(V, "V", any_input));
+  LA_TRY(check_ptr(S_carry, "S_carry", any_state));
+  LA_TRY(check_ptr(z_carry, "z_carry", any_state));
+  LA_TRY(check_ws(p, ws, ws_bytes));
+  const size_t nb = io_bytes(p);
+  if (overlap(S_carry, s_bytes(p), ws, ws_bytes) || overlap(z_carry, z_bytes(p), ws, ws_bytes) ||
+      overlap(S_carry, s_bytes(p), z_carry, z_bytes(p)) ||
+      (uses_q && (overlap(O, nb, Q, nb) || overlap(O, nb, K, nb) || overlap(O, nb, V, nb) ||
+                  overlap(O, nb, ws, ws_bytes) || overlap(O, nb, S_carry, s_bytes(p)) ||
+                  overlap(O, nb, z_carry, z_bytes(p)))))
+    return fail(LA_ERR_INVALID_ARG, "O, the carry and the workspace must not overlap");
+  if (!any_state) return LA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const WsLayout L = workspace_layout(p);
+  float* Sw = reinterpret_cast<float*>(w + L.state_S);
+  float* zw = reinterpret_cast<float*>(w + L.state_z);
+  // total = carry + own, formed once; written to the workspace for the apply
+  // and, when updating, to the carry as well.
+  const bool to_ws = uses_q;
+  const bool to_carry = update >= 1;
+  const StateOut out = {S_carry, z_carry, to_ws ? Sw : nullptr, to_ws ? zw : nullptr,
+                        to_carry ? S_carry : nullptr, to_carry ? z_carry : nullptr};
+  LA_TRY(run_reduce(p, K, V, w, out, st));
+  if (!uses_q || !any_input) return LA_OK;
+  const cudaError_t e = launch_apply(p, Q, Sw, zw, O, st);
+  if (e != cudaSuccess) return cuda_fail(e, "apply");
+  return LA_OK;
+}
+
+la_status la_state_reset(float* S, float* z, int B, int H, int D, la_stream stream) {
+  if (B < 0 || H < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d", B, H);
+  if (D != kD) return fail(LA_ERR_UNSUPPORTED, "head width D=%d (only 32 is built)", D);
+  const bool any = B > 0 && H > 0;
+  LA_TRY(check_ptr(S, "S", any));
+  LA_TRY(check_ptr(z, "z", any));
+  if (!any) return LA_OK;
+  const size_t bh = static_cast<size_t>(B) * H;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(S, 0, bh * kD * kD * sizeof(float), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(z, 0, bh * kD * sizeof(float), st);
+  if (e != cudaSuccess) return cuda_fail(e, "state reset");
+  return LA_OK;
+}
+
+const char* la_status_string(la_status status) {
+  switch (status) {
+    case LA_OK: return "LA_OK";
+    case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG: invalid argument";
+    case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: unsupported request";
+    case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE: workspace missing or too small";
+    case LA_ERR_CUDA: return "LA_ERR_CUDA: CUDA runtime or launch failure";
+  }
+  return "unknown la_status";
+}
+
+const char* la_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// Internal interface between the C-ABI layer (la_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace la {
+
+constexpr int kD = 32;                 // head width (the only one supported)
+constexpr int kStateFloats = kD * kD + kD;  // one (S, z) pair: 32x32 + 32
+constexpr int kNumSMs = 148;           // B200; used for the shape-only split rule
+constexpr int kTileTokens = 128;       // token granularity of a split
+
+// 3D RoPE: per pair j in [0,16) the axis (0 = t, 1 = h, 2 = w) and the inverse
+// frequency base^(-2k/d) of its segment, computed on the host in double.
+struct Rope {
+  int enabled;
+  int T, Hh, W, t_offset;
+  double inv_freq[kD / 2];
+  int axis[kD / 2];
+};
+
+struct Problem {
+  int B, N, H;
+  int io;      // 0 bf16, 1 float32
+  float eps;
+  int splits;  // token splits of the state reduce (shape-only)
+  int chunk;   // tokens per split (multiple of kTileTokens)
+  Rope rope;
+};
+
+// Workspace layout (byte offsets, 256-aligned), a pure function of the shape.
+struct WsLayout {
+  size_t counters;  // [B*H] uint32 arrival counters; zero between calls
+  size_t partials;  // [B*H][splits][kStateFloats] float32
+  size_t state_S;   // [B*H][32*32] float32
+  size_t state_z;   // [B*H][32] float32
+  size_t total;
+};
+WsLayout workspace_layout(const Problem& p);
+
+// Where the reduce puts its result: the fixed-order sum of the split
+// partials, plus carry_* when given, is written to out1_* and/or out2_*
+// (each may be null; out2 may alias carry). All [B*H][32*32] / [B*H][32].
+struct StateOut {
+  const float* carry_S;
+  const float* carry_z;
+  float* out1_S;
+  float* out1_z;
+  float* out2_S;
+  float* out2_z;
+};
+
+// State reduce in one launch: every CTA writes its split's partial (S, z)
+// to `partials`; the last CTA to arrive for a head (counted in `counters`)
+// sums the partials in split order, applies StateOut, and re-zeroes the
+// counter. Deterministic: the sum order depends on the shape only.
+cudaError_t launch_reduce(const Problem& p, const void* K, const void* V, float* partials,
+                          unsigned* counters, const StateOut& out, cudaStream_t s);
+// O = phi(Q) S / (ReLU(Q) . z + eps).
+cudaError_t launch_apply(const Problem& p, const void* Q, const float* S,
+                         const float* z, void* O, cudaStream_t s);
+
+}  // namespace la

@@ -8,6 +8,20 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def _ensure_library_built():
+    # The CUDA library is built in-tree; rebuild it if a source is newer. The
+    # build script is loaded by path: importing the package needs the library.
+    import importlib.util
+    path = os.path.join(ROOT, "linear_attention_diffusion_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_la_b200_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
+_ensure_library_built()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size parity case")

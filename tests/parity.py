@@ -1,0 +1,104 @@
+"""Helpers of the GPU parity tests: run the CUDA path, compute the oracle, and
+compare them element by element with tolerances stated here.
+
+Tolerances.
+
+* Spec bar for O: |gpu - ref| <= 2e-3 + 2e-2 |ref| for bf16 output and
+  |gpu - ref| <= 1e-4 + 1e-4 |ref| for float32 output.
+* A tighter bar derived from the arithmetic, checked as well. With
+  A = sum_n |phi(k_n)|^T |v_n| (the magnitude of every term of S):
+    S:  |S_gpu - S_ref| <= tol_s * A
+    z:  |z_gpu - z_ref| <= 1e-5 * z_ref          (a sum of non-negative terms)
+    O:  |O_gpu - O_ref| <= out_round * |O_ref| + tol_o * (|phi(q)| A) / den
+  where den = ReLU(q).z + eps. out_round is the output rounding (2^-8 for
+  bf16, 1e-6 for float32). tol_s / tol_o are the relative errors of the
+  operands the kernels feed their contractions: 2e-5 when they are exact (bf16
+  inputs without RoPE) or float32, 2^-8 / 2^-7 when a rotated feature or the
+  state is rounded to bf16 for the tensor cores.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import linear_attention_diffusion_b200 as la
+import oracle as orc
+
+NS_BF16 = (2e-2, 2e-3)   # (rtol, atol)
+NS_F32 = (1e-4, 1e-4)
+
+
+def theta_for(w_rope, T, Hh, W, t_offset=0, base=10000.0):
+    return orc.rope_angles(T, Hh, W, t_offset, base) if w_rope else None
+
+
+def to_dev(*xs, dtype=None):
+    out = []
+    for x in xs:
+        x = x if dtype is None else x.to(dtype)
+        out.append(x.contiguous().cuda())
+    return out
+
+
+def gpu_attention(Q, K, V, eps, rope_grid=None, t_offset=0):
+    """Run la_attention on device copies of CPU tensors; return CPU O, S, z."""
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    O, S, z = la.attention(Qd, Kd, Vd, eps=eps, rope_grid=rope_grid, t_offset=t_offset)
+    torch.cuda.synchronize()
+    return O.cpu(), S.cpu(), z.cpu()
+
+
+def magnitude_state(K, V, theta):
+    kf = orc.to_f64(K)
+    vf = orc.to_f64(V)
+    phik = np.abs(orc.feature_map(kf, theta))
+    return np.matmul(phik.transpose(0, 2, 3, 1), np.abs(vf).transpose(0, 2, 1, 3))
+
+
+def check_state(S_gpu, z_gpu, S_ref, z_ref, A, tol_s, what=""):
+    S_gpu = orc.to_f64(S_gpu)
+    z_gpu = orc.to_f64(z_gpu)
+    err = np.abs(S_gpu - S_ref)
+    bound = tol_s * A + 1e-30
+    bad = err > bound
+    assert not bad.any(), (f"{what} S: {bad.sum()} of {bad.size} outside tol; worst ratio "
+                           f"{float((err / bound).max()):.3g}")
+    zerr = np.abs(z_gpu - z_ref)
+    zb = 1e-5 * np.abs(z_ref) + 1e-30
+    assert not (zerr > zb).any(), f"{what} z: worst ratio {float((zerr / zb).max()):.3g}"
+
+
+def check_output(O_gpu, O_ref, io, tol_o, Q=None, theta=None, A=None, z_ref=None, eps=None,
+                 rows=None, what=""):
+    """Spec tolerance always; the derived bound when Q, A, z_ref are given."""
+    O_gpu = orc.to_f64(O_gpu)
+    rtol, atol = NS_BF16 if io == "bf16" else NS_F32
+    err = np.abs(O_gpu - O_ref)
+    assert np.isfinite(O_gpu).all(), f"{what}: non-finite output"
+    ns = atol + rtol * np.abs(O_ref)
+    assert not (err > ns).any(), (f"{what}: {(err > ns).sum()} elements outside the "
+                                  f"north-star tolerance; max err {err.max():.3g}")
+    if Q is None:
+        return
+    qf = orc.to_f64(Q)
+    th = theta
+    if rows is not None:
+        qf = qf[:, rows]
+        th = None if theta is None else theta[rows]
+    phq = np.abs(orc.feature_map(qf, th))
+    num_abs = np.matmul(phq.transpose(0, 2, 1, 3), A).transpose(0, 2, 1, 3)
+    den = np.einsum("bnhd,bhd->bnh", orc.relu(qf), z_ref) + eps
+    out_round = 2.0 ** -8 if io == "bf16" else 1e-6
+    bound = out_round * np.abs(O_ref) + tol_o * num_abs / den[..., None] + 1e-30
+    bad = err > bound
+    assert not bad.any(), (f"{what}: {bad.sum()} elements outside the derived bound; worst "
+                           f"ratio {float((err / bound).max()):.3g}")
+
+
+def tolerances(io, rope):
+    """(tol_s, tol_o) of the current kernels for this I/O type and feature map."""
+    if io == "bf16" and rope:
+        return 2.0 ** -8, 2.0 ** -7
+    if io == "bf16":
+        return 2e-5, 2.0 ** -7
+    return 2e-5, 2e-5
