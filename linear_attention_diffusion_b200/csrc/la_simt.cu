@@ -48,9 +48,10 @@ template <typename T>
 __global__ void __launch_bounds__(kRedThreads)
 reduce_simt(const Problem p, const T* __restrict__ K, const T* __restrict__ V,
             float* partials, unsigned* counters, const StateOut out) {
-  __shared__ float ks[kRedTile][kD + 4];
-  __shared__ float vs[kRedTile][kD + 4];
-  __shared__ float red[4][kD * kD];
+  // float4 reads below: the staging arrays must be 16-byte aligned.
+  __shared__ __align__(16) float ks[kRedTile][kD + 4];
+  __shared__ __align__(16) float vs[kRedTile][kD + 4];
+  __shared__ __align__(16) float red[4][kD * kD];
   __shared__ float zred[kRedThreads / 4][kD / 8][8];
 
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
