@@ -367,7 +367,7 @@ def run_la(args, w, rank, world, local_rank):
         ms_max = float(t.item())
 
     # end-to-end through the public API with host buffers
-    e2e = run_e2e(args, w, dev, stream, la, rank)
+    e2e = run_e2e(args, w, dev, stream, la, rank) if args.e2e_steps > 0 else None
     clocks = sampler.summary(t0, t1)
     sampler.stop()
     del g_chunk, g_rem
@@ -458,6 +458,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["la", "reference"], default="la")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.WORKLOADS))
+    # --e2e-steps 0 and --cpu-seconds 0 leave out the end-to-end and CPU
+    # legs (for profiler runs; the timed region is the same either way).
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--soak", type=float, default=1.0)
@@ -516,11 +518,12 @@ def main():
                                    "frac": round(v["gbs"] / peak, 4)}
                                for k, v in kernels.items()}}
     e = r["e2e"]
-    e2e = {"value": world * e["tokens_per_step"] / (e["ms_per_step"] / 1e3), "unit": "tokens/s",
-           "h2d_bytes_per_step": e["h2d_bytes_per_step"],
-           "d2h_bytes_per_step": e["d2h_bytes_per_step"], "steps": e["steps"],
-           "ms_per_step": round(e["ms_per_step"], 4),
-           "api": "la_block_causal_step" if w.block_causal else "la_attention"}
+    e2e = None if e is None else {
+        "value": world * e["tokens_per_step"] / (e["ms_per_step"] / 1e3), "unit": "tokens/s",
+        "h2d_bytes_per_step": e["h2d_bytes_per_step"],
+        "d2h_bytes_per_step": e["d2h_bytes_per_step"], "steps": e["steps"],
+        "ms_per_step": round(e["ms_per_step"], 4),
+        "api": "la_block_causal_step" if w.block_causal else "la_attention"}
     out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
            "latency_us": ms_step * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -529,7 +532,7 @@ def main():
            "roofline": roofline, "e2e": e2e,
            "gpu_launches": r["launches_per_step"] * args.steps,
            "clocks": r["clocks"], "graph_chunk_steps": r["chunk"], "soak_s": args.soak}
-    if world == 1:
+    if world == 1 and args.cpu_seconds > 0:
         tps, desc, cores, _, _ = oracle_sample(w, args.cpu_seconds)
         out["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores,
                                "kind": "oracle", "sample": desc}
