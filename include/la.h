@@ -152,6 +152,29 @@ la_status la_block_causal_step(const la_shape* shape, const void* Q,
 la_status la_state_reset(float* S, float* z, int B, int H, int D,
                          la_stream stream);
 
+/* State reduce without a workspace, for callers that cannot allocate device
+ * memory where they run it: a plugin inside a host application that owns
+ * every device buffer, a fixed-footprint runtime that forbids allocation
+ * after start-up, or a latency-critical loop that must not call cudaMalloc
+ * (cudaMalloc can synchronise the device). The pages have no counterpart of
+ * this entry point; it computes exactly what la_state_reduce computes, with
+ * the same kernel and the same split order, so S and z are identical.
+ *
+ * Scratch: a fixed 8 MiB array in the library's own device memory. Every GPU
+ * that loads the library holds it until the process exits. A shape whose
+ * scratch (split partials + per-head counters) does not fit returns
+ * LA_ERR_UNSUPPORTED before any launch; la_state_reduce with a workspace
+ * handles it. The call allocates nothing and frees nothing; it clears the
+ * counters it needs (cudaMemsetAsync on `stream`) before the kernel.
+ * All calls on one GPU share the array: calls whose kernels may overlap on
+ * the GPU (different streams or host threads) race and must be ordered.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture. */
+la_status la_state_reduce_static(const la_shape* shape, const void* K,
+                                 const void* V, float* S, float* z,
+                                 la_stream stream);
+
 /* Static description of a status code. Never NULL. */
 const char* la_status_string(la_status status);
 

@@ -59,6 +59,8 @@ _lib.la_workspace_bytes.argtypes = [_shape_p]
 _lib.la_workspace_bytes.restype = _sz
 _lib.la_state_reduce.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.la_state_reduce.restype = _i
+_lib.la_state_reduce_static.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp]
+_lib.la_state_reduce_static.restype = _i
 _lib.la_apply.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp]
 _lib.la_apply.restype = _i
 _lib.la_attention.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
@@ -119,6 +121,13 @@ def la_workspace_bytes(shape: LaShape) -> int:
 def la_state_reduce(shape: LaShape, K, V, S, z, ws, stream=None) -> None:
     _check(_lib.la_state_reduce(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(S), _ptr(z),
                                 _ptr(ws), _nbytes(ws), _stream(stream)), "la_state_reduce")
+
+
+def la_state_reduce_static(shape: LaShape, K, V, S, z, stream=None) -> None:
+    """la_state_reduce without a workspace: the scratch is the library's own
+    fixed device array (for callers that cannot allocate; see include/la.h)."""
+    _check(_lib.la_state_reduce_static(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(S), _ptr(z),
+                                       _stream(stream)), "la_state_reduce_static")
 
 
 def la_apply(shape: LaShape, Q, S, z, O, stream=None) -> None:

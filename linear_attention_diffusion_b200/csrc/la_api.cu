@@ -10,7 +10,7 @@
 #include "la_internal.h"
 
 namespace la {
-namespace {
+namespace detail {
 
 thread_local std::string g_last_error;
 
@@ -144,9 +144,10 @@ la_status run_reduce(const Problem& p, const void* K, const void* V, char* ws,
   return LA_OK;
 }
 
-}  // namespace
+}  // namespace detail
 
 WsLayout workspace_layout(const Problem& p) {
+  using detail::align256;
   WsLayout L;
   const size_t bh = static_cast<size_t>(p.B) * p.H;
   L.counters = 0;
@@ -161,6 +162,7 @@ WsLayout workspace_layout(const Problem& p) {
 }  // namespace la
 
 using namespace la;
+using namespace la::detail;
 
 extern "C" {
 

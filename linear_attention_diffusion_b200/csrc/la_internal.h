@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "la.h"
+
 namespace la {
 
 constexpr int kD = 32;                 // head width (the only one supported)
@@ -60,5 +62,15 @@ cudaError_t launch_reduce(const Problem& p, const void* K, const void* V, float*
 // O = phi(Q) S / (ReLU(Q) . z + eps).
 cudaError_t launch_apply(const Problem& p, const void* Q, const float* S,
                          const float* z, void* O, cudaStream_t s);
+
+// Host-side helpers of the C-ABI layer (la_api.cu).
+namespace detail {
+la_status fail(la_status st, const char* fmt, ...);
+la_status cuda_fail(cudaError_t e, const char* where);
+la_status make_problem(const la_shape* s, Problem& p);
+la_status check_ptr(const void* ptr, const char* name, bool needed);
+bool overlap(const void* a, size_t na, const void* b, size_t nb);
+size_t align256(size_t x);
+}  // namespace detail
 
 }  // namespace la

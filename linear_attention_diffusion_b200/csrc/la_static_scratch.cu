@@ -1,0 +1,98 @@
+// la_state_reduce_static: the state reduce for callers that cannot hand the
+// library a workspace.
+//
+// Some callers have no way to allocate device memory at the point where they
+// run the reduce: a plugin inside a host application that owns every device
+// buffer, a fixed-footprint runtime that forbids allocation once it has
+// started, or a latency-critical loop that must not call cudaMalloc (which
+// can synchronise the whole device). This entry point lets them run the
+// reduce with only their inputs and outputs: its scratch (the per-split
+// partial states and the per-head arrival counters) lives in a fixed array in
+// the library's own device memory, declared below.
+//
+// Cost of that choice: every GPU that loads the library holds the array
+// (kStaticScratchBytes) until the process exits, and all calls on one GPU
+// share it. Calls whose kernels may run at the same time on one GPU (other
+// streams, other host threads) race on the array and must be ordered by the
+// caller.
+#include <mutex>
+
+#include "la_internal.h"
+
+namespace la {
+namespace {
+
+// 8 MiB: enough for B*H*splits*(32*32+32) floats of every workload this
+// library targets (at most 4.7 MB: 70 heads x 16 splits, or 4 x 70 heads x
+// 4 splits) plus the counters.
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device, looked up once per
+// device. In host code the array's name only stands for the symbol; the
+// address a kernel may use comes from cudaGetSymbolAddress.
+la_status scratch_address(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return detail::cuda_fail(e, "la_state_reduce_static: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices)
+    return detail::fail(LA_ERR_UNSUPPORTED, "la_state_reduce_static: device %d", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+    if (e != cudaSuccess || ptr == nullptr)
+      return detail::cuda_fail(e, "la_state_reduce_static: cudaGetSymbolAddress");
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return LA_OK;
+}
+
+}  // namespace
+}  // namespace la
+
+using namespace la;
+
+extern "C" la_status la_state_reduce_static(const la_shape* shape, const void* K, const void* V,
+                                            float* S, float* z, la_stream stream) {
+  Problem p;
+  la_status st = detail::make_problem(shape, p);
+  if (st != LA_OK) return st;
+  const bool any_state = p.B > 0 && p.H > 0;
+  const bool any_input = any_state && p.N > 0;
+  if ((st = detail::check_ptr(K, "K", any_input)) != LA_OK) return st;
+  if ((st = detail::check_ptr(V, "V", any_input)) != LA_OK) return st;
+  if ((st = detail::check_ptr(S, "S", any_state)) != LA_OK) return st;
+  if ((st = detail::check_ptr(z, "z", any_state)) != LA_OK) return st;
+  const size_t bh = static_cast<size_t>(p.B) * p.H;
+  if (detail::overlap(S, bh * kD * kD * 4, z, bh * kD * 4))
+    return detail::fail(LA_ERR_INVALID_ARG, "S and z must not overlap");
+  // Scratch layout: counters first, then the split partials.
+  const size_t counters_bytes = detail::align256(bh * sizeof(unsigned));
+  const size_t need = counters_bytes + bh * p.splits * kStateFloats * sizeof(float);
+  if (need > kStaticScratchBytes)
+    return detail::fail(LA_ERR_UNSUPPORTED,
+                        "la_state_reduce_static: this shape needs %zu bytes of scratch but the "
+                        "library's static array holds %zu; use la_state_reduce with a workspace",
+                        need, kStaticScratchBytes);
+  if (!any_state) return LA_OK;
+  void* base = nullptr;
+  if ((st = scratch_address(&base)) != LA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* scratch = static_cast<unsigned char*>(base);
+  // The counters must start at zero; the array keeps whatever the previous
+  // call (or a failed one) left there.
+  cudaError_t e = cudaMemsetAsync(scratch, 0, bh * sizeof(unsigned), s);
+  if (e != cudaSuccess) return detail::cuda_fail(e, "la_state_reduce_static: clear counters");
+  const StateOut out = {nullptr, nullptr, S, z, nullptr, nullptr};
+  e = launch_reduce(p, K, V, reinterpret_cast<float*>(scratch + counters_bytes),
+                    reinterpret_cast<unsigned*>(scratch), out, s);
+  if (e != cudaSuccess) return detail::cuda_fail(e, "la_state_reduce_static");
+  return LA_OK;
+}
