@@ -182,6 +182,13 @@ const char* la_status_string(la_status status);
  * string if none). The pointer stays valid until the thread's next call. */
 const char* la_last_error(void);
 
+/* Device-side error word of the current device: non-zero when a kernel of
+ * this library gave up on a bounded wait (a pipeline stage that never
+ * arrived; the kernel then drained its copies and returned without a valid
+ * result). Synchronous: waits for the device's pending work. `reset` != 0
+ * clears the word afterwards. */
+la_status la_device_error(unsigned* code, int reset);
+
 #ifdef __cplusplus
 }
 #endif

@@ -73,6 +73,8 @@ _lib.la_status_string.argtypes = [_i]
 _lib.la_status_string.restype = ctypes.c_char_p
 _lib.la_last_error.argtypes = []
 _lib.la_last_error.restype = ctypes.c_char_p
+_lib.la_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), _i]
+_lib.la_device_error.restype = _i
 
 
 def make_shape(B: int, N: int, H: int, D: int = HEAD_DIM, io_dtype: str = "bf16",
@@ -159,6 +161,13 @@ def la_status_string(status: int) -> str:
 
 def la_last_error() -> str:
     return _lib.la_last_error().decode()
+
+
+def la_device_error(reset: bool = False) -> int:
+    """The device error word of the current device (0: no kernel gave up a wait)."""
+    code = ctypes.c_uint(0)
+    _check(_lib.la_device_error(ctypes.byref(code), int(bool(reset))), "la_device_error")
+    return int(code.value)
 
 
 # ---------------------------------------------------------------------------

@@ -34,11 +34,12 @@ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // Token splits of the state reduce: a function of (B, N, H) only, so that
 // the reduction order, and with it every bit of S and z, is fixed per shape.
-// About two CTAs of four heads per SM, at least one 128-token tile per split.
+// One wave of CTAs of four heads (one CTA per SM), at least one 128-token
+// tile per split.
 void choose_splits(Problem& p) {
   const int groups = ceil_div(p.H, 4);
   const long long units = static_cast<long long>(p.B) * groups;
-  int splits = units > 0 ? static_cast<int>((2LL * kNumSMs) / units) : 1;
+  int splits = units > 0 ? static_cast<int>(kNumSMs / units) : 1;
   const int max_splits = p.N > 0 ? ceil_div(p.N, kTileTokens) : 1;
   if (splits > max_splits) splits = max_splits;
   if (splits > 64) splits = 64;
@@ -145,6 +146,18 @@ la_status run_reduce(const Problem& p, const void* K, const void* V, char* ws,
 }
 
 }  // namespace detail
+
+cudaError_t launch_reduce(const Problem& p, const void* K, const void* V, float* partials,
+                          unsigned* counters, const StateOut& out, cudaStream_t s) {
+  if (p.io == LA_IO_BF16 && p.N > 0) return launch_reduce_tc(p, K, V, partials, counters, out, s);
+  return launch_reduce_simt(p, K, V, partials, counters, out, s);
+}
+
+cudaError_t launch_apply(const Problem& p, const void* Q, const float* S, const float* z,
+                         void* O, cudaStream_t s) {
+  if (p.io == LA_IO_BF16) return launch_apply_tc(p, Q, S, z, O, s);
+  return launch_apply_simt(p, Q, S, z, O, s);
+}
 
 WsLayout workspace_layout(const Problem& p) {
   using detail::align256;
@@ -314,5 +327,12 @@ const char* la_status_string(la_status status) {
 }
 
 const char* la_last_error(void) { return g_last_error.c_str(); }
+
+la_status la_device_error(unsigned* code, int reset) {
+  if (code == nullptr) return fail(LA_ERR_INVALID_ARG, "code is NULL");
+  const cudaError_t e = read_device_error(code, reset != 0);
+  if (e != cudaSuccess) return cuda_fail(e, "la_device_error");
+  return LA_OK;
+}
 
 }  // extern "C"

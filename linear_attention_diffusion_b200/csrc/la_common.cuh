@@ -88,21 +88,41 @@ __device__ __forceinline__ void finish_reduce(const Problem& p, int b, int h0, i
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int hh = 0; hh < nh && h0 + hh < p.H; ++hh) {
+  // Each thread sums float4 columns of the partials; the loads of up to 8
+  // splits are issued together and then added in split order.
+  constexpr int kVec = kStateFloats / 4;
+  const int heads = min(nh, p.H - h0);
+  for (int v = threadIdx.x; v < heads * kVec; v += blockDim.x) {
+    const int hh = v / kVec, i = (v - hh * kVec) * 4;
     const size_t bh = static_cast<size_t>(b) * p.H + h0 + hh;
-    const float* src = partials + bh * p.splits * kStateFloats;
-    for (int i = threadIdx.x; i < kStateFloats; i += blockDim.x) {
-      float acc = 0.0f;
-      for (int s = 0; s < p.splits; ++s) acc += __ldcg(src + static_cast<size_t>(s) * kStateFloats + i);
-      const bool is_s = i < kD * kD;
-      const size_t o = is_s ? bh * kD * kD + i : bh * kD + (i - kD * kD);
-      const float* c = is_s ? out.carry_S : out.carry_z;
-      if (c != nullptr) acc = c[o] + acc;
-      float* d1 = is_s ? out.out1_S : out.out1_z;
-      float* d2 = is_s ? out.out2_S : out.out2_z;
-      if (d1 != nullptr) d1[o] = acc;
-      if (d2 != nullptr) d2[o] = acc;
+    const float* src = partials + bh * p.splits * kStateFloats + i;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int s0 = 0; s0 < p.splits; s0 += 8) {
+      float4 t[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (s0 + k < p.splits)
+          t[k] = __ldcg(reinterpret_cast<const float4*>(src + static_cast<size_t>(s0 + k) * kStateFloats));
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (s0 + k < p.splits) {
+          acc.x += t[k].x;
+          acc.y += t[k].y;
+          acc.z += t[k].z;
+          acc.w += t[k].w;
+        }
     }
+    const bool is_s = i < kD * kD;
+    const size_t o = is_s ? bh * kD * kD + i : bh * kD + (i - kD * kD);
+    const float* c = is_s ? out.carry_S : out.carry_z;
+    if (c != nullptr) {
+      const float4 cv = *reinterpret_cast<const float4*>(c + o);
+      acc = make_float4(cv.x + acc.x, cv.y + acc.y, cv.z + acc.z, cv.w + acc.w);
+    }
+    float* d1 = is_s ? out.out1_S : out.out1_z;
+    float* d2 = is_s ? out.out2_S : out.out2_z;
+    if (d1 != nullptr) *reinterpret_cast<float4*>(d1 + o) = acc;
+    if (d2 != nullptr) *reinterpret_cast<float4*>(d2 + o) = acc;
   }
   if (threadIdx.x == 0) counters[static_cast<size_t>(b) * p.H + h0] = 0u;
 }

@@ -63,6 +63,20 @@ cudaError_t launch_reduce(const Problem& p, const void* K, const void* V, float*
 cudaError_t launch_apply(const Problem& p, const void* Q, const float* S,
                          const float* z, void* O, cudaStream_t s);
 
+// The two implementations behind launch_reduce / launch_apply: tensor-core
+// kernels for bf16 I/O (la_tc.cu), CUDA-core kernels for float32 I/O and the
+// empty sequence (la_simt.cu).
+cudaError_t launch_reduce_tc(const Problem& p, const void* K, const void* V, float* partials,
+                             unsigned* counters, const StateOut& out, cudaStream_t s);
+cudaError_t launch_apply_tc(const Problem& p, const void* Q, const float* S, const float* z,
+                            void* O, cudaStream_t s);
+cudaError_t launch_reduce_simt(const Problem& p, const void* K, const void* V, float* partials,
+                               unsigned* counters, const StateOut& out, cudaStream_t s);
+cudaError_t launch_apply_simt(const Problem& p, const void* Q, const float* S, const float* z,
+                              void* O, cudaStream_t s);
+// Device error word of the tensor-core kernels (bounded waits that gave up).
+cudaError_t read_device_error(unsigned* code, bool reset);
+
 // Host-side helpers of the C-ABI layer (la_api.cu).
 namespace detail {
 la_status fail(la_status st, const char* fmt, ...);

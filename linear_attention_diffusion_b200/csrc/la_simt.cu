@@ -196,8 +196,8 @@ apply_simt(const Problem p, const T* __restrict__ Q, const float* __restrict__ S
 
 }  // namespace
 
-cudaError_t launch_reduce(const Problem& p, const void* K, const void* V, float* partials,
-                          unsigned* counters, const StateOut& out, cudaStream_t s) {
+cudaError_t launch_reduce_simt(const Problem& p, const void* K, const void* V, float* partials,
+                               unsigned* counters, const StateOut& out, cudaStream_t s) {
   const dim3 grid(p.splits, p.H, p.B);
   if (p.io == 0)
     reduce_simt<__nv_bfloat16><<<grid, kRedThreads, 0, s>>>(
@@ -210,8 +210,8 @@ cudaError_t launch_reduce(const Problem& p, const void* K, const void* V, float*
   return cudaGetLastError();
 }
 
-cudaError_t launch_apply(const Problem& p, const void* Q, const float* S, const float* z,
-                         void* O, cudaStream_t s) {
+cudaError_t launch_apply_simt(const Problem& p, const void* Q, const float* S, const float* z,
+                              void* O, cudaStream_t s) {
   const dim3 grid((p.N + kApplyTile - 1) / kApplyTile, p.H, p.B);
   if (p.io == 0)
     apply_simt<__nv_bfloat16><<<grid, kApplyThreads, 0, s>>>(

@@ -45,6 +45,7 @@ def gpu_attention(Q, K, V, eps, rope_grid=None, t_offset=0):
     Qd, Kd, Vd = to_dev(Q, K, V)
     O, S, z = la.attention(Qd, Kd, Vd, eps=eps, rope_grid=rope_grid, t_offset=t_offset)
     torch.cuda.synchronize()
+    assert la.la_device_error() == 0, "a kernel gave up a bounded wait"
     return O.cpu(), S.cpu(), z.cpu()
 
 
