@@ -314,19 +314,21 @@ def run_la(args, w, rank, world, local_rank):
     chunk = min(chunk, args.steps) if args.steps > 0 else chunk
     chunk = max(1, chunk - chunk % n_sets) if chunk >= n_sets else chunk
 
-    def capture(nsteps):
+    def capture(nsteps, with_events):
         evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
                for _ in range(nsteps)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for i in range(nsteps):
-                step(i, evs[i])
+                step(i, evs[i] if with_events else None)
         check_status()
         return g, evs
 
-    g_chunk, ev_chunk = capture(chunk)
+    g_chunk, _ = capture(chunk, with_events=False)
     full, rem = divmod(args.steps, chunk)
-    g_rem, ev_rem = capture(rem) if rem else (None, None)
+    g_rem = capture(rem, with_events=False)[0] if rem else None
+    # a second graph with an event after every launch, for per-launch durations
+    g_ev, ev_chunk = capture(chunk, with_events=True)
 
     # soak: the same graph, untimed, for about a second, so that clocks settle
     torch.cuda.synchronize(dev)
@@ -336,6 +338,9 @@ def run_la(args, w, rank, world, local_rank):
             g_chunk.replay()
             torch.cuda.synchronize(dev)
 
+    # timed region 1: exactly K steps, graph replays back to back (no events
+    # between launches, so consecutive kernels overlap through programmatic
+    # dependent launch exactly as they do for a user's stream)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
@@ -355,10 +360,13 @@ def run_la(args, w, rank, world, local_rank):
         torch.distributed.barrier()
     ms = start.elapsed_time(end)
 
-    # per-launch durations from the last replay of the chunk graph
-    evs = ev_chunk if full > 0 else ev_rem
-    seg = [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(n_ev - 1)]
-    seg_us = [1000.0 * statistics.mean(s) for s in seg]
+    # timed region 2: the event graph, for the duration of each launch
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g_ev.replay()
+    torch.cuda.synchronize(dev)
+    seg = [[e[j].elapsed_time(e[j + 1]) for e in ev_chunk] for j in range(n_ev - 1)]
+    seg_us = [1000.0 * statistics.mean(x) for x in seg]
 
     ms_max = ms
     if world > 1:
@@ -370,7 +378,7 @@ def run_la(args, w, rank, world, local_rank):
     e2e = run_e2e(args, w, dev, stream, la, rank) if args.e2e_steps > 0 else None
     clocks = sampler.summary(t0, t1)
     sampler.stop()
-    del g_chunk, g_rem
+    del g_chunk, g_rem, g_ev
     return {"ms": ms_max, "seg_us": seg_us, "kernel_names": kernel_names, "e2e": e2e,
             "clocks": clocks, "launches_per_step": launches_per_step, "n_sets": n_sets,
             "chunk": chunk, "per_set_bytes": per_set}

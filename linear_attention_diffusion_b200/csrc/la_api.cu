@@ -154,8 +154,8 @@ cudaError_t launch_reduce(const Problem& p, const void* K, const void* V, float*
 }
 
 cudaError_t launch_apply(const Problem& p, const void* Q, const float* S, const float* z,
-                         void* O, cudaStream_t s) {
-  if (p.io == LA_IO_BF16) return launch_apply_tc(p, Q, S, z, O, s);
+                         void* O, bool after_own_reduce, cudaStream_t s) {
+  if (p.io == LA_IO_BF16) return launch_apply_tc(p, Q, S, z, O, after_own_reduce && p.N > 0, s);
   return launch_apply_simt(p, Q, S, z, O, s);
 }
 
@@ -217,7 +217,8 @@ la_status la_apply(const la_shape* shape, const void* Q, const float* S, const f
       overlap(O, io_bytes(p), z, z_bytes(p)))
     return fail(LA_ERR_INVALID_ARG, "O must not overlap Q, S or z");
   if (!any) return LA_OK;
-  const cudaError_t e = launch_apply(p, Q, S, z, O, reinterpret_cast<cudaStream_t>(stream));
+  const cudaError_t e =
+      launch_apply(p, Q, S, z, O, false, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "apply");
   return LA_OK;
 }
@@ -253,7 +254,7 @@ la_status la_attention(const la_shape* shape, const void* Q, const void* K, cons
   const StateOut out = {nullptr, nullptr, Sw, zw, S, z};
   LA_TRY(run_reduce(p, K, V, w, out, st));
   if (!any_input) return LA_OK;
-  const cudaError_t e = launch_apply(p, Q, Sw, zw, O, st);
+  const cudaError_t e = launch_apply(p, Q, Sw, zw, O, true, st);
   if (e != cudaSuccess) return cuda_fail(e, "apply");
   return LA_OK;
 }
@@ -295,7 +296,7 @@ la_status la_block_causal_step(const la_shape* shape, const void* Q, const void*
                         to_carry ? S_carry : nullptr, to_carry ? z_carry : nullptr};
   LA_TRY(run_reduce(p, K, V, w, out, st));
   if (!uses_q || !any_input) return LA_OK;
-  const cudaError_t e = launch_apply(p, Q, Sw, zw, O, st);
+  const cudaError_t e = launch_apply(p, Q, Sw, zw, O, true, st);
   if (e != cudaSuccess) return cuda_fail(e, "apply");
   return LA_OK;
 }

@@ -59,9 +59,10 @@ struct StateOut {
 // counter. Deterministic: the sum order depends on the shape only.
 cudaError_t launch_reduce(const Problem& p, const void* K, const void* V, float* partials,
                           unsigned* counters, const StateOut& out, cudaStream_t s);
-// O = phi(Q) S / (ReLU(Q) . z + eps).
+// O = phi(Q) S / (ReLU(Q) . z + eps). after_own_reduce: the previous kernel
+// on the stream is this library's state reduce (so Q may be read early).
 cudaError_t launch_apply(const Problem& p, const void* Q, const float* S,
-                         const float* z, void* O, cudaStream_t s);
+                         const float* z, void* O, bool after_own_reduce, cudaStream_t s);
 
 // The two implementations behind launch_reduce / launch_apply: tensor-core
 // kernels for bf16 I/O (la_tc.cu), CUDA-core kernels for float32 I/O and the
@@ -69,7 +70,7 @@ cudaError_t launch_apply(const Problem& p, const void* Q, const float* S,
 cudaError_t launch_reduce_tc(const Problem& p, const void* K, const void* V, float* partials,
                              unsigned* counters, const StateOut& out, cudaStream_t s);
 cudaError_t launch_apply_tc(const Problem& p, const void* Q, const float* S, const float* z,
-                            void* O, cudaStream_t s);
+                            void* O, bool after_own_reduce, cudaStream_t s);
 cudaError_t launch_reduce_simt(const Problem& p, const void* K, const void* V, float* partials,
                                unsigned* counters, const StateOut& out, cudaStream_t s);
 cudaError_t launch_apply_simt(const Problem& p, const void* Q, const float* S, const float* z,

@@ -31,6 +31,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <utility>
 
 #include "la_common.cuh"
 #include "la_sm100.cuh"
@@ -193,11 +194,75 @@ struct RedSmem {
   static constexpr int zred = stages + kRedStages * kRedStageBytes;    // [256][8] float
   static constexpr int rope = zred + kMathThreads * 8 * 4;             // float2[kRopeTableMax]
   static constexpr int bars = rope + kRopeTableMax * 8;                // mbarriers
-  static constexpr int nbars = 3 * kRedStages + 2;
+  static constexpr int nbars = 3 * kRedStages + 3;
   static constexpr int misc = bars + nbars * 8;                        // tmem base, abort
   static constexpr int bytes = misc + 16;
 };
 constexpr int kRedSmemBytes = RedSmem::bytes + 1024;
+
+// Second phase of the reduce for a group of 4 heads: the CTA that arrives
+// last for the group copies the group's partials (contiguous: heads x splits
+// x 1056 floats) into shared memory with bulk copies, sums them in split
+// order, adds the carry when given, writes the outputs and re-zeroes the
+// counter. Falls back to the register version when they do not fit.
+__device__ __forceinline__ void finish_reduce_bulk(const Problem& p, int b, int h0,
+                                                   const float* partials, unsigned* counters,
+                                                   const StateOut& out, uint8_t* smem,
+                                                   uint64_t* comb_full, volatile int* abort_flag) {
+  const int heads = min(kGroupHeads, p.H - h0);
+  const uint32_t per_head = static_cast<uint32_t>(p.splits) * kStateFloats * 4;
+  if (static_cast<size_t>(heads) * per_head > static_cast<size_t>(kRedStages) * kRedStageBytes) {
+    finish_reduce(p, b, h0, kGroupHeads, partials, counters, out);
+    return;
+  }
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  const size_t cidx = static_cast<size_t>(b) * p.H + h0;
+  if (threadIdx.x == 0) {
+    const unsigned prev = atomicAdd(&counters[cidx], 1u);
+    s_last = prev == static_cast<unsigned>(p.splits - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const float* src = partials + cidx * p.splits * kStateFloats;
+  float* buf = reinterpret_cast<float*>(smem + RedSmem::stages);
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(comb_full, heads * per_head);
+    for (int hh = 0; hh < heads; ++hh)
+      bulk_load(reinterpret_cast<uint8_t*>(buf) + hh * per_head,
+                reinterpret_cast<const uint8_t*>(src) + hh * per_head, per_head, comb_full);
+  }
+  const bool ok = mbar_wait(comb_full, 0, abort_flag, &g_tc_error, kErrWait);
+  if (!ok) return;  // the counter stays raised: the device error word reports it
+  constexpr int kVec = kStateFloats / 4;
+  for (int v = threadIdx.x; v < heads * kVec; v += blockDim.x) {
+    const int hh = v / kVec, i = (v - hh * kVec) * 4;
+    const float4* col = reinterpret_cast<const float4*>(buf + hh * p.splits * kStateFloats + i);
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int sp = 0; sp < p.splits; ++sp) {
+      const float4 t = col[sp * (kStateFloats / 4)];
+      acc.x += t.x;
+      acc.y += t.y;
+      acc.z += t.z;
+      acc.w += t.w;
+    }
+    const size_t bh = cidx + hh;
+    const bool is_s = i < kD * kD;
+    const size_t o = is_s ? bh * kD * kD + i : bh * kD + (i - kD * kD);
+    const float* c = is_s ? out.carry_S : out.carry_z;
+    if (c != nullptr) {
+      const float4 cv = *reinterpret_cast<const float4*>(c + o);
+      acc = make_float4(cv.x + acc.x, cv.y + acc.y, cv.z + acc.z, cv.w + acc.w);
+    }
+    float* d1 = is_s ? out.out1_S : out.out1_z;
+    float* d2 = is_s ? out.out2_S : out.out2_z;
+    if (d1 != nullptr) *reinterpret_cast<float4*>(d1 + o) = acc;
+    if (d2 != nullptr) *reinterpret_cast<float4*>(d2 + o) = acc;
+  }
+  if (threadIdx.x == 0) counters[cidx] = 0u;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -211,6 +276,7 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
   uint64_t* empty = ready + kRedStages;
   uint64_t* acc_full = empty + kRedStages;
   uint64_t* mma_done = acc_full + 1;
+  uint64_t* comb_full = mma_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + RedSmem::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + RedSmem::misc + 4);
   float* zred = reinterpret_cast<float*>(smem + RedSmem::zred);
@@ -231,6 +297,7 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
+    mbar_init(comb_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -249,6 +316,10 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(smem);
+  // Everything above overlaps the previous kernel's tail; global memory is
+  // touched only after it has completed. Then the next kernel may launch.
+  pdl_wait();
+  if (tid == 0) pdl_trigger();
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA
@@ -389,7 +460,7 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     tmem_dealloc(tmem, kRedTmemCols);
   }
   if (*abort_flag) return;  // partials incomplete: leave the counter alone
-  finish_reduce(p, b, h0, kGroupHeads, partials, counters, out);
+  finish_reduce_bulk(p, b, h0, partials, counters, out, smem, comb_full, abort_flag);
 }
 
 // ================================================================= apply
@@ -407,7 +478,7 @@ struct ApSmem {
   static constexpr int zs = bop + 2 * 32 * 128;                        // [4][32] float
   static constexpr int rope = zs + kGroupHeads * kD * 4;               // float2[kRopeTableMax]
   static constexpr int bars = rope + kRopeTableMax * 8;
-  static constexpr int nbars = 3 * kApStages + 2 + 2 + 1;
+  static constexpr int nbars = 3 * kApStages + 2 + 2 + 2;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int bytes = misc + 16;
 };
@@ -416,7 +487,7 @@ constexpr int kApSmemBytes = ApSmem::bytes + 1024;
 __global__ void __launch_bounds__(kThreads, 1)
 apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
          const Problem p, const RopeTable rt, const float* __restrict__ S,
-         const float* __restrict__ z, int tiles_per_cta) {
+         const float* __restrict__ z, int tiles_per_cta, int q_before_wait) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -426,6 +497,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   uint64_t* t_full = q_empty + kApStages;   // [2]
   uint64_t* t_empty = t_full + 2;           // [2]
   uint64_t* mma_done = t_empty + 2;
+  uint64_t* b_ready = mma_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + ApSmem::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + ApSmem::misc + 4);
   float* zs = reinterpret_cast<float*>(smem + ApSmem::zs);
@@ -449,6 +521,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       mbar_init(&t_empty[a], 128);
     }
     mbar_init(mma_done, 1);
+    mbar_init(b_ready, kMathThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -461,7 +534,20 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_o);
   }
+  if (tid >= 64 && rt.enabled && !rt.on_the_fly)
+    build_rope_table(p.rope, rope_tab, tid - 64, kMathThreads);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sbase = smem_u32(smem);
+
+  // Programmatic dependent launch: S and z come from the previous kernel, so
+  // they are read only after pdl_wait(). Q may be fetched before it when the
+  // caller knows the previous kernel does not write Q (q_before_wait).
+  if (warp == 0 && !q_before_wait) pdl_wait();
   if (tid >= 64) {
+    pdl_wait();
+    if (tid == 64) pdl_trigger();
     const int mt = tid - 64;
     // B operands: for head pair j, row e holds S[h][0..31][e] of heads 2j and
     // 2j+1 as bf16 (K-major, 128-byte swizzled)
@@ -484,13 +570,10 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       const int h = h0 + idx / kD;
       zs[idx] = h < p.H ? z[(static_cast<size_t>(b) * p.H + h) * kD + idx % kD] : 0.0f;
     }
-    if (rt.enabled && !rt.on_the_fly) build_rope_table(p.rope, rope_tab, mt, kMathThreads);
     fence_proxy_async_smem();
+    mbar_arrive(b_ready);
+    named_bar_sync(3, kMathThreads);  // zs visible to every math thread
   }
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t sbase = smem_u32(smem);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -513,7 +596,8 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, 32, 0, 0);
       const uint32_t bop = sbase + ApSmem::bop;
-      for (int i = 0; i < ntiles; ++i) {
+      const bool have_b = ntiles == 0 || mbar_wait(b_ready, 0, abort_flag, &g_tc_error, kErrWait);
+      for (int i = 0; have_b && i < ntiles; ++i) {
         const int s = i % kApStages;
         const uint32_t ph = (i / kApStages) & 1;
         const int a = i & 1;
@@ -699,6 +783,25 @@ cudaError_t ensure_smem_attr(int which, const void* fn, int bytes) {
 
 }  // namespace
 
+// Launch with programmatic dependent launch: the kernel's prologue may
+// overlap the previous kernel in the stream; its pdl_wait() orders every
+// access to global memory after that kernel.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, int smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 cudaError_t launch_reduce_tc(const Problem& p, const void* K, const void* V, float* partials,
                              unsigned* counters, const StateOut& out, cudaStream_t s) {
   CUtensorMap mk, mv;
@@ -710,12 +813,13 @@ cudaError_t launch_reduce_tc(const Problem& p, const void* K, const void* V, flo
     return e;
   const RopeTable rt = rope_table_for(p);
   const dim3 grid(p.splits, (p.H + kGroupHeads - 1) / kGroupHeads, p.B);
-  reduce_tc<<<grid, kThreads, kRedSmemBytes, s>>>(mk, mv, p, rt, partials, counters, out);
+  e = launch_pdl(reduce_tc, grid, kRedSmemBytes, s, mk, mv, p, rt, partials, counters, out);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_apply_tc(const Problem& p, const void* Q, const float* S, const float* z,
-                            void* O, cudaStream_t s) {
+                            void* O, bool after_own_reduce, cudaStream_t s) {
   CUtensorMap mq, mo;
   cudaError_t e;
   if ((e = make_map(&mq, Q, p, kApT)) != cudaSuccess) return e;
@@ -726,13 +830,19 @@ cudaError_t launch_apply_tc(const Problem& p, const void* Q, const float* S, con
   const int groups = (p.H + kGroupHeads - 1) / kGroupHeads;
   const int ntiles = (p.N + kApT - 1) / kApT;
   const long long units = static_cast<long long>(groups) * p.B;
-  int ctas_per_unit = static_cast<int>(std::max<long long>(1, kNumSMs / std::max<long long>(1, units)));
+  int ctas_per_unit =
+      static_cast<int>(std::max<long long>(1, kNumSMs / std::max<long long>(1, units)));
   ctas_per_unit = std::min(ctas_per_unit, ntiles);
   const int tiles_per_cta = (ntiles + ctas_per_unit - 1) / ctas_per_unit;
   ctas_per_unit = (ntiles + tiles_per_cta - 1) / tiles_per_cta;
   const RopeTable rt = rope_table_for(p);
   const dim3 grid(ctas_per_unit, groups, p.B);
-  apply_tc<<<grid, kThreads, kApSmemBytes, s>>>(mq, mo, p, rt, S, z, tiles_per_cta);
+  // Q may be read before the previous kernel completes only when that kernel
+  // is this library's own state reduce, which does not write Q and itself
+  // started reading only after everything before it had completed.
+  e = launch_pdl(apply_tc, grid, kApSmemBytes, s, mq, mo, p, rt, S, z, tiles_per_cta,
+                 after_own_reduce ? 1 : 0);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
