@@ -113,18 +113,19 @@ __device__ __forceinline__ void token_pos_advance(const Rope& r, TokPos& tp, int
   }
 }
 
-// (cos, sin) of pair j (0..15) at token position tp.
-__device__ __forceinline__ float2 rope_cs(const Rope& r, const RopeTable& rt, const float2* tab,
-                                          const TokPos& tp, int j) {
-  if (rt.on_the_fly) {
-    const int pos = j < 4 ? r.t_offset + tp.t : (j < 10 ? tp.h : tp.w);
-    float c, sn;
-    rope_cos_sin(pos, r.inv_freq[j], c, sn);
-    return make_float2(c, sn);
-  }
-  if (j < 4) return tab[tp.t * 4 + j];
-  if (j < 10) return tab[4 * r.T + tp.h * 6 + (j - 4)];
-  return tab[4 * r.T + 6 * r.Hh + tp.w * 6 + (j - 10)];
+// RoPE feature-map variants a kernel is compiled for.
+enum RopeMode : int { kNoRope = 0, kRopeTable = 1, kRopeOnTheFly = 2 };
+
+// Segment (0 = time, 1 = height, 2 = width) and index inside it of pair j.
+__host__ __device__ constexpr int pair_axis(int j) { return j < 4 ? 0 : (j < 10 ? 1 : 2); }
+__host__ __device__ constexpr int pair_off(int j) { return j < 4 ? j : (j < 10 ? j - 4 : j - 10); }
+
+// Table offsets of the three segments' rows for token position tp.
+struct RopeBases {
+  int t, h, w;
+};
+__device__ __forceinline__ RopeBases rope_bases(const Rope& r, const TokPos& tp) {
+  return {tp.t * 4, 4 * r.T + tp.h * 6, 4 * r.T + 6 * r.Hh + tp.w * 6};
 }
 
 // Barrier over `threads` threads of named barrier `id` that also ORs `pred`
@@ -264,6 +265,7 @@ __device__ __forceinline__ void finish_reduce_bulk(const Problem& p, int b, int 
   if (threadIdx.x == 0) counters[cidx] = 0u;
 }
 
+template <int kRope>
 __global__ void __launch_bounds__(kThreads, 1)
 reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
           const Problem p, const RopeTable rt, float* partials, unsigned* counters,
@@ -310,8 +312,7 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
   }
-  if (tid >= 64 && rt.enabled && !rt.on_the_fly)
-    build_rope_table(p.rope, rope_tab, tid - 64, kMathThreads);
+  if (kRope == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kMathThreads);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
@@ -373,9 +374,17 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     const int box = c >> 3, cc = c & 7;
     const int dpos = (cc & 3) * 8;  // first dim of the chunk inside its head
     float zacc[8] = {};
-    // this thread's tokens are n_begin + rg + 16 j, j = 0, 1, ...
+    // this thread's tokens are n_begin + rg + 16 j, j = 0, 1, ...; its chunk
+    // holds RoPE pairs j0 .. j0+3 (fixed per thread)
     TokPos tp = {0, 0, 0};
-    if (rt.enabled) tp = token_pos(p.rope, n_begin + rg);
+    if (kRope != kNoRope) tp = token_pos(p.rope, n_begin + rg);
+    const int j0 = dpos / 2;
+    int sel[4], off[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      sel[q] = pair_axis(j0 + q);
+      off[q] = pair_off(j0 + q);
+    }
     for (int i = 0; i < ntiles; ++i) {
       const int s = i % kRedStages;
       const uint32_t ph = (i / kRedStages) & 1;
@@ -395,11 +404,18 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         unpack8(u, x);
 #pragma unroll
         for (int e = 0; e < 8; ++e) zacc[e] += x[e];
-        if (rt.enabled) {
+        if (kRope != kNoRope) {
           if (y0 + r < p.N) {
+            const RopeBases rb = rope_bases(p.rope, tp);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const float2 cs = rope_cs(p.rope, rt, rope_tab, tp, dpos / 2 + q);
+              float2 cs;
+              if (kRope == kRopeTable) {
+                cs = rope_tab[(sel[q] == 0 ? rb.t : (sel[q] == 1 ? rb.h : rb.w)) + off[q]];
+              } else {
+                const int pos = sel[q] == 0 ? p.rope.t_offset + tp.t : (sel[q] == 1 ? tp.h : tp.w);
+                rope_cos_sin(pos, p.rope.inv_freq[j0 + q], cs.x, cs.y);
+              }
               const float x0 = x[2 * q], x1 = x[2 * q + 1];
               x[2 * q] = fmaf(x0, cs.x, -x1 * cs.y);
               x[2 * q + 1] = fmaf(x0, cs.y, x1 * cs.x);
@@ -484,6 +500,7 @@ struct ApSmem {
 };
 constexpr int kApSmemBytes = ApSmem::bytes + 1024;
 
+template <int kRope>
 __global__ void __launch_bounds__(kThreads, 1)
 apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
          const Problem p, const RopeTable rt, const float* __restrict__ S,
@@ -534,8 +551,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_o);
   }
-  if (tid >= 64 && rt.enabled && !rt.on_the_fly)
-    build_rope_table(p.rope, rope_tab, tid - 64, kMathThreads);
+  if (kRope == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kMathThreads);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
@@ -637,10 +653,20 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       const int n0 = (tile_begin + i) * kApT;
       const int n = n0 + row;
       float2 cs[16];
-      if (rt.enabled) {
+      if (kRope != kNoRope) {
         const TokPos tp = token_pos(p.rope, min(n, p.N - 1));
+        const RopeBases rb = rope_bases(p.rope, tp);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) cs[j] = rope_cs(p.rope, rt, rope_tab, tp, j);
+        for (int j = 0; j < 16; ++j) {
+          if (kRope == kRopeTable) {
+            const int a = pair_axis(j);
+            cs[j] = rope_tab[(a == 0 ? rb.t : (a == 1 ? rb.h : rb.w)) + pair_off(j)];
+          } else {
+            const int a = pair_axis(j);
+            const int pos = a == 0 ? p.rope.t_offset + tp.t : (a == 1 ? tp.h : tp.w);
+            rope_cos_sin(pos, p.rope.inv_freq[j], cs[j].x, cs[j].y);
+          }
+        }
       }
       float den[kGroupHeads] = {0.0f, 0.0f, 0.0f, 0.0f};
       const uint32_t st = sbase + ApSmem::stages + s * kApStageBytes;
@@ -665,7 +691,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         den[hh] = fmaf(x[5], zb.y, den[hh]);
         den[hh] = fmaf(x[6], zb.z, den[hh]);
         den[hh] = fmaf(x[7], zb.w, den[hh]);
-        if (rt.enabled) {
+        if (kRope != kNoRope) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float2 r = cs[d0 / 2 + q];
@@ -764,7 +790,7 @@ RopeTable rope_table_for(const Problem& p) {
 }
 
 constexpr int kMaxDev = 64;
-bool g_attr_set[2][kMaxDev] = {};
+bool g_attr_set[6][kMaxDev] = {};
 std::mutex g_attr_mu;
 
 cudaError_t ensure_smem_attr(int which, const void* fn, int bytes) {
@@ -808,12 +834,16 @@ cudaError_t launch_reduce_tc(const Problem& p, const void* K, const void* V, flo
   cudaError_t e;
   if ((e = make_map(&mk, K, p, kRedT)) != cudaSuccess) return e;
   if ((e = make_map(&mv, V, p, kRedT)) != cudaSuccess) return e;
-  if ((e = ensure_smem_attr(0, reinterpret_cast<const void*>(reduce_tc), kRedSmemBytes)) !=
+  const RopeTable rt = rope_table_for(p);
+  const int mode = !rt.enabled ? kNoRope : (rt.on_the_fly ? kRopeOnTheFly : kRopeTable);
+  void (*kern)(CUtensorMap, CUtensorMap, Problem, RopeTable, float*, unsigned*, StateOut) =
+      mode == kNoRope ? reduce_tc<kNoRope>
+                      : (mode == kRopeTable ? reduce_tc<kRopeTable> : reduce_tc<kRopeOnTheFly>);
+  if ((e = ensure_smem_attr(mode, reinterpret_cast<const void*>(kern), kRedSmemBytes)) !=
       cudaSuccess)
     return e;
-  const RopeTable rt = rope_table_for(p);
   const dim3 grid(p.splits, (p.H + kGroupHeads - 1) / kGroupHeads, p.B);
-  e = launch_pdl(reduce_tc, grid, kRedSmemBytes, s, mk, mv, p, rt, partials, counters, out);
+  e = launch_pdl(kern, grid, kRedSmemBytes, s, mk, mv, p, rt, partials, counters, out);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -824,9 +854,6 @@ cudaError_t launch_apply_tc(const Problem& p, const void* Q, const float* S, con
   cudaError_t e;
   if ((e = make_map(&mq, Q, p, kApT)) != cudaSuccess) return e;
   if ((e = make_map(&mo, O, p, kApT)) != cudaSuccess) return e;
-  if ((e = ensure_smem_attr(1, reinterpret_cast<const void*>(apply_tc), kApSmemBytes)) !=
-      cudaSuccess)
-    return e;
   const int groups = (p.H + kGroupHeads - 1) / kGroupHeads;
   const int ntiles = (p.N + kApT - 1) / kApT;
   const long long units = static_cast<long long>(groups) * p.B;
@@ -836,11 +863,19 @@ cudaError_t launch_apply_tc(const Problem& p, const void* Q, const float* S, con
   const int tiles_per_cta = (ntiles + ctas_per_unit - 1) / ctas_per_unit;
   ctas_per_unit = (ntiles + tiles_per_cta - 1) / tiles_per_cta;
   const RopeTable rt = rope_table_for(p);
+  const int mode = !rt.enabled ? kNoRope : (rt.on_the_fly ? kRopeOnTheFly : kRopeTable);
+  void (*kern)(CUtensorMap, CUtensorMap, Problem, RopeTable, const float*, const float*, int,
+               int) = mode == kNoRope ? apply_tc<kNoRope>
+                                      : (mode == kRopeTable ? apply_tc<kRopeTable>
+                                                            : apply_tc<kRopeOnTheFly>);
+  if ((e = ensure_smem_attr(3 + mode, reinterpret_cast<const void*>(kern), kApSmemBytes)) !=
+      cudaSuccess)
+    return e;
   const dim3 grid(ctas_per_unit, groups, p.B);
   // Q may be read before the previous kernel completes only when that kernel
   // is this library's own state reduce, which does not write Q and itself
   // started reading only after everything before it had completed.
-  e = launch_pdl(apply_tc, grid, kApSmemBytes, s, mq, mo, p, rt, S, z, tiles_per_cta,
+  e = launch_pdl(kern, grid, kApSmemBytes, s, mq, mo, p, rt, S, z, tiles_per_cta,
                  after_own_reduce ? 1 : 0);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

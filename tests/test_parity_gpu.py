@@ -43,6 +43,7 @@ SMALL = [
     (1, 1, 1, None, 0),             # one token, one head
     (1, 129, 70, (1, 3, 43), 0),    # one frame, 70 heads
     (2, 4096, 7, (4, 32, 32), 11),  # several splits per head
+    (1, 512, 5, (1, 2, 256), 7),    # RoPE table too large for shared memory: per-token angles
 ]
 
 
