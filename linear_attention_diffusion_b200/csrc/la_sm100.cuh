@@ -75,6 +75,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 
 // ------------------------------------------------------------------ fences
 
+// Release/acquire at GPU scope, issued by one thread after (or before) a CTA
+// barrier: the barrier orders the other threads' accesses with this fence.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -46,8 +46,11 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;
-constexpr int kMathThreads = 256;
+constexpr int kApWG = 3;            // apply: math warpgroups, one tile each in turn
+constexpr int kThreads = 64 + 128 * kApWG;  // apply: TMA warp, MMA warp, math warpgroups
+constexpr int kMathThreads = 128 * kApWG;
+constexpr int kRedMath = 512;       // reduce: 16 math warps
+constexpr int kRedThreads = 64 + kRedMath;
 constexpr int kGroupHeads = 4;
 constexpr int kRopeTableMax = 1536;  // float2 entries of the per-CTA RoPE table
 
@@ -192,8 +195,8 @@ constexpr int kRedTmemCols = 128;
 struct RedSmem {
   // offsets from the 1024-aligned base
   static constexpr int stages = 0;
-  static constexpr int zred = stages + kRedStages * kRedStageBytes;    // [256][8] float
-  static constexpr int rope = zred + kMathThreads * 8 * 4;             // float2[kRopeTableMax]
+  static constexpr int zred = stages + kRedStages * kRedStageBytes;    // [512][8] float
+  static constexpr int rope = zred + kRedMath * 8 * 4;                 // float2[kRopeTableMax]
   static constexpr int bars = rope + kRopeTableMax * 8;                // mbarriers
   static constexpr int nbars = 3 * kRedStages + 3;
   static constexpr int misc = bars + nbars * 8;                        // tmem base, abort
@@ -217,16 +220,18 @@ __device__ __forceinline__ void finish_reduce_bulk(const Problem& p, int b, int 
     return;
   }
   __shared__ int s_last;
-  __threadfence();
+  // The CTA barrier orders every thread's partial stores before thread 0's
+  // release fence; the CTA that arrives last acquires all groups' stores.
   __syncthreads();
   const size_t cidx = static_cast<size_t>(b) * p.H + h0;
   if (threadIdx.x == 0) {
+    fence_acq_rel_gpu();
     const unsigned prev = atomicAdd(&counters[cidx], 1u);
     s_last = prev == static_cast<unsigned>(p.splits - 1);
+    if (s_last) fence_acq_rel_gpu();
   }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   const float* src = partials + cidx * p.splits * kStateFloats;
   float* buf = reinterpret_cast<float*>(smem + RedSmem::stages);
   if (threadIdx.x == 0) {
@@ -266,7 +271,7 @@ __device__ __forceinline__ void finish_reduce_bulk(const Problem& p, int b, int 
 }
 
 template <int kRope>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kRedThreads, 1)
 reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
           const Problem p, const RopeTable rt, float* partials, unsigned* counters,
           const StateOut out) {
@@ -294,7 +299,7 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
   if (tid == 0) {
     for (int s = 0; s < kRedStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&ready[s], kMathThreads);
+      mbar_init(&ready[s], kRedMath);
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
@@ -312,7 +317,7 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
   }
-  if (kRope == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kMathThreads);
+  if (kRope == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kRedMath);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
@@ -370,11 +375,11 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     // ------------------------------------------------- feature map + key sum
     const int wt = tid - 64;
     const int c = wt & 15;        // 16-byte chunk column: box c/8, chunk c%8 of the row
-    const int rg = wt >> 4;       // row group: rows rg, rg+16, rg+32, rg+48
+    const int rg = wt >> 4;       // row group: rows rg and rg + 32 of every stage
     const int box = c >> 3, cc = c & 7;
     const int dpos = (cc & 3) * 8;  // first dim of the chunk inside its head
-    float zacc[8] = {};
-    // this thread's tokens are n_begin + rg + 16 j, j = 0, 1, ...; its chunk
+    float2 zacc[4] = {};
+    // this thread's tokens are n_begin + rg + 32 j, j = 0, 1, ...; its chunk
     // holds RoPE pairs j0 .. j0+3 (fixed per thread)
     TokPos tp = {0, 0, 0};
     if (kRope != kNoRope) tp = token_pos(p.rope, n_begin + rg);
@@ -392,8 +397,8 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       const uint32_t kb = sbase + RedSmem::stages + s * kRedStageBytes + box * kRedBox;
       const int y0 = n_begin + i * kRedT;
 #pragma unroll
-      for (int k = 0; k < kRedT / 16; ++k) {
-        const int r = rg + 16 * k;
+      for (int k = 0; k < kRedT / 32; ++k) {
+        const int r = rg + 32 * k;
         const uint32_t addr = kb + sw128_offset(r, cc);
         uint4 u = ld_shared_v4(addr);
         u.x = relu_bf16x2(u.x);
@@ -403,7 +408,7 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         float x[8];
         unpack8(u, x);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) zacc[e] += x[e];
+        for (int e = 0; e < 4; ++e) zacc[e] = __fadd2_rn(zacc[e], make_float2(x[2 * e], x[2 * e + 1]));
         if (kRope != kNoRope) {
           if (y0 + r < p.N) {
             const RopeBases rb = rope_bases(p.rope, tp);
@@ -416,13 +421,15 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
                 const int pos = sel[q] == 0 ? p.rope.t_offset + tp.t : (sel[q] == 1 ? tp.h : tp.w);
                 rope_cos_sin(pos, p.rope.inv_freq[j0 + q], cs.x, cs.y);
               }
-              const float x0 = x[2 * q], x1 = x[2 * q + 1];
-              x[2 * q] = fmaf(x0, cs.x, -x1 * cs.y);
-              x[2 * q + 1] = fmaf(x0, cs.y, x1 * cs.x);
+              const float2 t = __fmul2_rn(make_float2(x[2 * q + 1], x[2 * q + 1]),
+                                          make_float2(-cs.y, cs.x));
+              const float2 y = __ffma2_rn(make_float2(x[2 * q], x[2 * q]), cs, t);
+              x[2 * q] = y.x;
+              x[2 * q + 1] = y.y;
             }
             u = pack8(x);
           }
-          token_pos_advance(p.rope, tp, 16);
+          token_pos_advance(p.rope, tp, 32);
         }
         st_shared_v4(addr, u);
       }
@@ -430,8 +437,11 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       mbar_arrive(&ready[s]);
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) zred[wt * 8 + e] = zacc[e];
-    named_bar_sync(1, kMathThreads);
+    for (int e = 0; e < 4; ++e) {
+      zred[wt * 8 + 2 * e] = zacc[e].x;
+      zred[wt * 8 + 2 * e + 1] = zacc[e].y;
+    }
+    named_bar_sync(1, kRedMath);
 
     // state of the four heads: the 32x32 diagonal blocks of the accumulator
     if (warp >= 2 && warp < 6) {
@@ -457,11 +467,11 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       }
     }
     if (wt < 128) {
-      // key sum of dim wt of the group: 16 row groups, in order
+      // key sum of dim wt of the group: 32 row groups, in order
       const int q = wt >> 5, d = wt & 31;
       const int col = wt >> 3, e = wt & 7;  // chunk column and element holding this dim
       float s = 0.0f;
-      for (int r = 0; r < 16; ++r) s += zred[(r * 16 + col) * 8 + e];
+      for (int r = 0; r < kRedMath / 16; ++r) s += zred[(r * 16 + col) * 8 + e];
       const int h = h0 + q;
       if (h < p.H)
         partials[((static_cast<size_t>(b) * p.H + h) * p.splits + split) * kStateFloats +
@@ -482,19 +492,20 @@ reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
 // ================================================================= apply
 
 constexpr int kApT = 128;                          // tokens per tile
-constexpr int kApStages = 4;
+constexpr int kApStages = 5;
 constexpr int kApBox = kApT * 128;                 // [128 tokens][64 dims] bf16
 constexpr int kApStageBytes = 2 * kApBox;
-constexpr int kApTmemCols = 256;                   // two 128-column accumulators
+constexpr int kApTmemCols = 512;                   // kApWG 128-column accumulators
 
+// A stage holds a tile's Q, then phi(Q) for the MMA, then the tile's O for the
+// TMA store: it is released to the producer once the store has read it.
 struct ApSmem {
   static constexpr int stages = 0;
-  static constexpr int obuf = stages + kApStages * kApStageBytes;      // [2 WG][2 boxes]
-  static constexpr int bop = obuf + 2 * kApStageBytes;                 // [2 pairs][32][128 B]
+  static constexpr int bop = stages + kApStages * kApStageBytes;       // [2 pairs][32][128 B]
   static constexpr int zs = bop + 2 * 32 * 128;                        // [4][32] float
   static constexpr int rope = zs + kGroupHeads * kD * 4;               // float2[kRopeTableMax]
   static constexpr int bars = rope + kRopeTableMax * 8;
-  static constexpr int nbars = 3 * kApStages + 2 + 2 + 2;
+  static constexpr int nbars = 3 * kApStages + 2 * kApWG + 2;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int bytes = misc + 16;
 };
@@ -511,9 +522,9 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + ApSmem::bars);
   uint64_t* q_ready = q_full + kApStages;
   uint64_t* q_empty = q_ready + kApStages;
-  uint64_t* t_full = q_empty + kApStages;   // [2]
-  uint64_t* t_empty = t_full + 2;           // [2]
-  uint64_t* mma_done = t_empty + 2;
+  uint64_t* t_full = q_empty + kApStages;   // [kApWG]
+  uint64_t* t_empty = t_full + kApWG;       // [kApWG]
+  uint64_t* mma_done = t_empty + kApWG;
   uint64_t* b_ready = mma_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + ApSmem::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + ApSmem::misc + 4);
@@ -533,7 +544,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       mbar_init(&q_ready[s], 128);
       mbar_init(&q_empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kApWG; ++a) {
       mbar_init(&t_full[a], 1);
       mbar_init(&t_empty[a], 128);
     }
@@ -588,7 +599,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     }
     fence_proxy_async_smem();
     mbar_arrive(b_ready);
-    named_bar_sync(3, kMathThreads);  // zs visible to every math thread
+    named_bar_sync(1 + kApWG, kMathThreads);  // zs visible to every math thread
   }
 
   if (warp == 0) {
@@ -616,9 +627,9 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       for (int i = 0; have_b && i < ntiles; ++i) {
         const int s = i % kApStages;
         const uint32_t ph = (i / kApStages) & 1;
-        const int a = i & 1;
+        const int a = i % kApWG;
         if (!mbar_wait(&q_ready[s], ph, abort_flag, &g_tc_error, kErrWait)) break;
-        if (!mbar_wait(&t_empty[a], ((i >> 1) & 1) ^ 1, abort_flag, &g_tc_error, kErrWait))
+        if (!mbar_wait(&t_empty[a], ((i / kApWG) & 1) ^ 1, abort_flag, &g_tc_error, kErrWait))
           break;
         tc_fence_after();
         const uint32_t st = sbase + ApSmem::stages + s * kApStageBytes;
@@ -632,7 +643,6 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
             mma_bf16(tmem + a * 128 + hh * 32, ad, bd, idesc, kk);
           }
         }
-        mma_commit(&q_empty[s]);
         mma_commit(&t_full[a]);
       }
       mma_commit(mma_done);
@@ -643,9 +653,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const bool leader = (warp == 2 + 4 * wg) && lane == 0;
-    uint8_t* ob = smem + ApSmem::obuf + wg * kApStageBytes;
-    const uint32_t ob_u = smem_u32(ob);
-    for (int i = wg; i < ntiles; i += 2) {
+    for (int i = wg; i < ntiles; i += kApWG) {
       const int s = i % kApStages;
       const uint32_t ph = (i / kApStages) & 1;
       bool ok = mbar_wait(&q_full[s], ph, abort_flag, &g_tc_error, kErrWait);
@@ -695,9 +703,11 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float2 r = cs[d0 / 2 + q];
-            const float x0 = x[2 * q], x1 = x[2 * q + 1];
-            x[2 * q] = fmaf(x0, r.x, -x1 * r.y);
-            x[2 * q + 1] = fmaf(x0, r.y, x1 * r.x);
+            const float2 t = __fmul2_rn(make_float2(x[2 * q + 1], x[2 * q + 1]),
+                                        make_float2(-r.y, r.x));
+            const float2 y = __ffma2_rn(make_float2(x[2 * q], x[2 * q]), r, t);
+            x[2 * q] = y.x;
+            x[2 * q + 1] = y.y;
           }
           u = pack8(x);
         }
@@ -706,11 +716,11 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       fence_proxy_async_smem();
       mbar_arrive(&q_ready[s]);
 
-      // epilogue: O = num / den, staged in shared memory, stored with TMA
+      // epilogue: O = num / den, written over the tile in shared memory (the
+      // MMA has finished reading it), stored with TMA
       const int a = wg;
-      ok = mbar_wait(&t_full[a], (i >> 1) & 1, abort_flag, &g_tc_error, kErrWait);
+      ok = mbar_wait(&t_full[a], (i / kApWG) & 1, abort_flag, &g_tc_error, kErrWait);
       tc_fence_after();
-      if (leader) bulk_wait_read<0>();
       if (bar_any(1 + wg, 128, !ok || *abort_flag)) break;
 #pragma unroll
       for (int hh = 0; hh < kGroupHeads; ++hh) {
@@ -723,7 +733,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           float x[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[e] = v[8 * k + e] * inv;
-          st_shared_v4(ob_u + (hh >> 1) * kApBox + sw128_offset(row, (hh & 1) * 4 + k), pack8(x));
+          st_shared_v4(st + (hh >> 1) * kApBox + sw128_offset(row, (hh & 1) * 4 + k), pack8(x));
         }
       }
       tc_fence_before();
@@ -731,9 +741,12 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       fence_proxy_async_smem();
       named_bar_sync(1 + wg, 128);
       if (leader) {
-        tma_store_3d(&tm_o, ob, h0 * 32, n0, b);
-        tma_store_3d(&tm_o, ob + kApBox, h0 * 32 + 64, n0, b);
+        uint8_t* tile = smem + ApSmem::stages + s * kApStageBytes;
+        tma_store_3d(&tm_o, tile, h0 * 32, n0, b);
+        tma_store_3d(&tm_o, tile + kApBox, h0 * 32 + 64, n0, b);
         bulk_commit();
+        bulk_wait_read<0>();      // the store has read the stage
+        mbar_arrive(&q_empty[s]);  // hand the stage back to the producer
       }
     }
     if (leader) bulk_wait<0>();
@@ -813,11 +826,11 @@ cudaError_t ensure_smem_attr(int which, const void* fn, int bytes) {
 // overlap the previous kernel in the stream; its pdl_wait() orders every
 // access to global memory after that kernel.
 template <typename... Params, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, int smem, cudaStream_t s,
-                       Args&&... args) {
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, int threads, int smem,
+                       cudaStream_t s, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -843,7 +856,8 @@ cudaError_t launch_reduce_tc(const Problem& p, const void* K, const void* V, flo
       cudaSuccess)
     return e;
   const dim3 grid(p.splits, (p.H + kGroupHeads - 1) / kGroupHeads, p.B);
-  e = launch_pdl(kern, grid, kRedSmemBytes, s, mk, mv, p, rt, partials, counters, out);
+  e = launch_pdl(kern, grid, kRedThreads, kRedSmemBytes, s, mk, mv, p, rt, partials, counters,
+                 out);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -875,7 +889,7 @@ cudaError_t launch_apply_tc(const Problem& p, const void* Q, const float* S, con
   // Q may be read before the previous kernel completes only when that kernel
   // is this library's own state reduce, which does not write Q and itself
   // started reading only after everything before it had completed.
-  e = launch_pdl(kern, grid, kApSmemBytes, s, mq, mo, p, rt, S, z, tiles_per_cta,
+  e = launch_pdl(kern, grid, kThreads, kApSmemBytes, s, mq, mo, p, rt, S, z, tiles_per_cta,
                  after_own_reduce ? 1 : 0);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
