@@ -55,6 +55,28 @@ def env_int(name, default):
         return default
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """The largest value of x over all ranks (x itself on a single process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaled_value(tokens_per_step: int, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank processes its own copy of the workload,
+    and the job takes as long as its slowest rank."""
+    return world * tokens_per_step * steps / (ms_max / 1e3)
+
+
+def rank_seed(rank: int) -> int:
+    """Base input seed of a rank: each replica draws its own batch."""
+    return 1000 * int(rank)
+
+
 def layer_bytes(w, io_bytes=2):
     """Algorithmic HBM bytes of one layer: read Q, K, V, write O, write/read the state."""
     th = w.B * w.N * w.H
@@ -239,9 +261,9 @@ def run_la(args, w, rank, world, local_rank):
     sets = []
     for i in range(n_sets):
         if w.block_causal:
-            q, k, v = wl.make_qkv(w, 1000 * rank, block=0, step=i)
+            q, k, v = wl.make_qkv(w, rank_seed(rank), block=0, step=i)
         else:
-            q, k, v = wl.make_qkv(w, 1000 * rank + 10 * i)
+            q, k, v = wl.make_qkv(w, rank_seed(rank) + 10 * i)
         q, k, v = (x.to(dev) for x in (q, k, v))
         sets.append((q, k, v, torch.empty_like(q)))
     S = torch.zeros((w.B, w.H, D, D), device=dev)
@@ -368,11 +390,7 @@ def run_la(args, w, rank, world, local_rank):
     seg = [[e[j].elapsed_time(e[j + 1]) for e in ev_chunk] for j in range(n_ev - 1)]
     seg_us = [1000.0 * statistics.mean(x) for x in seg]
 
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dev)
 
     # end-to-end through the public API with host buffers
     e2e = run_e2e(args, w, dev, stream, la, rank) if args.e2e_steps > 0 else None
@@ -499,7 +517,7 @@ def main():
 
     ms_step = r["ms"] / args.steps
     tokens_step = (w.M * w.N * w.B) if w.block_causal else w.B * w.N
-    value = world * tokens_step * args.steps / (r["ms"] / 1e3)
+    value = weak_scaled_value(tokens_step, args.steps, world, r["ms"])
     peak, peak_src = peaks()
     lb = layer_bytes(w)
     if w.block_causal:
