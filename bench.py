@@ -78,11 +78,10 @@ def rank_seed(rank: int) -> int:
 
 
 def layer_bytes(w, io_bytes=2):
-    """Algorithmic HBM bytes of one layer: read Q, K, V, write O, write/read the state."""
+    """Algorithmic HBM bytes of one layer: read Q, K, V, write O, write the state."""
     th = w.B * w.N * w.H
     state = w.B * w.H * (D * D + D) * 4
-    return {"state_reduce": 2 * th * D * io_bytes + state,   # read K, V; write S, z
-            "apply": 2 * th * D * io_bytes + state}          # read Q, S, z; write O
+    return {"attention_layer": 4 * th * D * io_bytes + state}
 
 
 def peaks():
@@ -284,7 +283,8 @@ def run_la(args, w, rank, world, local_rank):
 
     if w.block_causal:
         calls_per_step = w.M * (w.steps + 1)
-        launches_per_step = 2 * calls_per_step  # reduce + apply per call; reset is memsets
+        # one or two kernels per call (see la_attention_launches); reset is memsets
+        launches_per_step = la.la_attention_launches(keep[0]) * calls_per_step
 
         def step(i, evs=None):
             status.append(lib.la_state_reset(S_p, z_p, w.B, w.H, D, sp))
@@ -302,19 +302,16 @@ def run_la(args, w, rank, world, local_rank):
                     c += 1
         kernel_names = ("la_block_causal_step",)
     else:
-        launches_per_step = 2
+        launches_per_step = la.la_attention_launches(keep[0])
 
         def step(i, evs=None):
             q, k, v, o = ptrs[i % n_sets]
             if evs is not None:
                 evs[0].record(stream)
-            status.append(lib.la_state_reduce(shapes[0], k, v, S_p, z_p, ws_p, ws_n, sp))
+            status.append(lib.la_attention(shapes[0], q, k, v, S_p, z_p, o, ws_p, ws_n, sp))
             if evs is not None:
                 evs[1].record(stream)
-            status.append(lib.la_apply(shapes[0], q, S_p, z_p, o, sp))
-            if evs is not None:
-                evs[2].record(stream)
-        kernel_names = ("state_reduce", "apply")
+        kernel_names = ("attention_layer",)
 
     def check_status():
         bad = [s for s in status if s != 0]
@@ -331,7 +328,7 @@ def run_la(args, w, rank, world, local_rank):
     check_status()
 
     # chunk graph: C steps, with an event after every launch
-    n_ev = 3 if not w.block_causal else 2
+    n_ev = 2
     chunk = n_sets * max(1, 100 // n_sets) if not w.block_causal else 1
     chunk = min(chunk, args.steps) if args.steps > 0 else chunk
     chunk = max(1, chunk - chunk % n_sets) if chunk >= n_sets else chunk
@@ -525,14 +522,16 @@ def main():
         alg = 4 * w.B * w.N * w.H * D * 2 + 2 * w.B * w.H * (D * D + D) * 4
         dur_us = r["seg_us"][0]
         kernels = {name: {"avg_us": dur_us, "algorithmic_bytes": alg,
-                          "gbs": alg / (dur_us * 1e-6) / 1e9, "launches": 2}}
+                          "gbs": alg / (dur_us * 1e-6) / 1e9,
+                          "launches": r["launches_per_step"] // (w.M * (w.steps + 1))}}
         dom = name
         traffic = None
     else:
         kernels = {}
         for nm, us in zip(r["kernel_names"], r["seg_us"]):
             kernels[nm] = {"avg_us": us, "algorithmic_bytes": lb[nm],
-                           "gbs": lb[nm] / (us * 1e-6) / 1e9, "launches": 1}
+                           "gbs": lb[nm] / (us * 1e-6) / 1e9,
+                           "launches": r["launches_per_step"]}
         dom = max(kernels, key=lambda k: kernels[k]["avg_us"])
         traffic = profiled_traffic(w.name, dom)
     kd = kernels[dom]

@@ -73,6 +73,8 @@ _lib.la_status_string.argtypes = [_i]
 _lib.la_status_string.restype = ctypes.c_char_p
 _lib.la_last_error.argtypes = []
 _lib.la_last_error.restype = ctypes.c_char_p
+_lib.la_attention_launches.argtypes = [_shape_p]
+_lib.la_attention_launches.restype = _i
 _lib.la_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), _i]
 _lib.la_device_error.restype = _i
 
@@ -153,6 +155,11 @@ def la_block_causal_step(shape: LaShape, Q, K, V, S_carry, z_carry, O, update: i
 def la_state_reset(S, z, B: int, H: int, D: int = HEAD_DIM, stream=None) -> None:
     _check(_lib.la_state_reset(_ptr(S), _ptr(z), int(B), int(H), int(D), _stream(stream)),
            "la_state_reset")
+
+
+def la_attention_launches(shape: LaShape) -> int:
+    """Kernel launches of la_attention / la_block_causal_step (update 0, 1)."""
+    return int(_lib.la_attention_launches(ctypes.byref(shape)))
 
 
 def la_status_string(status: int) -> str:

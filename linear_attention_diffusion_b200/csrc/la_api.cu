@@ -164,7 +164,7 @@ WsLayout workspace_layout(const Problem& p) {
   WsLayout L;
   const size_t bh = static_cast<size_t>(p.B) * p.H;
   L.counters = 0;
-  L.partials = align256(bh * sizeof(unsigned));
+  L.partials = align256(3 * bh * sizeof(unsigned));
   L.state_S = align256(L.partials + bh * p.splits * kStateFloats * sizeof(float));
   L.state_z = align256(L.state_S + bh * kD * kD * sizeof(float));
   L.total = align256(L.state_z + bh * kD * sizeof(float));
@@ -252,6 +252,14 @@ la_status la_attention(const la_shape* shape, const void* Q, const void* K, cons
   float* Sw = reinterpret_cast<float*>(w + L.state_S);
   float* zw = reinterpret_cast<float*>(w + L.state_z);
   const StateOut out = {nullptr, nullptr, Sw, zw, S, z};
+  if (any_input && layer_fusable(p)) {
+    const cudaError_t e = launch_layer_tc(p, Q, K, V, O, reinterpret_cast<float*>(w + L.partials),
+                                          reinterpret_cast<unsigned*>(w + L.counters), out, st);
+    if (e == cudaSuccess) return LA_OK;
+    if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge)
+      return cuda_fail(e, "attention layer");
+    (void)cudaGetLastError();  // clear the refused launch, take the two-kernel path
+  }
   LA_TRY(run_reduce(p, K, V, w, out, st));
   if (!any_input) return LA_OK;
   const cudaError_t e = launch_apply(p, Q, Sw, zw, O, true, st);
@@ -294,6 +302,14 @@ la_status la_block_causal_step(const la_shape* shape, const void* Q, const void*
   const bool to_carry = update >= 1;
   const StateOut out = {S_carry, z_carry, to_ws ? Sw : nullptr, to_ws ? zw : nullptr,
                         to_carry ? S_carry : nullptr, to_carry ? z_carry : nullptr};
+  if (uses_q && any_input && layer_fusable(p)) {
+    const cudaError_t e = launch_layer_tc(p, Q, K, V, O, reinterpret_cast<float*>(w + L.partials),
+                                          reinterpret_cast<unsigned*>(w + L.counters), out, st);
+    if (e == cudaSuccess) return LA_OK;
+    if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge)
+      return cuda_fail(e, "block-causal layer");
+    (void)cudaGetLastError();
+  }
   LA_TRY(run_reduce(p, K, V, w, out, st));
   if (!uses_q || !any_input) return LA_OK;
   const cudaError_t e = launch_apply(p, Q, Sw, zw, O, true, st);
@@ -314,6 +330,14 @@ la_status la_state_reset(float* S, float* z, int B, int H, int D, la_stream stre
   if (e == cudaSuccess) e = cudaMemsetAsync(z, 0, bh * kD * sizeof(float), st);
   if (e != cudaSuccess) return cuda_fail(e, "state reset");
   return LA_OK;
+}
+
+int la_attention_launches(const la_shape* shape) {
+  Problem p;
+  if (make_problem(shape, p) != LA_OK) return 0;
+  if (p.B == 0 || p.H == 0) return 0;
+  if (p.N == 0) return 1;
+  return layer_fusable(p) ? 1 : 2;
 }
 
 const char* la_status_string(la_status status) {

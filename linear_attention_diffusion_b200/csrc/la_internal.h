@@ -33,7 +33,7 @@ struct Problem {
 
 // Workspace layout (byte offsets, 256-aligned), a pure function of the shape.
 struct WsLayout {
-  size_t counters;  // [B*H] uint32 arrival counters; zero between calls
+  size_t counters;  // [3][B*H] uint32 arrival / ready / departure words; zero between calls
   size_t partials;  // [B*H][splits][kStateFloats] float32
   size_t state_S;   // [B*H][32*32] float32
   size_t state_z;   // [B*H][32] float32
@@ -75,6 +75,14 @@ cudaError_t launch_reduce_simt(const Problem& p, const void* K, const void* V, f
                                unsigned* counters, const StateOut& out, cudaStream_t s);
 cudaError_t launch_apply_simt(const Problem& p, const void* Q, const float* S, const float* z,
                               void* O, cudaStream_t s);
+// The whole layer (state reduce, then apply) in one cooperative launch; the
+// reduce's combined state goes to `out` (out.out1_* must be set: the apply
+// reads it there). Returns cudaErrorNotSupported when the shape does not fit
+// one wave of co-resident CTAs; the caller then launches reduce and apply.
+bool layer_fusable(const Problem& p);
+cudaError_t launch_layer_tc(const Problem& p, const void* Q, const void* K, const void* V,
+                            void* O, float* partials, unsigned* counters, const StateOut& out,
+                            cudaStream_t s);
 // Device error word of the tensor-core kernels (bounded waits that gave up).
 cudaError_t read_device_error(unsigned* code, bool reset);
 

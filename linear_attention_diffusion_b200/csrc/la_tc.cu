@@ -30,6 +30,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 #include <utility>
 
@@ -46,11 +47,6 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kApWG = 3;            // apply: math warpgroups, one tile each in turn
-constexpr int kThreads = 64 + 128 * kApWG;  // apply: TMA warp, MMA warp, math warpgroups
-constexpr int kMathThreads = 128 * kApWG;
-constexpr int kRedMath = 512;       // reduce: 16 math warps
-constexpr int kRedThreads = 64 + kRedMath;
 constexpr int kGroupHeads = 4;
 constexpr int kRopeTableMax = 1536;  // float2 entries of the per-CTA RoPE table
 
@@ -184,77 +180,98 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
                : "memory");
 }
 
-// ================================================================ reduce
+// ============================================================ the kernel
 
-constexpr int kRedT = 64;                          // tokens per stage
-constexpr int kRedStages = 5;
-constexpr int kRedBox = kRedT * 128;               // bytes of one [64 tokens][64 dims] box
-constexpr int kRedStageBytes = 4 * kRedBox;        // K box 0, K box 1, V box 0, V box 1
-constexpr int kRedTmemCols = 128;
+// One kernel template serves three launches: the state reduce alone, the
+// apply alone, and the fused layer (reduce, a per-head-group hand-off, then
+// apply). All share one TMA stage ring: a ring position p uses stage p % 5
+// with phase parity (p / 5) & 1, whichever operation the tile belongs to.
+enum Phases : int { kReduceOnly = 1, kApplyOnly = 2, kFusedLayer = 3 };
 
-struct RedSmem {
-  // offsets from the 1024-aligned base
+constexpr int kMath = 512;                   // 16 math warps (warps 2..17)
+constexpr int kThreadsTc = 64 + kMath;       // + TMA warp + MMA warp
+constexpr int kApWG = kMath / 128;           // apply: 4 warpgroups, one tile each in turn
+constexpr int kStages = 5;
+constexpr int kStageBytes = 32768;
+constexpr int kRedT = 64;                    // reduce: tokens per stage (K and V, 4 heads)
+constexpr int kRedBox = kRedT * 128;         // [64 tokens][64 dims] bf16
+constexpr int kApT = 128;                    // apply: tokens per tile (Q, 4 heads)
+constexpr int kApBox = kApT * 128;           // [128 tokens][64 dims] bf16
+constexpr int kTmemCols = 512;               // reduce: cols [0,128); apply: kApWG x 128
+
+// named barriers: 0 = whole CTA, 1 = all math threads, 2.. = apply warpgroups
+constexpr int kBarMath = 1;
+constexpr int kBarWG0 = 2;
+
+struct Smem {  // byte offsets from the 1024-aligned base
   static constexpr int stages = 0;
-  static constexpr int zred = stages + kRedStages * kRedStageBytes;    // [512][8] float
-  static constexpr int rope = zred + kRedMath * 8 * 4;                 // float2[kRopeTableMax]
-  static constexpr int bars = rope + kRopeTableMax * 8;                // mbarriers
-  static constexpr int nbars = 3 * kRedStages + 3;
-  static constexpr int misc = bars + nbars * 8;                        // tmem base, abort
+  static constexpr int zred = stages + kStages * kStageBytes;  // [512][8] f32; then S scratch
+  static constexpr int bop = zred + kMath * 8 * 4;             // [2 pairs][32 rows][128 B]
+  static constexpr int zs = bop + 2 * 32 * 128;                // [4][32] f32
+  static constexpr int rope = zs + kGroupHeads * kD * 4;       // float2[kRopeTableMax]
+  static constexpr int bars = rope + kRopeTableMax * 8;
+  // full[5] empty[5] ready[5] t_full[4] t_empty[4] acc_full mma_done b_ready
+  static constexpr int nbars = 3 * kStages + 2 * kApWG + 3;
+  static constexpr int misc = bars + nbars * 8;                // tmem base, abort, last flag
   static constexpr int bytes = misc + 16;
 };
-constexpr int kRedSmemBytes = RedSmem::bytes + 1024;
+constexpr int kSmemBytes = Smem::bytes + 1024;
 
-// Second phase of the reduce for a group of 4 heads: the CTA that arrives
-// last for the group copies the group's partials (contiguous: heads x splits
-// x 1056 floats) into shared memory with bulk copies, sums them in split
-// order, adds the carry when given, writes the outputs and re-zeroes the
-// counter. Falls back to the register version when they do not fit.
-__device__ __forceinline__ void finish_reduce_bulk(const Problem& p, int b, int h0,
-                                                   const float* partials, unsigned* counters,
-                                                   const StateOut& out, uint8_t* smem,
-                                                   uint64_t* comb_full, volatile int* abort_flag) {
-  const int heads = min(kGroupHeads, p.H - h0);
-  const uint32_t per_head = static_cast<uint32_t>(p.splits) * kStateFloats * 4;
-  if (static_cast<size_t>(heads) * per_head > static_cast<size_t>(kRedStages) * kRedStageBytes) {
-    finish_reduce(p, b, h0, kGroupHeads, partials, counters, out);
-    return;
-  }
-  __shared__ int s_last;
-  // The CTA barrier orders every thread's partial stores before thread 0's
-  // release fence; the CTA that arrives last acquires all groups' stores.
-  __syncthreads();
-  const size_t cidx = static_cast<size_t>(b) * p.H + h0;
-  if (threadIdx.x == 0) {
-    fence_acq_rel_gpu();
-    const unsigned prev = atomicAdd(&counters[cidx], 1u);
-    s_last = prev == static_cast<unsigned>(p.splits - 1);
-    if (s_last) fence_acq_rel_gpu();
-  }
-  __syncthreads();
-  if (!s_last) return;
-  const float* src = partials + cidx * p.splits * kStateFloats;
-  float* buf = reinterpret_cast<float*>(smem + RedSmem::stages);
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(comb_full, heads * per_head);
-    for (int hh = 0; hh < heads; ++hh)
-      bulk_load(reinterpret_cast<uint8_t*>(buf) + hh * per_head,
-                reinterpret_cast<const uint8_t*>(src) + hh * per_head, per_head, comb_full);
-  }
-  const bool ok = mbar_wait(comb_full, 0, abort_flag, &g_tc_error, kErrWait);
-  if (!ok) return;  // the counter stays raised: the device error word reports it
-  constexpr int kVec = kStateFloats / 4;
-  for (int v = threadIdx.x; v < heads * kVec; v += blockDim.x) {
-    const int hh = v / kVec, i = (v - hh * kVec) * 4;
-    const float4* col = reinterpret_cast<const float4*>(buf + hh * p.splits * kStateFloats + i);
-    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    for (int sp = 0; sp < p.splits; ++sp) {
-      const float4 t = col[sp * (kStateFloats / 4)];
-      acc.x += t.x;
-      acc.y += t.y;
-      acc.z += t.z;
-      acc.w += t.w;
+struct LayerArgs {
+  float* partials;     // [B*H][splits][kStateFloats]
+  unsigned* arrive;    // [B*H] per head-group arrival counters (index b*H + h0)
+  unsigned* ready;     // [B*H] fused layer: "combined state written" flags
+  unsigned* depart;    // [B*H] fused layer: departure counters
+  StateOut out;        // where the reduce's combined state goes
+  const float* S_in;   // apply: state to apply (fused: out.out1_S)
+  const float* z_in;
+  int tiles_per_cta;   // apply: 128-token tiles per CTA
+  int q_before_wait;   // apply only: Q may be read before the previous grid completes
+};
+
+__device__ __forceinline__ bool spin_flag(const unsigned* flag, volatile int* abort_flag) {
+  if (ld_acquire_gpu(flag) != 0u) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (ld_acquire_gpu(flag) != 0u) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicOr(&g_tc_error, kErrWait);
+      return false;
     }
+    __nanosleep(64);
+  }
+}
+
+// Sum of the head group's split partials in split order (+ carry), written to
+// StateOut; by the math threads of the CTA that arrived last, from registers
+// (the stage ring may already hold prefetched tiles).
+__device__ __forceinline__ void combine_from_global(const Problem& p, int b, int h0, int mt,
+                                                    const float* partials, const StateOut& out) {
+  constexpr int kVec = kStateFloats / 4;
+  const int heads = min(kGroupHeads, p.H - h0);
+  const size_t cidx = static_cast<size_t>(b) * p.H + h0;
+  for (int v = mt; v < heads * kVec; v += kMath) {
+    const int hh = v / kVec, i = (v - hh * kVec) * 4;
     const size_t bh = cidx + hh;
+    const float* src = partials + bh * p.splits * kStateFloats + i;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int s0 = 0; s0 < p.splits; s0 += 8) {
+      float4 t[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (s0 + k < p.splits)
+          t[k] = __ldcg(reinterpret_cast<const float4*>(src + static_cast<size_t>(s0 + k) * kStateFloats));
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (s0 + k < p.splits) {
+          acc.x += t[k].x;
+          acc.y += t[k].y;
+          acc.z += t[k].z;
+          acc.w += t[k].w;
+        }
+    }
     const bool is_s = i < kD * kD;
     const size_t o = is_s ? bh * kD * kD + i : bh * kD + (i - kD * kD);
     const float* c = is_s ? out.carry_S : out.carry_z;
@@ -267,372 +284,160 @@ __device__ __forceinline__ void finish_reduce_bulk(const Problem& p, int b, int 
     if (d1 != nullptr) *reinterpret_cast<float4*>(d1 + o) = acc;
     if (d2 != nullptr) *reinterpret_cast<float4*>(d2 + o) = acc;
   }
-  if (threadIdx.x == 0) counters[cidx] = 0u;
 }
 
-template <int kRope>
-__global__ void __launch_bounds__(kRedThreads, 1)
-reduce_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-          const Problem p, const RopeTable rt, float* partials, unsigned* counters,
-          const StateOut out) {
+template <int kRope, int kPh>
+__global__ void __launch_bounds__(kThreadsTc, 1)
+layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+         const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
+         const Problem p, const RopeTable rt, const LayerArgs a) {
+  constexpr bool kRed = (kPh & kReduceOnly) != 0;
+  constexpr bool kApp = (kPh & kApplyOnly) != 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + RedSmem::bars);
-  uint64_t* ready = full + kRedStages;
-  uint64_t* empty = ready + kRedStages;
-  uint64_t* acc_full = empty + kRedStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Smem::bars);
+  uint64_t* empty = full + kStages;
+  uint64_t* ready = empty + kStages;
+  uint64_t* t_full = ready + kStages;   // [kApWG]
+  uint64_t* t_empty = t_full + kApWG;   // [kApWG]
+  uint64_t* acc_full = t_empty + kApWG;
   uint64_t* mma_done = acc_full + 1;
-  uint64_t* comb_full = mma_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + RedSmem::misc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + RedSmem::misc + 4);
-  float* zred = reinterpret_cast<float*>(smem + RedSmem::zred);
-  float2* rope_tab = reinterpret_cast<float2*>(smem + RedSmem::rope);
+  uint64_t* b_ready = mma_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + Smem::misc + 8);
+  float* zred = reinterpret_cast<float*>(smem + Smem::zred);
+  float* zs = reinterpret_cast<float*>(smem + Smem::zs);
+  float2* rope_tab = reinterpret_cast<float2*>(smem + Smem::rope);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int split = blockIdx.x, group = blockIdx.y, b = blockIdx.z;
+  const int group = blockIdx.y, b = blockIdx.z;
   const int h0 = group * kGroupHeads;
-  const int n_begin = split * p.chunk;
+  const size_t cidx = static_cast<size_t>(b) * p.H + h0;
+  // reduce work: the token split blockIdx.x, in 64-token stages
+  const int n_begin = blockIdx.x * p.chunk;
   const int n_end = min(p.N, n_begin + p.chunk);
-  const int ntiles = n_end > n_begin ? (n_end - n_begin + kRedT - 1) / kRedT : 0;
+  const int nA = kRed && n_end > n_begin ? (n_end - n_begin + kRedT - 1) / kRedT : 0;
+  // apply work: a range of 128-token tiles
+  const int ntiles_all = (p.N + kApT - 1) / kApT;
+  const int tile_begin = blockIdx.x * a.tiles_per_cta;
+  const int nB = kApp ? max(0, min(ntiles_all, tile_begin + a.tiles_per_cta) - tile_begin) : 0;
 
   if (tid == 0) {
-    for (int s = 0; s < kRedStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&ready[s], kRedMath);
       mbar_init(&empty[s], 1);
+      mbar_init(&ready[s], 1);
+    }
+    for (int w = 0; w < kApWG; ++w) {
+      mbar_init(&t_full[w], 1);
+      mbar_init(&t_empty[w], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
-    mbar_init(comb_full, 1);
+    mbar_init(b_ready, 1);
     *abort_flag = 0;
+    *last_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kRedTmemCols);
+    tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
     tc_fence_before();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_k);
-    prefetch_tmap(&tm_v);
+    if (kRed) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+    }
+    if (kApp) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_o);
+    }
   }
-  if (kRope == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kRedMath);
+  if (kRope == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kMath);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(smem);
-  // Everything above overlaps the previous kernel's tail; global memory is
-  // touched only after it has completed. Then the next kernel may launch.
-  pdl_wait();
-  if (tid == 0) pdl_trigger();
+
+  // Programmatic dependent launch: global memory is touched only after the
+  // previous grid has completed -- except Q in an apply whose previous grid is
+  // this library's own reduce (q_before_wait), which the TMA warp may fetch
+  // early. The next grid may then be scheduled.
+  const bool early_q = kPh == kApplyOnly && a.q_before_wait;
+  if (!(warp == 0 && early_q)) pdl_wait();
+  if (tid == 64) pdl_trigger();
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- TMA
+    // ------------------------------------------------------------ TMA loads
     if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int s = i % kRedStages;
-        const uint32_t ph = (i / kRedStages) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, &g_tc_error, kErrWait)) break;
-        mbar_arrive_expect_tx(&full[s], kRedStageBytes);
-        uint8_t* st = smem + RedSmem::stages + s * kRedStageBytes;
+      int pos = 0;
+      bool ok = true;
+      for (int i = 0; ok && i < nA; ++i, ++pos) {
+        const int s = pos % kStages;
+        if (!(ok = mbar_wait(&empty[s], ((pos / kStages) & 1) ^ 1, abort_flag, &g_tc_error,
+                             kErrWait)))
+          break;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        uint8_t* st = smem + Smem::stages + s * kStageBytes;
         const int y = n_begin + i * kRedT;
         tma_load_3d(st, &tm_k, &full[s], h0 * 32, y, b);
         tma_load_3d(st + kRedBox, &tm_k, &full[s], h0 * 32 + 64, y, b);
         tma_load_3d(st + 2 * kRedBox, &tm_v, &full[s], h0 * 32, y, b);
         tma_load_3d(st + 3 * kRedBox, &tm_v, &full[s], h0 * 32 + 64, y, b);
-        issued = i + 1;
+      }
+      for (int i = 0; ok && i < nB; ++i, ++pos) {
+        const int s = pos % kStages;
+        if (!(ok = mbar_wait(&empty[s], ((pos / kStages) & 1) ^ 1, abort_flag, &g_tc_error,
+                             kErrWait)))
+          break;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        uint8_t* st = smem + Smem::stages + s * kStageBytes;
+        const int y = (tile_begin + i) * kApT;
+        tma_load_3d(st, &tm_q, &full[s], h0 * 32, y, b);
+        tma_load_3d(st + kApBox, &tm_q, &full[s], h0 * 32 + 64, y, b);
       }
       // drain: every load issued must have landed before the CTA exits
-      for (int i = max(0, issued - kRedStages); i < issued; ++i)
-        mbar_wait(&full[i % kRedStages], (i / kRedStages) & 1, abort_flag, nullptr, 0);
+      for (int q = max(0, pos - kStages); q < pos; ++q)
+        mbar_wait(&full[q % kStages], (q / kStages) & 1, abort_flag, nullptr, 0);
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA
+    // ------------------------------------------------------------------ MMA
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, 128, 1, 1);
-      for (int i = 0; i < ntiles; ++i) {
-        const int s = i % kRedStages;
-        const uint32_t ph = (i / kRedStages) & 1;
-        if (!mbar_wait(&ready[s], ph, abort_flag, &g_tc_error, kErrWait)) break;
+      int pos = 0;
+      bool ok = true;
+      const uint32_t id_red = idesc_bf16_f32(128, 128, 1, 1);
+      for (int i = 0; i < nA; ++i, ++pos) {
+        const int s = pos % kStages;
+        if (!(ok = mbar_wait(&ready[s], (pos / kStages) & 1, abort_flag, &g_tc_error, kErrWait)))
+          break;
         tc_fence_after();
-        const uint32_t st = sbase + RedSmem::stages + s * kRedStageBytes;
+        const uint32_t st = sbase + Smem::stages + s * kStageBytes;
 #pragma unroll
         for (int kk = 0; kk < kRedT / 16; ++kk) {
-          // 16 tokens = two 8-row groups of 128 bytes
+          // 16 tokens = two 8-row groups of 128 bytes; LBO = the second 64-dim box
           const uint64_t ad = smem_desc_sw128(st + kk * 2048, kRedBox, 1024);
           const uint64_t bd = smem_desc_sw128(st + 2 * kRedBox + kk * 2048, kRedBox, 1024);
-          mma_bf16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16(tmem, ad, bd, id_red, (i > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&empty[s]);
       }
-      mma_commit(acc_full);
-      mma_commit(mma_done);
-      mbar_wait(mma_done, 0, abort_flag, nullptr, 0);
-    }
-  } else {
-    // ------------------------------------------------- feature map + key sum
-    const int wt = tid - 64;
-    const int c = wt & 15;        // 16-byte chunk column: box c/8, chunk c%8 of the row
-    const int rg = wt >> 4;       // row group: rows rg and rg + 32 of every stage
-    const int box = c >> 3, cc = c & 7;
-    const int dpos = (cc & 3) * 8;  // first dim of the chunk inside its head
-    float2 zacc[4] = {};
-    // this thread's tokens are n_begin + rg + 32 j, j = 0, 1, ...; its chunk
-    // holds RoPE pairs j0 .. j0+3 (fixed per thread)
-    TokPos tp = {0, 0, 0};
-    if (kRope != kNoRope) tp = token_pos(p.rope, n_begin + rg);
-    const int j0 = dpos / 2;
-    int sel[4], off[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      sel[q] = pair_axis(j0 + q);
-      off[q] = pair_off(j0 + q);
-    }
-    for (int i = 0; i < ntiles; ++i) {
-      const int s = i % kRedStages;
-      const uint32_t ph = (i / kRedStages) & 1;
-      if (!mbar_wait(&full[s], ph, abort_flag, &g_tc_error, kErrWait)) break;
-      const uint32_t kb = sbase + RedSmem::stages + s * kRedStageBytes + box * kRedBox;
-      const int y0 = n_begin + i * kRedT;
-#pragma unroll
-      for (int k = 0; k < kRedT / 32; ++k) {
-        const int r = rg + 32 * k;
-        const uint32_t addr = kb + sw128_offset(r, cc);
-        uint4 u = ld_shared_v4(addr);
-        u.x = relu_bf16x2(u.x);
-        u.y = relu_bf16x2(u.y);
-        u.z = relu_bf16x2(u.z);
-        u.w = relu_bf16x2(u.w);
-        float x[8];
-        unpack8(u, x);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) zacc[e] = __fadd2_rn(zacc[e], make_float2(x[2 * e], x[2 * e + 1]));
-        if (kRope != kNoRope) {
-          if (y0 + r < p.N) {
-            const RopeBases rb = rope_bases(p.rope, tp);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float2 cs;
-              if (kRope == kRopeTable) {
-                cs = rope_tab[(sel[q] == 0 ? rb.t : (sel[q] == 1 ? rb.h : rb.w)) + off[q]];
-              } else {
-                const int pos = sel[q] == 0 ? p.rope.t_offset + tp.t : (sel[q] == 1 ? tp.h : tp.w);
-                rope_cos_sin(pos, p.rope.inv_freq[j0 + q], cs.x, cs.y);
-              }
-              const float2 t = __fmul2_rn(make_float2(x[2 * q + 1], x[2 * q + 1]),
-                                          make_float2(-cs.y, cs.x));
-              const float2 y = __ffma2_rn(make_float2(x[2 * q], x[2 * q]), cs, t);
-              x[2 * q] = y.x;
-              x[2 * q + 1] = y.y;
-            }
-            u = pack8(x);
-          }
-          token_pos_advance(p.rope, tp, 32);
-        }
-        st_shared_v4(addr, u);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&ready[s]);
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      zred[wt * 8 + 2 * e] = zacc[e].x;
-      zred[wt * 8 + 2 * e + 1] = zacc[e].y;
-    }
-    named_bar_sync(1, kRedMath);
-
-    // state of the four heads: the 32x32 diagonal blocks of the accumulator
-    if (warp >= 2 && warp < 6) {
-      const int q = warp & 3;  // TMEM lane quadrant = head in the group
-      float v[32];
-      bool ok = ntiles > 0 && mbar_wait(acc_full, 0, abort_flag, &g_tc_error, kErrWait);
-      ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld is warp-collective
-      if (ok) {
-        tc_fence_after();
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32 * q, v);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = 0.0f;
-      }
-      const int h = h0 + q;
-      if (h < p.H) {
-        float* dst = partials +
-                     ((static_cast<size_t>(b) * p.H + h) * p.splits + split) * kStateFloats +
-                     lane * kD;
-#pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-      }
-    }
-    if (wt < 128) {
-      // key sum of dim wt of the group: 32 row groups, in order
-      const int q = wt >> 5, d = wt & 31;
-      const int col = wt >> 3, e = wt & 7;  // chunk column and element holding this dim
-      float s = 0.0f;
-      for (int r = 0; r < kRedMath / 16; ++r) s += zred[(r * 16 + col) * 8 + e];
-      const int h = h0 + q;
-      if (h < p.H)
-        partials[((static_cast<size_t>(b) * p.H + h) * p.splits + split) * kStateFloats +
-                 kD * kD + d] = s;
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kRedTmemCols);
-  }
-  if (*abort_flag) return;  // partials incomplete: leave the counter alone
-  finish_reduce_bulk(p, b, h0, partials, counters, out, smem, comb_full, abort_flag);
-}
-
-// ================================================================= apply
-
-constexpr int kApT = 128;                          // tokens per tile
-constexpr int kApStages = 5;
-constexpr int kApBox = kApT * 128;                 // [128 tokens][64 dims] bf16
-constexpr int kApStageBytes = 2 * kApBox;
-constexpr int kApTmemCols = 512;                   // kApWG 128-column accumulators
-
-// A stage holds a tile's Q, then phi(Q) for the MMA, then the tile's O for the
-// TMA store: it is released to the producer once the store has read it.
-struct ApSmem {
-  static constexpr int stages = 0;
-  static constexpr int bop = stages + kApStages * kApStageBytes;       // [2 pairs][32][128 B]
-  static constexpr int zs = bop + 2 * 32 * 128;                        // [4][32] float
-  static constexpr int rope = zs + kGroupHeads * kD * 4;               // float2[kRopeTableMax]
-  static constexpr int bars = rope + kRopeTableMax * 8;
-  static constexpr int nbars = 3 * kApStages + 2 * kApWG + 2;
-  static constexpr int misc = bars + nbars * 8;
-  static constexpr int bytes = misc + 16;
-};
-constexpr int kApSmemBytes = ApSmem::bytes + 1024;
-
-template <int kRope>
-__global__ void __launch_bounds__(kThreads, 1)
-apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
-         const Problem p, const RopeTable rt, const float* __restrict__ S,
-         const float* __restrict__ z, int tiles_per_cta, int q_before_wait) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + ApSmem::bars);
-  uint64_t* q_ready = q_full + kApStages;
-  uint64_t* q_empty = q_ready + kApStages;
-  uint64_t* t_full = q_empty + kApStages;   // [kApWG]
-  uint64_t* t_empty = t_full + kApWG;       // [kApWG]
-  uint64_t* mma_done = t_empty + kApWG;
-  uint64_t* b_ready = mma_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + ApSmem::misc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + ApSmem::misc + 4);
-  float* zs = reinterpret_cast<float*>(smem + ApSmem::zs);
-  float2* rope_tab = reinterpret_cast<float2*>(smem + ApSmem::rope);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int group = blockIdx.y, b = blockIdx.z;
-  const int h0 = group * kGroupHeads;
-  const int ntiles_all = (p.N + kApT - 1) / kApT;
-  const int tile_begin = blockIdx.x * tiles_per_cta;
-  const int ntiles = max(0, min(ntiles_all, tile_begin + tiles_per_cta) - tile_begin);
-
-  if (tid == 0) {
-    for (int s = 0; s < kApStages; ++s) {
-      mbar_init(&q_full[s], 1);
-      mbar_init(&q_ready[s], 128);
-      mbar_init(&q_empty[s], 1);
-    }
-    for (int a = 0; a < kApWG; ++a) {
-      mbar_init(&t_full[a], 1);
-      mbar_init(&t_empty[a], 128);
-    }
-    mbar_init(mma_done, 1);
-    mbar_init(b_ready, kMathThreads);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, kApTmemCols);
-    tmem_relinquish();
-    tc_fence_before();
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_q);
-    prefetch_tmap(&tm_o);
-  }
-  if (kRope == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kMathThreads);
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t sbase = smem_u32(smem);
-
-  // Programmatic dependent launch: S and z come from the previous kernel, so
-  // they are read only after pdl_wait(). Q may be fetched before it when the
-  // caller knows the previous kernel does not write Q (q_before_wait).
-  if (warp == 0 && !q_before_wait) pdl_wait();
-  if (tid >= 64) {
-    pdl_wait();
-    if (tid == 64) pdl_trigger();
-    const int mt = tid - 64;
-    // B operands: for head pair j, row e holds S[h][0..31][e] of heads 2j and
-    // 2j+1 as bf16 (K-major, 128-byte swizzled)
-    for (int idx = mt; idx < 2 * 32 * 8; idx += kMathThreads) {
-      const int j = idx >> 8, e = (idx >> 3) & 31, c = idx & 7;
-      const int hh = 2 * j + (c >> 2), d0 = (c & 3) * 8;
-      const int h = h0 + hh;
-      float x[8];
-      if (h < p.H) {
-        const float* src = S + ((static_cast<size_t>(b) * p.H + h) * kD + d0) * kD + e;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) x[k] = src[k * kD];
-      } else {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) x[k] = 0.0f;
-      }
-      st_shared_v4(smem_u32(smem + ApSmem::bop + j * 4096) + sw128_offset(e, c), pack8(x));
-    }
-    for (int idx = mt; idx < kGroupHeads * kD; idx += kMathThreads) {
-      const int h = h0 + idx / kD;
-      zs[idx] = h < p.H ? z[(static_cast<size_t>(b) * p.H + h) * kD + idx % kD] : 0.0f;
-    }
-    fence_proxy_async_smem();
-    mbar_arrive(b_ready);
-    named_bar_sync(1 + kApWG, kMathThreads);  // zs visible to every math thread
-  }
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int s = i % kApStages;
-        const uint32_t ph = (i / kApStages) & 1;
-        if (!mbar_wait(&q_empty[s], ph ^ 1, abort_flag, &g_tc_error, kErrWait)) break;
-        mbar_arrive_expect_tx(&q_full[s], kApStageBytes);
-        uint8_t* st = smem + ApSmem::stages + s * kApStageBytes;
-        const int y = (tile_begin + i) * kApT;
-        tma_load_3d(st, &tm_q, &q_full[s], h0 * 32, y, b);
-        tma_load_3d(st + kApBox, &tm_q, &q_full[s], h0 * 32 + 64, y, b);
-        issued = i + 1;
-      }
-      for (int i = max(0, issued - kApStages); i < issued; ++i)
-        mbar_wait(&q_full[i % kApStages], (i / kApStages) & 1, abort_flag, nullptr, 0);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, 32, 0, 0);
-      const uint32_t bop = sbase + ApSmem::bop;
-      const bool have_b = ntiles == 0 || mbar_wait(b_ready, 0, abort_flag, &g_tc_error, kErrWait);
-      for (int i = 0; have_b && i < ntiles; ++i) {
-        const int s = i % kApStages;
-        const uint32_t ph = (i / kApStages) & 1;
-        const int a = i % kApWG;
-        if (!mbar_wait(&q_ready[s], ph, abort_flag, &g_tc_error, kErrWait)) break;
-        if (!mbar_wait(&t_empty[a], ((i / kApWG) & 1) ^ 1, abort_flag, &g_tc_error, kErrWait))
+      if (kRed) mma_commit(acc_full);
+      if (ok && kApp && nB > 0) ok = mbar_wait(b_ready, 0, abort_flag, &g_tc_error, kErrWait);
+      const uint32_t id_ap = idesc_bf16_f32(128, 32, 0, 0);
+      const uint32_t bop = sbase + Smem::bop;
+      for (int j = 0; ok && j < nB; ++j, ++pos) {
+        const int s = pos % kStages;
+        const int w = j % kApWG;
+        if (!(ok = mbar_wait(&ready[s], (pos / kStages) & 1, abort_flag, &g_tc_error, kErrWait)))
+          break;
+        if (!(ok = mbar_wait(&t_empty[w], ((j / kApWG) & 1) ^ 1, abort_flag, &g_tc_error,
+                             kErrWait)))
           break;
         tc_fence_after();
-        const uint32_t st = sbase + ApSmem::stages + s * kApStageBytes;
+        const uint32_t st = sbase + Smem::stages + s * kStageBytes;
 #pragma unroll
         for (int hh = 0; hh < kGroupHeads; ++hh) {
           const uint32_t koff = (hh & 1) * 64;
@@ -640,123 +445,306 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           for (int kk = 0; kk < 2; ++kk) {
             const uint64_t ad = smem_desc_sw128(st + (hh >> 1) * kApBox + koff + kk * 32, 16, 1024);
             const uint64_t bd = smem_desc_sw128(bop + (hh >> 1) * 4096 + koff + kk * 32, 16, 1024);
-            mma_bf16(tmem + a * 128 + hh * 32, ad, bd, idesc, kk);
+            mma_bf16(tmem + w * 128 + hh * 32, ad, bd, id_ap, kk);
           }
         }
-        mma_commit(&t_full[a]);
+        mma_commit(&t_full[w]);
       }
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, abort_flag, nullptr, 0);
     }
   } else {
-    const int wg = (warp - 2) >> 2;
-    const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    const bool leader = (warp == 2 + 4 * wg) && lane == 0;
-    for (int i = wg; i < ntiles; i += kApWG) {
-      const int s = i % kApStages;
-      const uint32_t ph = (i / kApStages) & 1;
-      bool ok = mbar_wait(&q_full[s], ph, abort_flag, &g_tc_error, kErrWait);
-      if (bar_any(1 + wg, 128, !ok || *abort_flag)) break;
-      const int n0 = (tile_begin + i) * kApT;
-      const int n = n0 + row;
-      float2 cs[16];
-      if (kRope != kNoRope) {
-        const TokPos tp = token_pos(p.rope, min(n, p.N - 1));
-        const RopeBases rb = rope_bases(p.rope, tp);
+    // ---------------------------------------------------------- math warps
+    const int mt = tid - 64;
+    bool alive = true;
+    if (kRed) {
+      // feature map of K, key sum: thread mt owns 16-byte chunk column c of
+      // rows rg and rg + 32 of every stage
+      const int c = mt & 15, rg = mt >> 4;
+      const int box = c >> 3, cc = c & 7;
+      const int dpos = (cc & 3) * 8;  // first dim of the chunk inside its head
+      float2 zacc[4] = {};
+      TokPos tp = {0, 0, 0};
+      if (kRope != kNoRope) tp = token_pos(p.rope, n_begin + rg);
+      const int j0 = dpos / 2;
+      int sel[4], off[4];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          if (kRope == kRopeTable) {
-            const int a = pair_axis(j);
-            cs[j] = rope_tab[(a == 0 ? rb.t : (a == 1 ? rb.h : rb.w)) + pair_off(j)];
-          } else {
-            const int a = pair_axis(j);
-            const int pos = a == 0 ? p.rope.t_offset + tp.t : (a == 1 ? tp.h : tp.w);
-            rope_cos_sin(pos, p.rope.inv_freq[j], cs[j].x, cs[j].y);
-          }
-        }
+      for (int q = 0; q < 4; ++q) {
+        sel[q] = pair_axis(j0 + q);
+        off[q] = pair_off(j0 + q);
       }
-      float den[kGroupHeads] = {0.0f, 0.0f, 0.0f, 0.0f};
-      const uint32_t st = sbase + ApSmem::stages + s * kApStageBytes;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int hh = c >> 2, d0 = (c & 3) * 8;
-        const uint32_t addr = st + (c >> 3) * kApBox + sw128_offset(row, c & 7);
-        uint4 u = ld_shared_v4(addr);
-        u.x = relu_bf16x2(u.x);
-        u.y = relu_bf16x2(u.y);
-        u.z = relu_bf16x2(u.z);
-        u.w = relu_bf16x2(u.w);
-        float x[8];
-        unpack8(u, x);
-        const float4 za = *reinterpret_cast<const float4*>(zs + hh * kD + d0);
-        const float4 zb = *reinterpret_cast<const float4*>(zs + hh * kD + d0 + 4);
-        den[hh] = fmaf(x[0], za.x, den[hh]);
-        den[hh] = fmaf(x[1], za.y, den[hh]);
-        den[hh] = fmaf(x[2], za.z, den[hh]);
-        den[hh] = fmaf(x[3], za.w, den[hh]);
-        den[hh] = fmaf(x[4], zb.x, den[hh]);
-        den[hh] = fmaf(x[5], zb.y, den[hh]);
-        den[hh] = fmaf(x[6], zb.z, den[hh]);
-        den[hh] = fmaf(x[7], zb.w, den[hh]);
-        if (kRope != kNoRope) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 r = cs[d0 / 2 + q];
-            const float2 t = __fmul2_rn(make_float2(x[2 * q + 1], x[2 * q + 1]),
-                                        make_float2(-r.y, r.x));
-            const float2 y = __ffma2_rn(make_float2(x[2 * q], x[2 * q]), r, t);
-            x[2 * q] = y.x;
-            x[2 * q + 1] = y.y;
-          }
-          u = pack8(x);
+      for (int i = 0; i < nA; ++i) {
+        const int s = i % kStages;
+        const bool ok = mbar_wait(&full[s], (i / kStages) & 1, abort_flag, &g_tc_error, kErrWait);
+        if (bar_any(kBarMath, kMath, !ok || *abort_flag)) {
+          alive = false;
+          break;
         }
-        st_shared_v4(addr, u);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&q_ready[s]);
-
-      // epilogue: O = num / den, written over the tile in shared memory (the
-      // MMA has finished reading it), stored with TMA
-      const int a = wg;
-      ok = mbar_wait(&t_full[a], (i / kApWG) & 1, abort_flag, &g_tc_error, kErrWait);
-      tc_fence_after();
-      if (bar_any(1 + wg, 128, !ok || *abort_flag)) break;
+        const uint32_t kb = sbase + Smem::stages + s * kStageBytes + box * kRedBox;
+        const int y0 = n_begin + i * kRedT;
 #pragma unroll
-      for (int hh = 0; hh < kGroupHeads; ++hh) {
-        float v[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + a * 128 + hh * 32,
-                           v);
-        const float inv = 1.0f / (den[hh] + p.eps);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < kRedT / 32; ++k) {
+          const int r = rg + 32 * k;
+          const uint32_t addr = kb + sw128_offset(r, cc);
+          uint4 u = ld_shared_v4(addr);
+          u.x = relu_bf16x2(u.x);
+          u.y = relu_bf16x2(u.y);
+          u.z = relu_bf16x2(u.z);
+          u.w = relu_bf16x2(u.w);
           float x[8];
+          unpack8(u, x);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = v[8 * k + e] * inv;
-          st_shared_v4(st + (hh >> 1) * kApBox + sw128_offset(row, (hh & 1) * 4 + k), pack8(x));
+          for (int e = 0; e < 4; ++e)
+            zacc[e] = __fadd2_rn(zacc[e], make_float2(x[2 * e], x[2 * e + 1]));
+          if (kRope != kNoRope) {
+            if (y0 + r < p.N) {
+              const RopeBases rb = rope_bases(p.rope, tp);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                float2 cs;
+                if (kRope == kRopeTable) {
+                  cs = rope_tab[(sel[q] == 0 ? rb.t : (sel[q] == 1 ? rb.h : rb.w)) + off[q]];
+                } else {
+                  const int pos = sel[q] == 0 ? p.rope.t_offset + tp.t : (sel[q] == 1 ? tp.h : tp.w);
+                  rope_cos_sin(pos, p.rope.inv_freq[j0 + q], cs.x, cs.y);
+                }
+                const float2 t = __fmul2_rn(make_float2(x[2 * q + 1], x[2 * q + 1]),
+                                            make_float2(-cs.y, cs.x));
+                const float2 y = __ffma2_rn(make_float2(x[2 * q], x[2 * q]), cs, t);
+                x[2 * q] = y.x;
+                x[2 * q + 1] = y.y;
+              }
+              u = pack8(x);
+            }
+            token_pos_advance(p.rope, tp, 32);
+          }
+          st_shared_v4(addr, u);
         }
+        fence_proxy_async_smem();
+        named_bar_sync(kBarMath, kMath);
+        if (mt == 0) mbar_arrive(&ready[s]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        zred[mt * 8 + 2 * e] = zacc[e].x;
+        zred[mt * 8 + 2 * e + 1] = zacc[e].y;
+      }
+      named_bar_sync(kBarMath, kMath);
+      // state of the four heads: the 32x32 diagonal blocks of the accumulator
+      if (warp >= 2 && warp < 6) {
+        const int q = warp & 3;  // TMEM lane quadrant = head in the group
+        float v[32];
+        bool got = alive && nA > 0 && mbar_wait(acc_full, 0, abort_flag, &g_tc_error, kErrWait);
+        got = __all_sync(0xffffffffu, got);  // tcgen05.ld is warp-collective
+        if (got) {
+          tc_fence_after();
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32 * q, v);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0.0f;
+        }
+        const int h = h0 + q;
+        if (h < p.H) {
+          float* dst = a.partials + ((cidx + q) * p.splits + blockIdx.x) * kStateFloats + lane * kD;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
+      }
+      if (mt < 128) {
+        // key sum of dim mt of the group: 32 row groups, in order
+        const int q = mt >> 5, d = mt & 31;
+        const int col = mt >> 3, e = mt & 7;  // chunk column and element holding this dim
+        float sum = 0.0f;
+        for (int r = 0; r < kMath / 16; ++r) sum += zred[(r * 16 + col) * 8 + e];
+        if (h0 + q < p.H)
+          a.partials[((cidx + q) * p.splits + blockIdx.x) * kStateFloats + kD * kD + d] = sum;
       }
       tc_fence_before();
-      mbar_arrive(&t_empty[a]);
-      fence_proxy_async_smem();
-      named_bar_sync(1 + wg, 128);
-      if (leader) {
-        uint8_t* tile = smem + ApSmem::stages + s * kApStageBytes;
-        tma_store_3d(&tm_o, tile, h0 * 32, n0, b);
-        tma_store_3d(&tm_o, tile + kApBox, h0 * 32 + 64, n0, b);
-        bulk_commit();
-        bulk_wait_read<0>();      // the store has read the stage
-        mbar_arrive(&q_empty[s]);  // hand the stage back to the producer
+    }
+
+    if (kRed) {
+      // ---- second phase of the reduce: the head group's CTA that arrives
+      // last sums every split's partial in split order (+ carry) and writes
+      // the state. The named barrier orders each math thread's partial stores
+      // before the release fence of the arriving thread.
+      named_bar_sync(kBarMath, kMath);
+      if (mt == 0) {
+        fence_acq_rel_gpu();
+        const unsigned prev = atomicAdd(&a.arrive[cidx], 1u);
+        *last_flag = prev == gridDim.x - 1;
+        if (*last_flag) fence_acq_rel_gpu();
+      }
+      named_bar_sync(kBarMath, kMath);
+      const bool last = *last_flag != 0;
+      if (last && alive) combine_from_global(p, b, h0, mt, a.partials, a.out);
+      named_bar_sync(kBarMath, kMath);
+      if (kPh == kReduceOnly) {
+        if (mt == 0 && last) a.arrive[cidx] = 0u;  // ready for the next call
+      } else {
+        // fused layer: the other CTAs of the group wait for the last one's
+        // flag (the launch is cooperative: all CTAs are resident)
+        if (mt == 0) {
+          if (last) {
+            fence_acq_rel_gpu();
+            st_release_gpu(&a.ready[cidx], 1u);
+          } else {
+            spin_flag(&a.ready[cidx], abort_flag);
+          }
+        }
+        named_bar_sync(kBarMath, kMath);
+        if (*abort_flag) alive = false;
       }
     }
-    if (leader) bulk_wait<0>();
+
+    if (kApp && alive) {
+      // ---- the state of the four heads as the MMA's B operand: row e of head
+      // pair j holds S[h][0..31][e] of heads 2j and 2j+1 in bf16 (K-major,
+      // 128-byte swizzle); S goes through shared memory with 16-byte loads
+      float* sbuf = zred;  // [4][32][32] f32, free once the reduce is done
+      for (int idx = mt; idx < kGroupHeads * kD * kD / 4; idx += kMath) {
+        const int hh = idx >> 8, h = h0 + hh;
+        float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (h < p.H)
+          v = __ldcg(reinterpret_cast<const float4*>(a.S_in + (cidx + hh) * kD * kD) + (idx & 255));
+        *reinterpret_cast<float4*>(sbuf + idx * 4) = v;
+      }
+      if (mt < kGroupHeads * kD) {
+        const int h = h0 + mt / kD;
+        zs[mt] = h < p.H ? __ldcg(a.z_in + cidx * kD + mt) : 0.0f;
+      }
+      named_bar_sync(kBarMath, kMath);
+      {
+        const int idx = mt;  // 2 pairs x 32 rows x 8 chunks = 512 = kMath
+        const int j = idx >> 8, e = (idx >> 3) & 31, c = idx & 7;
+        const int hh = 2 * j + (c >> 2), d0 = (c & 3) * 8;
+        float x[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] = sbuf[hh * kD * kD + (d0 + k) * kD + e];
+        st_shared_v4(sbase + Smem::bop + j * 4096 + sw128_offset(e, c), pack8(x));
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(kBarMath, kMath);
+      if (mt == 0) mbar_arrive(b_ready);
+      if (kPh == kFusedLayer && mt == 0) {
+        // the state is read: the last CTA to leave resets the group's words
+        const unsigned prev = atomicAdd(&a.depart[cidx], 1u);
+        if (prev == gridDim.x - 1) {
+          a.arrive[cidx] = 0u;
+          a.ready[cidx] = 0u;
+          a.depart[cidx] = 0u;
+        }
+      }
+
+      // ---- apply: warpgroup wg owns tiles wg, wg + 4, ...; thread = token row
+      const int wg = (warp - 2) >> 2;
+      const int quad = warp & 3;
+      const int row = quad * 32 + lane;
+      const bool leader = (warp == 2 + 4 * wg) && lane == 0;
+      for (int j = wg; j < nB; j += kApWG) {
+        const int pos = nA + j;
+        const int s = pos % kStages;
+        bool ok = mbar_wait(&full[s], (pos / kStages) & 1, abort_flag, &g_tc_error, kErrWait);
+        if (bar_any(kBarWG0 + wg, 128, !ok || *abort_flag)) break;
+        const int n0 = (tile_begin + j) * kApT;
+        const int n = n0 + row;
+        float2 cs[16];
+        if (kRope != kNoRope) {
+          const TokPos tp = token_pos(p.rope, min(n, p.N - 1));
+          const RopeBases rb = rope_bases(p.rope, tp);
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int ax = pair_axis(jj);
+            if (kRope == kRopeTable) {
+              cs[jj] = rope_tab[(ax == 0 ? rb.t : (ax == 1 ? rb.h : rb.w)) + pair_off(jj)];
+            } else {
+              const int pp = ax == 0 ? p.rope.t_offset + tp.t : (ax == 1 ? tp.h : tp.w);
+              rope_cos_sin(pp, p.rope.inv_freq[jj], cs[jj].x, cs[jj].y);
+            }
+          }
+        }
+        float den[kGroupHeads] = {0.0f, 0.0f, 0.0f, 0.0f};
+        const uint32_t st = sbase + Smem::stages + s * kStageBytes;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int hh = c >> 2, d0 = (c & 3) * 8;
+          const uint32_t addr = st + (c >> 3) * kApBox + sw128_offset(row, c & 7);
+          uint4 u = ld_shared_v4(addr);
+          u.x = relu_bf16x2(u.x);
+          u.y = relu_bf16x2(u.y);
+          u.z = relu_bf16x2(u.z);
+          u.w = relu_bf16x2(u.w);
+          float x[8];
+          unpack8(u, x);
+          const float4 za = *reinterpret_cast<const float4*>(zs + hh * kD + d0);
+          const float4 zb = *reinterpret_cast<const float4*>(zs + hh * kD + d0 + 4);
+          den[hh] = fmaf(x[0], za.x, den[hh]);
+          den[hh] = fmaf(x[1], za.y, den[hh]);
+          den[hh] = fmaf(x[2], za.z, den[hh]);
+          den[hh] = fmaf(x[3], za.w, den[hh]);
+          den[hh] = fmaf(x[4], zb.x, den[hh]);
+          den[hh] = fmaf(x[5], zb.y, den[hh]);
+          den[hh] = fmaf(x[6], zb.z, den[hh]);
+          den[hh] = fmaf(x[7], zb.w, den[hh]);
+          if (kRope != kNoRope) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float2 r = cs[d0 / 2 + q];
+              const float2 t = __fmul2_rn(make_float2(x[2 * q + 1], x[2 * q + 1]),
+                                          make_float2(-r.y, r.x));
+              const float2 y = __ffma2_rn(make_float2(x[2 * q], x[2 * q]), r, t);
+              x[2 * q] = y.x;
+              x[2 * q + 1] = y.y;
+            }
+            u = pack8(x);
+          }
+          st_shared_v4(addr, u);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(kBarWG0 + wg, 128);
+        if (leader) mbar_arrive(&ready[s]);
+
+        // epilogue: O = num / den over the tile in shared memory (the MMA has
+        // read it), stored with TMA; the stage returns once the store read it
+        ok = mbar_wait(&t_full[wg], (j / kApWG) & 1, abort_flag, &g_tc_error, kErrWait);
+        tc_fence_after();
+        if (bar_any(kBarWG0 + wg, 128, !ok || *abort_flag)) break;
+#pragma unroll
+        for (int hh = 0; hh < kGroupHeads; ++hh) {
+          float v[32];
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + wg * 128 + hh * 32,
+                             v);
+          const float inv = 1.0f / (den[hh] + p.eps);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = v[8 * k + e] * inv;
+            st_shared_v4(st + (hh >> 1) * kApBox + sw128_offset(row, (hh & 1) * 4 + k), pack8(x));
+          }
+        }
+        tc_fence_before();
+        fence_proxy_async_smem();
+        named_bar_sync(kBarWG0 + wg, 128);
+        if (leader) {
+          mbar_arrive(&t_empty[wg]);
+          uint8_t* tile = smem + Smem::stages + s * kStageBytes;
+          tma_store_3d(&tm_o, tile, h0 * 32, n0, b);
+          tma_store_3d(&tm_o, tile + kApBox, h0 * 32 + 64, n0, b);
+          bulk_commit();
+          bulk_wait_read<0>();      // the store has read the stage
+          mbar_arrive(&empty[s]);   // hand the stage back to the TMA warp
+        }
+      }
+      if (leader) bulk_wait<0>();
+    }
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kApTmemCols);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -803,7 +791,7 @@ RopeTable rope_table_for(const Problem& p) {
 }
 
 constexpr int kMaxDev = 64;
-bool g_attr_set[6][kMaxDev] = {};
+bool g_attr_set[9][kMaxDev] = {};
 std::mutex g_attr_mu;
 
 cudaError_t ensure_smem_attr(int which, const void* fn, int bytes) {
@@ -820,26 +808,69 @@ cudaError_t ensure_smem_attr(int which, const void* fn, int bytes) {
   return cudaSuccess;
 }
 
-}  // namespace
-
-// Launch with programmatic dependent launch: the kernel's prologue may
-// overlap the previous kernel in the stream; its pdl_wait() orders every
-// access to global memory after that kernel.
-template <typename... Params, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, int threads, int smem,
-                       cudaStream_t s, Args&&... args) {
+// Launch of layer_tc with programmatic dependent launch (the prologue may
+// overlap the previous kernel in the stream) and, for the fused layer, as a
+// cooperative launch (its CTAs wait on each other, so all must be resident).
+cudaError_t launch_layer(void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, Problem,
+                                      RopeTable, LayerArgs),
+                         dim3 grid, cudaStream_t s, bool cooperative, const CUtensorMap& mk,
+                         const CUtensorMap& mv, const CUtensorMap& mq, const CUtensorMap& mo,
+                         const Problem& p, const RopeTable& rt, const LayerArgs& a) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(threads, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.blockDim = dim3(kThreadsTc, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(kSmemBytes);
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  // A cooperative launch that the runtime refuses with the programmatic
+  // attribute is retried without it (the kernel's griddepcontrol
+  // instructions are then no-ops); the outcome is remembered.
+  static std::atomic<int> coop_pdl{1};
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    const bool pdl = !cooperative || coop_pdl.load() != 0;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (pdl) {
+      attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[n].val.programmaticStreamSerializationAllowed = 1;
+      ++n;
+    }
+    if (cooperative) {
+      attr[n].id = cudaLaunchAttributeCooperative;
+      attr[n].val.cooperative = 1;
+      ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mk, mv, mq, mo, p, rt, a);
+    if (e == cudaSuccess || !cooperative || !pdl || e == cudaErrorCooperativeLaunchTooLarge)
+      return e;
+    (void)cudaGetLastError();
+    coop_pdl.store(0);
+  }
+  return cudaErrorUnknown;
 }
+
+using LayerKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, Problem,
+                             RopeTable, LayerArgs);
+
+template <int kPh>
+LayerKernel pick_kernel(int mode) {
+  return mode == kNoRope ? layer_tc<kNoRope, kPh>
+                         : (mode == kRopeTable ? layer_tc<kRopeTable, kPh>
+                                               : layer_tc<kRopeOnTheFly, kPh>);
+}
+
+int rope_mode(const RopeTable& rt) {
+  return !rt.enabled ? kNoRope : (rt.on_the_fly ? kRopeOnTheFly : kRopeTable);
+}
+
+// 128-token tiles per CTA when `ctas` CTAs share a head group's tiles.
+int apply_tiles_per_cta(const Problem& p, int ctas) {
+  const int ntiles = (p.N + kApT - 1) / kApT;
+  return (ntiles + ctas - 1) / ctas;
+}
+
+}  // namespace
 
 cudaError_t launch_reduce_tc(const Problem& p, const void* K, const void* V, float* partials,
                              unsigned* counters, const StateOut& out, cudaStream_t s) {
@@ -848,16 +879,16 @@ cudaError_t launch_reduce_tc(const Problem& p, const void* K, const void* V, flo
   if ((e = make_map(&mk, K, p, kRedT)) != cudaSuccess) return e;
   if ((e = make_map(&mv, V, p, kRedT)) != cudaSuccess) return e;
   const RopeTable rt = rope_table_for(p);
-  const int mode = !rt.enabled ? kNoRope : (rt.on_the_fly ? kRopeOnTheFly : kRopeTable);
-  void (*kern)(CUtensorMap, CUtensorMap, Problem, RopeTable, float*, unsigned*, StateOut) =
-      mode == kNoRope ? reduce_tc<kNoRope>
-                      : (mode == kRopeTable ? reduce_tc<kRopeTable> : reduce_tc<kRopeOnTheFly>);
-  if ((e = ensure_smem_attr(mode, reinterpret_cast<const void*>(kern), kRedSmemBytes)) !=
-      cudaSuccess)
+  const int mode = rope_mode(rt);
+  LayerKernel kern = pick_kernel<kReduceOnly>(mode);
+  if ((e = ensure_smem_attr(mode, reinterpret_cast<const void*>(kern), kSmemBytes)) != cudaSuccess)
     return e;
+  LayerArgs a = {};
+  a.partials = partials;
+  a.arrive = counters;
+  a.out = out;
   const dim3 grid(p.splits, (p.H + kGroupHeads - 1) / kGroupHeads, p.B);
-  e = launch_pdl(kern, grid, kRedThreads, kRedSmemBytes, s, mk, mv, p, rt, partials, counters,
-                 out);
+  e = launch_layer(kern, grid, s, false, mk, mv, mk, mk, p, rt, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -868,29 +899,76 @@ cudaError_t launch_apply_tc(const Problem& p, const void* Q, const float* S, con
   cudaError_t e;
   if ((e = make_map(&mq, Q, p, kApT)) != cudaSuccess) return e;
   if ((e = make_map(&mo, O, p, kApT)) != cudaSuccess) return e;
+  const RopeTable rt = rope_table_for(p);
+  const int mode = rope_mode(rt);
+  LayerKernel kern = pick_kernel<kApplyOnly>(mode);
+  if ((e = ensure_smem_attr(3 + mode, reinterpret_cast<const void*>(kern), kSmemBytes)) !=
+      cudaSuccess)
+    return e;
   const int groups = (p.H + kGroupHeads - 1) / kGroupHeads;
   const int ntiles = (p.N + kApT - 1) / kApT;
   const long long units = static_cast<long long>(groups) * p.B;
-  int ctas_per_unit =
-      static_cast<int>(std::max<long long>(1, kNumSMs / std::max<long long>(1, units)));
-  ctas_per_unit = std::min(ctas_per_unit, ntiles);
-  const int tiles_per_cta = (ntiles + ctas_per_unit - 1) / ctas_per_unit;
-  ctas_per_unit = (ntiles + tiles_per_cta - 1) / tiles_per_cta;
-  const RopeTable rt = rope_table_for(p);
-  const int mode = !rt.enabled ? kNoRope : (rt.on_the_fly ? kRopeOnTheFly : kRopeTable);
-  void (*kern)(CUtensorMap, CUtensorMap, Problem, RopeTable, const float*, const float*, int,
-               int) = mode == kNoRope ? apply_tc<kNoRope>
-                                      : (mode == kRopeTable ? apply_tc<kRopeTable>
-                                                            : apply_tc<kRopeOnTheFly>);
-  if ((e = ensure_smem_attr(3 + mode, reinterpret_cast<const void*>(kern), kApSmemBytes)) !=
-      cudaSuccess)
-    return e;
-  const dim3 grid(ctas_per_unit, groups, p.B);
+  int ctas = static_cast<int>(std::max<long long>(1, kNumSMs / std::max<long long>(1, units)));
+  ctas = std::min(ctas, ntiles);
+  const int tpc = apply_tiles_per_cta(p, ctas);
+  ctas = (ntiles + tpc - 1) / tpc;
+  LayerArgs a = {};
+  a.S_in = S;
+  a.z_in = z;
+  a.tiles_per_cta = tpc;
   // Q may be read before the previous kernel completes only when that kernel
   // is this library's own state reduce, which does not write Q and itself
   // started reading only after everything before it had completed.
-  e = launch_pdl(kern, grid, kThreads, kApSmemBytes, s, mq, mo, p, rt, S, z, tiles_per_cta,
-                 after_own_reduce ? 1 : 0);
+  a.q_before_wait = after_own_reduce ? 1 : 0;
+  const dim3 grid(ctas, groups, p.B);
+  e = launch_layer(kern, grid, s, false, mq, mq, mq, mo, p, rt, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// The single-launch layer pays off where launch, ramp-up and the hand-off
+// between the two operations dominate: layers of up to 2^19 token-heads
+// (128 MiB of Q, K, V and O in bf16). Larger layers run as reduce + apply with
+// programmatic dependent launch, which measured faster there. Both paths give
+// bitwise identical results (same split order, same combine, same apply).
+constexpr long long kFuseMaxTokenHeads = 1LL << 19;
+
+bool layer_fusable(const Problem& p) {
+  const long long ctas =
+      static_cast<long long>(p.splits) * ((p.H + kGroupHeads - 1) / kGroupHeads) * p.B;
+  const long long token_heads = static_cast<long long>(p.B) * p.N * p.H;
+  return p.io == LA_IO_BF16 && p.N > 0 && ctas <= kNumSMs && token_heads <= kFuseMaxTokenHeads;
+}
+
+cudaError_t launch_layer_tc(const Problem& p, const void* Q, const void* K, const void* V,
+                            void* O, float* partials, unsigned* counters, const StateOut& out,
+                            cudaStream_t s) {
+  if (!layer_fusable(p) || out.out1_S == nullptr || out.out1_z == nullptr)
+    return cudaErrorNotSupported;
+  CUtensorMap mk, mv, mq, mo;
+  cudaError_t e;
+  if ((e = make_map(&mk, K, p, kRedT)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, V, p, kRedT)) != cudaSuccess) return e;
+  if ((e = make_map(&mq, Q, p, kApT)) != cudaSuccess) return e;
+  if ((e = make_map(&mo, O, p, kApT)) != cudaSuccess) return e;
+  const RopeTable rt = rope_table_for(p);
+  const int mode = rope_mode(rt);
+  LayerKernel kern = pick_kernel<kFusedLayer>(mode);
+  if ((e = ensure_smem_attr(6 + mode, reinterpret_cast<const void*>(kern), kSmemBytes)) !=
+      cudaSuccess)
+    return e;
+  const size_t bh = static_cast<size_t>(p.B) * p.H;
+  LayerArgs a = {};
+  a.partials = partials;
+  a.arrive = counters;
+  a.ready = counters + bh;
+  a.depart = counters + 2 * bh;
+  a.out = out;
+  a.S_in = out.out1_S;
+  a.z_in = out.out1_z;
+  a.tiles_per_cta = apply_tiles_per_cta(p, p.splits);
+  const dim3 grid(p.splits, (p.H + kGroupHeads - 1) / kGroupHeads, p.B);
+  e = launch_layer(kern, grid, s, true, mk, mv, mq, mo, p, rt, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -127,3 +127,32 @@ def test_stream_argument_is_honoured(cuda_device):
     s.synchronize()
     O_ref, S_ref, z_ref = P.gpu_attention(Q, K, V, eps)
     assert torch.equal(O.cpu(), O_ref) and torch.equal(S.cpu(), S_ref)
+
+
+def test_single_launch_layer_and_two_kernel_fallback(cuda_device):
+    """la_attention runs a small layer as one cooperative launch when one wave of
+    CTAs covers it, else as reduce + apply; both match the oracle and each
+    other bit for bit."""
+    assert la.la_attention_launches(la.make_shape(4, 1024, 70)) == 1
+    assert la.la_attention_launches(la.make_shape(1, 16384, 70)) == 2   # large: two kernels
+    assert la.la_attention_launches(la.make_shape(4, 1024, 70, io_dtype="f32")) == 2
+    # 80 batch elements x 2 head groups = 160 CTAs > one wave: two kernels
+    shape = la.make_shape(80, 200, 8)
+    assert la.la_attention_launches(shape) == 2
+    Q, K, V, th, eps = _case(80, 200, 8, 99)
+    _full_check(Q, K, V, th, eps, "bf16", what="two-kernel fallback")
+
+
+def test_fused_and_two_kernel_paths_are_bitwise_equal(cuda_device):
+    w = wl.WORKLOADS["sana1.6b_1024px"]
+    Q, K, V = P.to_dev(*wl.make_qkv(w, 17))
+    shape = la.shape_for(Q, eps=w.eps)
+    assert la.la_attention_launches(shape) == 1
+    O1, S1, z1 = la.attention(Q, K, V, eps=w.eps)          # single launch
+    S2 = torch.empty_like(S1)
+    z2 = torch.empty_like(z1)
+    O2 = torch.empty_like(O1)
+    la.la_state_reduce(shape, K, V, S2, z2, la.workspace(shape))
+    la.la_apply(shape, Q, S2, z2, O2)                       # two kernels
+    torch.cuda.synchronize()
+    assert torch.equal(S1, S2) and torch.equal(z1, z2) and torch.equal(O1, O2)
