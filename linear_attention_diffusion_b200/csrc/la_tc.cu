@@ -245,44 +245,64 @@ __device__ __forceinline__ bool spin_flag(const unsigned* flag, volatile int* ab
 }
 
 // Sum of the head group's split partials in split order (+ carry), written to
-// StateOut; by the math threads of the CTA that arrived last, from registers
-// (the stage ring may already hold prefetched tiles).
+// StateOut, by the math threads of the CTA that arrived last. Each thread owns
+// at most kPerThread float4 columns and issues the loads of all of them for 4
+// splits at once before adding, so the combine costs one L2 round trip per 4
+// splits.
 __device__ __forceinline__ void combine_from_global(const Problem& p, int b, int h0, int mt,
                                                     const float* partials, const StateOut& out) {
-  constexpr int kVec = kStateFloats / 4;
+  constexpr int kVec = kStateFloats / 4;                     // 264 float4 per head
+  constexpr int kPerThread = (kGroupHeads * kVec + kMath - 1) / kMath;  // 3
   const int heads = min(kGroupHeads, p.H - h0);
   const size_t cidx = static_cast<size_t>(b) * p.H + h0;
-  for (int v = mt; v < heads * kVec; v += kMath) {
+  float4 acc[kPerThread];
+  const float* src[kPerThread];
+  bool own[kPerThread];
+#pragma unroll
+  for (int u = 0; u < kPerThread; ++u) {
+    const int v = mt + u * kMath;
+    own[u] = v < heads * kVec;
+    const int hh = own[u] ? v / kVec : 0, i = own[u] ? (v - hh * kVec) * 4 : 0;
+    src[u] = partials + (cidx + hh) * p.splits * kStateFloats + i;
+    acc[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  }
+  for (int s0 = 0; s0 < p.splits; s0 += 4) {
+    float4 t[kPerThread][4];
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u)
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (own[u] && s0 + k < p.splits)
+          t[u][k] = __ldcg(reinterpret_cast<const float4*>(src[u] + static_cast<size_t>(s0 + k) * kStateFloats));
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u)
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (own[u] && s0 + k < p.splits) {
+          acc[u].x += t[u][k].x;
+          acc[u].y += t[u][k].y;
+          acc[u].z += t[u][k].z;
+          acc[u].w += t[u][k].w;
+        }
+  }
+#pragma unroll
+  for (int u = 0; u < kPerThread; ++u) {
+    if (!own[u]) continue;
+    const int v = mt + u * kMath;
     const int hh = v / kVec, i = (v - hh * kVec) * 4;
     const size_t bh = cidx + hh;
-    const float* src = partials + bh * p.splits * kStateFloats + i;
-    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    for (int s0 = 0; s0 < p.splits; s0 += 8) {
-      float4 t[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        if (s0 + k < p.splits)
-          t[k] = __ldcg(reinterpret_cast<const float4*>(src + static_cast<size_t>(s0 + k) * kStateFloats));
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        if (s0 + k < p.splits) {
-          acc.x += t[k].x;
-          acc.y += t[k].y;
-          acc.z += t[k].z;
-          acc.w += t[k].w;
-        }
-    }
     const bool is_s = i < kD * kD;
     const size_t o = is_s ? bh * kD * kD + i : bh * kD + (i - kD * kD);
     const float* c = is_s ? out.carry_S : out.carry_z;
+    float4 r = acc[u];
     if (c != nullptr) {
       const float4 cv = *reinterpret_cast<const float4*>(c + o);
-      acc = make_float4(cv.x + acc.x, cv.y + acc.y, cv.z + acc.z, cv.w + acc.w);
+      r = make_float4(cv.x + r.x, cv.y + r.y, cv.z + r.z, cv.w + r.w);
     }
     float* d1 = is_s ? out.out1_S : out.out1_z;
     float* d2 = is_s ? out.out2_S : out.out2_z;
-    if (d1 != nullptr) *reinterpret_cast<float4*>(d1 + o) = acc;
-    if (d2 != nullptr) *reinterpret_cast<float4*>(d2 + o) = acc;
+    if (d1 != nullptr) *reinterpret_cast<float4*>(d1 + o) = r;
+    if (d2 != nullptr) *reinterpret_cast<float4*>(d2 + o) = r;
   }
 }
 
