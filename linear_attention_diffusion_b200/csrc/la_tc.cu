@@ -210,8 +210,8 @@ struct Smem {  // byte offsets from the 1024-aligned base
   static constexpr int zs = bop + 2 * 32 * 128;                // [4][32] f32
   static constexpr int rope = zs + kGroupHeads * kD * 4;       // float2[kRopeTableMax]
   static constexpr int bars = rope + kRopeTableMax * 8;
-  // full[5] empty[5] ready[5] t_full[4] t_empty[4] acc_full mma_done b_ready
-  static constexpr int nbars = 3 * kStages + 2 * kApWG + 3;
+  // full[5] empty[5] ready_a[5] ready_b[5] t_full[4] t_empty[4] acc_full mma_done b_ready
+  static constexpr int nbars = 4 * kStages + 2 * kApWG + 3;
   static constexpr int misc = bars + nbars * 8;                // tmem base, abort, last flag
   static constexpr int bytes = misc + 16;
 };
@@ -318,8 +318,9 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Smem::bars);
   uint64_t* empty = full + kStages;
-  uint64_t* ready = empty + kStages;
-  uint64_t* t_full = ready + kStages;   // [kApWG]
+  uint64_t* ready_a = empty + kStages;  // reduce stage transformed: 512 arrivals
+  uint64_t* ready_b = ready_a + kStages; // apply tile transformed: 128 arrivals
+  uint64_t* t_full = ready_b + kStages;  // [kApWG]
   uint64_t* t_empty = t_full + kApWG;   // [kApWG]
   uint64_t* acc_full = t_empty + kApWG;
   uint64_t* mma_done = acc_full + 1;
@@ -348,7 +349,8 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&ready[s], 1);
+      mbar_init(&ready_a[s], kMath);
+      mbar_init(&ready_b[s], 128);
     }
     for (int w = 0; w < kApWG; ++w) {
       mbar_init(&t_full[w], 1);
@@ -431,7 +433,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       const uint32_t id_red = idesc_bf16_f32(128, 128, 1, 1);
       for (int i = 0; i < nA; ++i, ++pos) {
         const int s = pos % kStages;
-        if (!(ok = mbar_wait(&ready[s], (pos / kStages) & 1, abort_flag, &g_tc_error, kErrWait)))
+        if (!(ok = mbar_wait(&ready_a[s], (i / kStages) & 1, abort_flag, &g_tc_error, kErrWait)))
           break;
         tc_fence_after();
         const uint32_t st = sbase + Smem::stages + s * kStageBytes;
@@ -451,7 +453,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       for (int j = 0; ok && j < nB; ++j, ++pos) {
         const int s = pos % kStages;
         const int w = j % kApWG;
-        if (!(ok = mbar_wait(&ready[s], (pos / kStages) & 1, abort_flag, &g_tc_error, kErrWait)))
+        if (!(ok = mbar_wait(&ready_b[s], (j / kStages) & 1, abort_flag, &g_tc_error, kErrWait)))
           break;
         if (!(ok = mbar_wait(&t_empty[w], ((j / kApWG) & 1) ^ 1, abort_flag, &g_tc_error,
                              kErrWait)))
@@ -495,8 +497,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       }
       for (int i = 0; i < nA; ++i) {
         const int s = i % kStages;
-        const bool ok = mbar_wait(&full[s], (i / kStages) & 1, abort_flag, &g_tc_error, kErrWait);
-        if (bar_any(kBarMath, kMath, !ok || *abort_flag)) {
+        if (!mbar_wait(&full[s], (i / kStages) & 1, abort_flag, &g_tc_error, kErrWait)) {
           alive = false;
           break;
         }
@@ -541,15 +542,14 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
           st_shared_v4(addr, u);
         }
         fence_proxy_async_smem();
-        named_bar_sync(kBarMath, kMath);
-        if (mt == 0) mbar_arrive(&ready[s]);
+        mbar_arrive(&ready_a[s]);
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         zred[mt * 8 + 2 * e] = zacc[e].x;
         zred[mt * 8 + 2 * e + 1] = zacc[e].y;
       }
-      named_bar_sync(kBarMath, kMath);
+      alive = !bar_any(kBarMath, kMath, !alive || *abort_flag);
       // state of the four heads: the 32x32 diagonal blocks of the accumulator
       if (warp >= 2 && warp < 6) {
         const int q = warp & 3;  // TMEM lane quadrant = head in the group
@@ -721,8 +721,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
           st_shared_v4(addr, u);
         }
         fence_proxy_async_smem();
-        named_bar_sync(kBarWG0 + wg, 128);
-        if (leader) mbar_arrive(&ready[s]);
+        mbar_arrive(&ready_b[s]);
 
         // epilogue: O = num / den over the tile in shared memory (the MMA has
         // read it), stored with TMA; the stage returns once the store read it
