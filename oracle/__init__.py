@@ -24,4 +24,6 @@ from .linear_attention import (  # noqa: F401
     block_causal_bruteforce,
     apply_rows,
     to_f64,
+    rope_unrotate,
+    backward,
 )

@@ -24,6 +24,9 @@ Sources (page title, then section):
         denoising steps against it, and after the last step the block's own
         state is folded in once.
 [SVS2]  same page, "Stage 2": 3D RoPE over time, height and width.
+[SI]    "Sana: Efficient High-Resolution Image Synthesis with Linear Diffusion
+        Transformers", section "Infra": the linear attention has a fused
+        forward and backward (the backward pass below is its gradient).
 [MJ]    SANA-Video article (mjgaz.cn), section "设计细节": later blocks integrate
         earlier blocks' features through the linear state, earlier blocks never
         see later ones, and each block sums the accumulated KV with its own.
@@ -227,3 +230,42 @@ def block_causal_bruteforce(blocks: List[dict], eps: float) -> List[List[np.ndar
         past_v.append(to_f64(Vu))
         past_th.append(thu)
     return outs
+
+
+def rope_unrotate(x: np.ndarray, theta: np.ndarray) -> np.ndarray:
+    """The inverse (transpose) of rope_rotate: rotate the pairs by -theta."""
+    return rope_rotate(x, -theta)
+
+
+def backward(Q, K, V, dO, eps: float, theta: Optional[np.ndarray] = None):
+    """Gradient of the non-causal layer O = attention(Q, K, V) [SI], by hand.
+
+    With den_i = ReLU(q_i).z + eps, num_i = phi(q_i) S, O_i = num_i / den_i:
+      dnum_i = dO_i / den_i,  dden_i = -(dO_i . O_i) / den_i
+      dS = sum_i phi(q_i)^T dnum_i,   dz = sum_i dden_i ReLU(q_i)
+      dq_i = [R_i^T (dnum_i S^T) + dden_i z] * [q_i > 0]
+      dk_j = [R_j^T (dS v_j) + dz] * [k_j > 0],   dv_j = phi(k_j) dS
+    (R = the RoPE rotation, identity without RoPE; the ReLU derivative is 0 at
+    0.) Returns dQ, dK, dV [B, N, H, D] and dS [B, H, D, D], dz [B, H, D].
+    """
+    Q, K, V, dO = to_f64(Q), to_f64(K), to_f64(V), to_f64(dO)
+    qp, kp = relu(Q), relu(K)
+    phq = qp if theta is None else rope_rotate(qp, theta)
+    phk = kp if theta is None else rope_rotate(kp, theta)
+    S = np.matmul(phk.transpose(0, 2, 3, 1), V.transpose(0, 2, 1, 3))      # [B,H,D,E]
+    z = kp.sum(axis=1)                                                      # [B,H,D]
+    den = np.einsum("bnhd,bhd->bnh", qp, z) + float(eps)                    # [B,N,H]
+    num = np.einsum("bnhd,bhde->bnhe", phq, S)
+    O = num / den[..., None]
+    dnum = dO / den[..., None]
+    dden = -np.einsum("bnhe,bnhe->bnh", dO, O) / den
+    dS = np.einsum("bnhd,bnhe->bhde", phq, dnum)
+    dz = np.einsum("bnh,bnhd->bhd", dden, qp)
+    dphq = np.einsum("bnhe,bhde->bnhd", dnum, S)
+    dqp = (dphq if theta is None else rope_unrotate(dphq, theta)) + dden[..., None] * z[:, None]
+    dQ = dqp * (Q > 0)
+    dphk = np.einsum("bhde,bnhe->bnhd", dS, V)
+    dkp = (dphk if theta is None else rope_unrotate(dphk, theta)) + dz[:, None]
+    dK = dkp * (K > 0)
+    dV = np.einsum("bnhd,bhde->bnhe", phk, dS)
+    return dQ, dK, dV, dS, dz

@@ -294,3 +294,77 @@ def test_single_block_is_noncausal_and_update1_matches():
     S_own, z_own = orc.state_reduce(K, V)
     np.testing.assert_array_equal(S1, S_own)
     np.testing.assert_array_equal(z1, z_own)
+
+
+# --------------------------------------------------------------------------
+# Backward pass: pinned to central finite differences of the quadratic form
+
+
+def _fd_grad(f, X, h=1e-6):
+    g = np.zeros_like(X)
+    it = np.nditer(X, flags=["multi_index"])
+    for _ in it:
+        idx = it.multi_index
+        Xp = X.copy()
+        Xm = X.copy()
+        Xp[idx] += h
+        Xm[idx] -= h
+        g[idx] = (f(Xp) - f(Xm)) / (2 * h)
+    return g
+
+
+def _away_from_kinks(X, margin=0.05):
+    # keep every entry at least `margin` away from 0 so ReLU is smooth there
+    return np.where(np.abs(X) < margin, np.sign(X + 1e-12) * margin, X)
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_backward_matches_finite_differences_of_the_quadratic_form(rope):
+    T, Hh, W = 2, 2, 3
+    N, H = T * Hh * W, 2
+    Q, K, V = (_away_from_kinks(x) for x in _qkv(1, N, H, 300))
+    G = _rand(V.shape, 304)          # dL/dO for L = sum(O * G)
+    eps = 0.1
+    th = orc.rope_angles(T, Hh, W, 3) if rope else None
+
+    def loss_q(Qx):
+        return float((orc.attention_bruteforce(Qx, K, V, eps, th, th) * G).sum())
+
+    def loss_k(Kx):
+        return float((orc.attention_bruteforce(Q, Kx, V, eps, th, th) * G).sum())
+
+    def loss_v(Vx):
+        return float((orc.attention_bruteforce(Q, K, Vx, eps, th, th) * G).sum())
+
+    dQ, dK, dV, _, _ = orc.backward(Q, K, V, G, eps, th)
+    np.testing.assert_allclose(dQ, _fd_grad(loss_q, Q), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dK, _fd_grad(loss_k, K), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dV, _fd_grad(loss_v, V), rtol=1e-6, atol=1e-8)
+
+
+def test_backward_state_gradients_are_the_chain_rule_through_S_and_z():
+    # dS and dz: perturbing S (or z) directly in the apply changes the loss by
+    # <dS, dS_pert> (resp. <dz, dz_pert>) to first order.
+    Q, K, V = _qkv(1, 20, 2, 310)
+    G = _rand(V.shape, 311)
+    eps = 0.05
+    S, z = orc.state_reduce(K, V)
+    _, _, _, dS, dz = orc.backward(Q, K, V, G, eps)
+    P = _rand(S.shape, 312)
+    h = 1e-6
+    lp = (orc.apply(Q, S + h * P, z, eps) * G).sum()
+    lm = (orc.apply(Q, S - h * P, z, eps) * G).sum()
+    np.testing.assert_allclose((lp - lm) / (2 * h), (dS * P).sum(), rtol=1e-6)
+    Pz = np.abs(_rand(z.shape, 313))
+    lp = (orc.apply(Q, S, z + h * Pz, eps) * G).sum()
+    lm = (orc.apply(Q, S, z - h * Pz, eps) * G).sum()
+    np.testing.assert_allclose((lp - lm) / (2 * h), (dz * Pz).sum(), rtol=1e-6)
+
+
+def test_backward_negative_inputs_get_zero_gradient():
+    Q, K, V = _qkv(1, 16, 1, 320)
+    Q[0, :4] = -np.abs(Q[0, :4])
+    K[0, :4] = -np.abs(K[0, :4])
+    dQ, dK, dV, _, _ = orc.backward(Q, K, V, _rand(V.shape, 321), 1e-3)
+    assert np.all(dQ[0, :4] == 0) and np.all(dK[0, :4] == 0)
+    assert np.all(dV[0, :4] == 0)  # an all-negative key carries no value
