@@ -252,20 +252,26 @@ def backward(Q, K, V, dO, eps: float, theta: Optional[np.ndarray] = None):
     qp, kp = relu(Q), relu(K)
     phq = qp if theta is None else rope_rotate(qp, theta)
     phk = kp if theta is None else rope_rotate(kp, theta)
-    S = np.matmul(phk.transpose(0, 2, 3, 1), V.transpose(0, 2, 1, 3))      # [B,H,D,E]
-    z = kp.sum(axis=1)                                                      # [B,H,D]
-    den = np.einsum("bnhd,bhd->bnh", qp, z) + float(eps)                    # [B,N,H]
-    num = np.einsum("bnhd,bhde->bnhe", phq, S)
-    O = num / den[..., None]
+
+    def heads(x):  # [B, N, H, D] -> [B, H, N, D], for batched matmuls
+        return x.transpose(0, 2, 1, 3)
+
+    def tokens(x):  # [B, H, N, D] -> [B, N, H, D]
+        return x.transpose(0, 2, 1, 3)
+
+    S = np.matmul(heads(phk).transpose(0, 1, 3, 2), heads(V))            # [B,H,D,E]
+    z = kp.sum(axis=1)                                                    # [B,H,D]
+    den = np.einsum("bnhd,bhd->bnh", qp, z) + float(eps)                  # [B,N,H]
+    O = tokens(np.matmul(heads(phq), S)) / den[..., None]
     dnum = dO / den[..., None]
     dden = -np.einsum("bnhe,bnhe->bnh", dO, O) / den
-    dS = np.einsum("bnhd,bnhe->bhde", phq, dnum)
+    dS = np.matmul(heads(phq).transpose(0, 1, 3, 2), heads(dnum))         # sum_n phq^T dnum
     dz = np.einsum("bnh,bnhd->bhd", dden, qp)
-    dphq = np.einsum("bnhe,bhde->bnhd", dnum, S)
+    dphq = tokens(np.matmul(heads(dnum), S.transpose(0, 1, 3, 2)))        # dnum S^T
     dqp = (dphq if theta is None else rope_unrotate(dphq, theta)) + dden[..., None] * z[:, None]
     dQ = dqp * (Q > 0)
-    dphk = np.einsum("bhde,bnhe->bnhd", dS, V)
+    dphk = tokens(np.matmul(heads(V), dS.transpose(0, 1, 3, 2)))          # (dS v^T)^T
     dkp = (dphk if theta is None else rope_unrotate(dphk, theta)) + dz[:, None]
     dK = dkp * (K > 0)
-    dV = np.einsum("bnhd,bhde->bnhe", phk, dS)
+    dV = tokens(np.matmul(heads(phk), dS))                                # phk dS
     return dQ, dK, dV, dS, dz
