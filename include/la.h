@@ -147,6 +147,32 @@ la_status la_block_causal_step(const la_shape* shape, const void* Q,
                                float* z_carry, void* O, int update, void* ws,
                                size_t ws_bytes, la_stream stream);
 
+/* Backward of la_attention, for training (Sana, section Infra: the linear
+ * attention is trained with a fused forward and backward kernel). Given the
+ * forward's inputs, its state (S, z) and the output gradient dO, with
+ * den_n = ReLU(q_n) . z + eps:
+ *   dnum_n = dO_n / den_n,  dden_n = -(dO_n . O_n) / den_n,
+ *   dS = sum_n phi(q_n)^T dnum_n,  dz = sum_n dden_n ReLU(q_n),
+ *   dq_n = [R_n^T (S dnum_n^T) + dden_n z] * [q_n > 0],
+ *   dk_n = [R_n^T (dS v_n^T) + dz] * [k_n > 0],  dv_n = phi(k_n) dS,
+ * R_n the token's RoPE rotation (identity when shape->rope == 0), [x > 0]
+ * taken elementwise (the gradient of ReLU at 0 is taken as 0).
+ * Q, K, V, dO: [B,N,H,D] io_dtype (device, read). S [B,H,D,D], z [B,H,D]
+ * float32 (device, read): the state the forward produced; both NULL makes the
+ * call reduce it again from (K, V) into the workspace first. dQ, dK, dV:
+ * [B,N,H,D] io_dtype (device, written; bf16 rounded to nearest-even).
+ * dS [B,H,D,D], dz [B,H,D] float32 (device, written): the gradients of the
+ * state. O is not an input: dO_n . O_n = phi(q_n) . (S dnum_n^T) / den_n.
+ * ws: as for la_attention (same size). Two launches (three when the state is
+ * recomputed); dS and dz are summed over the same shape-only token splits
+ * as the state reduce, so results are bitwise reproducible.
+ * None of the outputs may overlap each other, an input or the workspace. */
+la_status la_attention_backward(const la_shape* shape, const void* Q,
+                                const void* K, const void* V, const float* S,
+                                const float* z, const void* dO, void* dQ,
+                                void* dK, void* dV, float* dS, float* dz,
+                                void* ws, size_t ws_bytes, la_stream stream);
+
 /* Reset of the KV cache at the start of a video (SANA-Video section 4: the
  * cache starts empty): S[B,H,D,D] = 0, z[B,H,D] = 0 on `stream`. */
 la_status la_state_reset(float* S, float* z, int B, int H, int D,

@@ -67,6 +67,8 @@ _lib.la_attention.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, 
 _lib.la_attention.restype = _i
 _lib.la_block_causal_step.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]
 _lib.la_block_causal_step.restype = _i
+_lib.la_attention_backward.argtypes = [_shape_p] + [_vp] * 11 + [_vp, _sz, _vp]
+_lib.la_attention_backward.restype = _i
 _lib.la_state_reset.argtypes = [_vp, _vp, _i, _i, _i, _vp]
 _lib.la_state_reset.restype = _i
 _lib.la_status_string.argtypes = [_i]
@@ -152,6 +154,15 @@ def la_block_causal_step(shape: LaShape, Q, K, V, S_carry, z_carry, O, update: i
            "la_block_causal_step")
 
 
+def la_attention_backward(shape: LaShape, Q, K, V, S, z, dO, dQ, dK, dV, dS, dz, ws,
+                          stream=None) -> None:
+    """Gradients of la_attention; S and z None makes the call reduce the state again."""
+    _check(_lib.la_attention_backward(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(S),
+                                      _ptr(z), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dS),
+                                      _ptr(dz), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "la_attention_backward")
+
+
 def la_state_reset(S, z, B: int, H: int, D: int = HEAD_DIM, stream=None) -> None:
     _check(_lib.la_state_reset(_ptr(S), _ptr(z), int(B), int(H), int(D), _stream(stream)),
            "la_state_reset")
@@ -212,3 +223,17 @@ def attention(Q, K, V, eps: float = 1e-6, rope_grid=None, t_offset: int = 0,
     O = torch.empty_like(Q)
     la_attention(shape, Q, K, V, S, z, O, workspace(shape, Q.device), stream)
     return O, S, z
+
+
+def attention_backward(Q, K, V, dO, S=None, z=None, eps: float = 1e-6, rope_grid=None,
+                       t_offset: int = 0, rope_base: float = 10000.0, stream=None):
+    """dQ, dK, dV, dS, dz of non-causal ReLU linear attention for [B, N, H, 32] CUDA tensors."""
+    import torch
+    shape = shape_for(Q, eps, rope_grid, t_offset, rope_base)
+    B, N, H, D = Q.shape
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    dS = torch.empty((B, H, D, D), dtype=torch.float32, device=Q.device)
+    dz = torch.empty((B, H, D), dtype=torch.float32, device=Q.device)
+    la_attention_backward(shape, Q, K, V, S, z, dO, dQ, dK, dV, dS, dz,
+                          workspace(shape, Q.device), stream)
+    return dQ, dK, dV, dS, dz

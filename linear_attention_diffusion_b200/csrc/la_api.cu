@@ -317,6 +317,66 @@ la_status la_block_causal_step(const la_shape* shape, const void* Q, const void*
   return LA_OK;
 }
 
+la_status la_attention_backward(const la_shape* shape, const void* Q, const void* K,
+                                const void* V, const float* S, const float* z, const void* dO,
+                                void* dQ, void* dK, void* dV, float* dS, float* dz, void* ws,
+                                size_t ws_bytes, la_stream stream) {
+  Problem p;
+  LA_TRY(make_problem(shape, p));
+  const bool any_state = p.B > 0 && p.H > 0;
+  const bool any_input = any_state && p.N > 0;
+  if ((S == nullptr) != (z == nullptr))
+    return fail(LA_ERR_INVALID_ARG, "S and z must both be given or both be NULL");
+  const bool recompute = S == nullptr;
+  LA_TRY(check_ptr(Q, "Q", any_input));
+  LA_TRY(check_ptr(K, "K", any_input));
+  LA_TRY(check_ptr(V, "V", any_input));
+  LA_TRY(check_ptr(dO, "dO", any_input));
+  LA_TRY(check_ptr(S, "S", any_state && !recompute));
+  LA_TRY(check_ptr(z, "z", any_state && !recompute));
+  LA_TRY(check_ptr(dQ, "dQ", any_input));
+  LA_TRY(check_ptr(dK, "dK", any_input));
+  LA_TRY(check_ptr(dV, "dV", any_input));
+  LA_TRY(check_ptr(dS, "dS", any_state));
+  LA_TRY(check_ptr(dz, "dz", any_state));
+  LA_TRY(check_ws(p, ws, ws_bytes));
+  const size_t nb = io_bytes(p), sb = s_bytes(p), zb = z_bytes(p);
+  const void* outs[5] = {dQ, dK, dV, dS, dz};
+  const size_t out_n[5] = {nb, nb, nb, sb, zb};
+  const void* ins[7] = {Q, K, V, dO, S, z, ws};
+  const size_t in_n[7] = {nb, nb, nb, nb, sb, zb, ws_bytes};
+  for (int i = 0; i < 5; ++i) {
+    for (int j = i + 1; j < 5; ++j)
+      if (overlap(outs[i], out_n[i], outs[j], out_n[j]))
+        return fail(LA_ERR_INVALID_ARG, "the gradients must not overlap each other");
+    for (int j = 0; j < 7; ++j)
+      if (overlap(outs[i], out_n[i], ins[j], in_n[j]))
+        return fail(LA_ERR_INVALID_ARG, "a gradient overlaps an input or the workspace");
+  }
+  if (!recompute && (overlap(S, sb, ws, ws_bytes) || overlap(z, zb, ws, ws_bytes)))
+    return fail(LA_ERR_INVALID_ARG, "S and z must not overlap the workspace");
+  if (!any_state) return LA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const WsLayout L = workspace_layout(p);
+  float* partials = reinterpret_cast<float*>(w + L.partials);
+  unsigned* counters = reinterpret_cast<unsigned*>(w + L.counters);
+  if (recompute) {
+    float* Sw = reinterpret_cast<float*>(w + L.state_S);
+    float* zw = reinterpret_cast<float*>(w + L.state_z);
+    LA_TRY(run_reduce(p, K, V, w, StateOut{nullptr, nullptr, Sw, zw, nullptr, nullptr}, st));
+    S = Sw;
+    z = zw;
+  }
+  const StateOut grads = {nullptr, nullptr, dS, dz, nullptr, nullptr};
+  cudaError_t e = launch_backward_q(p, Q, dO, S, z, dQ, partials, counters, grads, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward (query side)");
+  if (!any_input) return LA_OK;
+  e = launch_backward_kv(p, K, V, dS, dz, dK, dV, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward (key side)");
+  return LA_OK;
+}
+
 la_status la_state_reset(float* S, float* z, int B, int H, int D, la_stream stream) {
   if (B < 0 || H < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d", B, H);
   if (D != kD) return fail(LA_ERR_UNSUPPORTED, "head width D=%d (only 32 is built)", D);

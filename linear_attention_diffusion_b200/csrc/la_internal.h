@@ -83,6 +83,15 @@ bool layer_fusable(const Problem& p);
 cudaError_t launch_layer_tc(const Problem& p, const void* Q, const void* K, const void* V,
                             void* O, float* partials, unsigned* counters, const StateOut& out,
                             cudaStream_t s);
+// Backward of the non-causal layer (la_backward.cu). Query side: dQ, and the
+// state gradients reduced over the token splits into `out` (same partials,
+// counters and split order as the state reduce). Key side: dK and dV from
+// the combined dS, dz.
+cudaError_t launch_backward_q(const Problem& p, const void* Q, const void* dO, const float* S,
+                              const float* z, void* dQ, float* partials, unsigned* counters,
+                              const StateOut& out, cudaStream_t s);
+cudaError_t launch_backward_kv(const Problem& p, const void* K, const void* V, const float* dS,
+                               const float* dz, void* dK, void* dV, cudaStream_t s);
 // Device error word of the tensor-core kernels (bounded waits that gave up).
 cudaError_t read_device_error(unsigned* code, bool reset);
 

@@ -103,3 +103,67 @@ def tolerances(io, rope):
     if io == "bf16":
         return 2e-5, 2.0 ** -7
     return 2e-5, 2e-5
+
+
+# ---------------------------------------------------------------------------
+# Backward pass.
+#
+# The GPU is given the oracle's (S, z) rounded to float32, so the comparison
+# isolates the backward kernels. Their arithmetic is float32 sums of products
+# whose magnitudes are written out below with absolute values (M_*); each
+# gradient must satisfy
+#     |g_gpu - g_ref| <= out_round * |g_ref| + tol_b * M
+# with out_round the output rounding (2^-8 for bf16 gradients, 1e-6 for
+# float32, 0 for dS/dz which are float32 sums) and tol_b = 1e-4 (the longest
+# float32 running sum is a few thousand terms per thread, well inside it).
+# Elements whose ReLU input is <= 0 must be exactly zero in dQ and dK.
+
+TOL_B = 1e-4
+
+
+def _pair_sum(x):
+    """|R^T y|_d <= |y_d| + |y_{d xor 1}| for a rotation R of the pairs (2i, 2i+1)."""
+    y = x.copy()
+    y[..., 0::2] += x[..., 1::2]
+    y[..., 1::2] += x[..., 0::2]
+    return y
+
+
+def backward_magnitudes(Q, K, V, dO, eps, theta, S, z):
+    """Magnitudes M of every term of each gradient (float64, same shapes)."""
+    qf, kf, vf, gf = (orc.to_f64(x) for x in (Q, K, V, dO))
+    qp, kp = orc.relu(qf), orc.relu(kf)
+    phq = np.abs(orc.feature_map(qf, theta))
+    phk = np.abs(orc.feature_map(kf, theta))
+    den = np.einsum("bnhd,bhd->bnh", qp, z) + eps
+    adnum = np.abs(gf) / den[..., None]
+    heads = lambda x: x.transpose(0, 2, 1, 3)
+    aS = np.abs(S)
+    Mt = heads(np.matmul(heads(adnum), aS.transpose(0, 1, 3, 2)))          # |S| |dnum|
+    Mdden = np.einsum("bnhd,bnhd->bnh", phq, Mt) / den                      # >= |dden|
+    M_dS = np.matmul(heads(phq).transpose(0, 1, 3, 2), heads(adnum))
+    M_dz = np.einsum("bnh,bnhd->bhd", Mdden, qp)
+    rot = _pair_sum if theta is not None else (lambda x: x)
+    M_dQ = rot(Mt) + Mdden[..., None] * z[:, None]
+    M_dK = rot(heads(np.matmul(heads(np.abs(vf)), M_dS.transpose(0, 1, 3, 2)))) + M_dz[:, None]
+    M_dV = heads(np.matmul(heads(phk), M_dS))
+    return M_dQ, M_dK, M_dV, M_dS, M_dz
+
+
+def check_backward(got, ref, mags, io, Q, K, what=""):
+    """got/ref/mags: (dQ, dK, dV, dS, dz). Element by element, with the bound above."""
+    names = ("dQ", "dK", "dV", "dS", "dz")
+    out_round = 2.0 ** -8 if io == "bf16" else 1e-6
+    for i, (name, g, r, m) in enumerate(zip(names, got, ref, mags)):
+        g = orc.to_f64(g)
+        assert g.shape == r.shape, f"{what} {name}: shape {g.shape} != {r.shape}"
+        assert np.isfinite(g).all(), f"{what} {name}: non-finite values"
+        rr = out_round if i < 3 else 0.0
+        err = np.abs(g - r)
+        bound = rr * np.abs(r) + TOL_B * m + 1e-30
+        bad = err > bound
+        assert not bad.any(), (f"{what} {name}: {bad.sum()} of {bad.size} outside the derived "
+                               f"bound; worst ratio {float((err / bound).max()):.3g}")
+    for name, g, x in (("dQ", got[0], Q), ("dK", got[1], K)):
+        masked = orc.to_f64(x) <= 0
+        assert (orc.to_f64(g)[masked] == 0).all(), f"{what} {name}: non-zero where the input <= 0"
