@@ -2,12 +2,14 @@
 """Benchmark of one ReLU linear-attention layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl la|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--op layer|backward]
 
 A step is one pass of the layer's hot path over one batch of synthetic input:
 the state reduce (S = sum phi(K)^T V, z = sum ReLU(K)) and the apply
 (O = phi(Q) S / (ReLU(Q).z + eps)) of the default workload, or a whole
 block-causal video (reset, 12 blocks x 5 calls) for the LongSANA workload.
+With --op backward a step is the layer's backward instead (dQ, dK, dV and the
+state gradients from Q, K, V, the state and dO; non-causal workloads).
 Rank 0 prints one JSON line. Multi-GPU runs are weak-scaled: every rank runs
 its own copy of the workload (heads and batches are independent), with no
 collective on the data path; the time is the max over ranks.
@@ -38,6 +40,7 @@ if ROOT not in sys.path:
 import workloads as wl  # noqa: E402
 
 METRIC = "linear-attn tokens/s per layer at 1 B200; achieved HBM GB/s vs peak"
+METRIC_BWD = "linear-attn backward tokens/s per layer at 1 B200; achieved HBM GB/s vs peak"
 DEFAULT_WORKLOAD = "sana1.6b_1024px"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
@@ -81,7 +84,9 @@ def layer_bytes(w, io_bytes=2):
     """Algorithmic HBM bytes of one layer: read Q, K, V, write O, write the state."""
     th = w.B * w.N * w.H
     state = w.B * w.H * (D * D + D) * 4
-    return {"attention_layer": 4 * th * D * io_bytes + state}
+    # backward: read Q, K, V, dO and (S, z); write dQ, dK, dV and (dS, dz)
+    return {"attention_layer": 4 * th * D * io_bytes + state,
+            "attention_backward": 7 * th * D * io_bytes + 2 * state}
 
 
 def peaks():
@@ -190,7 +195,7 @@ def cpu_cores_used():
         return os.cpu_count() or 1
 
 
-def oracle_sample(w, seconds, max_reps=None):
+def oracle_sample(w, seconds, max_reps=None, op="layer"):
     """Time the float64 oracle on a bounded sample of workload `w`.
 
     One call covers a subset of heads sized so that it takes at most about
@@ -199,8 +204,12 @@ def oracle_sample(w, seconds, max_reps=None):
     import numpy as np
     import oracle as orc
 
+    dOa = wl.make_tensor((w.B, w.N, w.H, w.D), 3) if op == "backward" else None
+
     def run(h_sub, Q, K, V, th):
-        if w.block_causal:
+        if op == "backward":
+            orc.backward(Q, K, V, dOa[:, :, :h_sub], w.eps, th)
+        elif w.block_causal:
             Sc = np.zeros((w.B, h_sub, D, D))
             zc = np.zeros((w.B, h_sub, D))
             orc.block_causal_step(Q, K, V, Sc, zc, 1, w.eps, th)
@@ -231,7 +240,8 @@ def oracle_sample(w, seconds, max_reps=None):
                 f"{reps} calls in {el:.1f} s, scaled to {w.H} heads x {calls} calls per video")
     else:
         tokens_per_s = w.B * w.N / full_call
-        desc = (f"oracle attention on {h_sub} of {w.H} heads (B={w.B}, N={w.N}), {reps} calls "
+        what = "backward" if op == "backward" else "attention"
+        desc = (f"oracle {what} on {h_sub} of {w.H} heads (B={w.B}, N={w.N}), {reps} calls "
                 f"in {el:.1f} s, scaled to {w.H} heads")
     return tokens_per_s, desc, cpu_cores_used(), per_call, h_sub
 
@@ -253,7 +263,8 @@ def run_la(args, w, rank, world, local_rank):
     lib = la._lib
     sp = stream.cuda_stream
 
-    per_set = 3 * w.B * w.N * w.H * D * 2
+    bwd = args.op == "backward"
+    per_set = (4 if bwd else 3) * w.B * w.N * w.H * D * 2
     n_sets = max(1, min(8, math.ceil(2 * L2_BYTES / per_set)))
     if w.block_causal:
         n_sets = 5  # one set per call of a block; each set is far above L2
@@ -264,9 +275,20 @@ def run_la(args, w, rank, world, local_rank):
         else:
             q, k, v = wl.make_qkv(w, rank_seed(rank) + 10 * i)
         q, k, v = (x.to(dev) for x in (q, k, v))
-        sets.append((q, k, v, torch.empty_like(q)))
+        if bwd:
+            # the set's dO and its forward state (computed once, untimed)
+            g = wl.make_tensor(tuple(q.shape), rank_seed(rank) + 10 * i + 3).to(dev)
+            _, Si, zi = la.attention(q, k, v, eps=w.eps,
+                                     rope_grid=(w.T, w.Hh, w.W) if w.rope else None)
+            sets.append((q, k, v, g, Si, zi))
+        else:
+            sets.append((q, k, v, torch.empty_like(q)))
     S = torch.zeros((w.B, w.H, D, D), device=dev)
     z = torch.zeros((w.B, w.H, D), device=dev)
+    if bwd:
+        grads = [torch.empty_like(sets[0][0]) for _ in range(3)] + [torch.empty_like(S),
+                                                                    torch.empty_like(z)]
+        grad_p = [t.data_ptr() for t in grads]
 
     def shape_at(t_offset=0):
         return la.make_shape(w.B, w.N, w.H, D, "bf16", w.rope, w.T, w.Hh, w.W, t_offset,
@@ -281,7 +303,19 @@ def run_la(args, w, rank, world, local_rank):
     shapes = [ctypes.byref(s) for s in keep]
     status = []
 
-    if w.block_causal:
+    if bwd:
+        launches_per_step = 2  # query side, then key side
+
+        def step(i, evs=None):
+            q, k, v, g, Si, zi = ptrs[i % n_sets]
+            if evs is not None:
+                evs[0].record(stream)
+            status.append(lib.la_attention_backward(shapes[0], q, k, v, Si, zi, g, *grad_p,
+                                                    ws_p, ws_n, sp))
+            if evs is not None:
+                evs[1].record(stream)
+        kernel_names = ("attention_backward",)
+    elif w.block_causal:
         calls_per_step = w.M * (w.steps + 1)
         # one or two kernels per call (see la_attention_launches); reset is memsets
         launches_per_step = la.la_attention_launches(keep[0]) * calls_per_step
@@ -390,7 +424,12 @@ def run_la(args, w, rank, world, local_rank):
     ms_max = max_over_ranks(ms, dev)
 
     # end-to-end through the public API with host buffers
-    e2e = run_e2e(args, w, dev, stream, la, rank) if args.e2e_steps > 0 else None
+    if args.e2e_steps <= 0:
+        e2e = None
+    elif bwd:
+        e2e = run_e2e_backward(args, w, dev, stream, la, rank)
+    else:
+        e2e = run_e2e(args, w, dev, stream, la, rank)
     clocks = sampler.summary(t0, t1)
     sampler.stop()
     del g_chunk, g_rem, g_ev
@@ -454,6 +493,48 @@ def run_e2e(args, w, dev, stream, la, rank):
             "h2d_bytes_per_step": 3 * nb * passes, "d2h_bytes_per_step": nb * passes}
 
 
+def run_e2e_backward(args, w, dev, stream, la, rank):
+    """The backward through la_attention_backward with pinned host Q, K, V, dO
+    copied in and dQ, dK, dV copied out inside the timed region; the state is
+    reduced again inside the call (S = z = NULL), as a caller holding only
+    host tensors would do."""
+    import torch
+    steps = max(1, min(args.steps, args.e2e_steps))
+    q, k, v = wl.make_qkv(w, 1000 * rank + 7)
+    g = wl.make_tensor(tuple(q.shape), 1000 * rank + 10)
+    hin = [x.pin_memory() for x in (q, k, v, g)]
+    hout = [torch.empty_like(hin[0]).pin_memory() for _ in range(3)]
+    din = [torch.empty_like(x, device=dev) for x in hin]
+    dout = [torch.empty_like(x, device=dev) for x in hout]
+    dS = torch.empty((w.B, w.H, D, D), device=dev)
+    dz = torch.empty((w.B, w.H, D), device=dev)
+    shape = la.make_shape(w.B, w.N, w.H, D, "bf16", w.rope, w.T, w.Hh, w.W, 0, w.rope_base,
+                          w.eps)
+    ws = la.workspace(shape, dev)
+
+    def one_step():
+        for d_, h_ in zip(din, hin):
+            d_.copy_(h_, non_blocking=True)
+        la.la_attention_backward(shape, din[0], din[1], din[2], None, None, din[3], *dout, dS,
+                                 dz, ws, stream)
+        for h_, d_ in zip(hout, dout):
+            h_.copy_(d_, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        one_step()
+        torch.cuda.synchronize(dev)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            one_step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    nb = hin[0].numel() * hin[0].element_size()
+    return {"ms_per_step": a.elapsed_time(b) / steps, "tokens_per_step": w.B * w.N,
+            "steps": steps, "h2d_bytes_per_step": 4 * nb, "d2h_bytes_per_step": 3 * nb}
+
+
 # ---------------------------------------------------------------------------
 
 
@@ -486,11 +567,16 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--soak", type=float, default=1.0)
+    ap.add_argument("--op", choices=["layer", "backward"], default="layer")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
+    if args.op == "backward" and w.block_causal:
+        ap.error("--op backward covers the non-causal workloads")
     if args.steps is None:
         per_step_us = {"sana0.6b_512px": 10, "sana1.6b_1024px": 30, "sana1.6b_4k": 120,
                        "sanavideo_480p": 250, "longsana_block_causal": 12000}[w.name]
+        if args.op == "backward":
+            per_step_us *= 10
         args.steps = max(10, int(0.5e6 / per_step_us))
     args.warmup = max(args.warmup, 3)
 
@@ -548,17 +634,20 @@ def main():
         "h2d_bytes_per_step": e["h2d_bytes_per_step"],
         "d2h_bytes_per_step": e["d2h_bytes_per_step"], "steps": e["steps"],
         "ms_per_step": round(e["ms_per_step"], 4),
-        "api": "la_block_causal_step" if w.block_causal else "la_attention"}
-    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "api": ("la_attention_backward" if args.op == "backward" else
+                "la_block_causal_step" if w.block_causal else "la_attention")}
+    bwd = args.op == "backward"
+    out = {"metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
            "latency_us": ms_step * 1e3, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), bf16)",
-           "config": config_of(w, world, r["n_sets"], r["per_set_bytes"]),
+           "config": dict(config_of(w, world, r["n_sets"], r["per_set_bytes"]),
+                          **({"op": "backward (dQ, dK, dV, dS, dz)"} if bwd else {})),
            "roofline": roofline, "e2e": e2e,
            "gpu_launches": r["launches_per_step"] * args.steps,
            "clocks": r["clocks"], "graph_chunk_steps": r["chunk"], "soak_s": args.soak}
     if world == 1 and args.cpu_seconds > 0:
-        tps, desc, cores, _, _ = oracle_sample(w, args.cpu_seconds)
+        tps, desc, cores, _, _ = oracle_sample(w, args.cpu_seconds, op=args.op)
         out["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores,
                                "kind": "oracle", "sample": desc}
     print(json.dumps(out), flush=True)
@@ -570,15 +659,19 @@ def main_reference(args, w, rank, world):
         return
     budget = 150.0  # seconds for warm-up + timed steps together
     per = budget / (args.steps + args.warmup)
-    _, _, cores, per_call, h_sub = oracle_sample(w, min(per, 3.0), max_reps=1)
+    _, _, cores, per_call, h_sub = oracle_sample(w, min(per, 3.0), max_reps=1, op=args.op)
     # each step: one oracle call on h_sub heads (at most `per` seconds)
     import oracle as orc
     import numpy as np
     th = orc.rope_angles(w.T, w.Hh, w.W, 0, w.rope_base) if w.rope else None
     Q, K, V = (x[:, :, :h_sub].contiguous() for x in wl.make_qkv(w, 0))
+    bwd = args.op == "backward"
+    dO = wl.make_tensor((w.B, w.N, w.H, w.D), 3)[:, :, :h_sub].contiguous() if bwd else None
 
     def call():
-        if w.block_causal:
+        if bwd:
+            orc.backward(Q, K, V, dO, w.eps, th)
+        elif w.block_causal:
             orc.block_causal_step(Q, K, V, np.zeros((w.B, h_sub, D, D)),
                                   np.zeros((w.B, h_sub, D)), 1, w.eps, th)
         else:
@@ -601,12 +694,14 @@ def main_reference(args, w, rank, world):
     else:
         value = w.B * w.N / full_call
         ms_step = full_call * 1e3
-        sample = f"each step: oracle attention on {h_sub} of {w.H} heads; scaled to {w.H} heads"
-    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        what = "backward" if bwd else "attention"
+        sample = f"each step: oracle {what} on {h_sub} of {w.H} heads; scaled to {w.H} heads"
+    out = {"impl": "reference", "metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": "tokens/s",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic (seeded N(0,1), bf16 inputs read exactly)",
-           "config": config_of(w, world),
+           "config": dict(config_of(w, world),
+                          **({"op": "backward (dQ, dK, dV, dS, dz)"} if bwd else {})),
            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,

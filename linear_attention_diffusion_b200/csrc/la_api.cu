@@ -159,6 +159,21 @@ cudaError_t launch_apply(const Problem& p, const void* Q, const float* S, const 
   return launch_apply_simt(p, Q, S, z, O, s);
 }
 
+cudaError_t launch_backward_q(const Problem& p, const void* Q, const void* dO, const float* S,
+                              const float* z, void* dQ, float* partials, unsigned* counters,
+                              const StateOut& out, cudaStream_t s) {
+  if (p.io == LA_IO_BF16 && p.N > 0)
+    return launch_backward_q_tc(p, Q, dO, S, z, dQ, partials, counters, out, s);
+  return launch_backward_q_simt(p, Q, dO, S, z, dQ, partials, counters, out, s);
+}
+
+cudaError_t launch_backward_kv(const Problem& p, const void* K, const void* V, const float* dS,
+                               const float* dz, void* dK, void* dV, bool after_own_q,
+                               cudaStream_t s) {
+  if (p.io == LA_IO_BF16) return launch_backward_kv_tc(p, K, V, dS, dz, dK, dV, after_own_q, s);
+  return launch_backward_kv_simt(p, K, V, dS, dz, dK, dV, s);
+}
+
 WsLayout workspace_layout(const Problem& p) {
   using detail::align256;
   WsLayout L;
@@ -372,7 +387,7 @@ la_status la_attention_backward(const la_shape* shape, const void* Q, const void
   cudaError_t e = launch_backward_q(p, Q, dO, S, z, dQ, partials, counters, grads, st);
   if (e != cudaSuccess) return cuda_fail(e, "backward (query side)");
   if (!any_input) return LA_OK;
-  e = launch_backward_kv(p, K, V, dS, dz, dK, dV, st);
+  e = launch_backward_kv(p, K, V, dS, dz, dK, dV, true, st);
   if (e != cudaSuccess) return cuda_fail(e, "backward (key side)");
   return LA_OK;
 }
@@ -415,8 +430,11 @@ const char* la_last_error(void) { return g_last_error.c_str(); }
 
 la_status la_device_error(unsigned* code, int reset) {
   if (code == nullptr) return fail(LA_ERR_INVALID_ARG, "code is NULL");
-  const cudaError_t e = read_device_error(code, reset != 0);
+  unsigned fwd = 0, bwd = 0;
+  cudaError_t e = read_device_error(&fwd, reset != 0);
+  if (e == cudaSuccess) e = read_device_error_bwd(&bwd, reset != 0);
   if (e != cudaSuccess) return cuda_fail(e, "la_device_error");
+  *code = fwd | bwd;
   return LA_OK;
 }
 

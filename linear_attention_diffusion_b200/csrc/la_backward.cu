@@ -1,4 +1,5 @@
-// Backward pass of the non-causal layer on CUDA cores (float32 and bf16 I/O).
+// Backward pass of the non-causal layer on CUDA cores (the float32-I/O path;
+// bf16 I/O runs on the tensor cores, la_backward_tc.cu).
 //
 // "Sana: Efficient High-Resolution Image Synthesis with Linear Diffusion
 // Transformers", section Infra, runs the linear attention with a fused forward
@@ -235,9 +236,9 @@ bwd_kv_simt(const Problem p, const T* __restrict__ K, const T* __restrict__ V,
 
 }  // namespace
 
-cudaError_t launch_backward_q(const Problem& p, const void* Q, const void* dO, const float* S,
-                              const float* z, void* dQ, float* partials, unsigned* counters,
-                              const StateOut& out, cudaStream_t s) {
+cudaError_t launch_backward_q_simt(const Problem& p, const void* Q, const void* dO, const float* S,
+                                   const float* z, void* dQ, float* partials,
+                                   unsigned* counters, const StateOut& out, cudaStream_t s) {
   const dim3 grid(p.splits, p.H, p.B);
   if (p.io == 0)
     bwd_q_simt<__nv_bfloat16><<<grid, kBThreads, 0, s>>>(
@@ -250,8 +251,8 @@ cudaError_t launch_backward_q(const Problem& p, const void* Q, const void* dO, c
   return cudaGetLastError();
 }
 
-cudaError_t launch_backward_kv(const Problem& p, const void* K, const void* V, const float* dS,
-                               const float* dz, void* dK, void* dV, cudaStream_t s) {
+cudaError_t launch_backward_kv_simt(const Problem& p, const void* K, const void* V, const float* dS,
+                                    const float* dz, void* dK, void* dV, cudaStream_t s) {
   const dim3 grid((p.N + kKT - 1) / kKT, p.H, p.B);
   if (p.io == 0)
     bwd_kv_simt<__nv_bfloat16><<<grid, kBThreads, 0, s>>>(

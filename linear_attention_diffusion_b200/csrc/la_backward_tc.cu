@@ -1,0 +1,846 @@
+// Tensor-core (tcgen05) backward of the bf16 layer. What it computes is the
+// gradient of the Sana Linear DiT's ReLU linear attention ("Sana: Efficient
+// High-Resolution Image Synthesis with Linear Diffusion Transformers", section
+// Infra: the attention is trained with a fused forward and backward kernel),
+// with the RoPE-after-ReLU numerator of "SANA-Video: Efficient Video
+// Generation with Block Linear Diffusion Transformer", section 2.2. With
+// den_n = ReLU(q_n) . z + eps and R_n the token's rotation:
+//
+//   dnum_n = dO_n / den_n,   t_n = S dnum_n^T,   u_n = R_n^T t_n
+//   dden_n = -(ReLU(q_n) . u_n) / den_n      (= -(dO_n . O_n) / den_n)
+//   dQ_n   = [u_n + dden_n z] * [q_n > 0]
+//   dS     = sum_n phi(q_n)^T dnum_n,        dz = sum_n dden_n ReLU(q_n)
+//   dK_n   = [R_n^T (dS v_n^T) + dz] * [k_n > 0],   dV_n = phi(k_n) dS
+//
+// Query side (one launch, grid = token splits x head groups x batch, as the
+// state reduce): per 128-token tile of a 4-head group,
+//   transform  Q -> ReLU(Q) and dO -> dnum (bf16) in place in shared memory;
+//   MMA 1      t = dnum S^T per head (M = 128 tokens, N = 32, K = 32) into TMEM;
+//   epilogue   dden, dQ (stored straight from registers), dz on CUDA cores;
+//   rewrite    ReLU(Q) -> phi(Q) in place (RoPE only);
+//   MMA 2      dS += phi(Q)^T dnum (M = N = 128 dims, K = 16 tokens; the four
+//              32x32 diagonal blocks are the heads' dS).
+// The split partials of (dS, dz) are combined by the last CTA of each head
+// group in split order, exactly like the state reduce: deterministic.
+//
+// Key side (one launch, grid = tile ranges x head groups x batch): per tile,
+//   transform  K -> phi(K) in place (the sign mask stays in registers);
+//   MMA 1      dphi(K) = V dS^T per head; epilogue dK = R^T dphi(K) + dz,
+//              masked, written over the V tile (MMA 1 has read it);
+//   MMA 2      dV = phi(K) dS per head, in the same TMEM columns; dV written
+//              over the K tile; dK and dV stored with TMA.
+//
+// Warp roles: warp 0 TMA, warp 1 MMA (one elected lane), warps 2..13 three
+// math warpgroups. Warpgroup w owns stage w, TMEM columns [128 w, 128 w + 128)
+// and the tiles j = w (mod 3), so every mbarrier has one consumer that waits
+// for its phases in order (a parity wait cannot tell phase k from k + 2).
+// Every wait is bounded and raises the device error word when it gives up.
+#include <algorithm>
+
+#include "la_tc_common.cuh"
+
+namespace la {
+
+// Device error word of the backward kernels (same meaning as the forward's).
+__device__ unsigned g_bwd_tc_error;
+
+namespace {
+
+constexpr int kBT = 128;                // tokens per tile
+constexpr int kBBox = kBT * 128;        // [128 tokens][64 dims] bf16 = 16 KB
+constexpr int kBTile = 4 * kBBox;       // two tensors x two boxes = 64 KB
+constexpr int kBStages = 3;
+constexpr int kBWG = 3;                 // math warpgroups (one per stage)
+constexpr int kBMath = kBWG * 128;
+constexpr int kBThreads = 64 + kBMath;
+constexpr int kBTmemCols = 512;
+constexpr int kBarAll = 1;              // named barrier over the math threads
+constexpr int kBarW0 = 2;               // + warpgroup
+
+struct QSmem {  // query side, byte offsets from the 1024-aligned base
+  static constexpr int stages = 0;                          // [3][Q box0, Q box1, dO box0, dO box1]
+  static constexpr int bop = stages + kBStages * kBTile;    // S as B operand: [2][32 rows][128 B]
+  static constexpr int zs = bop + 8192;                     // [4][32] f32
+  static constexpr int dden = zs + 512;                     // [3][128 rows][4] f32
+  static constexpr int rope = dden + kBWG * kBT * 4 * 4;    // float2[kRopeTableMax]
+  static constexpr int bars = rope + kRopeTableMax * 8;
+  // full[3] empty[3] ready_t[3] ready_s[3] t_full[3] acc_full mma_done b_ready
+  static constexpr int nbars = 5 * kBStages + 3;
+  static constexpr int misc = bars + nbars * 8;
+  static constexpr int bytes = misc + 16;
+};
+struct KVSmem {  // key side
+  static constexpr int stages = 0;                          // [3][K box0, K box1, V box0, V box1]
+  static constexpr int bop1 = stages + kBStages * kBTile;   // dS rows d (K = e)
+  static constexpr int bop2 = bop1 + 8192;                  // dS^T rows e (K = d)
+  static constexpr int zs = bop2 + 8192;                    // dz [4][32] f32
+  static constexpr int rope = zs + 512;
+  static constexpr int bars = rope + kRopeTableMax * 8;
+  // full[3] empty[3] ready[3] t_full[3] t_empty[3] b_ready mma_done
+  static constexpr int nbars = 5 * kBStages + 2;
+  static constexpr int misc = bars + nbars * 8;
+  static constexpr int bytes = misc + 16;
+};
+constexpr int kQSmemBytes = QSmem::bytes + 1024;
+constexpr int kKVSmemBytes = KVSmem::bytes + 1024;
+static_assert(kQSmemBytes <= 232448 && kKVSmemBytes <= 232448, "shared memory per CTA");
+
+struct BwdArgs {
+  float* partials;        // query side: [B*H][splits][kStateFloats]
+  unsigned* arrive;       // query side: per head-group arrival counters (index b*H + h0)
+  StateOut out;           // query side: where the combined (dS, dz) goes
+  const float* S;         // query side: the forward state; key side: dS
+  const float* z;         // query side: z; key side: dz
+  __nv_bfloat16* dQ;      // query side output
+  int tiles_per_cta;      // key side
+  int kv_before_wait;     // key side: K, V may be fetched before the previous grid completes
+};
+
+// (cos, sin) of the 16 pairs of token n (the row's RoPE rotation).
+template <int kRope>
+__device__ __forceinline__ void row_angles(const Problem& p, const float2* tab, int n,
+                                           float2 (&cs)[16]) {
+  const TokPos tp = token_pos(p.rope, min(n, p.N - 1));
+  const RopeBases rb = rope_bases(p.rope, tp);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int ax = pair_axis(j);
+    if (kRope == kRopeTable) {
+      cs[j] = tab[(ax == 0 ? rb.t : (ax == 1 ? rb.h : rb.w)) + pair_off(j)];
+    } else {
+      const int pp = ax == 0 ? p.rope.t_offset + tp.t : (ax == 1 ? tp.h : tp.w);
+      rope_cos_sin(pp, p.rope.inv_freq[j], cs[j].x, cs[j].y);
+    }
+  }
+}
+
+// x <- R x (sign = +1) or R^T x (sign = -1) for the 4 pairs of a chunk whose
+// first pair is j0.
+template <int kSign>
+__device__ __forceinline__ void rotate_chunk(const float2 (&cs)[16], int j0, float (&x)[8]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 r = cs[j0 + q];
+    const float sn = kSign > 0 ? r.y : -r.y;
+    const float2 t = __fmul2_rn(make_float2(x[2 * q + 1], x[2 * q + 1]), make_float2(-sn, r.x));
+    const float2 y = __ffma2_rn(make_float2(x[2 * q], x[2 * q]), make_float2(r.x, sn), t);
+    x[2 * q] = y.x;
+    x[2 * q + 1] = y.y;
+  }
+}
+
+// Build a 4-head B operand in shared memory from a float32 [heads][32][32]
+// global array M: row r of head pair j holds M[h][r][0..31] (transpose = 0) or
+// M[h][0..31][r] (transpose = 1) of heads 2j and 2j+1, in bf16, K-major with
+// the 128-byte swizzle. Missing heads are zero.
+__device__ __forceinline__ void build_bop(uint32_t bop, const float* M, size_t cidx, int h0,
+                                          int H, bool transpose, int mt, int nthreads) {
+  for (int idx = mt; idx < 2 * 32 * 8; idx += nthreads) {
+    const int j = idx >> 8, r = (idx >> 3) & 31, c = idx & 7;
+    const int hh = 2 * j + (c >> 2), k0 = (c & 3) * 8;
+    float x[8];
+    if (h0 + hh < H) {
+      const float* m = M + (cidx + hh) * kD * kD;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[k] = transpose ? __ldcg(m + (k0 + k) * kD + r) : __ldcg(m + r * kD + k0 + k);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[k] = 0.0f;
+    }
+    st_shared_v4(bop + j * 4096 + sw128_offset(r, c), pack8(x));
+  }
+}
+
+// ================================================================ query side
+
+template <int kRope>
+__global__ void __launch_bounds__(kBThreads, 1)
+bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
+         const Problem p, const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + QSmem::bars);
+  uint64_t* empty = full + kBStages;
+  uint64_t* ready_t = empty + kBStages;   // tile transformed (128 arrivals)
+  uint64_t* ready_s = ready_t + kBStages; // phi(Q) in place, dz done (128 arrivals)
+  uint64_t* t_full = ready_s + kBStages;  // t of the stage's tile is in TMEM
+  uint64_t* acc_full = t_full + kBStages;
+  uint64_t* mma_done = acc_full + 1;
+  uint64_t* b_ready = mma_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + QSmem::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + QSmem::misc + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + QSmem::misc + 8);
+  float* zs = reinterpret_cast<float*>(smem + QSmem::zs);
+  float* dden_buf = reinterpret_cast<float*>(smem + QSmem::dden);
+  float2* rope_tab = reinterpret_cast<float2*>(smem + QSmem::rope);
+  unsigned* err = &g_bwd_tc_error;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int group = blockIdx.y, b = blockIdx.z;
+  const int h0 = group * kGroupHeads;
+  const size_t cidx = static_cast<size_t>(b) * p.H + h0;
+  const int n_begin = blockIdx.x * p.chunk;
+  const int n_end = min(p.N, n_begin + p.chunk);
+  const int nT = n_end > n_begin ? (n_end - n_begin + kBT - 1) / kBT : 0;
+
+  if (tid == 0) {
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&ready_t[s], 128);
+      mbar_init(&ready_s[s], 128);
+      mbar_init(&t_full[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(mma_done, 1);
+    mbar_init(b_ready, 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kBTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_g);
+  }
+  if (kRope == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kBMath);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sbase = smem_u32(smem);
+  pdl_wait();
+  if (tid == 64) pdl_trigger();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA loads
+    if (lane == 0) {
+      int i = 0;
+      for (; i < nT; ++i) {
+        const int s = i % kBStages;
+        if (!mbar_wait(&empty[s], ((i / kBStages) & 1) ^ 1, abort_flag, err, kErrWait)) break;
+        mbar_arrive_expect_tx(&full[s], kBTile);
+        uint8_t* st = smem + QSmem::stages + s * kBTile;
+        const int y = n_begin + i * kBT;
+        tma_load_3d(st, &tm_q, &full[s], h0 * 32, y, b);
+        tma_load_3d(st + kBBox, &tm_q, &full[s], h0 * 32 + 64, y, b);
+        tma_load_3d(st + 2 * kBBox, &tm_g, &full[s], h0 * 32, y, b);
+        tma_load_3d(st + 3 * kBBox, &tm_g, &full[s], h0 * 32 + 64, y, b);
+      }
+      for (int q = max(0, i - kBStages); q < i; ++q)
+        mbar_drain(&full[q % kBStages], (q / kBStages) & 1, err, kErrWait);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0) {
+      bool ok = nT == 0 || mbar_wait(b_ready, 0, abort_flag, err, kErrWait);
+      const uint32_t id_t = idesc_bf16_f32(128, 32, 0, 0);
+      const uint32_t id_s = idesc_bf16_f32(128, 128, 1, 1);
+      const uint32_t bop = sbase + QSmem::bop;
+      // MMA 2 of tile i - 1 is issued after MMA 1 of tile i
+      for (int i = 0; ok && i <= nT; ++i) {
+        if (i < nT) {
+          const int s = i % kBStages;
+          if (!(ok = mbar_wait(&ready_t[s], (i / kBStages) & 1, abort_flag, err, kErrWait))) break;
+          tc_fence_after();
+          const uint32_t st = sbase + QSmem::stages + s * kBTile;
+#pragma unroll
+          for (int hh = 0; hh < kGroupHeads; ++hh) {
+            const uint32_t koff = (hh & 1) * 64;
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              const uint64_t ad =
+                  smem_desc_sw128(st + 2 * kBBox + (hh >> 1) * kBBox + koff + kk * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(bop + (hh >> 1) * 4096 + koff + kk * 32, 16, 1024);
+              mma_bf16(tmem + 128 + s * 128 + hh * 32, ad, bd, id_t, kk);
+            }
+          }
+          mma_commit(&t_full[s]);
+        }
+        const int k = i - 1;
+        if (k >= 0) {
+          const int s = k % kBStages;
+          if (!(ok = mbar_wait(&ready_s[s], (k / kBStages) & 1, abort_flag, err, kErrWait))) break;
+          tc_fence_after();
+          const uint32_t st = sbase + QSmem::stages + s * kBTile;
+#pragma unroll
+          for (int kk = 0; kk < kBT / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(st + kk * 2048, kBBox, 1024);
+            const uint64_t bd = smem_desc_sw128(st + 2 * kBBox + kk * 2048, kBBox, 1024);
+            mma_bf16(tmem, ad, bd, id_s, (k > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+        }
+      }
+      mma_commit(acc_full);
+      mma_commit(mma_done);
+      mbar_drain(mma_done, 0, err, kErrWait);
+    }
+  } else {
+    // ---------------------------------------------------------- math warps
+    const int mt = tid - 64;
+    const int wg = mt >> 7, wt = mt & 127;
+    const int quad = warp & 3;            // TMEM lane quadrant of this warp
+    const int row = quad * 32 + lane;     // token row of the tile (thread = row)
+    bool alive = true;
+
+    // S as the B operand of MMA 1 (rows d, K = e), z of the four heads
+    build_bop(sbase + QSmem::bop, a.S, cidx, h0, p.H, false, mt, kBMath);
+    if (mt < kGroupHeads * kD) zs[mt] = h0 + mt / kD < p.H ? __ldcg(a.z + cidx * kD + mt) : 0.0f;
+    fence_proxy_async_smem();
+    named_bar_sync(kBarAll, kBMath);
+    if (mt == 0) mbar_arrive(b_ready);
+
+    // dz of dims [(c&3)*8, +8) of head c>>2 over rows rg, rg + 8, ...
+    const int zc = wt & 15, zrg = wt >> 4;
+    float zacc[8] = {};
+    float* my_dden = dden_buf + wg * kBT * 4;
+
+    for (int j = wg; j < nT; j += kBWG) {
+      const int s = wg;  // j % kBStages
+      const uint32_t par = (j / kBStages) & 1;
+      bool ok = mbar_wait(&full[s], par, abort_flag, err, kErrWait);
+      if (bar_any(kBarW0 + wg, 128, !ok || *abort_flag)) {
+        alive = false;
+        break;
+      }
+      const uint32_t st = sbase + QSmem::stages + s * kBTile;
+      const int n0 = n_begin + j * kBT;
+      const int n = n0 + row;
+      float2 cs[16];
+      if (kRope != kNoRope) row_angles<kRope>(p, rope_tab, n, cs);
+
+      // ---- transform: ReLU(Q) in place, den, dnum = dO / den in place
+      float inv[kGroupHeads];
+#pragma unroll
+      for (int hh = 0; hh < kGroupHeads; ++hh) {
+        float den = 0.0f;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int c = hh * 4 + c4;
+          const uint32_t addr = st + (c >> 3) * kBBox + sw128_offset(row, c & 7);
+          uint4 u = ld_shared_v4(addr);
+          u.x = relu_bf16x2(u.x);
+          u.y = relu_bf16x2(u.y);
+          u.z = relu_bf16x2(u.z);
+          u.w = relu_bf16x2(u.w);
+          float x[8];
+          unpack8(u, x);
+          const float* zz = zs + hh * kD + c4 * 8;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) den = fmaf(x[e], zz[e], den);
+          st_shared_v4(addr, u);
+        }
+        inv[hh] = 1.0f / (den + p.eps);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int c = hh * 4 + c4;
+          const uint32_t addr = st + 2 * kBBox + (c >> 3) * kBBox + sw128_offset(row, c & 7);
+          float x[8];
+          unpack8(ld_shared_v4(addr), x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] *= inv[hh];
+          st_shared_v4(addr, pack8(x));
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&ready_t[s]);
+
+      // ---- epilogue: u = R^T t, dden, dQ, per head
+      ok = mbar_wait(&t_full[s], par, abort_flag, err, kErrWait);
+      tc_fence_after();
+      if (bar_any(kBarW0 + wg, 128, !ok || *abort_flag)) {
+        alive = false;
+        break;
+      }
+      const bool row_ok = n < n_end;
+#pragma unroll
+      for (int hh = 0; hh < kGroupHeads; ++hh) {
+        float t[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 128 + s * 128 + hh * 32,
+                           t);
+        if (kRope != kNoRope) {
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            float y[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = t[c4 * 8 + e];
+            rotate_chunk<-1>(cs, c4 * 4, y);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) t[c4 * 8 + e] = y[e];
+          }
+        }
+        // ReLU(q) is read from shared memory twice rather than held in registers
+        float dot = 0.0f;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int c = hh * 4 + c4;
+          float x[8];
+          unpack8(ld_shared_v4(st + (c >> 3) * kBBox + sw128_offset(row, c & 7)), x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dot = fmaf(x[e], t[c4 * 8 + e], dot);
+        }
+        const float dden = -dot * inv[hh];
+        my_dden[row * 4 + hh] = dden;
+        if (row_ok && h0 + hh < p.H) {
+          const float* zz = zs + hh * kD;
+          __nv_bfloat16* dst = a.dQ + ((static_cast<size_t>(b) * p.N + n) * p.H + h0 + hh) * kD;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int c = hh * 4 + c4;
+            float x[8];
+            unpack8(ld_shared_v4(st + (c >> 3) * kBBox + sw128_offset(row, c & 7)), x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int d = c4 * 8 + e;
+              x[e] = x[e] > 0.0f ? fmaf(dden, zz[d], t[d]) : 0.0f;
+            }
+            *reinterpret_cast<uint4*>(dst + c4 * 8) = pack8(x);
+          }
+        }
+      }
+      tc_fence_before();
+      named_bar_sync(kBarW0 + wg, 128);
+
+      // ---- dz over the tile's rows (fixed order per thread)
+      {
+        const int hh = zc >> 2;
+#pragma unroll 4
+        for (int r = zrg; r < kBT; r += 8) {
+          float x[8];
+          unpack8(ld_shared_v4(st + (zc >> 3) * kBBox + sw128_offset(r, zc & 7)), x);
+          const float dd = my_dden[r * 4 + hh];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) zacc[e] = fmaf(dd, x[e], zacc[e]);
+        }
+      }
+      named_bar_sync(kBarW0 + wg, 128);
+
+      // ---- rewrite ReLU(Q) -> phi(Q) for MMA 2
+      if (kRope != kNoRope) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const uint32_t addr = st + (c >> 3) * kBBox + sw128_offset(row, c & 7);
+          float x[8];
+          unpack8(ld_shared_v4(addr), x);
+          rotate_chunk<1>(cs, (c & 3) * 4, x);
+          st_shared_v4(addr, pack8(x));
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&ready_s[s]);
+    }
+
+    // ---- partial (dS, dz) of this split
+    alive = !bar_any(kBarAll, kBMath, !alive || *abort_flag);
+    float* scratch = reinterpret_cast<float*>(smem + QSmem::stages);  // [kBMath][8] after the MMAs
+    if (warp >= 2 && warp < 6) {
+      const int q = warp & 3;
+      float v[32];
+      bool got = alive && nT > 0 && mbar_wait(acc_full, 0, abort_flag, err, kErrWait);
+      got = __all_sync(0xffffffffu, got);
+      if (got) {
+        tc_fence_after();
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32 * q, v);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0.0f;
+      }
+      if (h0 + q < p.H) {
+        float* dst = a.partials + ((cidx + q) * p.splits + blockIdx.x) * kStateFloats + lane * kD;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+      }
+    }
+    // every MMA has completed (acc_full) before the stages are reused as scratch
+    bool drained = !alive || nT == 0 || mbar_wait(acc_full, 0, abort_flag, err, kErrWait);
+    alive = !bar_any(kBarAll, kBMath, !drained || *abort_flag) && alive;
+    if (alive) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) scratch[mt * 8 + e] = zacc[e];
+    }
+    named_bar_sync(kBarAll, kBMath);
+    if (alive && mt < kGroupHeads * kD) {
+      const int q = mt >> 5, d = mt & 31;
+      const int col = q * 4 + (d >> 3), e = d & 7;
+      float sum = 0.0f;
+      for (int w = 0; w < kBWG; ++w)
+        for (int rg = 0; rg < 8; ++rg) sum += scratch[(w * 128 + rg * 16 + col) * 8 + e];
+      if (h0 + q < p.H)
+        a.partials[((cidx + q) * p.splits + blockIdx.x) * kStateFloats + kD * kD + d] = sum;
+    }
+    tc_fence_before();
+
+    // ---- last CTA of the head group: sum the splits in order
+    named_bar_sync(kBarAll, kBMath);
+    if (mt == 0) {
+      fence_acq_rel_gpu();
+      const unsigned prev = atomicAdd(&a.arrive[cidx], 1u);
+      *last_flag = prev == gridDim.x - 1;
+      if (*last_flag) fence_acq_rel_gpu();
+    }
+    named_bar_sync(kBarAll, kBMath);
+    const bool last = *last_flag != 0;
+    if (last && alive) combine_from_global<kBMath>(p, b, h0, mt, a.partials, a.out);
+    named_bar_sync(kBarAll, kBMath);
+    if (mt == 0 && last) a.arrive[cidx] = 0u;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBTmemCols);
+  }
+}
+
+// ================================================================== key side
+
+template <int kRope>
+__global__ void __launch_bounds__(kBThreads, 1)
+bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+          const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
+          const Problem p, const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + KVSmem::bars);
+  uint64_t* empty = full + kBStages;
+  uint64_t* ready = empty + kBStages;    // tile transformed (128 arrivals)
+  uint64_t* t_full = ready + kBStages;   // MMA 1, then MMA 2, of the stage's tile done
+  uint64_t* t_empty = t_full + kBStages; // their results read out of TMEM
+  uint64_t* b_ready = t_empty + kBStages;
+  uint64_t* mma_done = b_ready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + KVSmem::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + KVSmem::misc + 4);
+  float* zs = reinterpret_cast<float*>(smem + KVSmem::zs);
+  float2* rope_tab = reinterpret_cast<float2*>(smem + KVSmem::rope);
+  unsigned* err = &g_bwd_tc_error;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int group = blockIdx.y, b = blockIdx.z;
+  const int h0 = group * kGroupHeads;
+  const size_t cidx = static_cast<size_t>(b) * p.H + h0;
+  const int ntiles_all = (p.N + kBT - 1) / kBT;
+  const int tile_begin = blockIdx.x * a.tiles_per_cta;
+  const int nT = max(0, min(ntiles_all, tile_begin + a.tiles_per_cta) - tile_begin);
+
+  if (tid == 0) {
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&ready[s], 128);
+      mbar_init(&t_full[s], 1);
+      mbar_init(&t_empty[s], 1);
+    }
+    mbar_init(b_ready, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kBTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_dk);
+    prefetch_tmap(&tm_dv);
+  }
+  if (kRope == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kBMath);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sbase = smem_u32(smem);
+  // K and V are inputs the query side does not write: the TMA warp may fetch
+  // them before that grid completes; dS and dz are read after the wait.
+  if (!(warp == 0 && a.kv_before_wait)) pdl_wait();
+  if (tid == 64) pdl_trigger();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int i = 0;
+      for (; i < nT; ++i) {
+        const int s = i % kBStages;
+        if (!mbar_wait(&empty[s], ((i / kBStages) & 1) ^ 1, abort_flag, err, kErrWait)) break;
+        mbar_arrive_expect_tx(&full[s], kBTile);
+        uint8_t* st = smem + KVSmem::stages + s * kBTile;
+        const int y = (tile_begin + i) * kBT;
+        tma_load_3d(st, &tm_k, &full[s], h0 * 32, y, b);
+        tma_load_3d(st + kBBox, &tm_k, &full[s], h0 * 32 + 64, y, b);
+        tma_load_3d(st + 2 * kBBox, &tm_v, &full[s], h0 * 32, y, b);
+        tma_load_3d(st + 3 * kBBox, &tm_v, &full[s], h0 * 32 + 64, y, b);
+      }
+      for (int q = max(0, i - kBStages); q < i; ++q)
+        mbar_drain(&full[q % kBStages], (q / kBStages) & 1, err, kErrWait);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = nT == 0 || mbar_wait(b_ready, 0, abort_flag, err, kErrWait);
+      const uint32_t id = idesc_bf16_f32(128, 32, 0, 0);
+      const uint32_t bop1 = sbase + KVSmem::bop1, bop2 = sbase + KVSmem::bop2;
+      // t_empty[s] completes twice per tile (MMA 1's and MMA 2's results
+      // read), so the waits alternate parity 1 (before MMA 1) and 0 (before
+      // MMA 2). MMA 2 of tile i - 1 is issued after MMA 1 of tile i.
+      for (int i = 0; ok && i <= nT; ++i) {
+        if (i < nT) {
+          const int s = i % kBStages;
+          if (!(ok = mbar_wait(&ready[s], (i / kBStages) & 1, abort_flag, err, kErrWait))) break;
+          if (!(ok = mbar_wait(&t_empty[s], 1, abort_flag, err, kErrWait))) break;
+          tc_fence_after();
+          const uint32_t st = sbase + KVSmem::stages + s * kBTile;
+#pragma unroll
+          for (int hh = 0; hh < kGroupHeads; ++hh) {
+            const uint32_t koff = (hh & 1) * 64;
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              // dphi(K)[n][d] = sum_e V[n][e] dS[d][e]
+              const uint64_t av =
+                  smem_desc_sw128(st + 2 * kBBox + (hh >> 1) * kBBox + koff + kk * 32, 16, 1024);
+              const uint64_t bd =
+                  smem_desc_sw128(bop1 + (hh >> 1) * 4096 + koff + kk * 32, 16, 1024);
+              mma_bf16(tmem + s * 128 + hh * 32, av, bd, id, kk);
+            }
+          }
+          mma_commit(&t_full[s]);
+        }
+        const int k = i - 1;
+        if (k >= 0) {
+          const int s = k % kBStages;
+          if (!(ok = mbar_wait(&t_empty[s], 0, abort_flag, err, kErrWait))) break;
+          tc_fence_after();
+          const uint32_t st = sbase + KVSmem::stages + s * kBTile;
+#pragma unroll
+          for (int hh = 0; hh < kGroupHeads; ++hh) {
+            const uint32_t koff = (hh & 1) * 64;
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              // dV[n][e] = sum_d phi(K)[n][d] dS[d][e]
+              const uint64_t ak = smem_desc_sw128(st + (hh >> 1) * kBBox + koff + kk * 32, 16, 1024);
+              const uint64_t bd =
+                  smem_desc_sw128(bop2 + (hh >> 1) * 4096 + koff + kk * 32, 16, 1024);
+              mma_bf16(tmem + s * 128 + hh * 32, ak, bd, id, kk);
+            }
+          }
+          mma_commit(&t_full[s]);
+        }
+      }
+      mma_commit(mma_done);
+      mbar_drain(mma_done, 0, err, kErrWait);
+    }
+  } else {
+    const int mt = tid - 64;
+    const int wg = mt >> 7, wt = mt & 127;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const bool leader = wt == 0;
+
+    build_bop(sbase + KVSmem::bop1, a.S, cidx, h0, p.H, false, mt, kBMath);
+    build_bop(sbase + KVSmem::bop2, a.S, cidx, h0, p.H, true, mt, kBMath);
+    if (mt < kGroupHeads * kD) zs[mt] = h0 + mt / kD < p.H ? __ldcg(a.z + cidx * kD + mt) : 0.0f;
+    fence_proxy_async_smem();
+    named_bar_sync(kBarAll, kBMath);
+    if (mt == 0) mbar_arrive(b_ready);
+
+    for (int j = wg; j < nT; j += kBWG) {
+      const int s = wg;  // j % kBStages
+      bool ok = mbar_wait(&full[s], (j / kBStages) & 1, abort_flag, err, kErrWait);
+      if (bar_any(kBarW0 + wg, 128, !ok || *abort_flag)) break;
+      const uint32_t st = sbase + KVSmem::stages + s * kBTile;
+      const int n0 = (tile_begin + j) * kBT;
+      float2 cs[16];
+      if (kRope != kNoRope) row_angles<kRope>(p, rope_tab, n0 + row, cs);
+
+      // ---- transform: K -> phi(K) in place; keep the sign mask of K
+      uint32_t mask[kGroupHeads] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint32_t addr = st + (c >> 3) * kBBox + sw128_offset(row, c & 7);
+        uint4 v = ld_shared_v4(addr);
+        v.x = relu_bf16x2(v.x);
+        v.y = relu_bf16x2(v.y);
+        v.z = relu_bf16x2(v.z);
+        v.w = relu_bf16x2(v.w);
+        float x[8];
+        unpack8(v, x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (x[e] > 0.0f) mask[c >> 2] |= 1u << ((c & 3) * 8 + e);
+        if (kRope != kNoRope) {
+          rotate_chunk<1>(cs, (c & 3) * 4, x);
+          v = pack8(x);
+        }
+        st_shared_v4(addr, v);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&ready[s]);
+
+      const uint32_t tcol = tmem + (static_cast<uint32_t>(quad * 32) << 16) + s * 128;
+      // ---- dK = R^T dphi(K) + dz, masked, over the V tile (MMA 1 has read it)
+      ok = mbar_wait(&t_full[s], 0, abort_flag, err, kErrWait);
+      tc_fence_after();
+      if (bar_any(kBarW0 + wg, 128, !ok || *abort_flag)) break;
+#pragma unroll
+      for (int hh = 0; hh < kGroupHeads; ++hh) {
+        float g[32];
+        tmem_ld_32x32b_x32(tcol + hh * 32, g);
+        const float* zz = zs + hh * kD;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = g[c4 * 8 + e];
+          if (kRope != kNoRope) rotate_chunk<-1>(cs, c4 * 4, x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int d = c4 * 8 + e;
+            x[e] = (mask[hh] >> d) & 1u ? x[e] + zz[d] : 0.0f;
+          }
+          const int c = hh * 4 + c4;
+          st_shared_v4(st + 2 * kBBox + (c >> 3) * kBBox + sw128_offset(row, c & 7), pack8(x));
+        }
+      }
+      tc_fence_before();
+      named_bar_sync(kBarW0 + wg, 128);
+      if (leader) mbar_arrive(&t_empty[s]);
+
+      // ---- dV over the K tile (MMA 2 has read phi(K)), then both stores
+      ok = mbar_wait(&t_full[s], 1, abort_flag, err, kErrWait);
+      tc_fence_after();
+      if (bar_any(kBarW0 + wg, 128, !ok || *abort_flag)) break;
+#pragma unroll
+      for (int hh = 0; hh < kGroupHeads; ++hh) {
+        float g[32];
+        tmem_ld_32x32b_x32(tcol + hh * 32, g);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = g[c4 * 8 + e];
+          const int c = hh * 4 + c4;
+          st_shared_v4(st + (c >> 3) * kBBox + sw128_offset(row, c & 7), pack8(x));
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      named_bar_sync(kBarW0 + wg, 128);
+      if (leader) {
+        mbar_arrive(&t_empty[s]);
+        uint8_t* tile = smem + KVSmem::stages + s * kBTile;
+        tma_store_3d(&tm_dk, tile + 2 * kBBox, h0 * 32, n0, b);
+        tma_store_3d(&tm_dk, tile + 3 * kBBox, h0 * 32 + 64, n0, b);
+        tma_store_3d(&tm_dv, tile, h0 * 32, n0, b);
+        tma_store_3d(&tm_dv, tile + kBBox, h0 * 32 + 64, n0, b);
+        bulk_commit();
+        bulk_wait_read<0>();
+        mbar_arrive(&empty[s]);
+      }
+    }
+    if (leader) bulk_wait<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBTmemCols);
+  }
+}
+
+// ============================================================== host side
+
+// Launch with programmatic dependent launch: the prologue (barriers, TMEM,
+// RoPE table) may overlap the previous kernel in the stream.
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl(Kernel kern, dim3 grid, int smem, cudaStream_t s, const Args&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kBThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+}  // namespace
+
+cudaError_t launch_backward_q_tc(const Problem& p, const void* Q, const void* dO, const float* S,
+                                 const float* z, void* dQ, float* partials, unsigned* counters,
+                                 const StateOut& out, cudaStream_t s) {
+  CUtensorMap mq, mg;
+  cudaError_t e;
+  if ((e = make_map(&mq, Q, p, kBT)) != cudaSuccess) return e;
+  if ((e = make_map(&mg, dO, p, kBT)) != cudaSuccess) return e;
+  const int mode = rope_mode(rope_table_for(p));
+  auto kern = mode == kNoRope ? bwd_q_tc<kNoRope>
+                              : (mode == kRopeTable ? bwd_q_tc<kRopeTable> : bwd_q_tc<kRopeOnTheFly>);
+  if ((e = ensure_smem_attr(mode, reinterpret_cast<const void*>(kern), kQSmemBytes)) != cudaSuccess)
+    return e;
+  BwdArgs a = {};
+  a.partials = partials;
+  a.arrive = counters;
+  a.out = out;
+  a.S = S;
+  a.z = z;
+  a.dQ = static_cast<__nv_bfloat16*>(dQ);
+  const dim3 grid(p.splits, (p.H + kGroupHeads - 1) / kGroupHeads, p.B);
+  e = launch_pdl(kern, grid, kQSmemBytes, s, mq, mg, p, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_backward_kv_tc(const Problem& p, const void* K, const void* V, const float* dS,
+                                  const float* dz, void* dK, void* dV, bool after_own_q,
+                                  cudaStream_t s) {
+  CUtensorMap mk, mv, mdk, mdv;
+  cudaError_t e;
+  if ((e = make_map(&mk, K, p, kBT)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, V, p, kBT)) != cudaSuccess) return e;
+  if ((e = make_map(&mdk, dK, p, kBT)) != cudaSuccess) return e;
+  if ((e = make_map(&mdv, dV, p, kBT)) != cudaSuccess) return e;
+  const int mode = rope_mode(rope_table_for(p));
+  auto kern = mode == kNoRope
+                  ? bwd_kv_tc<kNoRope>
+                  : (mode == kRopeTable ? bwd_kv_tc<kRopeTable> : bwd_kv_tc<kRopeOnTheFly>);
+  if ((e = ensure_smem_attr(3 + mode, reinterpret_cast<const void*>(kern), kKVSmemBytes)) !=
+      cudaSuccess)
+    return e;
+  const int groups = (p.H + kGroupHeads - 1) / kGroupHeads;
+  const int ntiles = (p.N + kBT - 1) / kBT;
+  const long long units = static_cast<long long>(groups) * p.B;
+  int ctas = static_cast<int>(std::max<long long>(1, kNumSMs / std::max<long long>(1, units)));
+  ctas = std::min(ctas, ntiles);
+  const int tpc = (ntiles + ctas - 1) / ctas;
+  ctas = (ntiles + tpc - 1) / tpc;
+  BwdArgs a = {};
+  a.S = dS;
+  a.z = dz;
+  a.tiles_per_cta = tpc;
+  a.kv_before_wait = after_own_q ? 1 : 0;
+  const dim3 grid(ctas, groups, p.B);
+  e = launch_pdl(kern, grid, kKVSmemBytes, s, mk, mv, mdk, mdv, p, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t read_device_error_bwd(unsigned* code, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(code, g_bwd_tc_error, sizeof(unsigned));
+  if (e == cudaSuccess && reset) {
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_bwd_tc_error, &zero, sizeof(unsigned));
+  }
+  return e;
+}
+
+}  // namespace la

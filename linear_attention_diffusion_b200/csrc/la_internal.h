@@ -83,17 +83,33 @@ bool layer_fusable(const Problem& p);
 cudaError_t launch_layer_tc(const Problem& p, const void* Q, const void* K, const void* V,
                             void* O, float* partials, unsigned* counters, const StateOut& out,
                             cudaStream_t s);
-// Backward of the non-causal layer (la_backward.cu). Query side: dQ, and the
-// state gradients reduced over the token splits into `out` (same partials,
-// counters and split order as the state reduce). Key side: dK and dV from
-// the combined dS, dz.
+// Backward of the non-causal layer. Query side: dQ, and the state gradients
+// reduced over the token splits into `out` (same partials, counters and split
+// order as the state reduce). Key side: dK and dV from the combined dS, dz.
+// Tensor-core kernels for bf16 I/O (la_backward_tc.cu), CUDA-core kernels for
+// float32 I/O and the empty sequence (la_backward.cu).
 cudaError_t launch_backward_q(const Problem& p, const void* Q, const void* dO, const float* S,
                               const float* z, void* dQ, float* partials, unsigned* counters,
                               const StateOut& out, cudaStream_t s);
 cudaError_t launch_backward_kv(const Problem& p, const void* K, const void* V, const float* dS,
-                               const float* dz, void* dK, void* dV, cudaStream_t s);
-// Device error word of the tensor-core kernels (bounded waits that gave up).
+                               const float* dz, void* dK, void* dV, bool after_own_q,
+                               cudaStream_t s);
+cudaError_t launch_backward_q_tc(const Problem& p, const void* Q, const void* dO, const float* S,
+                                 const float* z, void* dQ, float* partials, unsigned* counters,
+                                 const StateOut& out, cudaStream_t s);
+cudaError_t launch_backward_kv_tc(const Problem& p, const void* K, const void* V, const float* dS,
+                                  const float* dz, void* dK, void* dV, bool after_own_q,
+                                  cudaStream_t s);
+cudaError_t launch_backward_q_simt(const Problem& p, const void* Q, const void* dO,
+                                   const float* S, const float* z, void* dQ, float* partials,
+                                   unsigned* counters, const StateOut& out, cudaStream_t s);
+cudaError_t launch_backward_kv_simt(const Problem& p, const void* K, const void* V,
+                                    const float* dS, const float* dz, void* dK, void* dV,
+                                    cudaStream_t s);
+// Device error words of the tensor-core kernels (bounded waits that gave up):
+// the forward's (la_tc.cu) and the backward's (la_backward_tc.cu).
 cudaError_t read_device_error(unsigned* code, bool reset);
+cudaError_t read_device_error_bwd(unsigned* code, bool reset);
 
 // Host-side helpers of the C-ABI layer (la_api.cu).
 namespace detail {

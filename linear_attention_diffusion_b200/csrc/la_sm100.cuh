@@ -73,6 +73,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Wait for work this CTA issued itself (TMA copies, MMAs) before it frees
+// the memory that work uses: unlike mbar_wait it does not stop when another
+// warp has given up, since that work completes regardless; it is still
+// bounded by kWaitLimitNs, after which it raises the error word.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, unsigned* error_word,
+                                           unsigned code) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (error_word != nullptr) atomicOr(error_word, code);
+      return false;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ fences
 
 // Release/acquire at GPU scope, issued by one thread after (or before) a CTA

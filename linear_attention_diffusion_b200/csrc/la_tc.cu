@@ -22,20 +22,15 @@
 //           dims, K-major, straight from the TMA tile) and B = S^T (bf16,
 //           K-major); D = 128 x 32 fp32 per head in tensor memory.
 //
-// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 allocates tensor
-// memory and issues the MMAs (one elected lane), warps 2..9 transform tiles
+// Warp roles (576 threads): warp 0 issues TMA loads, warp 1 allocates tensor
+// memory and issues the MMAs (one elected lane), warps 2..17 transform tiles
 // in shared memory and run the epilogue. Every mbarrier wait is bounded; a
 // wait that gives up raises the library's device error word and the CTA
 // drains its copies and MMAs and frees its tensor memory before returning.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include <atomic>
-#include <mutex>
 #include <utility>
 
-#include "la_common.cuh"
-#include "la_sm100.cuh"
+#include "la_tc_common.cuh"
 
 namespace la {
 
@@ -46,139 +41,6 @@ __device__ unsigned g_tc_error;
 namespace {
 
 using namespace sm100;
-
-constexpr int kGroupHeads = 4;
-constexpr int kRopeTableMax = 1536;  // float2 entries of the per-CTA RoPE table
-
-enum : unsigned { kErrWait = 1u };
-
-// ------------------------------------------------------------------ RoPE
-
-// Per-CTA table of (cos, sin) for every position of the block: T frames x 4
-// pairs (time), then Hh x 6 pairs (height), then W x 6 pairs (width). Angles
-// are formed and reduced to [-pi, pi] in double, then evaluated in float. When
-// the table does not fit in shared memory the angles are evaluated per token
-// instead.
-struct RopeTable {
-  int enabled;
-  int on_the_fly;
-};
-
-__host__ __device__ inline int rope_table_entries(const Rope& r) {
-  return 4 * r.T + 6 * r.Hh + 6 * r.W;
-}
-
-__device__ void build_rope_table(const Rope& r, float2* tab, int tid, int nthreads) {
-  const int total = rope_table_entries(r);
-  for (int i = tid; i < total; i += nthreads) {
-    int pos, j;
-    if (i < 4 * r.T) {
-      pos = r.t_offset + i / 4;
-      j = i % 4;
-    } else if (i < 4 * r.T + 6 * r.Hh) {
-      const int k = i - 4 * r.T;
-      pos = k / 6;
-      j = 4 + k % 6;
-    } else {
-      const int k = i - 4 * r.T - 6 * r.Hh;
-      pos = k / 6;
-      j = 10 + k % 6;
-    }
-    float cs, sn;
-    rope_cos_sin(pos, r.inv_freq[j], cs, sn);
-    tab[i] = make_float2(cs, sn);
-  }
-}
-
-struct TokPos {
-  int t, h, w;  // local frame, row, column of a token
-};
-
-__device__ __forceinline__ TokPos token_pos(const Rope& r, int n) {
-  const int hw = n / r.W;
-  const int t = hw / r.Hh;
-  return {t, hw - t * r.Hh, n - hw * r.W};
-}
-
-// Position of token n + step from that of token n (raster order, step >= 0).
-__device__ __forceinline__ void token_pos_advance(const Rope& r, TokPos& tp, int step) {
-  tp.w += step;
-  while (tp.w >= r.W) {
-    tp.w -= r.W;
-    if (++tp.h == r.Hh) {
-      tp.h = 0;
-      ++tp.t;
-    }
-  }
-}
-
-// RoPE feature-map variants a kernel is compiled for.
-enum RopeMode : int { kNoRope = 0, kRopeTable = 1, kRopeOnTheFly = 2 };
-
-// Segment (0 = time, 1 = height, 2 = width) and index inside it of pair j.
-__host__ __device__ constexpr int pair_axis(int j) { return j < 4 ? 0 : (j < 10 ? 1 : 2); }
-__host__ __device__ constexpr int pair_off(int j) { return j < 4 ? j : (j < 10 ? j - 4 : j - 10); }
-
-// Table offsets of the three segments' rows for token position tp.
-struct RopeBases {
-  int t, h, w;
-};
-__device__ __forceinline__ RopeBases rope_bases(const Rope& r, const TokPos& tp) {
-  return {tp.t * 4, 4 * r.T + tp.h * 6, 4 * r.T + 6 * r.Hh + tp.w * 6};
-}
-
-// Barrier over `threads` threads of named barrier `id` that also ORs `pred`
-// across them: every participant gets the same answer.
-__device__ __forceinline__ bool bar_any(int id, int threads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(threads)
-      : "memory");
-  return r != 0;
-}
-
-__device__ __forceinline__ void unpack8(const uint4& u, float (&x)[8]) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    x[2 * i] = __uint_as_float(w[i] << 16);
-    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
-}
-
-__device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
-  uint4 u;
-  u.x = pack_bf16x2(x[0], x[1]);
-  u.y = pack_bf16x2(x[2], x[3]);
-  u.z = pack_bf16x2(x[4], x[5]);
-  u.w = pack_bf16x2(x[6], x[7]);
-  return u;
-}
-
-// max(x, 0) on packed bf16 pairs: exact.
-__device__ __forceinline__ uint32_t relu_bf16x2(uint32_t v) {
-  uint32_t r;
-  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(0u));
-  return r;
-}
-
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-               "r"(v.z), "r"(v.w)
-               : "memory");
-}
 
 // ============================================================ the kernel
 
@@ -228,83 +90,6 @@ struct LayerArgs {
   int tiles_per_cta;   // apply: 128-token tiles per CTA
   int q_before_wait;   // apply only: Q may be read before the previous grid completes
 };
-
-__device__ __forceinline__ bool spin_flag(const unsigned* flag, volatile int* abort_flag) {
-  if (ld_acquire_gpu(flag) != 0u) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    if (ld_acquire_gpu(flag) != 0u) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
-      atomicOr(&g_tc_error, kErrWait);
-      return false;
-    }
-    __nanosleep(64);
-  }
-}
-
-// Sum of the head group's split partials in split order (+ carry), written to
-// StateOut, by the math threads of the CTA that arrived last. Each thread owns
-// at most kPerThread float4 columns and issues the loads of all of them for 4
-// splits at once before adding, so the combine costs one L2 round trip per 4
-// splits.
-__device__ __forceinline__ void combine_from_global(const Problem& p, int b, int h0, int mt,
-                                                    const float* partials, const StateOut& out) {
-  constexpr int kVec = kStateFloats / 4;                     // 264 float4 per head
-  constexpr int kPerThread = (kGroupHeads * kVec + kMath - 1) / kMath;  // 3
-  const int heads = min(kGroupHeads, p.H - h0);
-  const size_t cidx = static_cast<size_t>(b) * p.H + h0;
-  float4 acc[kPerThread];
-  const float* src[kPerThread];
-  bool own[kPerThread];
-#pragma unroll
-  for (int u = 0; u < kPerThread; ++u) {
-    const int v = mt + u * kMath;
-    own[u] = v < heads * kVec;
-    const int hh = own[u] ? v / kVec : 0, i = own[u] ? (v - hh * kVec) * 4 : 0;
-    src[u] = partials + (cidx + hh) * p.splits * kStateFloats + i;
-    acc[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  }
-  for (int s0 = 0; s0 < p.splits; s0 += 4) {
-    float4 t[kPerThread][4];
-#pragma unroll
-    for (int u = 0; u < kPerThread; ++u)
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (own[u] && s0 + k < p.splits)
-          t[u][k] = __ldcg(reinterpret_cast<const float4*>(src[u] + static_cast<size_t>(s0 + k) * kStateFloats));
-#pragma unroll
-    for (int u = 0; u < kPerThread; ++u)
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (own[u] && s0 + k < p.splits) {
-          acc[u].x += t[u][k].x;
-          acc[u].y += t[u][k].y;
-          acc[u].z += t[u][k].z;
-          acc[u].w += t[u][k].w;
-        }
-  }
-#pragma unroll
-  for (int u = 0; u < kPerThread; ++u) {
-    if (!own[u]) continue;
-    const int v = mt + u * kMath;
-    const int hh = v / kVec, i = (v - hh * kVec) * 4;
-    const size_t bh = cidx + hh;
-    const bool is_s = i < kD * kD;
-    const size_t o = is_s ? bh * kD * kD + i : bh * kD + (i - kD * kD);
-    const float* c = is_s ? out.carry_S : out.carry_z;
-    float4 r = acc[u];
-    if (c != nullptr) {
-      const float4 cv = *reinterpret_cast<const float4*>(c + o);
-      r = make_float4(cv.x + r.x, cv.y + r.y, cv.z + r.z, cv.w + r.w);
-    }
-    float* d1 = is_s ? out.out1_S : out.out1_z;
-    float* d2 = is_s ? out.out2_S : out.out2_z;
-    if (d1 != nullptr) *reinterpret_cast<float4*>(d1 + o) = r;
-    if (d2 != nullptr) *reinterpret_cast<float4*>(d2 + o) = r;
-  }
-}
 
 template <int kRope, int kPh>
 __global__ void __launch_bounds__(kThreadsTc, 1)
@@ -423,7 +208,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       }
       // drain: every load issued must have landed before the CTA exits
       for (int q = max(0, pos - kStages); q < pos; ++q)
-        mbar_wait(&full[q % kStages], (q / kStages) & 1, abort_flag, nullptr, 0);
+        mbar_drain(&full[q % kStages], (q / kStages) & 1, &g_tc_error, kErrWait);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
@@ -473,7 +258,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
         mma_commit(&t_full[w]);
       }
       mma_commit(mma_done);
-      mbar_wait(mma_done, 0, abort_flag, nullptr, 0);
+      mbar_drain(mma_done, 0, &g_tc_error, kErrWait);
     }
   } else {
     // ---------------------------------------------------------- math warps
@@ -597,7 +382,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       }
       named_bar_sync(kBarMath, kMath);
       const bool last = *last_flag != 0;
-      if (last && alive) combine_from_global(p, b, h0, mt, a.partials, a.out);
+      if (last && alive) combine_from_global<kMath>(p, b, h0, mt, a.partials, a.out);
       named_bar_sync(kBarMath, kMath);
       if (kPh == kReduceOnly) {
         if (mt == 0 && last) a.arrive[cidx] = 0u;  // ready for the next call
@@ -609,7 +394,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
             fence_acq_rel_gpu();
             st_release_gpu(&a.ready[cidx], 1u);
           } else {
-            spin_flag(&a.ready[cidx], abort_flag);
+            spin_flag(&a.ready[cidx], abort_flag, &g_tc_error);
           }
         }
         named_bar_sync(kBarMath, kMath);
@@ -664,7 +449,16 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       for (int j = wg; j < nB; j += kApWG) {
         const int pos = nA + j;
         const int s = pos % kStages;
-        bool ok = mbar_wait(&full[s], (pos / kStages) & 1, abort_flag, &g_tc_error, kErrWait);
+        // The stage's previous apply tile (pos - kStages) belonged to another
+        // warpgroup. A parity wait cannot tell phase k from k + 2, so wait for
+        // that tile's release first: then the full phase awaited next is
+        // unambiguous. (Every earlier release precedes the load of this
+        // warpgroup's previous tile, which it has already consumed.)
+        bool ok = true;
+        if (pos - kStages >= nA)
+          ok = mbar_wait(&empty[s], ((pos - kStages) / kStages) & 1, abort_flag, &g_tc_error,
+                         kErrWait);
+        ok = ok && mbar_wait(&full[s], (pos / kStages) & 1, abort_flag, &g_tc_error, kErrWait);
         if (bar_any(kBarWG0 + wg, 128, !ok || *abort_flag)) break;
         const int n0 = (tile_begin + j) * kApT;
         const int n = n0 + row;
@@ -769,64 +563,6 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
 
 // ============================================================== host side
 
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
-cudaError_t g_encode_err = cudaSuccess;
-
-cudaError_t get_encoder() {
-  std::call_once(g_encode_once, [] {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    g_encode_err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-    if (g_encode_err == cudaSuccess && (q != cudaDriverEntryPointSuccess || fn == nullptr))
-      g_encode_err = cudaErrorNotSupported;
-    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  });
-  return g_encode_err;
-}
-
-// [B][N][H*32] bf16 viewed as a 3D tensor; box = 64 dims x rows tokens x 1.
-cudaError_t make_map(CUtensorMap* m, const void* base, const Problem& p, int rows) {
-  cudaError_t e = get_encoder();
-  if (e != cudaSuccess) return e;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p.H) * kD, static_cast<cuuint64_t>(p.N),
-                              static_cast<cuuint64_t>(p.B)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p.H) * kD * 2,
-                                 static_cast<cuuint64_t>(p.N) * p.H * kD * 2};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
-                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
-RopeTable rope_table_for(const Problem& p) {
-  RopeTable rt{};
-  rt.enabled = p.rope.enabled;
-  if (rt.enabled) rt.on_the_fly = rope_table_entries(p.rope) > kRopeTableMax;
-  return rt;
-}
-
-constexpr int kMaxDev = 64;
-bool g_attr_set[9][kMaxDev] = {};
-std::mutex g_attr_mu;
-
-cudaError_t ensure_smem_attr(int which, const void* fn, int bytes) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_attr_mu);
-  if (!g_attr_set[which][dev]) {
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    g_attr_set[which][dev] = true;
-  }
-  return cudaSuccess;
-}
-
 // Launch of layer_tc with programmatic dependent launch (the prologue may
 // overlap the previous kernel in the stream) and, for the fused layer, as a
 // cooperative launch (its CTAs wait on each other, so all must be resident).
@@ -877,10 +613,6 @@ LayerKernel pick_kernel(int mode) {
   return mode == kNoRope ? layer_tc<kNoRope, kPh>
                          : (mode == kRopeTable ? layer_tc<kRopeTable, kPh>
                                                : layer_tc<kRopeOnTheFly, kPh>);
-}
-
-int rope_mode(const RopeTable& rt) {
-  return !rt.enabled ? kNoRope : (rt.on_the_fly ? kRopeOnTheFly : kRopeTable);
 }
 
 // 128-token tiles per CTA when `ctas` CTAs share a head group's tiles.

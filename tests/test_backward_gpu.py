@@ -54,6 +54,10 @@ SMALL = [
     (1, 1, 1, None, 0),             # one token, one head
     (2, 4096, 7, (4, 32, 32), 11),  # several splits per head
     (1, 512, 5, (1, 2, 256), 7),    # a long axis: large angles
+    # 37 head groups: 8 tiles per CTA on both sides, so every stage, TMEM
+    # buffer and barrier of the tensor-core kernels goes through several phases
+    (1, 4096, 148, None, 0),
+    (1, 4096, 148, (4, 32, 32), 5),
 ]
 
 
