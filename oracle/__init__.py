@@ -26,4 +26,6 @@ from .linear_attention import (  # noqa: F401
     to_f64,
     rope_unrotate,
     backward,
+    causal_attention,
+    causal_bruteforce,
 )

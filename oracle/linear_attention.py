@@ -30,6 +30,10 @@ Sources (page title, then section):
 [MJ]    SANA-Video article (mjgaz.cn), section "设计细节": later blocks integrate
         earlier blocks' features through the linear state, earlier blocks never
         see later ones, and each block sums the accumulated KV with its own.
+[SV23t] SANA-Video section 2.3 read at token granularity (the pages' sum over
+        j up to i - 1 with j indexing tokens): query i sees keys j <= i. The
+        query's own token is included, as the block mode includes the block's
+        own state; a token-level block of one token gives exactly this.
 
 The pages lose the formulas of sections 2.1 and 2.3 in extraction. The
 readings taken here:
@@ -275,3 +279,45 @@ def backward(Q, K, V, dO, eps: float, theta: Optional[np.ndarray] = None):
     dK = dkp * (K > 0)
     dV = tokens(np.matmul(heads(phk), dS))                                # phk dS
     return dQ, dK, dV, dS, dz
+
+
+def causal_attention(Q, K, V, eps: float, theta: Optional[np.ndarray] = None,
+                     S0: Optional[np.ndarray] = None, z0: Optional[np.ndarray] = None):
+    """Token-causal ReLU linear attention [SV23t], by its recurrence.
+
+    With the state carried in (S0, z0) (zero when None):
+      S_i = S0 + sum_{j<=i} phi(k_j)^T v_j,   z_i = z0 + sum_{j<=i} ReLU(k_j),
+      O_i = phi(q_i) S_i / (ReLU(q_i) . z_i + eps).
+    The state is advanced one token at a time, in token order. Returns O
+    [B, N, H, D] and the final state (S_N, z_N).
+    """
+    Q, K, V = to_f64(Q), to_f64(K), to_f64(V)
+    B, N, H, D = Q.shape
+    qp, kp = relu(Q), relu(K)
+    phq = qp if theta is None else rope_rotate(qp, theta)
+    phk = kp if theta is None else rope_rotate(kp, theta)
+    S = np.zeros((B, H, D, D)) if S0 is None else np.array(S0, dtype=np.float64)
+    z = np.zeros((B, H, D)) if z0 is None else np.array(z0, dtype=np.float64)
+    O = np.empty((B, N, H, D))
+    for n in range(N):
+        S = S + phk[:, n, :, :, None] * V[:, n, :, None, :]
+        z = z + kp[:, n]
+        num = np.einsum("bhd,bhde->bhe", phq[:, n], S)
+        den = np.einsum("bhd,bhd->bh", qp[:, n], z) + float(eps)
+        O[:, n] = num / den[..., None]
+    return O, S, z
+
+
+def causal_bruteforce(Q, K, V, eps: float, theta: Optional[np.ndarray] = None) -> np.ndarray:
+    """The causal quadratic form: O_i = sum_{j<=i} (phi(q_i) . phi(k_j)) v_j /
+    (sum_{j<=i} ReLU(q_i) . ReLU(k_j) + eps). Tiny inputs only."""
+    Q, K, V = to_f64(Q), to_f64(K), to_f64(V)
+    N = Q.shape[1]
+    qp, kp = relu(Q), relu(K)
+    phq = qp if theta is None else rope_rotate(qp, theta)
+    phk = kp if theta is None else rope_rotate(kp, theta)
+    seen = np.tril(np.ones((N, N)))                          # [i, j]: j <= i
+    weights = np.einsum("bihd,bjhd->bhij", phq, phk) * seen
+    den = (np.einsum("bihd,bjhd->bhij", qp, kp) * seen).sum(axis=-1) + float(eps)
+    num = np.einsum("bhij,bjhe->bhie", weights, V)
+    return (num / den[..., None]).transpose(0, 2, 1, 3)

@@ -368,3 +368,76 @@ def test_backward_negative_inputs_get_zero_gradient():
     dQ, dK, dV, _, _ = orc.backward(Q, K, V, _rand(V.shape, 321), 1e-3)
     assert np.all(dQ[0, :4] == 0) and np.all(dK[0, :4] == 0)
     assert np.all(dV[0, :4] == 0)  # an all-negative key carries no value
+
+
+# --------------------------------------------------------------------------
+# Token-causal attention (a query sees the keys up to and including its own
+# token)
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_causal_recurrence_equals_masked_quadratic_form(rope):
+    T, Hh, W = 2, 3, 5
+    N = T * Hh * W
+    Q, K, V = _qkv(2, N, 3, 71)
+    th = orc.rope_angles(T, Hh, W, 2) if rope else None
+    O, S, z = orc.causal_attention(Q, K, V, 1e-6, th)
+    np.testing.assert_allclose(O, orc.causal_bruteforce(Q, K, V, 1e-6, th), rtol=1e-12,
+                               atol=1e-14)
+    # the final state is the whole sequence's state
+    S_ref, z_ref = orc.state_reduce(K, V, th)
+    np.testing.assert_allclose(S, S_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(z, z_ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_causal_last_token_is_noncausal_and_first_token_closed_form(rope):
+    T, Hh, W = 3, 2, 4
+    N = T * Hh * W
+    Q, K, V = _qkv(1, N, 2, 73)
+    th = orc.rope_angles(T, Hh, W, 0) if rope else None
+    O, _, _ = orc.causal_attention(Q, K, V, 1e-6, th)
+    full = orc.attention(Q, K, V, 1e-6, th)
+    np.testing.assert_allclose(O[:, -1], full[:, -1], rtol=1e-12, atol=1e-14)
+    # token 0 sees only itself
+    qp, kp = np.maximum(Q[:, 0], 0), np.maximum(K[:, 0], 0)
+    phq = qp if th is None else orc.rope_rotate(qp[:, None], th[:1])[:, 0]
+    phk = kp if th is None else orc.rope_rotate(kp[:, None], th[:1])[:, 0]
+    w = (phq * phk).sum(-1)
+    den = (qp * kp).sum(-1) + 1e-6
+    np.testing.assert_allclose(O[:, 0], (w / den)[..., None] * V[:, 0], rtol=1e-12, atol=1e-14)
+
+
+def test_causal_prefix_and_carry_compose():
+    # causality: the first m outputs do not depend on later tokens; streaming:
+    # running the second part from the first part's final state continues the
+    # sequence exactly
+    Q, K, V = _qkv(2, 40, 3, 75)
+    Q2, K2, V2 = Q.copy(), K.copy(), V.copy()
+    Q2[:, 25:] += 5.0
+    K2[:, 25:] *= -2.0
+    V2[:, 25:] = 7.0
+    a, _, _ = orc.causal_attention(Q, K, V, 1e-6)
+    b, _, _ = orc.causal_attention(Q2, K2, V2, 1e-6)
+    np.testing.assert_array_equal(a[:, :25], b[:, :25])
+    first, S1, z1 = orc.causal_attention(Q[:, :17], K[:, :17], V[:, :17], 1e-6)
+    rest, S2, z2 = orc.causal_attention(Q[:, 17:], K[:, 17:], V[:, 17:], 1e-6, None, S1, z1)
+    np.testing.assert_allclose(np.concatenate([first, rest], axis=1), a, rtol=1e-12, atol=1e-14)
+    _, S_all, z_all = orc.causal_attention(Q, K, V, 1e-6)
+    np.testing.assert_allclose(S2, S_all, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(z2, z_all, rtol=1e-12, atol=1e-12)
+
+
+def test_causal_is_block_causal_with_one_token_blocks():
+    # the block-causal mode with blocks of one token, each applied once with
+    # update = 1, is token-causal attention
+    T, Hh, W = 4, 1, 1
+    Q, K, V = _qkv(1, T, 2, 77)
+    th = orc.rope_angles(T, Hh, W, 0)
+    O, _, _ = orc.causal_attention(Q, K, V, 1e-6, th)
+    S = np.zeros((1, 2, D, D))
+    z = np.zeros((1, 2, D))
+    for t in range(T):
+        o, S, z = orc.block_causal_step(Q[:, t:t + 1], K[:, t:t + 1], V[:, t:t + 1], S, z, 1,
+                                        1e-6, th[t:t + 1])
+        np.testing.assert_allclose(o[:, 0], O[:, t], rtol=1e-12, atol=1e-14)
