@@ -173,6 +173,25 @@ la_status la_attention_backward(const la_shape* shape, const void* Q,
                                 void* dK, void* dV, float* dS, float* dz,
                                 void* ws, size_t ws_bytes, la_stream stream);
 
+/* Token-causal attention: query n sees keys 0..n (SANA-Video section 2.3
+ * read at token granularity; the block-causal mode with blocks of one token).
+ * With the carried state (S0, z0) = (S_carry, z_carry), or zero when both
+ * are NULL:
+ *   S_n = S0 + sum_{j<=n} phi(k_j)^T v_j,   z_n = z0 + sum_{j<=n} ReLU(k_j),
+ *   O_n = phi(q_n) S_n / (ReLU(q_n) . z_n + eps).
+ * update = 1 (needs the carry): afterwards the carry holds S_N, z_N, so a
+ * sequence can be fed in consecutive calls (prefill, then one token at a
+ * time); update = 0 leaves it unchanged. Q, K, V: [B,N,H,D] io_dtype (read);
+ * O: [B,N,H,D] io_dtype (written); carry [B,H,D,D] / [B,H,D] float32. ws: as
+ * for la_attention (same size). Two launches: the state reduce leaves each
+ * token split's partial state in the workspace; the causal kernel starts
+ * each split from the carry plus the earlier splits (summed in split order)
+ * and walks its tokens in chunks of 32 on CUDA cores. Deterministic. */
+la_status la_causal_attention(const la_shape* shape, const void* Q,
+                              const void* K, const void* V, float* S_carry,
+                              float* z_carry, void* O, int update, void* ws,
+                              size_t ws_bytes, la_stream stream);
+
 /* Reset of the KV cache at the start of a video (SANA-Video section 4: the
  * cache starts empty): S[B,H,D,D] = 0, z[B,H,D] = 0 on `stream`. */
 la_status la_state_reset(float* S, float* z, int B, int H, int D,

@@ -69,6 +69,8 @@ _lib.la_block_causal_step.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _vp, _i
 _lib.la_block_causal_step.restype = _i
 _lib.la_attention_backward.argtypes = [_shape_p] + [_vp] * 11 + [_vp, _sz, _vp]
 _lib.la_attention_backward.restype = _i
+_lib.la_causal_attention.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]
+_lib.la_causal_attention.restype = _i
 _lib.la_state_reset.argtypes = [_vp, _vp, _i, _i, _i, _vp]
 _lib.la_state_reset.restype = _i
 _lib.la_status_string.argtypes = [_i]
@@ -163,6 +165,15 @@ def la_attention_backward(shape: LaShape, Q, K, V, S, z, dO, dQ, dK, dV, dS, dz,
            "la_attention_backward")
 
 
+def la_causal_attention(shape: LaShape, Q, K, V, S_carry, z_carry, O, update: int, ws,
+                        stream=None) -> None:
+    """Token-causal attention; the carry (S_carry, z_carry) may be None when update = 0."""
+    _check(_lib.la_causal_attention(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V),
+                                    _ptr(S_carry), _ptr(z_carry), _ptr(O), int(update),
+                                    _ptr(ws), _nbytes(ws), _stream(stream)),
+           "la_causal_attention")
+
+
 def la_state_reset(S, z, B: int, H: int, D: int = HEAD_DIM, stream=None) -> None:
     _check(_lib.la_state_reset(_ptr(S), _ptr(z), int(B), int(H), int(D), _stream(stream)),
            "la_state_reset")
@@ -237,3 +248,14 @@ def attention_backward(Q, K, V, dO, S=None, z=None, eps: float = 1e-6, rope_grid
     la_attention_backward(shape, Q, K, V, S, z, dO, dQ, dK, dV, dS, dz,
                           workspace(shape, Q.device), stream)
     return dQ, dK, dV, dS, dz
+
+
+def causal_attention(Q, K, V, S_carry=None, z_carry=None, update: int = 0, eps: float = 1e-6,
+                     rope_grid=None, t_offset: int = 0, rope_base: float = 10000.0, stream=None):
+    """O of token-causal ReLU linear attention for [B, N, H, 32] CUDA tensors."""
+    shape = shape_for(Q, eps, rope_grid, t_offset, rope_base)
+    import torch
+    O = torch.empty_like(Q)
+    la_causal_attention(shape, Q, K, V, S_carry, z_carry, O, update,
+                        workspace(shape, Q.device), stream)
+    return O

@@ -392,6 +392,46 @@ la_status la_attention_backward(const la_shape* shape, const void* Q, const void
   return LA_OK;
 }
 
+la_status la_causal_attention(const la_shape* shape, const void* Q, const void* K,
+                              const void* V, float* S_carry, float* z_carry, void* O, int update,
+                              void* ws, size_t ws_bytes, la_stream stream) {
+  Problem p;
+  LA_TRY(make_problem(shape, p));
+  if (update < 0 || update > 1) return fail(LA_ERR_INVALID_ARG, "update=%d (0 or 1)", update);
+  if ((S_carry == nullptr) != (z_carry == nullptr))
+    return fail(LA_ERR_INVALID_ARG, "S_carry and z_carry must both be given or both be NULL");
+  if (update == 1 && S_carry == nullptr)
+    return fail(LA_ERR_INVALID_ARG, "update=1 needs S_carry and z_carry");
+  const bool any_state = p.B > 0 && p.H > 0;
+  const bool any_input = any_state && p.N > 0;
+  LA_TRY(check_ptr(Q, "Q", any_input));
+  LA_TRY(check_ptr(K, "K", any_input));
+  LA_TRY(check_ptr(V, "V", any_input));
+  LA_TRY(check_ptr(O, "O", any_input));
+  LA_TRY(check_ptr(S_carry, "S_carry", any_state && S_carry != nullptr));
+  LA_TRY(check_ptr(z_carry, "z_carry", any_state && z_carry != nullptr));
+  LA_TRY(check_ws(p, ws, ws_bytes));
+  const size_t nb = io_bytes(p);
+  if (overlap(O, nb, Q, nb) || overlap(O, nb, K, nb) || overlap(O, nb, V, nb) ||
+      overlap(O, nb, ws, ws_bytes) || overlap(O, nb, S_carry, s_bytes(p)) ||
+      overlap(O, nb, z_carry, z_bytes(p)) || overlap(S_carry, s_bytes(p), ws, ws_bytes) ||
+      overlap(z_carry, z_bytes(p), ws, ws_bytes) ||
+      overlap(S_carry, s_bytes(p), z_carry, z_bytes(p)))
+    return fail(LA_ERR_INVALID_ARG, "O, the carry and the workspace must not overlap");
+  if (!any_state) return LA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const WsLayout L = workspace_layout(p);
+  // the splits' partial states only: no combine
+  LA_TRY(run_reduce(p, K, V, w, StateOut{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr},
+                    st));
+  const cudaError_t e =
+      launch_causal(p, Q, K, V, reinterpret_cast<const float*>(w + L.partials), S_carry, z_carry,
+                    update, reinterpret_cast<unsigned*>(w + L.counters), O, st);
+  if (e != cudaSuccess) return cuda_fail(e, "causal attention");
+  return LA_OK;
+}
+
 la_status la_state_reset(float* S, float* z, int B, int H, int D, la_stream stream) {
   if (B < 0 || H < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d", B, H);
   if (D != kD) return fail(LA_ERR_UNSUPPORTED, "head width D=%d (only 32 is built)", D);

@@ -87,6 +87,11 @@ __device__ __forceinline__ void finish_reduce(const Problem& p, int b, int h0, i
   }
   __syncthreads();
   if (!s_last) return;
+  if (out.out1_S == nullptr && out.out1_z == nullptr && out.out2_S == nullptr &&
+      out.out2_z == nullptr) {  // partials only (the token-causal pass reads them)
+    if (threadIdx.x == 0) counters[static_cast<size_t>(b) * p.H + h0] = 0u;
+    return;
+  }
   __threadfence();
   // Each thread sums float4 columns of the partials; the loads of up to 8
   // splits are issued together and then added in split order.

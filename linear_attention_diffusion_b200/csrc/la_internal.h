@@ -106,6 +106,14 @@ cudaError_t launch_backward_q_simt(const Problem& p, const void* Q, const void* 
 cudaError_t launch_backward_kv_simt(const Problem& p, const void* K, const void* V,
                                     const float* dS, const float* dz, void* dK, void* dV,
                                     cudaStream_t s);
+// Token-causal attention (la_causal.cu): `partials` holds every token
+// split's partial state (the state reduce with no outputs requested); each
+// split starts from the carry plus the earlier splits' partials. update = 1
+// folds the whole sequence into the carry (read-before-write is ordered by
+// `counters`, which the kernel leaves zero).
+cudaError_t launch_causal(const Problem& p, const void* Q, const void* K, const void* V,
+                          const float* partials, float* S_carry, float* z_carry, int update,
+                          unsigned* counters, void* O, cudaStream_t s);
 // Device error words of the tensor-core kernels (bounded waits that gave up):
 // the forward's (la_tc.cu) and the backward's (la_backward_tc.cu).
 cudaError_t read_device_error(unsigned* code, bool reset);

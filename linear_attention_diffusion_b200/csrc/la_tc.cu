@@ -382,7 +382,9 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       }
       named_bar_sync(kBarMath, kMath);
       const bool last = *last_flag != 0;
-      if (last && alive) combine_from_global<kMath>(p, b, h0, mt, a.partials, a.out);
+      const bool wanted = a.out.out1_S != nullptr || a.out.out1_z != nullptr ||
+                          a.out.out2_S != nullptr || a.out.out2_z != nullptr;
+      if (last && alive && wanted) combine_from_global<kMath>(p, b, h0, mt, a.partials, a.out);
       named_bar_sync(kBarMath, kMath);
       if (kPh == kReduceOnly) {
         if (mt == 0 && last) a.arrive[cidx] = 0u;  // ready for the next call

@@ -175,3 +175,48 @@ def check_backward(got, ref, mags, io, Q, K, what=""):
     for name, g, x in (("dQ", got[0], Q), ("dK", got[1], K)):
         masked = orc.to_f64(x) <= 0
         assert (orc.to_f64(g)[masked] == 0).all(), f"{what} {name}: non-zero where the input <= 0"
+
+
+# ---------------------------------------------------------------------------
+# Token-causal attention.
+#
+# With M_i = |phi(q_i)| (|S0| + sum_{j<=i} |phi(k_j)|^T |v_j|) / den_i (every
+# term of the numerator in absolute value):
+#     |O_gpu - O_ref| <= out_round * |O_ref| + tol_c * M_i
+# tol_c = 1e-4 for float32 arithmetic on exact operands; 2^-8 when the split
+# partial states come from the tensor-core reduce with RoPE (the rotated key
+# feature is rounded to bf16 there, 2^-9 per term).
+
+
+def causal_magnitude(Q, K, V, eps, theta, S0=None, z0=None):
+    """M_i above, by the same token-order recurrence as the oracle."""
+    qf, kf, vf = orc.to_f64(Q), orc.to_f64(K), orc.to_f64(V)
+    B, N, H, D_ = qf.shape
+    phq = np.abs(orc.feature_map(qf, theta))
+    phk = np.abs(orc.feature_map(kf, theta))
+    qp, kp = orc.relu(qf), orc.relu(kf)
+    A = np.zeros((B, H, D_, D_)) if S0 is None else np.abs(np.asarray(S0, np.float64))
+    z = np.zeros((B, H, D_)) if z0 is None else np.asarray(z0, np.float64)
+    av = np.abs(vf)
+    M = np.empty((B, N, H, D_))
+    for n in range(N):
+        A = A + phk[:, n, :, :, None] * av[:, n, :, None, :]
+        z = z + kp[:, n]
+        den = np.einsum("bhd,bhd->bh", qp[:, n], z) + eps
+        M[:, n] = np.einsum("bhd,bhde->bhe", phq[:, n], A) / den[..., None]
+    return M
+
+
+def check_causal(O_gpu, O_ref, M, io, tol, what=""):
+    O_gpu = orc.to_f64(O_gpu)
+    assert np.isfinite(O_gpu).all(), f"{what}: non-finite output"
+    rtol, atol = NS_BF16 if io == "bf16" else NS_F32
+    err = np.abs(O_gpu - O_ref)
+    ns = atol + rtol * np.abs(O_ref)
+    assert not (err > ns).any(), (f"{what}: {(err > ns).sum()} elements outside the "
+                                  f"north-star tolerance; max err {err.max():.3g}")
+    out_round = 2.0 ** -8 if io == "bf16" else 1e-6
+    bound = out_round * np.abs(O_ref) + tol * M + 1e-30
+    bad = err > bound
+    assert not bad.any(), (f"{what}: {bad.sum()} elements outside the derived bound; worst "
+                           f"ratio {float((err / bound).max()):.3g}")
