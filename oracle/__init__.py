@@ -29,3 +29,4 @@ from .linear_attention import (  # noqa: F401
     causal_attention,
     causal_bruteforce,
 )
+from .temporal_conv import temporal_conv  # noqa: F401,E402

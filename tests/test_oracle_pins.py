@@ -441,3 +441,58 @@ def test_causal_is_block_causal_with_one_token_blocks():
         o, S, z = orc.block_causal_step(Q[:, t:t + 1], K[:, t:t + 1], V[:, t:t + 1], S, z, 1,
                                         1e-6, th[t:t + 1])
         np.testing.assert_allclose(o[:, 0], O[:, t], rtol=1e-12, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Temporal depth-wise convolution with the block-causal conv cache
+
+
+def _conv_inputs(B, T, Hh, W, C, seed):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, T, Hh, W, C)), rng.standard_normal((C, 3)),
+            rng.standard_normal(C))
+
+
+def test_temporal_conv_is_a_zero_padded_correlation_plus_shortcut():
+    from scipy.ndimage import correlate1d
+    x, w, b = _conv_inputs(2, 7, 3, 4, 5, 81)
+    y, f = orc.temporal_conv(x, w, b)
+    ref = np.empty_like(x)
+    for c in range(x.shape[-1]):
+        ref[..., c] = correlate1d(x[..., c], w[c], axis=1, mode="constant", cval=0.0)
+    np.testing.assert_allclose(y, x + b + ref, rtol=1e-13, atol=1e-13)
+    np.testing.assert_array_equal(f, x[:, -1])
+
+
+def test_temporal_conv_impulse_response_fixes_tap_order():
+    # a single non-zero frame t0: frame t0 - 1 sees it as its next frame (tap
+    # 2), frame t0 + 1 as its previous frame (tap 0)
+    B, T, Hh, W, C = 1, 6, 1, 1, 3
+    x = np.zeros((B, T, Hh, W, C))
+    x[0, 3, 0, 0] = [1.0, 2.0, -1.0]
+    w = np.array([[0.5, 0.25, 0.125], [1.0, 2.0, 3.0], [-1.0, 0.0, 1.0]])
+    y, _ = orc.temporal_conv(x, w)
+    v = x[0, 3, 0, 0]
+    np.testing.assert_allclose(y[0, 2, 0, 0], w[:, 2] * v)
+    np.testing.assert_allclose(y[0, 3, 0, 0], v + w[:, 1] * v)
+    np.testing.assert_allclose(y[0, 4, 0, 0], w[:, 0] * v)
+    assert not y[0, [0, 1, 5]].any()
+
+
+def test_temporal_conv_cache_carries_the_previous_block():
+    # block 2 run with block 1's cache equals block 2 alone plus the previous
+    # frame's contribution at its first frame; the cache is the last frame
+    x, w, b = _conv_inputs(2, 9, 2, 3, 4, 83)
+    x1, x2 = x[:, :5], x[:, 5:]
+    y1, f1 = orc.temporal_conv(x1, w, b)
+    y2, f2 = orc.temporal_conv(x2, w, b, f1)
+    alone, _ = orc.temporal_conv(x2, w, b)
+    np.testing.assert_array_equal(f1, x[:, 4])
+    np.testing.assert_array_equal(f2, x[:, 8])
+    np.testing.assert_allclose(y2[:, 1:], alone[:, 1:], rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(y2[:, 0], alone[:, 0] + w[:, 0] * x[:, 4], rtol=1e-13, atol=1e-13)
+    # and block 1's last frame does not see block 2 (block-causal), unlike a
+    # whole-clip convolution
+    whole, _ = orc.temporal_conv(x, w, b)
+    np.testing.assert_allclose(y1[:, 4] + w[:, 2] * x[:, 5], whole[:, 4], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(y2, whole[:, 5:], rtol=1e-13, atol=1e-13)
