@@ -2,14 +2,16 @@
 """Benchmark of one ReLU linear-attention layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl la|reference]
-                    [--workload NAME] [--op layer|backward]
+                    [--workload NAME] [--op layer|backward|causal]
 
 A step is one pass of the layer's hot path over one batch of synthetic input:
 the state reduce (S = sum phi(K)^T V, z = sum ReLU(K)) and the apply
 (O = phi(Q) S / (ReLU(Q).z + eps)) of the default workload, or a whole
 block-causal video (reset, 12 blocks x 5 calls) for the LongSANA workload.
 With --op backward a step is the layer's backward instead (dQ, dK, dV and the
-state gradients from Q, K, V, the state and dO; non-causal workloads).
+state gradients from Q, K, V, the state and dO); with --op causal it is
+token-causal attention over the workload's tokens (query n sees keys 0..n).
+Both cover the non-causal workloads' shapes.
 Rank 0 prints one JSON line. Multi-GPU runs are weak-scaled: every rank runs
 its own copy of the workload (heads and batches are independent), with no
 collective on the data path; the time is the max over ranks.
@@ -41,6 +43,11 @@ import workloads as wl  # noqa: E402
 
 METRIC = "linear-attn tokens/s per layer at 1 B200; achieved HBM GB/s vs peak"
 METRIC_BWD = "linear-attn backward tokens/s per layer at 1 B200; achieved HBM GB/s vs peak"
+METRIC_CAUSAL = ("token-causal linear-attn tokens/s per layer at 1 B200; "
+                 "achieved HBM GB/s vs peak")
+METRICS = {"layer": METRIC, "backward": METRIC_BWD, "causal": METRIC_CAUSAL}
+OP_CONFIG = {"layer": {}, "backward": {"op": "backward (dQ, dK, dV, dS, dz)"},
+             "causal": {"op": "token-causal (query n sees keys 0..n), no carry"}}
 DEFAULT_WORKLOAD = "sana1.6b_1024px"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
@@ -84,9 +91,11 @@ def layer_bytes(w, io_bytes=2):
     """Algorithmic HBM bytes of one layer: read Q, K, V, write O, write the state."""
     th = w.B * w.N * w.H
     state = w.B * w.H * (D * D + D) * 4
-    # backward: read Q, K, V, dO and (S, z); write dQ, dK, dV and (dS, dz)
+    # backward: read Q, K, V, dO and (S, z); write dQ, dK, dV and (dS, dz).
+    # causal: the minimum, Q, K, V read once and O written once.
     return {"attention_layer": 4 * th * D * io_bytes + state,
-            "attention_backward": 7 * th * D * io_bytes + 2 * state}
+            "attention_backward": 7 * th * D * io_bytes + 2 * state,
+            "causal_attention": 4 * th * D * io_bytes}
 
 
 def peaks():
@@ -209,6 +218,8 @@ def oracle_sample(w, seconds, max_reps=None, op="layer"):
     def run(h_sub, Q, K, V, th):
         if op == "backward":
             orc.backward(Q, K, V, dOa[:, :, :h_sub], w.eps, th)
+        elif op == "causal":
+            orc.causal_attention(Q, K, V, w.eps, th)
         elif w.block_causal:
             Sc = np.zeros((w.B, h_sub, D, D))
             zc = np.zeros((w.B, h_sub, D))
@@ -240,7 +251,7 @@ def oracle_sample(w, seconds, max_reps=None, op="layer"):
                 f"{reps} calls in {el:.1f} s, scaled to {w.H} heads x {calls} calls per video")
     else:
         tokens_per_s = w.B * w.N / full_call
-        what = "backward" if op == "backward" else "attention"
+        what = {"backward": "backward", "causal": "causal_attention"}.get(op, "attention")
         desc = (f"oracle {what} on {h_sub} of {w.H} heads (B={w.B}, N={w.N}), {reps} calls "
                 f"in {el:.1f} s, scaled to {w.H} heads")
     return tokens_per_s, desc, cpu_cores_used(), per_call, h_sub
@@ -303,7 +314,19 @@ def run_la(args, w, rank, world, local_rank):
     shapes = [ctypes.byref(s) for s in keep]
     status = []
 
-    if bwd:
+    if args.op == "causal":
+        launches_per_step = 2  # split states, then the causal pass
+
+        def step(i, evs=None):
+            q, k, v, o = ptrs[i % n_sets]
+            if evs is not None:
+                evs[0].record(stream)
+            status.append(lib.la_causal_attention(shapes[0], q, k, v, None, None, o, 0, ws_p,
+                                                  ws_n, sp))
+            if evs is not None:
+                evs[1].record(stream)
+        kernel_names = ("causal_attention",)
+    elif bwd:
         launches_per_step = 2  # query side, then key side
 
         def step(i, evs=None):
@@ -428,6 +451,8 @@ def run_la(args, w, rank, world, local_rank):
         e2e = None
     elif bwd:
         e2e = run_e2e_backward(args, w, dev, stream, la, rank)
+    elif args.op == "causal":
+        e2e = run_e2e(args, w, dev, stream, la, rank, causal=True)
     else:
         e2e = run_e2e(args, w, dev, stream, la, rank)
     clocks = sampler.summary(t0, t1)
@@ -438,7 +463,7 @@ def run_la(args, w, rank, world, local_rank):
             "chunk": chunk, "per_set_bytes": per_set}
 
 
-def run_e2e(args, w, dev, stream, la, rank):
+def run_e2e(args, w, dev, stream, la, rank, causal=False):
     """Same metric through la_attention / la_block_causal_step with pinned host
     inputs copied in and the output copied out inside the timed region."""
     import torch
@@ -460,7 +485,9 @@ def run_e2e(args, w, dev, stream, la, rank):
         dq.copy_(hq, non_blocking=True)
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
-        if w.block_causal:
+        if causal:
+            la.la_causal_attention(shape, dq, dk, dv, None, None, do, 0, ws, stream)
+        elif w.block_causal:
             la.la_block_causal_step(shape, dq, dk, dv, S, z, do, update, ws, stream)
         else:
             la.la_attention(shape, dq, dk, dv, S, z, do, ws, stream)
@@ -567,15 +594,15 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--soak", type=float, default=1.0)
-    ap.add_argument("--op", choices=["layer", "backward"], default="layer")
+    ap.add_argument("--op", choices=["layer", "backward", "causal"], default="layer")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
-    if args.op == "backward" and w.block_causal:
-        ap.error("--op backward covers the non-causal workloads")
+    if args.op != "layer" and w.block_causal:
+        ap.error(f"--op {args.op} covers the non-causal workloads")
     if args.steps is None:
         per_step_us = {"sana0.6b_512px": 10, "sana1.6b_1024px": 30, "sana1.6b_4k": 120,
                        "sanavideo_480p": 250, "longsana_block_causal": 12000}[w.name]
-        if args.op == "backward":
+        if args.op != "layer":
             per_step_us *= 10
         args.steps = max(10, int(0.5e6 / per_step_us))
     args.warmup = max(args.warmup, 3)
@@ -635,14 +662,14 @@ def main():
         "d2h_bytes_per_step": e["d2h_bytes_per_step"], "steps": e["steps"],
         "ms_per_step": round(e["ms_per_step"], 4),
         "api": ("la_attention_backward" if args.op == "backward" else
+                "la_causal_attention" if args.op == "causal" else
                 "la_block_causal_step" if w.block_causal else "la_attention")}
-    bwd = args.op == "backward"
-    out = {"metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+    out = {"metric": METRICS[args.op], "value": value, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
            "latency_us": ms_step * 1e3, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), bf16)",
            "config": dict(config_of(w, world, r["n_sets"], r["per_set_bytes"]),
-                          **({"op": "backward (dQ, dK, dV, dS, dz)"} if bwd else {})),
+                          **OP_CONFIG[args.op]),
            "roofline": roofline, "e2e": e2e,
            "gpu_launches": r["launches_per_step"] * args.steps,
            "clocks": r["clocks"], "graph_chunk_steps": r["chunk"], "soak_s": args.soak}
@@ -671,6 +698,8 @@ def main_reference(args, w, rank, world):
     def call():
         if bwd:
             orc.backward(Q, K, V, dO, w.eps, th)
+        elif args.op == "causal":
+            orc.causal_attention(Q, K, V, w.eps, th)
         elif w.block_causal:
             orc.block_causal_step(Q, K, V, np.zeros((w.B, h_sub, D, D)),
                                   np.zeros((w.B, h_sub, D)), 1, w.eps, th)
@@ -694,14 +723,13 @@ def main_reference(args, w, rank, world):
     else:
         value = w.B * w.N / full_call
         ms_step = full_call * 1e3
-        what = "backward" if bwd else "attention"
+        what = {"backward": "backward", "causal": "causal_attention"}.get(args.op, "attention")
         sample = f"each step: oracle {what} on {h_sub} of {w.H} heads; scaled to {w.H} heads"
-    out = {"impl": "reference", "metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": "tokens/s",
+    out = {"impl": "reference", "metric": METRICS[args.op], "value": value, "unit": "tokens/s",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic (seeded N(0,1), bf16 inputs read exactly)",
-           "config": dict(config_of(w, world),
-                          **({"op": "backward (dQ, dK, dV, dS, dz)"} if bwd else {})),
+           "config": dict(config_of(w, world), **OP_CONFIG[args.op]),
            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,

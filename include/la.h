@@ -192,6 +192,31 @@ la_status la_causal_attention(const la_shape* shape, const void* Q,
                               float* z_carry, void* O, int update, void* ws,
                               size_t ws_bytes, la_stream stream);
 
+/* Shape of a channels-last video feature map [B][T][Hh][W][C] (the DiT's
+ * tokens [B][N][C] with N = T*Hh*W in raster order). C must be a multiple
+ * of 8. */
+typedef struct {
+  int B, T, Hh, W, C;
+  int io_dtype; /* LA_IO_BF16 or LA_IO_F32 */
+} la_conv_shape;
+
+/* Temporal depth-wise convolution of the spatial-temporal Mix-FFN, entered
+ * through a shortcut, with the block-causal conv cache f (SANA-Video, Stage 2
+ * and section 4: the conv cache is the last frame of the temporal
+ * convolution, the third part of the KV cache):
+ *   y[t] = x[t] + bias + w[c][0] x[t-1] + w[c][1] x[t] + w[c][2] x[t+1]
+ * per channel c, with x[-1] = f_in (the previous block's last frame; zero
+ * when f_in is NULL, as for a whole clip or a first block) and x[T] = 0
+ * (later blocks are never seen). f_out (may be NULL) receives x[T-1], the
+ * cache for the next block. x, y: [B][T][Hh][W][C] io_dtype; f_in, f_out:
+ * [B][Hh][W][C] io_dtype; w: [C][3] float32; bias: [C] float32 or NULL. All
+ * device pointers, 16-byte aligned. y may be x (in place) and f_out may be
+ * f_in; no other overlap is allowed. Float32 arithmetic, one rounding of y.
+ * T = 0 leaves y empty and sets f_out to f_in (or zero). One launch. */
+la_status la_temporal_conv(const la_conv_shape* shape, const void* x,
+                           const float* w, const float* bias, const void* f_in,
+                           void* f_out, void* y, la_stream stream);
+
 /* Reset of the KV cache at the start of a video (SANA-Video section 4: the
  * cache starts empty): S[B,H,D,D] = 0, z[B,H,D] = 0 on `stream`. */
 la_status la_state_reset(float* S, float* z, int B, int H, int D,

@@ -43,6 +43,15 @@ class LaShape(ctypes.Structure):
     ]
 
 
+class LaConvShape(ctypes.Structure):
+    """Mirror of ``la_conv_shape`` in include/la.h."""
+
+    _fields_ = [
+        ("B", ctypes.c_int), ("T", ctypes.c_int), ("Hh", ctypes.c_int), ("W", ctypes.c_int),
+        ("C", ctypes.c_int), ("io_dtype", ctypes.c_int),
+    ]
+
+
 class LaError(RuntimeError):
     def __init__(self, status: int, func: str):
         self.status = status
@@ -71,6 +80,8 @@ _lib.la_attention_backward.argtypes = [_shape_p] + [_vp] * 11 + [_vp, _sz, _vp]
 _lib.la_attention_backward.restype = _i
 _lib.la_causal_attention.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]
 _lib.la_causal_attention.restype = _i
+_lib.la_temporal_conv.argtypes = [ctypes.POINTER(LaConvShape), _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.la_temporal_conv.restype = _i
 _lib.la_state_reset.argtypes = [_vp, _vp, _i, _i, _i, _vp]
 _lib.la_state_reset.restype = _i
 _lib.la_status_string.argtypes = [_i]
@@ -174,6 +185,17 @@ def la_causal_attention(shape: LaShape, Q, K, V, S_carry, z_carry, O, update: in
            "la_causal_attention")
 
 
+def make_conv_shape(B: int, T: int, Hh: int, W: int, C: int, io_dtype: str = "bf16") -> LaConvShape:
+    return LaConvShape(int(B), int(T), int(Hh), int(W), int(C),
+                       LA_IO_BF16 if io_dtype == "bf16" else LA_IO_F32)
+
+
+def la_temporal_conv(shape: LaConvShape, x, w, bias, f_in, f_out, y, stream=None) -> None:
+    """Temporal depth-wise conv with shortcut and conv cache (see include/la.h)."""
+    _check(_lib.la_temporal_conv(ctypes.byref(shape), _ptr(x), _ptr(w), _ptr(bias), _ptr(f_in),
+                                 _ptr(f_out), _ptr(y), _stream(stream)), "la_temporal_conv")
+
+
 def la_state_reset(S, z, B: int, H: int, D: int = HEAD_DIM, stream=None) -> None:
     _check(_lib.la_state_reset(_ptr(S), _ptr(z), int(B), int(H), int(D), _stream(stream)),
            "la_state_reset")
@@ -259,3 +281,14 @@ def causal_attention(Q, K, V, S_carry=None, z_carry=None, update: int = 0, eps: 
     la_causal_attention(shape, Q, K, V, S_carry, z_carry, O, update,
                         workspace(shape, Q.device), stream)
     return O
+
+
+def temporal_conv(x, w, bias=None, f_in=None, want_cache: bool = False, stream=None):
+    """y (and the next conv cache when ``want_cache``) for x [B, T, Hh, W, C] CUDA tensors."""
+    import torch
+    B, T, Hh, W, C = x.shape
+    shape = make_conv_shape(B, T, Hh, W, C, "bf16" if x.dtype == torch.bfloat16 else "f32")
+    y = torch.empty_like(x)
+    f_out = torch.empty((B, Hh, W, C), dtype=x.dtype, device=x.device) if want_cache else None
+    la_temporal_conv(shape, x, w, bias, f_in, f_out, y, stream)
+    return (y, f_out) if want_cache else y

@@ -432,6 +432,60 @@ la_status la_causal_attention(const la_shape* shape, const void* Q, const void* 
   return LA_OK;
 }
 
+la_status la_temporal_conv(const la_conv_shape* shape, const void* x, const float* w,
+                           const float* bias, const void* f_in, void* f_out, void* y,
+                           la_stream stream) {
+  if (shape == nullptr) return fail(LA_ERR_INVALID_ARG, "shape is NULL");
+  const la_conv_shape& s = *shape;
+  if (s.B < 0 || s.T < 0 || s.Hh < 0 || s.W < 0 || s.C < 0)
+    return fail(LA_ERR_INVALID_ARG, "negative size B=%d T=%d Hh=%d W=%d C=%d", s.B, s.T, s.Hh,
+                s.W, s.C);
+  if (s.C % 8 != 0) return fail(LA_ERR_UNSUPPORTED, "C=%d is not a multiple of 8", s.C);
+  if (s.io_dtype != LA_IO_BF16 && s.io_dtype != LA_IO_F32)
+    return fail(LA_ERR_INVALID_ARG, "io_dtype=%d", s.io_dtype);
+  const long long hw = 1LL * s.Hh * s.W;
+  const long long frame_elems = hw * s.C;
+  if (hw > 0x7fffffffLL || 1LL * s.B * s.T * frame_elems >= (1LL << 40))
+    return fail(LA_ERR_UNSUPPORTED, "feature map too large");
+  const size_t esz = s.io_dtype == LA_IO_BF16 ? 2 : 4;
+  const size_t nx = static_cast<size_t>(s.B) * s.T * frame_elems * esz;
+  const size_t nf = static_cast<size_t>(s.B) * frame_elems * esz;
+  const bool any_cols = s.B > 0 && hw > 0 && s.C > 0;
+  const bool any = any_cols && s.T > 0;
+  LA_TRY(check_ptr(x, "x", any));
+  LA_TRY(check_ptr(y, "y", any));
+  LA_TRY(check_ptr(w, "w", any));
+  LA_TRY(check_ptr(bias, "bias", any && bias != nullptr));
+  LA_TRY(check_ptr(f_in, "f_in", any_cols && f_in != nullptr));
+  LA_TRY(check_ptr(f_out, "f_out", any_cols && f_out != nullptr));
+  const size_t nw = static_cast<size_t>(s.C) * 3 * 4, nb = static_cast<size_t>(s.C) * 4;
+  // y == x and f_out == f_in are allowed exactly; any other overlap is not
+  if ((y != x && overlap(y, nx, x, nx)) || (f_out != f_in && overlap(f_out, nf, f_in, nf)) ||
+      overlap(y, nx, w, nw) || overlap(y, nx, bias, nb) || overlap(y, nx, f_in, nf) ||
+      overlap(y, nx, f_out, nf) || overlap(f_out, nf, x, nx) || overlap(f_out, nf, w, nw) ||
+      overlap(f_out, nf, bias, nb))
+    return fail(LA_ERR_INVALID_ARG, "y and f_out must not overlap the other buffers");
+  if (!any_cols) return LA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (s.T == 0) {
+    if (f_out == nullptr || f_out == f_in) return LA_OK;
+    const cudaError_t e = f_in != nullptr
+                              ? cudaMemcpyAsync(f_out, f_in, nf, cudaMemcpyDeviceToDevice, st)
+                              : cudaMemsetAsync(f_out, 0, nf, st);
+    if (e != cudaSuccess) return cuda_fail(e, "temporal conv (empty clip)");
+    return LA_OK;
+  }
+  ConvProblem cp;
+  cp.B = s.B;
+  cp.T = s.T;
+  cp.HW = static_cast<int>(hw);
+  cp.C = s.C;
+  cp.io = s.io_dtype;
+  const cudaError_t e = launch_temporal_conv(cp, x, w, bias, f_in, f_out, y, st);
+  if (e != cudaSuccess) return cuda_fail(e, "temporal conv");
+  return LA_OK;
+}
+
 la_status la_state_reset(float* S, float* z, int B, int H, int D, la_stream stream) {
   if (B < 0 || H < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d", B, H);
   if (D != kD) return fail(LA_ERR_UNSUPPORTED, "head width D=%d (only 32 is built)", D);
@@ -470,11 +524,12 @@ const char* la_last_error(void) { return g_last_error.c_str(); }
 
 la_status la_device_error(unsigned* code, int reset) {
   if (code == nullptr) return fail(LA_ERR_INVALID_ARG, "code is NULL");
-  unsigned fwd = 0, bwd = 0;
+  unsigned fwd = 0, bwd = 0, conv = 0;
   cudaError_t e = read_device_error(&fwd, reset != 0);
   if (e == cudaSuccess) e = read_device_error_bwd(&bwd, reset != 0);
+  if (e == cudaSuccess) e = read_device_error_conv(&conv, reset != 0);
   if (e != cudaSuccess) return cuda_fail(e, "la_device_error");
-  *code = fwd | bwd;
+  *code = fwd | bwd | conv;
   return LA_OK;
 }
 

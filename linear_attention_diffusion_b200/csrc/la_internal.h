@@ -114,10 +114,19 @@ cudaError_t launch_backward_kv_simt(const Problem& p, const void* K, const void*
 cudaError_t launch_causal(const Problem& p, const void* Q, const void* K, const void* V,
                           const float* partials, float* S_carry, float* z_carry, int update,
                           unsigned* counters, void* O, cudaStream_t s);
+// Temporal depth-wise convolution with the conv cache (la_conv.cu).
+struct ConvProblem {
+  int B, T, HW, C;  // C a multiple of 8
+  int io;           // 0 bf16, 1 float32
+};
+cudaError_t launch_temporal_conv(const ConvProblem& cp, const void* x, const float* w,
+                                 const float* bias, const void* f_in, void* f_out, void* y,
+                                 cudaStream_t s);
 // Device error words of the tensor-core kernels (bounded waits that gave up):
 // the forward's (la_tc.cu) and the backward's (la_backward_tc.cu).
 cudaError_t read_device_error(unsigned* code, bool reset);
 cudaError_t read_device_error_bwd(unsigned* code, bool reset);
+cudaError_t read_device_error_conv(unsigned* code, bool reset);  // la_conv.cu
 
 // Host-side helpers of the C-ABI layer (la_api.cu).
 namespace detail {
