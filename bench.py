@@ -2,7 +2,7 @@
 """Benchmark of one ReLU linear-attention layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl la|reference]
-                    [--workload NAME] [--op layer|backward|causal]
+                    [--workload NAME] [--op layer|backward|causal|tconv]
 
 A step is one pass of the layer's hot path over one batch of synthetic input:
 the state reduce (S = sum phi(K)^T V, z = sum ReLU(K)) and the apply
@@ -11,7 +11,10 @@ block-causal video (reset, 12 blocks x 5 calls) for the LongSANA workload.
 With --op backward a step is the layer's backward instead (dQ, dK, dV and the
 state gradients from Q, K, V, the state and dO); with --op causal it is
 token-causal attention over the workload's tokens (query n sees keys 0..n).
-Both cover the non-causal workloads' shapes.
+Both cover the non-causal workloads' shapes. With --op tconv a step is the
+Mix-FFN's temporal depth-wise convolution over the video workload's latent
+grid at the FFN width: a whole clip (sanavideo_480p), or one block reading and
+updating the conv cache (longsana_block_causal).
 Rank 0 prints one JSON line. Multi-GPU runs are weak-scaled: every rank runs
 its own copy of the workload (heads and batches are independent), with no
 collective on the data path; the time is the max over ranks.
@@ -45,9 +48,15 @@ METRIC = "linear-attn tokens/s per layer at 1 B200; achieved HBM GB/s vs peak"
 METRIC_BWD = "linear-attn backward tokens/s per layer at 1 B200; achieved HBM GB/s vs peak"
 METRIC_CAUSAL = ("token-causal linear-attn tokens/s per layer at 1 B200; "
                  "achieved HBM GB/s vs peak")
-METRICS = {"layer": METRIC, "backward": METRIC_BWD, "causal": METRIC_CAUSAL}
+METRIC_TCONV = "temporal-conv tokens/s per layer at 1 B200; achieved HBM GB/s vs peak"
+METRICS = {"layer": METRIC, "backward": METRIC_BWD, "causal": METRIC_CAUSAL,
+           "tconv": METRIC_TCONV}
+# Channels of the temporal convolution: the FFN width of Sana-1.6B, which
+# SANA-Video starts from (width 2240, FFN 5600).
+FFN_WIDTH = 5600
 OP_CONFIG = {"layer": {}, "backward": {"op": "backward (dQ, dK, dV, dS, dz)"},
-             "causal": {"op": "token-causal (query n sees keys 0..n), no carry"}}
+             "causal": {"op": "token-causal (query n sees keys 0..n), no carry"},
+             "tconv": {"op": "temporal depth-wise conv 3x1x1 + shortcut", "channels": FFN_WIDTH}}
 DEFAULT_WORKLOAD = "sana1.6b_1024px"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
@@ -261,6 +270,88 @@ def oracle_sample(w, seconds, max_reps=None, op="layer"):
 # the CUDA path
 
 
+def time_steps(args, step, stream, dev, world, n_sets, one_step_graphs, check_status):
+    """Warm-up, then exactly args.steps steps timed on the device.
+
+    ``step(i, evs)`` enqueues step i on ``stream`` (recording evs[0] and
+    evs[1] around its launches when given). Steps are captured in CUDA graphs
+    of ``chunk`` steps (one step per graph when ``one_step_graphs``) and
+    replayed back to back between two events; a second graph with events
+    around every step gives the per-step device durations. Returns
+    (ms over all ranks' max, per-step us list, chunk, wall t0, wall t1).
+    """
+    import torch
+    # warm-up, eager
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    torch.cuda.synchronize(dev)
+    check_status()
+
+    # chunk graph: C steps, with an event after every launch
+    n_ev = 2
+    chunk = n_sets * max(1, 100 // n_sets) if not one_step_graphs else 1
+    chunk = min(chunk, args.steps) if args.steps > 0 else chunk
+    chunk = max(1, chunk - chunk % n_sets) if chunk >= n_sets else chunk
+
+    def capture(nsteps, with_events):
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
+               for _ in range(nsteps)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(nsteps):
+                step(i, evs[i] if with_events else None)
+        check_status()
+        return g, evs
+
+    g_chunk, _ = capture(chunk, with_events=False)
+    full, rem = divmod(args.steps, chunk)
+    g_rem = capture(rem, with_events=False)[0] if rem else None
+    # a second graph with an event after every launch, for per-launch durations
+    g_ev, ev_chunk = capture(chunk, with_events=True)
+
+    # soak: the same graph, untimed, for about a second, so that clocks settle
+    torch.cuda.synchronize(dev)
+    t_soak = time.time()
+    with torch.cuda.stream(stream):
+        while time.time() - t_soak < args.soak:
+            g_chunk.replay()
+            torch.cuda.synchronize(dev)
+
+    # timed region 1: exactly K steps, graph replays back to back (no events
+    # between launches, so consecutive kernels overlap through programmatic
+    # dependent launch exactly as they do for a user's stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(full):
+            g_chunk.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        end.record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end)
+
+    # timed region 2: the event graph, for the duration of each launch
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g_ev.replay()
+    torch.cuda.synchronize(dev)
+    seg = [[e[j].elapsed_time(e[j + 1]) for e in ev_chunk] for j in range(n_ev - 1)]
+    seg_us = [1000.0 * statistics.mean(x) for x in seg]
+
+    del g_chunk, g_rem, g_ev  # release the graphs before any collective teardown
+    return max_over_ranks(ms, dev), seg_us, chunk, t0, t1
+
+
 def run_la(args, w, rank, world, local_rank):
     import torch
     import linear_attention_diffusion_b200 as la
@@ -377,74 +468,8 @@ def run_la(args, w, rank, world, local_rank):
             raise RuntimeError(f"library call failed: {la.la_status_string(bad[0])} "
                                f"{la.la_last_error()}")
 
-    # warm-up, eager
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            step(i)
-    torch.cuda.synchronize(dev)
-    check_status()
-
-    # chunk graph: C steps, with an event after every launch
-    n_ev = 2
-    chunk = n_sets * max(1, 100 // n_sets) if not w.block_causal else 1
-    chunk = min(chunk, args.steps) if args.steps > 0 else chunk
-    chunk = max(1, chunk - chunk % n_sets) if chunk >= n_sets else chunk
-
-    def capture(nsteps, with_events):
-        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
-               for _ in range(nsteps)]
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(nsteps):
-                step(i, evs[i] if with_events else None)
-        check_status()
-        return g, evs
-
-    g_chunk, _ = capture(chunk, with_events=False)
-    full, rem = divmod(args.steps, chunk)
-    g_rem = capture(rem, with_events=False)[0] if rem else None
-    # a second graph with an event after every launch, for per-launch durations
-    g_ev, ev_chunk = capture(chunk, with_events=True)
-
-    # soak: the same graph, untimed, for about a second, so that clocks settle
-    torch.cuda.synchronize(dev)
-    t_soak = time.time()
-    with torch.cuda.stream(stream):
-        while time.time() - t_soak < args.soak:
-            g_chunk.replay()
-            torch.cuda.synchronize(dev)
-
-    # timed region 1: exactly K steps, graph replays back to back (no events
-    # between launches, so consecutive kernels overlap through programmatic
-    # dependent launch exactly as they do for a user's stream)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    t0 = time.time()
-    with torch.cuda.stream(stream):
-        start.record(stream)
-        for _ in range(full):
-            g_chunk.replay()
-        if g_rem is not None:
-            g_rem.replay()
-        end.record(stream)
-    torch.cuda.synchronize(dev)
-    t1 = time.time()
-    if world > 1:
-        torch.distributed.barrier()
-    ms = start.elapsed_time(end)
-
-    # timed region 2: the event graph, for the duration of each launch
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            g_ev.replay()
-    torch.cuda.synchronize(dev)
-    seg = [[e[j].elapsed_time(e[j + 1]) for e in ev_chunk] for j in range(n_ev - 1)]
-    seg_us = [1000.0 * statistics.mean(x) for x in seg]
-
-    ms_max = max_over_ranks(ms, dev)
+    ms_max, seg_us, chunk, t0, t1 = time_steps(args, step, stream, dev, world, n_sets,
+                                               w.block_causal, check_status)
 
     # end-to-end through the public API with host buffers
     if args.e2e_steps <= 0:
@@ -457,10 +482,94 @@ def run_la(args, w, rank, world, local_rank):
         e2e = run_e2e(args, w, dev, stream, la, rank)
     clocks = sampler.summary(t0, t1)
     sampler.stop()
-    del g_chunk, g_rem, g_ev
     return {"ms": ms_max, "seg_us": seg_us, "kernel_names": kernel_names, "e2e": e2e,
             "clocks": clocks, "launches_per_step": launches_per_step, "n_sets": n_sets,
             "chunk": chunk, "per_set_bytes": per_set}
+
+
+def run_tconv(args, w, rank, world, local_rank):
+    """The temporal convolution over the video workload's latent grid."""
+    import torch
+    import linear_attention_diffusion_b200 as la
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(str(getattr(props, "uuid", "") or ""))
+    stream = torch.cuda.Stream(dev)
+    lib = la._lib
+    sp = stream.cuda_stream
+    C = FFN_WIDTH
+    cshape = la.make_conv_shape(w.B, w.T, w.Hh, w.W, C)
+    x = wl.make_tensor((w.B, w.T, w.Hh, w.W, C), rank_seed(rank) + 20).to(dev)
+    y = torch.empty_like(x)
+    wt = wl.make_tensor((C, 3), 21, torch.float32).to(dev)
+    bias = wl.make_tensor((C,), 22, torch.float32).to(dev)
+    # block-causal: the block reads the cache and leaves its last frame there
+    cache = wl.make_tensor((w.B, w.Hh, w.W, C), 23).to(dev) if w.block_causal else None
+    cache_p = None if cache is None else cache.data_ptr()
+    per_set = x.numel() * x.element_size()
+    status = []
+
+    def step(i, evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        status.append(lib.la_temporal_conv(ctypes.byref(cshape), x.data_ptr(), wt.data_ptr(),
+                                           bias.data_ptr(), cache_p, cache_p, y.data_ptr(), sp))
+        if evs is not None:
+            evs[1].record(stream)
+
+    def check_status():
+        bad = [v for v in status if v != 0]
+        status.clear()
+        if bad:
+            raise RuntimeError(f"library call failed: {la.la_status_string(bad[0])} "
+                               f"{la.la_last_error()}")
+
+    ms_max, seg_us, chunk, t0, t1 = time_steps(args, step, stream, dev, world, 1, False,
+                                               check_status)
+    e2e = None
+    if args.e2e_steps > 0:
+        steps = max(1, min(args.steps, args.e2e_steps))
+        hx = x.cpu().pin_memory()
+        hy = torch.empty_like(hx).pin_memory()
+        with torch.cuda.stream(stream):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(steps):
+                x.copy_(hx, non_blocking=True)
+                la.la_temporal_conv(cshape, x, wt, bias, cache, cache, y, stream)
+                hy.copy_(y, non_blocking=True)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e = {"ms_per_step": a.elapsed_time(b) / steps, "tokens_per_step": w.B * w.N,
+               "steps": steps, "h2d_bytes_per_step": per_set, "d2h_bytes_per_step": per_set}
+    clocks = sampler.summary(t0, t1)
+    sampler.stop()
+    return {"ms": ms_max, "seg_us": seg_us, "kernel_names": ("temporal_conv",), "e2e": e2e,
+            "clocks": clocks, "launches_per_step": 1, "n_sets": 1, "chunk": chunk,
+            "per_set_bytes": per_set, "cache_bytes": 0 if cache is None else 2 * per_set // w.T}
+
+
+def oracle_sample_tconv(w, seconds):
+    """The float64 temporal convolution on a channel subset, scaled to FFN_WIDTH."""
+    import oracle as orc
+    c_sub = 8
+    x = wl.make_tensor((w.B, w.T, w.Hh, w.W, c_sub), 20)
+    wt = wl.make_tensor((c_sub, 3), 21, __import__("torch").float32)
+    f = wl.make_tensor((w.B, w.Hh, w.W, c_sub), 23) if w.block_causal else None
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        orc.temporal_conv(x, wt, None, f)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    per_call = el / reps * FFN_WIDTH / c_sub
+    desc = (f"oracle temporal_conv on {c_sub} of {FFN_WIDTH} channels ({w.T}x{w.Hh}x{w.W}), "
+            f"{reps} calls in {el:.1f} s, scaled to {FFN_WIDTH} channels")
+    return w.B * w.N / per_call, desc, cpu_cores_used(), per_call
 
 
 def run_e2e(args, w, dev, stream, la, rank, causal=False):
@@ -594,16 +703,20 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--soak", type=float, default=1.0)
-    ap.add_argument("--op", choices=["layer", "backward", "causal"], default="layer")
+    ap.add_argument("--op", choices=["layer", "backward", "causal", "tconv"], default="layer")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
-    if args.op != "layer" and w.block_causal:
+    if args.op in ("backward", "causal") and w.block_causal:
         ap.error(f"--op {args.op} covers the non-causal workloads")
+    if args.op == "tconv" and not w.rope:
+        ap.error("--op tconv needs a video workload (sanavideo_480p, longsana_block_causal)")
     if args.steps is None:
         per_step_us = {"sana0.6b_512px": 10, "sana1.6b_1024px": 30, "sana1.6b_4k": 120,
                        "sanavideo_480p": 250, "longsana_block_causal": 12000}[w.name]
-        if args.op != "layer":
+        if args.op in ("backward", "causal"):
             per_step_us *= 10
+        elif args.op == "tconv":
+            per_step_us = 200
         args.steps = max(10, int(0.5e6 / per_step_us))
     args.warmup = max(args.warmup, 3)
 
@@ -619,18 +732,19 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
-    r = run_la(args, w, rank, world, local_rank)
+    r = (run_tconv if args.op == "tconv" else run_la)(args, w, rank, world, local_rank)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank != 0:
         return
 
     ms_step = r["ms"] / args.steps
-    tokens_step = (w.M * w.N * w.B) if w.block_causal else w.B * w.N
+    tokens_step = (w.M * w.N * w.B) if (w.block_causal and args.op == "layer") else w.B * w.N
     value = weak_scaled_value(tokens_step, args.steps, world, r["ms"])
     peak, peak_src = peaks()
     lb = layer_bytes(w)
-    if w.block_causal:
+    lb["temporal_conv"] = 2 * r["per_set_bytes"] + r.get("cache_bytes", 0)
+    if w.block_causal and args.op == "layer":
         name = "la_block_causal_step(update=0)"
         alg = 4 * w.B * w.N * w.H * D * 2 + 2 * w.B * w.H * (D * D + D) * 4
         dur_us = r["seg_us"][0]
@@ -663,6 +777,7 @@ def main():
         "ms_per_step": round(e["ms_per_step"], 4),
         "api": ("la_attention_backward" if args.op == "backward" else
                 "la_causal_attention" if args.op == "causal" else
+                "la_temporal_conv" if args.op == "tconv" else
                 "la_block_causal_step" if w.block_causal else "la_attention")}
     out = {"metric": METRICS[args.op], "value": value, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -673,7 +788,11 @@ def main():
            "roofline": roofline, "e2e": e2e,
            "gpu_launches": r["launches_per_step"] * args.steps,
            "clocks": r["clocks"], "graph_chunk_steps": r["chunk"], "soak_s": args.soak}
-    if world == 1 and args.cpu_seconds > 0:
+    if world == 1 and args.cpu_seconds > 0 and args.op == "tconv":
+        tps, desc, cores, _ = oracle_sample_tconv(w, args.cpu_seconds)
+        out["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores,
+                               "kind": "oracle", "sample": desc}
+    elif world == 1 and args.cpu_seconds > 0:
         tps, desc, cores, _, _ = oracle_sample(w, args.cpu_seconds, op=args.op)
         out["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores,
                                "kind": "oracle", "sample": desc}
@@ -686,6 +805,20 @@ def main_reference(args, w, rank, world):
         return
     budget = 150.0  # seconds for warm-up + timed steps together
     per = budget / (args.steps + args.warmup)
+    if args.op == "tconv":
+        tps, desc, cores, per_call = oracle_sample_tconv(w, min(per * args.steps, 60.0))
+        out = {"impl": "reference", "metric": METRICS[args.op], "value": tps, "unit": "tokens/s",
+               "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": per_call * 1e3, "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": "f64",
+               "data": "synthetic (seeded N(0,1), bf16 inputs read exactly)",
+               "config": dict(config_of(w, world), **OP_CONFIG[args.op]),
+               "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores,
+                                "kind": "oracle", "sample": desc},
+               "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                       "d2h_bytes_per_step": 0}}
+        print(json.dumps(out), flush=True)
+        return
     _, _, cores, per_call, h_sub = oracle_sample(w, min(per, 3.0), max_reps=1, op=args.op)
     # each step: one oracle call on h_sub heads (at most `per` seconds)
     import oracle as orc

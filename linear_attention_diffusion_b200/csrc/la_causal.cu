@@ -49,17 +49,35 @@ __device__ __forceinline__ void store4(float* p, const float (&x)[4]) {
 }
 
 template <typename T>
+__device__ __forceinline__ void load_row4(const Problem& p, const T* Q, const T* K, const T* V,
+                                          int b, int h, int n, bool row, int d0, float (&q)[4],
+                                          float (&k)[4], float (&v)[4]) {
+  if (row) {
+    const size_t off = ((static_cast<size_t>(b) * p.N + n) * p.H + h) * kD + d0;
+    load4(Q + off, q);
+    load4(K + off, k);
+    load4(V + off, v);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) q[i] = k[i] = v[i] = 0.0f;
+  }
+}
+
+// Shared-memory layout: every product below reads one 16-byte vector per
+// four FMAs (rows padded to 36 floats keep the vectors aligned and spread
+// the rows of a warp over the banks).
+template <typename T>
 __global__ void __launch_bounds__(kCThreads)
 causal_simt(const Problem p, const T* __restrict__ Q, const T* __restrict__ K,
             const T* __restrict__ V, const float* __restrict__ partials, float* S_carry,
             float* z_carry, int update, unsigned* counters, T* __restrict__ O) {
-  __shared__ float Rs[kD][kD + 1];                 // running state S[d][e]
-  __shared__ float Rz[kD];                         // running key sum
-  __shared__ __align__(16) float phq[kCT][kD + 4];
-  __shared__ __align__(16) float phk[kCT][kD + 4];
-  __shared__ __align__(16) float kcum[kCT][kD + 4];  // ReLU(k), then its prefix over rows
-  __shared__ __align__(16) float vs[kCT][kD + 4];
-  __shared__ float A[kCT][kCT + 1];                // (phi(q_i) . phi(k_j)) for j <= i
+  __shared__ __align__(16) float Rs[kD][kD + 4];      // running state S[d][e]
+  __shared__ __align__(16) float Rz[kD];              // running key sum
+  __shared__ __align__(16) float phq[kCT][kD + 4];    // phi(q)[i][d]
+  __shared__ __align__(16) float phkT[kD][kCT + 4];   // phi(k)[j][d], transposed: [d][j]
+  __shared__ __align__(16) float kcum[kCT][kD + 4];   // ReLU(k), then its prefix over rows
+  __shared__ __align__(16) float vs[kCT][kD + 4];     // v[j][e]
+  __shared__ __align__(16) float A[kCT][kCT + 4];     // phi(q_i) . phi(k_j) for j <= i, else 0
   __shared__ int s_last;
 
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -100,19 +118,14 @@ causal_simt(const Problem p, const T* __restrict__ Q, const T* __restrict__ K,
 
   const int n_begin = split * p.chunk;
   const int n_end = min(p.N, n_begin + p.chunk);
-  const int r = tid >> 3, d0 = (tid & 7) * 4;
+  const int r = tid >> 3, d0 = (tid & 7) * 4;  // token row, first of 4 dims (also e0, j0)
+  const int warp = tid >> 5, lane = tid & 31;
 
+  float q[4], k[4], v[4];
+  if (n_begin < n_end) load_row4(p, Q, K, V, b, h, n_begin + r, n_begin + r < n_end, d0, q, k, v);
   for (int n0 = n_begin; n0 < n_end; n0 += kCT) {
     const int n = n0 + r;
     const bool row = n < n_end;
-    float q[4] = {0.0f, 0.0f, 0.0f, 0.0f}, k[4] = {0.0f, 0.0f, 0.0f, 0.0f},
-          v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (row) {
-      const size_t off = ((static_cast<size_t>(b) * p.N + n) * p.H + h) * kD + d0;
-      load4(Q + off, q);
-      load4(K + off, k);
-      load4(V + off, v);
-    }
     float qp[4], pq[4], pk[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -135,62 +148,87 @@ causal_simt(const Problem p, const T* __restrict__ Q, const T* __restrict__ K,
         pk[2 * pr + 1] = fmaf(b0, s, b1 * c);
       }
     }
+    *reinterpret_cast<float4*>(&phq[r][d0]) = make_float4(pq[0], pq[1], pq[2], pq[3]);
+    *reinterpret_cast<float4*>(&kcum[r][d0]) = make_float4(k[0], k[1], k[2], k[3]);
+    *reinterpret_cast<float4*>(&vs[r][d0]) = make_float4(v[0], v[1], v[2], v[3]);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      phq[r][d0 + i] = pq[i];
-      phk[r][d0 + i] = pk[i];
-      kcum[r][d0 + i] = k[i];
-      vs[r][d0 + i] = v[i];
-    }
+    for (int i = 0; i < 4; ++i) phkT[d0 + i][r] = pk[i];
     __syncthreads();
+    // the next chunk's loads are in flight during this chunk's arithmetic
+    if (n0 + kCT < n_end) load_row4(p, Q, K, V, b, h, n + kCT, n + kCT < n_end, d0, q, k, v);
 
-    // ---- A[r][j] for j in [j0, j0 + 4), masked to j <= r; prefix of ReLU(k)
+    // ---- A[r][j0 .. j0+4), masked to j <= r
     {
-      const int j0 = (tid & 7) * 4;
       float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      if (j0 <= r) {
-#pragma unroll 8
+      if (d0 <= r) {
+#pragma unroll
         for (int d = 0; d < kD; d += 4) {
           const float4 x = *reinterpret_cast<const float4*>(&phq[r][d]);
+          const float xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            const float4 y = *reinterpret_cast<const float4*>(&phk[j0 + jj][d]);
-            a[jj] = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, a[jj]))));
+          for (int dd = 0; dd < 4; ++dd) {
+            const float4 y = *reinterpret_cast<const float4*>(&phkT[d + dd][d0]);
+            a[0] = fmaf(xs[dd], y.x, a[0]);
+            a[1] = fmaf(xs[dd], y.y, a[1]);
+            a[2] = fmaf(xs[dd], y.z, a[2]);
+            a[3] = fmaf(xs[dd], y.w, a[3]);
           }
         }
       }
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) A[r][j0 + jj] = j0 + jj <= r ? a[jj] : 0.0f;
+      for (int jj = 0; jj < 4; ++jj) a[jj] = d0 + jj <= r ? a[jj] : 0.0f;
+      *reinterpret_cast<float4*>(&A[r][d0]) = make_float4(a[0], a[1], a[2], a[3]);
     }
-    if (tid < kD) {
-      float c = 0.0f;
-      for (int j = 0; j < kCT; ++j) {
-        c += kcum[j][tid];
-        kcum[j][tid] = c;
+    // ---- inclusive prefix of ReLU(k) over the rows: warp w scans dims 4w..4w+3
+    {
+      float4 c = *reinterpret_cast<const float4*>(&kcum[lane][warp * 4]);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float4 u = make_float4(__shfl_up_sync(0xffffffffu, c.x, o),
+                                     __shfl_up_sync(0xffffffffu, c.y, o),
+                                     __shfl_up_sync(0xffffffffu, c.z, o),
+                                     __shfl_up_sync(0xffffffffu, c.w, o));
+        if (lane >= o) c = make_float4(c.x + u.x, c.y + u.y, c.z + u.z, c.w + u.w);
       }
+      __syncwarp();
+      *reinterpret_cast<float4*>(&kcum[lane][warp * 4]) = c;
     }
     __syncthreads();
 
     // ---- output of row r, dims [d0, d0 + 4)
     {
       float num[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 8
-      for (int d = 0; d < kD; ++d) {
-        const float x = phq[r][d];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) num[e] = fmaf(x, Rs[d][d0 + e], num[e]);
-      }
-      for (int j = 0; j <= r; ++j) {
-        const float a = A[r][j];
-        const float4 y = *reinterpret_cast<const float4*>(&vs[j][d0]);
-        num[0] = fmaf(a, y.x, num[0]);
-        num[1] = fmaf(a, y.y, num[1]);
-        num[2] = fmaf(a, y.z, num[2]);
-        num[3] = fmaf(a, y.w, num[3]);
-      }
-      float den = 0.0f;
+      for (int d = 0; d < kD; d += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(&phq[r][d]);
+        const float xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) den = fmaf(qp[i], Rz[d0 + i] + kcum[r][d0 + i], den);
+        for (int dd = 0; dd < 4; ++dd) {
+          const float4 y = *reinterpret_cast<const float4*>(&Rs[d + dd][d0]);
+          num[0] = fmaf(xs[dd], y.x, num[0]);
+          num[1] = fmaf(xs[dd], y.y, num[1]);
+          num[2] = fmaf(xs[dd], y.z, num[2]);
+          num[3] = fmaf(xs[dd], y.w, num[3]);
+        }
+      }
+      for (int j = 0; j <= r; j += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(&A[r][j]);  // zero beyond r
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const float4 y = *reinterpret_cast<const float4*>(&vs[j + jj][d0]);
+          num[0] = fmaf(xs[jj], y.x, num[0]);
+          num[1] = fmaf(xs[jj], y.y, num[1]);
+          num[2] = fmaf(xs[jj], y.z, num[2]);
+          num[3] = fmaf(xs[jj], y.w, num[3]);
+        }
+      }
+      const float4 rz = *reinterpret_cast<const float4*>(&Rz[d0]);
+      const float4 kc = *reinterpret_cast<const float4*>(&kcum[r][d0]);
+      float den = qp[0] * (rz.x + kc.x);
+      den = fmaf(qp[1], rz.y + kc.y, den);
+      den = fmaf(qp[2], rz.z + kc.z, den);
+      den = fmaf(qp[3], rz.w + kc.w, den);
       den += __shfl_xor_sync(0xffffffffu, den, 1);
       den += __shfl_xor_sync(0xffffffffu, den, 2);
       den += __shfl_xor_sync(0xffffffffu, den, 4);
@@ -206,19 +244,22 @@ causal_simt(const Problem p, const T* __restrict__ Q, const T* __restrict__ K,
 
     // ---- R += the chunk's state (rows beyond the split are zero)
     {
-      const int d = tid >> 3;  // state row, columns [d0, d0 + 4)
-      float acc[4] = {Rs[d][d0], Rs[d][d0 + 1], Rs[d][d0 + 2], Rs[d][d0 + 3]};
-#pragma unroll 8
-      for (int j = 0; j < kCT; ++j) {
-        const float x = phk[j][d];
-        const float4 y = *reinterpret_cast<const float4*>(&vs[j][d0]);
-        acc[0] = fmaf(x, y.x, acc[0]);
-        acc[1] = fmaf(x, y.y, acc[1]);
-        acc[2] = fmaf(x, y.z, acc[2]);
-        acc[3] = fmaf(x, y.w, acc[3]);
-      }
+      const int d = r;  // state row d, columns [d0, d0 + 4)
+      float4 acc = *reinterpret_cast<const float4*>(&Rs[d][d0]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) Rs[d][d0 + e] = acc[e];
+      for (int j = 0; j < kCT; j += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(&phkT[d][j]);
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const float4 y = *reinterpret_cast<const float4*>(&vs[j + jj][d0]);
+          acc.x = fmaf(xs[jj], y.x, acc.x);
+          acc.y = fmaf(xs[jj], y.y, acc.y);
+          acc.z = fmaf(xs[jj], y.z, acc.z);
+          acc.w = fmaf(xs[jj], y.w, acc.w);
+        }
+      }
+      *reinterpret_cast<float4*>(&Rs[d][d0]) = acc;
       if (tid < kD) Rz[tid] += kcum[kCT - 1][tid];
     }
     __syncthreads();
