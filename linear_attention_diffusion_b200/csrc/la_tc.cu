@@ -368,39 +368,50 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       tc_fence_before();
     }
 
+    float* sbuf = zred;  // [4][32][32] f32: the state for the apply, free once the reduce is done
     if (kRed) {
-      // ---- second phase of the reduce: the head group's CTA that arrives
-      // last sums every split's partial in split order (+ carry) and writes
-      // the state. The named barrier orders each math thread's partial stores
-      // before the release fence of the arriving thread.
+      // ---- second phase of the reduce. The named barrier orders each math
+      // thread's partial stores before the release fence of the arriving
+      // thread.
       named_bar_sync(kBarMath, kMath);
       if (mt == 0) {
         fence_acq_rel_gpu();
         const unsigned prev = atomicAdd(&a.arrive[cidx], 1u);
         *last_flag = prev == gridDim.x - 1;
-        if (*last_flag) fence_acq_rel_gpu();
+        if (kPh == kFusedLayer) {
+          // single-launch layer: every CTA of the head group waits for all the
+          // splits' partials (the launch is cooperative: all CTAs are resident)
+          spin_count(&a.arrive[cidx], gridDim.x, abort_flag, &g_tc_error);
+        } else if (*last_flag) {
+          fence_acq_rel_gpu();
+        }
       }
       named_bar_sync(kBarMath, kMath);
       const bool last = *last_flag != 0;
-      const bool wanted = a.out.out1_S != nullptr || a.out.out1_z != nullptr ||
-                          a.out.out2_S != nullptr || a.out.out2_z != nullptr;
-      if (last && alive && wanted) combine_from_global<kMath>(p, b, h0, mt, a.partials, a.out);
-      named_bar_sync(kBarMath, kMath);
       if (kPh == kReduceOnly) {
+        // the CTA that arrived last sums every split's partial in split order
+        // (+ carry) and writes the state
+        const bool wanted = a.out.out1_S != nullptr || a.out.out1_z != nullptr ||
+                            a.out.out2_S != nullptr || a.out.out2_z != nullptr;
+        if (last && alive && wanted) combine_from_global<kMath>(p, b, h0, mt, a.partials, a.out);
+        named_bar_sync(kBarMath, kMath);
         if (mt == 0 && last) a.arrive[cidx] = 0u;  // ready for the next call
       } else {
-        // fused layer: the other CTAs of the group wait for the last one's
-        // flag (the launch is cooperative: all CTAs are resident)
-        if (mt == 0) {
-          if (last) {
-            fence_acq_rel_gpu();
-            st_release_gpu(&a.ready[cidx], 1u);
-          } else {
-            spin_flag(&a.ready[cidx], abort_flag, &g_tc_error);
-          }
-        }
-        named_bar_sync(kBarMath, kMath);
+        // single-launch layer: every CTA sums the partials itself, in the same
+        // order as the reduce-only launch, straight into shared memory (so the
+        // results are bitwise those of reduce + apply); the state is written
+        // out by the last CTA to leave, once every CTA has read the carry
         if (*abort_flag) alive = false;
+        const int heads = min(kGroupHeads, p.H - h0);
+        for (int i = mt; i < (kGroupHeads - heads) * (kD * kD + kD); i += kMath) {
+          const int hh = heads + i / (kD * kD + kD), k = i % (kD * kD + kD);
+          if (k < kD * kD) sbuf[hh * kD * kD + k] = 0.0f;
+          else zs[hh * kD + k - kD * kD] = 0.0f;
+        }
+        const StateOut carry_only = {a.out.carry_S, a.out.carry_z, nullptr, nullptr, nullptr,
+                                     nullptr};
+        if (alive) combine_from_global<kMath>(p, b, h0, mt, a.partials, carry_only, sbuf, zs);
+        named_bar_sync(kBarMath, kMath);
       }
     }
 
@@ -408,19 +419,20 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       // ---- the state of the four heads as the MMA's B operand: row e of head
       // pair j holds S[h][0..31][e] of heads 2j and 2j+1 in bf16 (K-major,
       // 128-byte swizzle); S goes through shared memory with 16-byte loads
-      float* sbuf = zred;  // [4][32][32] f32, free once the reduce is done
-      for (int idx = mt; idx < kGroupHeads * kD * kD / 4; idx += kMath) {
-        const int hh = idx >> 8, h = h0 + hh;
-        float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        if (h < p.H)
-          v = __ldcg(reinterpret_cast<const float4*>(a.S_in + (cidx + hh) * kD * kD) + (idx & 255));
-        *reinterpret_cast<float4*>(sbuf + idx * 4) = v;
+      if (kPh == kApplyOnly) {  // the fused layer has it in shared memory already
+        for (int idx = mt; idx < kGroupHeads * kD * kD / 4; idx += kMath) {
+          const int hh = idx >> 8, h = h0 + hh;
+          float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          if (h < p.H)
+            v = __ldcg(reinterpret_cast<const float4*>(a.S_in + (cidx + hh) * kD * kD) + (idx & 255));
+          *reinterpret_cast<float4*>(sbuf + idx * 4) = v;
+        }
+        if (mt < kGroupHeads * kD) {
+          const int h = h0 + mt / kD;
+          zs[mt] = h < p.H ? __ldcg(a.z_in + cidx * kD + mt) : 0.0f;
+        }
+        named_bar_sync(kBarMath, kMath);
       }
-      if (mt < kGroupHeads * kD) {
-        const int h = h0 + mt / kD;
-        zs[mt] = h < p.H ? __ldcg(a.z_in + cidx * kD + mt) : 0.0f;
-      }
-      named_bar_sync(kBarMath, kMath);
       {
         const int idx = mt;  // 2 pairs x 32 rows x 8 chunks = 512 = kMath
         const int j = idx >> 8, e = (idx >> 3) & 31, c = idx & 7;
@@ -433,16 +445,6 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       fence_proxy_async_smem();
       named_bar_sync(kBarMath, kMath);
       if (mt == 0) mbar_arrive(b_ready);
-      if (kPh == kFusedLayer && mt == 0) {
-        // the state is read: the last CTA to leave resets the group's words
-        const unsigned prev = atomicAdd(&a.depart[cidx], 1u);
-        if (prev == gridDim.x - 1) {
-          a.arrive[cidx] = 0u;
-          a.ready[cidx] = 0u;
-          a.depart[cidx] = 0u;
-        }
-      }
-
       // ---- apply: warpgroup wg owns tiles wg, wg + 4, ...; thread = token row
       const int wg = (warp - 2) >> 2;
       const int quad = warp & 3;
@@ -552,6 +554,36 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
         }
       }
       if (leader) bulk_wait<0>();
+    }
+    if (kPh == kFusedLayer) {
+      // every CTA has read the carry and the partials once all have reached
+      // this point: the last to arrive here writes the state out (the carry
+      // may be updated in place) and resets the group's words
+      if (mt == 0) {
+        fence_acq_rel_gpu();
+        const unsigned prev = atomicAdd(&a.depart[cidx], 1u);
+        *last_flag = prev == gridDim.x - 1;
+        if (*last_flag) fence_acq_rel_gpu();
+      }
+      named_bar_sync(kBarMath, kMath);
+      if (*last_flag) {
+        const int heads = min(kGroupHeads, p.H - h0);
+        for (int i = mt; i < heads * (kD * kD + kD) / 4; i += kMath) {
+          const int hh = i / ((kD * kD + kD) / 4), k = (i % ((kD * kD + kD) / 4)) * 4;
+          const bool is_s = k < kD * kD;
+          const float4 v = is_s ? *reinterpret_cast<const float4*>(sbuf + hh * kD * kD + k)
+                                : *reinterpret_cast<const float4*>(zs + hh * kD + k - kD * kD);
+          const size_t o = is_s ? (cidx + hh) * kD * kD + k : (cidx + hh) * kD + k - kD * kD;
+          float* d1 = is_s ? a.out.out1_S : a.out.out1_z;
+          float* d2 = is_s ? a.out.out2_S : a.out.out2_z;
+          if (d1 != nullptr) *reinterpret_cast<float4*>(d1 + o) = v;
+          if (d2 != nullptr) *reinterpret_cast<float4*>(d2 + o) = v;
+        }
+        if (mt == 0) {
+          a.arrive[cidx] = 0u;
+          a.depart[cidx] = 0u;
+        }
+      }
     }
   }
 

@@ -177,7 +177,9 @@ __device__ __forceinline__ bool spin_flag(const unsigned* flag, volatile int* ab
 // splits.
 template <int kThreads>
 __device__ __forceinline__ void combine_from_global(const Problem& p, int b, int h0, int mt,
-                                                    const float* partials, const StateOut& out) {
+                                                    const float* partials, const StateOut& out,
+                                                    float* s_smem = nullptr,
+                                                    float* z_smem = nullptr) {
   constexpr int kVec = kStateFloats / 4;                     // 264 float4 per head
   constexpr int kPerThread = (kGroupHeads * kVec + kThreads - 1) / kThreads;
   const int heads = min(kGroupHeads, p.H - h0);
@@ -230,7 +232,27 @@ __device__ __forceinline__ void combine_from_global(const Problem& p, int b, int
     float* d2 = is_s ? out.out2_S : out.out2_z;
     if (d1 != nullptr) *reinterpret_cast<float4*>(d1 + o) = r;
     if (d2 != nullptr) *reinterpret_cast<float4*>(d2 + o) = r;
+    // shared-memory copy: S as [head][32][32], z as [head][32]
+    if (is_s && s_smem != nullptr) *reinterpret_cast<float4*>(s_smem + hh * kD * kD + i) = r;
+    if (!is_s && z_smem != nullptr) *reinterpret_cast<float4*>(z_smem + hh * kD + i - kD * kD) = r;
   }
+}
+
+// Wait until *counter >= target (acquire), for at most kWaitLimitNs; on
+// timeout raise the abort flag and `err` and return false.
+__device__ __forceinline__ bool spin_count(const unsigned* counter, unsigned target,
+                                           volatile int* abort_flag, unsigned* err) {
+  const uint64_t t0 = globaltimer_ns();
+  while (ld_acquire_gpu(counter) < target) {
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicOr(err, kErrWait);
+      return false;
+    }
+    __nanosleep(32);
+  }
+  return true;
 }
 
 // ------------------------------------------------------------------ host
