@@ -425,9 +425,12 @@ la_status la_causal_attention(const la_shape* shape, const void* Q, const void* 
   // the splits' partial states only: no combine
   LA_TRY(run_reduce(p, K, V, w, StateOut{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr},
                     st));
+  const float* partials = reinterpret_cast<const float*>(w + L.partials);
+  unsigned* counters = reinterpret_cast<unsigned*>(w + L.counters);
   const cudaError_t e =
-      launch_causal(p, Q, K, V, reinterpret_cast<const float*>(w + L.partials), S_carry, z_carry,
-                    update, reinterpret_cast<unsigned*>(w + L.counters), O, st);
+      causal_tc_supported(p)
+          ? launch_causal_tc(p, Q, K, V, partials, S_carry, z_carry, update, counters, O, st)
+          : launch_causal(p, Q, K, V, partials, S_carry, z_carry, update, counters, O, st);
   if (e != cudaSuccess) return cuda_fail(e, "causal attention");
   return LA_OK;
 }
@@ -524,12 +527,13 @@ const char* la_last_error(void) { return g_last_error.c_str(); }
 
 la_status la_device_error(unsigned* code, int reset) {
   if (code == nullptr) return fail(LA_ERR_INVALID_ARG, "code is NULL");
-  unsigned fwd = 0, bwd = 0, conv = 0;
+  unsigned fwd = 0, bwd = 0, conv = 0, causal = 0;
   cudaError_t e = read_device_error(&fwd, reset != 0);
   if (e == cudaSuccess) e = read_device_error_bwd(&bwd, reset != 0);
   if (e == cudaSuccess) e = read_device_error_conv(&conv, reset != 0);
+  if (e == cudaSuccess) e = read_device_error_causal(&causal, reset != 0);
   if (e != cudaSuccess) return cuda_fail(e, "la_device_error");
-  *code = fwd | bwd | conv;
+  *code = fwd | bwd | conv | causal;
   return LA_OK;
 }
 

@@ -114,6 +114,11 @@ cudaError_t launch_backward_kv_simt(const Problem& p, const void* K, const void*
 cudaError_t launch_causal(const Problem& p, const void* Q, const void* K, const void* V,
                           const float* partials, float* S_carry, float* z_carry, int update,
                           unsigned* counters, void* O, cudaStream_t s);
+// The tensor-core version (la_causal_tc.cu): bf16 I/O without RoPE.
+bool causal_tc_supported(const Problem& p);
+cudaError_t launch_causal_tc(const Problem& p, const void* Q, const void* K, const void* V,
+                             const float* partials, float* S_carry, float* z_carry, int update,
+                             unsigned* counters, void* O, cudaStream_t s);
 // Temporal depth-wise convolution with the conv cache (la_conv.cu).
 struct ConvProblem {
   int B, T, HW, C;  // C a multiple of 8
@@ -127,6 +132,7 @@ cudaError_t launch_temporal_conv(const ConvProblem& cp, const void* x, const flo
 cudaError_t read_device_error(unsigned* code, bool reset);
 cudaError_t read_device_error_bwd(unsigned* code, bool reset);
 cudaError_t read_device_error_conv(unsigned* code, bool reset);  // la_conv.cu
+cudaError_t read_device_error_causal(unsigned* code, bool reset);  // la_causal_tc.cu
 
 // Host-side helpers of the C-ABI layer (la_api.cu).
 namespace detail {

@@ -14,7 +14,14 @@ D = 32
 
 
 def _tol(io, rope):
-    return 2.0 ** -8 if (io == "bf16" and rope) else 1e-4
+    """Relative error per term: float32 arithmetic on exact operands (1e-4);
+    bf16 with RoPE: the split states come from the tensor-core reduce, whose
+    rotated key features are rounded to bf16 (2^-8); bf16 without RoPE: the
+    tensor-core kernel rounds the masked weights P and the running state R to
+    bf16 for its second MMA (2^-9 each, so 2^-7 with a factor 2 to spare)."""
+    if io != "bf16":
+        return 1e-4
+    return 2.0 ** -8 if rope else 2.0 ** -7
 
 
 def _inputs(B, N, H, seed, io):
