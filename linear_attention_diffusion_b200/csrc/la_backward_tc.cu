@@ -12,18 +12,19 @@
 //   dS     = sum_n phi(q_n)^T dnum_n,        dz = sum_n dden_n ReLU(q_n)
 //   dK_n   = [R_n^T (dS v_n^T) + dz] * [k_n > 0],   dV_n = phi(k_n) dS
 //
-// Query side (one launch, grid = token splits x head groups x batch, as the
-// state reduce): per 128-token tile of a 4-head group,
+// Query side (one launch, grid = token splits x head pairs x batch): per
+// 128-token tile of a head pair (one 64-dim TMA box per tensor),
 //   transform  Q -> ReLU(Q) and dO -> dnum (bf16) in place in shared memory;
 //   MMA 1      t = dnum S^T per head (M = 128 tokens, N = 32, K = 32) into TMEM;
 //   epilogue   dden, dQ (stored straight from registers), dz on CUDA cores;
 //   rewrite    ReLU(Q) -> phi(Q) in place (RoPE only);
-//   MMA 2      dS += phi(Q)^T dnum (M = N = 128 dims, K = 16 tokens; the four
-//              32x32 diagonal blocks are the heads' dS).
+//   MMA 2      dS += phi(Q)^T dnum (the reduce's MN-major form, M = 128 with
+//              the upper 64 rows unused, N = 64, K = 16 tokens; the two 32x32
+//              diagonal blocks are the heads' dS).
 // The split partials of (dS, dz) are combined by the last CTA of each head
-// group in split order, exactly like the state reduce: deterministic.
+// pair in split order, as in the state reduce: deterministic.
 //
-// Key side (one launch, grid = tile ranges x head groups x batch): per tile,
+// Key side (one launch, grid = tile ranges x head pairs x batch): per tile,
 //   transform  K -> phi(K) in place (the sign mask stays in registers);
 //   MMA 1      dphi(K) = V dS^T per head; epilogue dK = R^T dphi(K) + dz,
 //              masked, written over the V tile (MMA 1 has read it);
@@ -31,10 +32,15 @@
 //              over the K tile; dK and dV stored with TMA.
 //
 // Warp roles: warp 0 TMA, warp 1 MMA (one elected lane), warps 2..13 three
-// math warpgroups. Warpgroup w owns stage w, TMEM columns [128 w, 128 w + 128)
-// and the tiles j = w (mod 3), so every mbarrier has one consumer that waits
-// for its phases in order (a parity wait cannot tell phase k from k + 2).
-// Every wait is bounded and raises the device error word when it gives up.
+// math warpgroups. Six stages of 32 KB: tile j uses stage j mod 6 and TMEM
+// columns [64 s, 64 s + 64), and belongs to warpgroup j mod 3, so each
+// warpgroup owns two stages (its next tile loads while it works on the
+// current one) and every mbarrier has one consumer that waits for its phases
+// in order (a parity wait cannot tell phase k from k + 2). Two heads per CTA
+// keep the tiles small enough for six stages; the split count (query side)
+// and tile ranges (key side) are chosen for head pairs so the grid still
+// covers the SMs in one wave. Every wait is bounded and raises the device
+// error word when it gives up.
 #include <algorithm>
 
 #include "la_tc_common.cuh"
@@ -48,9 +54,11 @@ namespace {
 
 constexpr int kBT = 128;                // tokens per tile
 constexpr int kBBox = kBT * 128;        // [128 tokens][64 dims] bf16 = 16 KB
-constexpr int kBTile = 4 * kBBox;       // two tensors x two boxes = 64 KB
-constexpr int kBStages = 3;
-constexpr int kBWG = 3;                 // math warpgroups (one per stage)
+constexpr int kBTile = 2 * kBBox;       // two tensors = 32 KB
+constexpr int kBStages = 6;
+constexpr int kBWG = 3;                 // math warpgroups (two stages each)
+constexpr int kPair = 2;                // heads per CTA
+constexpr uint32_t kColDS = 64 * kBStages;  // query side: dS accumulator (64 columns)
 constexpr int kBMath = kBWG * 128;
 constexpr int kBThreads = 64 + kBMath;
 constexpr int kBTmemCols = 512;
@@ -58,25 +66,25 @@ constexpr int kBarAll = 1;              // named barrier over the math threads
 constexpr int kBarW0 = 2;               // + warpgroup
 
 struct QSmem {  // query side, byte offsets from the 1024-aligned base
-  static constexpr int stages = 0;                          // [3][Q box0, Q box1, dO box0, dO box1]
-  static constexpr int bop = stages + kBStages * kBTile;    // S as B operand: [2][32 rows][128 B]
-  static constexpr int zs = bop + 8192;                     // [4][32] f32
-  static constexpr int dden = zs + 512;                     // [3][128 rows][4] f32
-  static constexpr int rope = dden + kBWG * kBT * 4 * 4;    // float2[kRopeTableMax]
+  static constexpr int stages = 0;                          // [6][Q box, dO box]
+  static constexpr int bop = stages + kBStages * kBTile;    // S as B operand: [32 rows][128 B]
+  static constexpr int zs = bop + 4096;                     // [2][32] f32
+  static constexpr int dden = zs + 256;                     // [3][128 rows][2] f32
+  static constexpr int rope = dden + kBWG * kBT * kPair * 4;  // float2[kRopeTableMax]
   static constexpr int bars = rope + kRopeTableMax * 8;
-  // full[3] empty[3] ready_t[3] ready_s[3] t_full[3] acc_full mma_done b_ready
+  // full[6] empty[6] ready_t[6] ready_s[6] t_full[6] acc_full mma_done b_ready
   static constexpr int nbars = 5 * kBStages + 3;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int bytes = misc + 16;
 };
 struct KVSmem {  // key side
-  static constexpr int stages = 0;                          // [3][K box0, K box1, V box0, V box1]
+  static constexpr int stages = 0;                          // [6][K box, V box]
   static constexpr int bop1 = stages + kBStages * kBTile;   // dS rows d (K = e)
-  static constexpr int bop2 = bop1 + 8192;                  // dS^T rows e (K = d)
-  static constexpr int zs = bop2 + 8192;                    // dz [4][32] f32
-  static constexpr int rope = zs + 512;
+  static constexpr int bop2 = bop1 + 4096;                  // dS^T rows e (K = d)
+  static constexpr int zs = bop2 + 4096;                    // dz [2][32] f32
+  static constexpr int rope = zs + 256;
   static constexpr int bars = rope + kRopeTableMax * 8;
-  // full[3] empty[3] ready[3] t_full[3] t_empty[3] b_ready mma_done
+  // full[6] empty[6] ready[6] t_full[6] t_empty[6] b_ready mma_done
   static constexpr int nbars = 5 * kBStages + 2;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int bytes = misc + 16;
@@ -87,7 +95,7 @@ static_assert(kQSmemBytes <= 232448 && kKVSmemBytes <= 232448, "shared memory pe
 
 struct BwdArgs {
   float* partials;        // query side: [B*H][splits][kStateFloats]
-  unsigned* arrive;       // query side: per head-group arrival counters (index b*H + h0)
+  unsigned* arrive;       // query side: per head-pair arrival counters (index b*H + h0)
   StateOut out;           // query side: where the combined (dS, dz) goes
   const float* S;         // query side: the forward state; key side: dS
   const float* z;         // query side: z; key side: dz
@@ -129,15 +137,15 @@ __device__ __forceinline__ void rotate_chunk(const float2 (&cs)[16], int j0, flo
   }
 }
 
-// Build a 4-head B operand in shared memory from a float32 [heads][32][32]
-// global array M: row r of head pair j holds M[h][r][0..31] (transpose = 0) or
-// M[h][0..31][r] (transpose = 1) of heads 2j and 2j+1, in bf16, K-major with
-// the 128-byte swizzle. Missing heads are zero.
+// Build a head pair's B operand in shared memory from a float32 [heads][32][32]
+// global array M: row r holds M[h][r][0..31] (transpose = 0) or M[h][0..31][r]
+// (transpose = 1) of heads h0 and h0 + 1, in bf16, K-major with the 128-byte
+// swizzle. A missing head is zero.
 __device__ __forceinline__ void build_bop(uint32_t bop, const float* M, size_t cidx, int h0,
                                           int H, bool transpose, int mt, int nthreads) {
-  for (int idx = mt; idx < 2 * 32 * 8; idx += nthreads) {
-    const int j = idx >> 8, r = (idx >> 3) & 31, c = idx & 7;
-    const int hh = 2 * j + (c >> 2), k0 = (c & 3) * 8;
+  for (int idx = mt; idx < 32 * 8; idx += nthreads) {
+    const int r = idx >> 3, c = idx & 7;
+    const int hh = c >> 2, k0 = (c & 3) * 8;
     float x[8];
     if (h0 + hh < H) {
       const float* m = M + (cidx + hh) * kD * kD;
@@ -147,7 +155,7 @@ __device__ __forceinline__ void build_bop(uint32_t bop, const float* M, size_t c
 #pragma unroll
       for (int k = 0; k < 8; ++k) x[k] = 0.0f;
     }
-    st_shared_v4(bop + j * 4096 + sw128_offset(r, c), pack8(x));
+    st_shared_v4(bop + sw128_offset(r, c), pack8(x));
   }
 }
 
@@ -177,8 +185,8 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   unsigned* err = &g_bwd_tc_error;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int group = blockIdx.y, b = blockIdx.z;
-  const int h0 = group * kGroupHeads;
+  const int pair = blockIdx.y, b = blockIdx.z;
+  const int h0 = pair * kPair;
   const size_t cidx = static_cast<size_t>(b) * p.H + h0;
   const int n_begin = blockIdx.x * p.chunk;
   const int n_end = min(p.N, n_begin + p.chunk);
@@ -227,9 +235,7 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         uint8_t* st = smem + QSmem::stages + s * kBTile;
         const int y = n_begin + i * kBT;
         tma_load_3d(st, &tm_q, &full[s], h0 * 32, y, b);
-        tma_load_3d(st + kBBox, &tm_q, &full[s], h0 * 32 + 64, y, b);
-        tma_load_3d(st + 2 * kBBox, &tm_g, &full[s], h0 * 32, y, b);
-        tma_load_3d(st + 3 * kBBox, &tm_g, &full[s], h0 * 32 + 64, y, b);
+        tma_load_3d(st + kBBox, &tm_g, &full[s], h0 * 32, y, b);
       }
       for (int q = max(0, i - kBStages); q < i; ++q)
         mbar_drain(&full[q % kBStages], (q / kBStages) & 1, err, kErrWait);
@@ -239,7 +245,7 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     if (lane == 0) {
       bool ok = nT == 0 || mbar_wait(b_ready, 0, abort_flag, err, kErrWait);
       const uint32_t id_t = idesc_bf16_f32(128, 32, 0, 0);
-      const uint32_t id_s = idesc_bf16_f32(128, 128, 1, 1);
+      const uint32_t id_s = idesc_bf16_f32(128, 64, 1, 1);
       const uint32_t bop = sbase + QSmem::bop;
       // MMA 2 of tile i - 1 is issued after MMA 1 of tile i
       for (int i = 0; ok && i <= nT; ++i) {
@@ -249,14 +255,12 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           tc_fence_after();
           const uint32_t st = sbase + QSmem::stages + s * kBTile;
 #pragma unroll
-          for (int hh = 0; hh < kGroupHeads; ++hh) {
-            const uint32_t koff = (hh & 1) * 64;
+          for (int hh = 0; hh < kPair; ++hh) {
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
-              const uint64_t ad =
-                  smem_desc_sw128(st + 2 * kBBox + (hh >> 1) * kBBox + koff + kk * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(bop + (hh >> 1) * 4096 + koff + kk * 32, 16, 1024);
-              mma_bf16(tmem + 128 + s * 128 + hh * 32, ad, bd, id_t, kk);
+              const uint64_t ad = smem_desc_sw128(st + kBBox + hh * 64 + kk * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(bop + hh * 64 + kk * 32, 16, 1024);
+              mma_bf16(tmem + 64 * s + hh * 32, ad, bd, id_t, kk);
             }
           }
           mma_commit(&t_full[s]);
@@ -269,9 +273,11 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           const uint32_t st = sbase + QSmem::stages + s * kBTile;
 #pragma unroll
           for (int kk = 0; kk < kBT / 16; ++kk) {
+            // A: phi(Q) as M = 128 dims; its second 64-dim atom (LBO) is the
+            // dO box, whose rows of the product are not used
             const uint64_t ad = smem_desc_sw128(st + kk * 2048, kBBox, 1024);
-            const uint64_t bd = smem_desc_sw128(st + 2 * kBBox + kk * 2048, kBBox, 1024);
-            mma_bf16(tmem, ad, bd, id_s, (k > 0 || kk > 0) ? 1u : 0u);
+            const uint64_t bd = smem_desc_sw128(st + kBBox + kk * 2048, kBBox, 1024);
+            mma_bf16(tmem + kColDS, ad, bd, id_s, (k > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&empty[s]);
         }
@@ -288,20 +294,20 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     const int row = quad * 32 + lane;     // token row of the tile (thread = row)
     bool alive = true;
 
-    // S as the B operand of MMA 1 (rows d, K = e), z of the four heads
+    // S as the B operand of MMA 1 (rows d, K = e), z of the two heads
     build_bop(sbase + QSmem::bop, a.S, cidx, h0, p.H, false, mt, kBMath);
-    if (mt < kGroupHeads * kD) zs[mt] = h0 + mt / kD < p.H ? __ldcg(a.z + cidx * kD + mt) : 0.0f;
+    if (mt < kPair * kD) zs[mt] = h0 + mt / kD < p.H ? __ldcg(a.z + cidx * kD + mt) : 0.0f;
     fence_proxy_async_smem();
     named_bar_sync(kBarAll, kBMath);
     if (mt == 0) mbar_arrive(b_ready);
 
-    // dz of dims [(c&3)*8, +8) of head c>>2 over rows rg, rg + 8, ...
-    const int zc = wt & 15, zrg = wt >> 4;
+    // dz of dims [(c&3)*8, +8) of head c>>2 over rows rg, rg + 16, ...
+    const int zc = wt & 7, zrg = wt >> 3;
     float zacc[8] = {};
-    float* my_dden = dden_buf + wg * kBT * 4;
+    float* my_dden = dden_buf + wg * kBT * kPair;
 
     for (int j = wg; j < nT; j += kBWG) {
-      const int s = wg;  // j % kBStages
+      const int s = j % kBStages;  // wg or wg + 3
       const uint32_t par = (j / kBStages) & 1;
       bool ok = mbar_wait(&full[s], par, abort_flag, err, kErrWait);
       if (bar_any(kBarW0 + wg, 128, !ok || *abort_flag)) {
@@ -315,14 +321,14 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       if (kRope != kNoRope) row_angles<kRope>(p, rope_tab, n, cs);
 
       // ---- transform: ReLU(Q) in place, den, dnum = dO / den in place
-      float inv[kGroupHeads];
+      float inv[kPair];
 #pragma unroll
-      for (int hh = 0; hh < kGroupHeads; ++hh) {
+      for (int hh = 0; hh < kPair; ++hh) {
         float den = 0.0f;
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
           const int c = hh * 4 + c4;
-          const uint32_t addr = st + (c >> 3) * kBBox + sw128_offset(row, c & 7);
+          const uint32_t addr = st + sw128_offset(row, c);
           uint4 u = ld_shared_v4(addr);
           u.x = relu_bf16x2(u.x);
           u.y = relu_bf16x2(u.y);
@@ -339,7 +345,7 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
           const int c = hh * 4 + c4;
-          const uint32_t addr = st + 2 * kBBox + (c >> 3) * kBBox + sw128_offset(row, c & 7);
+          const uint32_t addr = st + kBBox + sw128_offset(row, c);
           float x[8];
           unpack8(ld_shared_v4(addr), x);
 #pragma unroll
@@ -359,10 +365,9 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       }
       const bool row_ok = n < n_end;
 #pragma unroll
-      for (int hh = 0; hh < kGroupHeads; ++hh) {
+      for (int hh = 0; hh < kPair; ++hh) {
         float t[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 128 + s * 128 + hh * 32,
-                           t);
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 64 * s + hh * 32, t);
         if (kRope != kNoRope) {
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
@@ -380,12 +385,12 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         for (int c4 = 0; c4 < 4; ++c4) {
           const int c = hh * 4 + c4;
           float x[8];
-          unpack8(ld_shared_v4(st + (c >> 3) * kBBox + sw128_offset(row, c & 7)), x);
+          unpack8(ld_shared_v4(st + sw128_offset(row, c)), x);
 #pragma unroll
           for (int e = 0; e < 8; ++e) dot = fmaf(x[e], t[c4 * 8 + e], dot);
         }
         const float dden = -dot * inv[hh];
-        my_dden[row * 4 + hh] = dden;
+        my_dden[row * kPair + hh] = dden;
         if (row_ok && h0 + hh < p.H) {
           const float* zz = zs + hh * kD;
           __nv_bfloat16* dst = a.dQ + ((static_cast<size_t>(b) * p.N + n) * p.H + h0 + hh) * kD;
@@ -393,7 +398,7 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           for (int c4 = 0; c4 < 4; ++c4) {
             const int c = hh * 4 + c4;
             float x[8];
-            unpack8(ld_shared_v4(st + (c >> 3) * kBBox + sw128_offset(row, c & 7)), x);
+            unpack8(ld_shared_v4(st + sw128_offset(row, c)), x);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const int d = c4 * 8 + e;
@@ -410,10 +415,10 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       {
         const int hh = zc >> 2;
 #pragma unroll 4
-        for (int r = zrg; r < kBT; r += 8) {
+        for (int r = zrg; r < kBT; r += 16) {
           float x[8];
-          unpack8(ld_shared_v4(st + (zc >> 3) * kBBox + sw128_offset(r, zc & 7)), x);
-          const float dd = my_dden[r * 4 + hh];
+          unpack8(ld_shared_v4(st + sw128_offset(r, zc)), x);
+          const float dd = my_dden[r * kPair + hh];
 #pragma unroll
           for (int e = 0; e < 8; ++e) zacc[e] = fmaf(dd, x[e], zacc[e]);
         }
@@ -423,8 +428,8 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       // ---- rewrite ReLU(Q) -> phi(Q) for MMA 2
       if (kRope != kNoRope) {
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint32_t addr = st + (c >> 3) * kBBox + sw128_offset(row, c & 7);
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t addr = st + sw128_offset(row, c);
           float x[8];
           unpack8(ld_shared_v4(addr), x);
           rotate_chunk<1>(cs, (c & 3) * 4, x);
@@ -438,14 +443,14 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     // ---- partial (dS, dz) of this split
     alive = !bar_any(kBarAll, kBMath, !alive || *abort_flag);
     float* scratch = reinterpret_cast<float*>(smem + QSmem::stages);  // [kBMath][8] after the MMAs
-    if (warp >= 2 && warp < 6) {
+    if (warp >= 2 && warp < 6 && (warp & 3) < kPair) {  // TMEM lanes of head q's dS rows
       const int q = warp & 3;
       float v[32];
       bool got = alive && nT > 0 && mbar_wait(acc_full, 0, abort_flag, err, kErrWait);
       got = __all_sync(0xffffffffu, got);
       if (got) {
         tc_fence_after();
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32 * q, v);
+        tmem_ld_32x32b_x32(tmem + kColDS + (static_cast<uint32_t>(32 * q) << 16) + 32 * q, v);
       } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = 0.0f;
@@ -465,12 +470,12 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       for (int e = 0; e < 8; ++e) scratch[mt * 8 + e] = zacc[e];
     }
     named_bar_sync(kBarAll, kBMath);
-    if (alive && mt < kGroupHeads * kD) {
+    if (alive && mt < kPair * kD) {
       const int q = mt >> 5, d = mt & 31;
       const int col = q * 4 + (d >> 3), e = d & 7;
       float sum = 0.0f;
       for (int w = 0; w < kBWG; ++w)
-        for (int rg = 0; rg < 8; ++rg) sum += scratch[(w * 128 + rg * 16 + col) * 8 + e];
+        for (int rg = 0; rg < 16; ++rg) sum += scratch[(w * 128 + rg * 8 + col) * 8 + e];
       if (h0 + q < p.H)
         a.partials[((cidx + q) * p.splits + blockIdx.x) * kStateFloats + kD * kD + d] = sum;
     }
@@ -486,7 +491,7 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     }
     named_bar_sync(kBarAll, kBMath);
     const bool last = *last_flag != 0;
-    if (last && alive) combine_from_global<kBMath>(p, b, h0, mt, a.partials, a.out);
+    if (last && alive) combine_from_global<kBMath, kPair>(p, b, h0, mt, a.partials, a.out);
     named_bar_sync(kBarAll, kBMath);
     if (mt == 0 && last) a.arrive[cidx] = 0u;
   }
@@ -523,8 +528,8 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
   unsigned* err = &g_bwd_tc_error;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int group = blockIdx.y, b = blockIdx.z;
-  const int h0 = group * kGroupHeads;
+  const int pair = blockIdx.y, b = blockIdx.z;
+  const int h0 = pair * kPair;
   const size_t cidx = static_cast<size_t>(b) * p.H + h0;
   const int ntiles_all = (p.N + kBT - 1) / kBT;
   const int tile_begin = blockIdx.x * a.tiles_per_cta;
@@ -574,9 +579,7 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         uint8_t* st = smem + KVSmem::stages + s * kBTile;
         const int y = (tile_begin + i) * kBT;
         tma_load_3d(st, &tm_k, &full[s], h0 * 32, y, b);
-        tma_load_3d(st + kBBox, &tm_k, &full[s], h0 * 32 + 64, y, b);
-        tma_load_3d(st + 2 * kBBox, &tm_v, &full[s], h0 * 32, y, b);
-        tma_load_3d(st + 3 * kBBox, &tm_v, &full[s], h0 * 32 + 64, y, b);
+        tma_load_3d(st + kBBox, &tm_v, &full[s], h0 * 32, y, b);
       }
       for (int q = max(0, i - kBStages); q < i; ++q)
         mbar_drain(&full[q % kBStages], (q / kBStages) & 1, err, kErrWait);
@@ -597,16 +600,13 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
           tc_fence_after();
           const uint32_t st = sbase + KVSmem::stages + s * kBTile;
 #pragma unroll
-          for (int hh = 0; hh < kGroupHeads; ++hh) {
-            const uint32_t koff = (hh & 1) * 64;
+          for (int hh = 0; hh < kPair; ++hh) {
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
               // dphi(K)[n][d] = sum_e V[n][e] dS[d][e]
-              const uint64_t av =
-                  smem_desc_sw128(st + 2 * kBBox + (hh >> 1) * kBBox + koff + kk * 32, 16, 1024);
-              const uint64_t bd =
-                  smem_desc_sw128(bop1 + (hh >> 1) * 4096 + koff + kk * 32, 16, 1024);
-              mma_bf16(tmem + s * 128 + hh * 32, av, bd, id, kk);
+              const uint64_t av = smem_desc_sw128(st + kBBox + hh * 64 + kk * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(bop1 + hh * 64 + kk * 32, 16, 1024);
+              mma_bf16(tmem + s * 64 + hh * 32, av, bd, id, kk);
             }
           }
           mma_commit(&t_full[s]);
@@ -618,15 +618,13 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
           tc_fence_after();
           const uint32_t st = sbase + KVSmem::stages + s * kBTile;
 #pragma unroll
-          for (int hh = 0; hh < kGroupHeads; ++hh) {
-            const uint32_t koff = (hh & 1) * 64;
+          for (int hh = 0; hh < kPair; ++hh) {
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
               // dV[n][e] = sum_d phi(K)[n][d] dS[d][e]
-              const uint64_t ak = smem_desc_sw128(st + (hh >> 1) * kBBox + koff + kk * 32, 16, 1024);
-              const uint64_t bd =
-                  smem_desc_sw128(bop2 + (hh >> 1) * 4096 + koff + kk * 32, 16, 1024);
-              mma_bf16(tmem + s * 128 + hh * 32, ak, bd, id, kk);
+              const uint64_t ak = smem_desc_sw128(st + hh * 64 + kk * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(bop2 + hh * 64 + kk * 32, 16, 1024);
+              mma_bf16(tmem + s * 64 + hh * 32, ak, bd, id, kk);
             }
           }
           mma_commit(&t_full[s]);
@@ -644,13 +642,13 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
 
     build_bop(sbase + KVSmem::bop1, a.S, cidx, h0, p.H, false, mt, kBMath);
     build_bop(sbase + KVSmem::bop2, a.S, cidx, h0, p.H, true, mt, kBMath);
-    if (mt < kGroupHeads * kD) zs[mt] = h0 + mt / kD < p.H ? __ldcg(a.z + cidx * kD + mt) : 0.0f;
+    if (mt < kPair * kD) zs[mt] = h0 + mt / kD < p.H ? __ldcg(a.z + cidx * kD + mt) : 0.0f;
     fence_proxy_async_smem();
     named_bar_sync(kBarAll, kBMath);
     if (mt == 0) mbar_arrive(b_ready);
 
     for (int j = wg; j < nT; j += kBWG) {
-      const int s = wg;  // j % kBStages
+      const int s = j % kBStages;  // wg or wg + 3
       bool ok = mbar_wait(&full[s], (j / kBStages) & 1, abort_flag, err, kErrWait);
       if (bar_any(kBarW0 + wg, 128, !ok || *abort_flag)) break;
       const uint32_t st = sbase + KVSmem::stages + s * kBTile;
@@ -659,10 +657,10 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       if (kRope != kNoRope) row_angles<kRope>(p, rope_tab, n0 + row, cs);
 
       // ---- transform: K -> phi(K) in place; keep the sign mask of K
-      uint32_t mask[kGroupHeads] = {0u, 0u, 0u, 0u};
+      uint32_t mask[kPair] = {0u, 0u};
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const uint32_t addr = st + (c >> 3) * kBBox + sw128_offset(row, c & 7);
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t addr = st + sw128_offset(row, c);
         uint4 v = ld_shared_v4(addr);
         v.x = relu_bf16x2(v.x);
         v.y = relu_bf16x2(v.y);
@@ -682,13 +680,13 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       fence_proxy_async_smem();
       mbar_arrive(&ready[s]);
 
-      const uint32_t tcol = tmem + (static_cast<uint32_t>(quad * 32) << 16) + s * 128;
+      const uint32_t tcol = tmem + (static_cast<uint32_t>(quad * 32) << 16) + s * 64;
       // ---- dK = R^T dphi(K) + dz, masked, over the V tile (MMA 1 has read it)
       ok = mbar_wait(&t_full[s], 0, abort_flag, err, kErrWait);
       tc_fence_after();
       if (bar_any(kBarW0 + wg, 128, !ok || *abort_flag)) break;
 #pragma unroll
-      for (int hh = 0; hh < kGroupHeads; ++hh) {
+      for (int hh = 0; hh < kPair; ++hh) {
         float g[32];
         tmem_ld_32x32b_x32(tcol + hh * 32, g);
         const float* zz = zs + hh * kD;
@@ -704,7 +702,7 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
             x[e] = (mask[hh] >> d) & 1u ? x[e] + zz[d] : 0.0f;
           }
           const int c = hh * 4 + c4;
-          st_shared_v4(st + 2 * kBBox + (c >> 3) * kBBox + sw128_offset(row, c & 7), pack8(x));
+          st_shared_v4(st + kBBox + sw128_offset(row, c), pack8(x));
         }
       }
       tc_fence_before();
@@ -716,7 +714,7 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       tc_fence_after();
       if (bar_any(kBarW0 + wg, 128, !ok || *abort_flag)) break;
 #pragma unroll
-      for (int hh = 0; hh < kGroupHeads; ++hh) {
+      for (int hh = 0; hh < kPair; ++hh) {
         float g[32];
         tmem_ld_32x32b_x32(tcol + hh * 32, g);
 #pragma unroll
@@ -725,7 +723,7 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[e] = g[c4 * 8 + e];
           const int c = hh * 4 + c4;
-          st_shared_v4(st + (c >> 3) * kBBox + sw128_offset(row, c & 7), pack8(x));
+          st_shared_v4(st + sw128_offset(row, c), pack8(x));
         }
       }
       tc_fence_before();
@@ -734,10 +732,8 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       if (leader) {
         mbar_arrive(&t_empty[s]);
         uint8_t* tile = smem + KVSmem::stages + s * kBTile;
-        tma_store_3d(&tm_dk, tile + 2 * kBBox, h0 * 32, n0, b);
-        tma_store_3d(&tm_dk, tile + 3 * kBBox, h0 * 32 + 64, n0, b);
+        tma_store_3d(&tm_dk, tile + kBBox, h0 * 32, n0, b);
         tma_store_3d(&tm_dv, tile, h0 * 32, n0, b);
-        tma_store_3d(&tm_dv, tile + kBBox, h0 * 32 + 64, n0, b);
         bulk_commit();
         bulk_wait_read<0>();
         mbar_arrive(&empty[s]);
@@ -794,8 +790,17 @@ cudaError_t launch_backward_q_tc(const Problem& p, const void* Q, const void* dO
   a.S = S;
   a.z = z;
   a.dQ = static_cast<__nv_bfloat16*>(dQ);
-  const dim3 grid(p.splits, (p.H + kGroupHeads - 1) / kGroupHeads, p.B);
-  e = launch_pdl(kern, grid, kQSmemBytes, s, mq, mg, p, a);
+  // token splits for head pairs (one wave); never more than the state
+  // reduce's, for which the workspace is sized
+  const int pairs = (p.H + kPair - 1) / kPair;
+  Problem pb = p;
+  const long long units = static_cast<long long>(pairs) * p.B;
+  int splits = static_cast<int>(std::max<long long>(1, kNumSMs / std::max<long long>(1, units)));
+  splits = std::min(splits, std::min(p.splits, (p.N + kBT - 1) / kBT));
+  pb.chunk = ((p.N + splits - 1) / splits + kBT - 1) / kBT * kBT;
+  pb.splits = (p.N + pb.chunk - 1) / pb.chunk;
+  const dim3 grid(pb.splits, pairs, p.B);
+  e = launch_pdl(kern, grid, kQSmemBytes, s, mq, mg, pb, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -816,7 +821,7 @@ cudaError_t launch_backward_kv_tc(const Problem& p, const void* K, const void* V
   if ((e = ensure_smem_attr(3 + mode, reinterpret_cast<const void*>(kern), kKVSmemBytes)) !=
       cudaSuccess)
     return e;
-  const int groups = (p.H + kGroupHeads - 1) / kGroupHeads;
+  const int groups = (p.H + kPair - 1) / kPair;
   const int ntiles = (p.N + kBT - 1) / kBT;
   const long long units = static_cast<long long>(groups) * p.B;
   int ctas = static_cast<int>(std::max<long long>(1, kNumSMs / std::max<long long>(1, units)));

@@ -175,14 +175,14 @@ __device__ __forceinline__ bool spin_flag(const unsigned* flag, volatile int* ab
 // at most kPerThread float4 columns and issues the loads of all of them for 4
 // splits at once before adding, so the combine costs one L2 round trip per 4
 // splits.
-template <int kThreads>
+template <int kThreads, int kHeads = kGroupHeads>
 __device__ __forceinline__ void combine_from_global(const Problem& p, int b, int h0, int mt,
                                                     const float* partials, const StateOut& out,
                                                     float* s_smem = nullptr,
                                                     float* z_smem = nullptr) {
   constexpr int kVec = kStateFloats / 4;                     // 264 float4 per head
-  constexpr int kPerThread = (kGroupHeads * kVec + kThreads - 1) / kThreads;
-  const int heads = min(kGroupHeads, p.H - h0);
+  constexpr int kPerThread = (kHeads * kVec + kThreads - 1) / kThreads;
+  const int heads = min(kHeads, p.H - h0);
   const size_t cidx = static_cast<size_t>(b) * p.H + h0;
   float4 acc[kPerThread];
   const float* src[kPerThread];
