@@ -247,9 +247,9 @@ la_status la_state_reduce_static(const la_shape* shape, const void* K,
 
 /* Kernel launches that la_attention, and la_block_causal_step with update 0
  * or 1, make for `shape`: 1 when the whole layer runs as one cooperative
- * launch (bf16 I/O, one wave of co-resident CTAs, at most 2^19 token-heads),
- * else 2 (state reduce, then apply). The two give bitwise identical results.
- * 0 for an invalid shape. Pure host function. */
+ * launch (bf16 I/O and a grid of splits x ceil(H/4) x B CTAs that fits one
+ * wave of co-resident CTAs), else 2 (state reduce, then apply). The two give
+ * bitwise identical results. 0 for an invalid shape. Pure host function. */
 int la_attention_launches(const la_shape* shape);
 
 /* Static description of a status code. Never NULL. */

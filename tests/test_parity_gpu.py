@@ -134,7 +134,7 @@ def test_single_launch_layer_and_two_kernel_fallback(cuda_device):
     CTAs covers it, else as reduce + apply; both match the oracle and each
     other bit for bit."""
     assert la.la_attention_launches(la.make_shape(4, 1024, 70)) == 1
-    assert la.la_attention_launches(la.make_shape(1, 16384, 70)) == 2   # large: two kernels
+    assert la.la_attention_launches(la.make_shape(1, 16384, 70)) == 1   # 144 CTAs: one wave
     assert la.la_attention_launches(la.make_shape(4, 1024, 70, io_dtype="f32")) == 2
     # 80 batch elements x 2 head groups = 160 CTAs > one wave: two kernels
     shape = la.make_shape(80, 200, 8)
@@ -143,8 +143,9 @@ def test_single_launch_layer_and_two_kernel_fallback(cuda_device):
     _full_check(Q, K, V, th, eps, "bf16", what="two-kernel fallback")
 
 
-def test_fused_and_two_kernel_paths_are_bitwise_equal(cuda_device):
-    w = wl.WORKLOADS["sana1.6b_1024px"]
+@pytest.mark.parametrize("name", ["sana1.6b_1024px", "sana1.6b_4k"])
+def test_fused_and_two_kernel_paths_are_bitwise_equal(cuda_device, name):
+    w = wl.WORKLOADS[name]
     Q, K, V = P.to_dev(*wl.make_qkv(w, 17))
     shape = la.shape_for(Q, eps=w.eps)
     assert la.la_attention_launches(shape) == 1
