@@ -259,6 +259,14 @@ const char* la_status_string(la_status status);
  * string if none). The pointer stays valid until the thread's next call. */
 const char* la_last_error(void);
 
+/* Health check of the device-side waits: one warp waits for a barrier phase
+ * that nothing completes; after limit_us microseconds (1 .. 10^7) it gives
+ * up, raises bit 0 of the device error word (see la_device_error) and
+ * returns, as a stalled pipeline stage of the library's kernels would. The
+ * context stays usable. Asynchronous on `stream`; LA_OK means the launch
+ * succeeded. */
+la_status la_wait_selftest(unsigned limit_us, la_stream stream);
+
 /* Device-side error word of the current device: non-zero when a kernel of
  * this library gave up on a bounded wait (a pipeline stage that never
  * arrived; the kernel then drained its copies and returned without a valid

@@ -91,6 +91,8 @@ _lib.la_last_error.restype = ctypes.c_char_p
 _lib.la_attention_launches.argtypes = [_shape_p]
 _lib.la_attention_launches.restype = _i
 _lib.la_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), _i]
+_lib.la_wait_selftest.argtypes = [ctypes.c_uint, _vp]
+_lib.la_wait_selftest.restype = _i
 _lib.la_device_error.restype = _i
 
 
@@ -212,6 +214,12 @@ def la_status_string(status: int) -> str:
 
 def la_last_error() -> str:
     return _lib.la_last_error().decode()
+
+
+def la_wait_selftest(limit_us: int, stream=None) -> None:
+    """Launch a warp whose wait nothing satisfies; it gives up after limit_us
+    and raises the device error word (see la_device_error)."""
+    _check(_lib.la_wait_selftest(int(limit_us), _stream(stream)), "la_wait_selftest")
 
 
 def la_device_error(reset: bool = False) -> int:

@@ -525,6 +525,14 @@ const char* la_status_string(la_status status) {
 
 const char* la_last_error(void) { return g_last_error.c_str(); }
 
+la_status la_wait_selftest(unsigned limit_us, la_stream stream) {
+  if (limit_us == 0 || limit_us > 10000000u)
+    return fail(LA_ERR_INVALID_ARG, "limit_us=%u (1 .. 10^7)", limit_us);
+  const cudaError_t e = launch_wait_selftest(limit_us, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "wait self-test");
+  return LA_OK;
+}
+
 la_status la_device_error(unsigned* code, int reset) {
   if (code == nullptr) return fail(LA_ERR_INVALID_ARG, "code is NULL");
   unsigned fwd = 0, bwd = 0, conv = 0, causal = 0;

@@ -130,6 +130,8 @@ cudaError_t launch_temporal_conv(const ConvProblem& cp, const void* x, const flo
 // Device error words of the tensor-core kernels (bounded waits that gave up):
 // the forward's (la_tc.cu) and the backward's (la_backward_tc.cu).
 cudaError_t read_device_error(unsigned* code, bool reset);
+// One warp waiting on a barrier that nothing completes, bounded by limit_us.
+cudaError_t launch_wait_selftest(unsigned limit_us, cudaStream_t s);
 cudaError_t read_device_error_bwd(unsigned* code, bool reset);
 cudaError_t read_device_error_conv(unsigned* code, bool reset);  // la_conv.cu
 cudaError_t read_device_error_causal(unsigned* code, bool reset);  // la_causal_tc.cu

@@ -595,6 +595,21 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
   }
 }
 
+// Health check of the bounded waits: one warp waits for a barrier phase that
+// nothing completes; the wait gives up after limit_ns and raises the error
+// word, exactly as a stalled pipeline stage of the kernels above would.
+__global__ void __launch_bounds__(32) wait_selftest(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);  // one arrival expected; none comes
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncwarp();
+  mbar_wait(&bar, 0, &abort_flag, &g_tc_error, kErrWait, limit_ns);
+}
+
 // ============================================================== host side
 
 // Launch of layer_tc with programmatic dependent launch (the prologue may
@@ -753,6 +768,11 @@ cudaError_t launch_layer_tc(const Problem& p, const void* Q, const void* K, cons
   const dim3 grid(p.splits, (p.H + kGroupHeads - 1) / kGroupHeads, p.B);
   e = launch_layer(kern, grid, s, true, mk, mv, mq, mo, p, rt, a);
   if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_selftest(unsigned limit_us, cudaStream_t s) {
+  wait_selftest<<<1, 32, 0, s>>>(static_cast<unsigned long long>(limit_us) * 1000ull);
   return cudaGetLastError();
 }
 

@@ -129,3 +129,10 @@ def test_binding_raises_with_detail():
     s = la.make_shape(1, 8, 1, D=16)
     with pytest.raises(la.LaError, match="only 32"):
         la._check(_call("la_apply", ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None), "la_apply")
+
+
+def test_wait_selftest_rejects_limits_out_of_range():
+    import linear_attention_diffusion_b200 as la
+    for bad in (0, 10_000_001):  # refused on the host, before any launch
+        with pytest.raises(la.LaError):
+            la.la_wait_selftest(bad, stream=0)
