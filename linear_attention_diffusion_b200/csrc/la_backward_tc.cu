@@ -164,7 +164,7 @@ __device__ __forceinline__ void build_bop(uint32_t bop, const float* M, size_t c
 template <int kRope>
 __global__ void __launch_bounds__(kBThreads, 1)
 bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
-         const Problem p, const BwdArgs a) {
+         const __grid_constant__ CUtensorMap tm_dq, const Problem p, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -215,6 +215,7 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_g);
+    prefetch_tmap(&tm_dq);
   }
   if (kRope == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kBMath);
   __syncthreads();
@@ -247,8 +248,30 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       const uint32_t id_t = idesc_bf16_f32(128, 32, 0, 0);
       const uint32_t id_s = idesc_bf16_f32(128, 64, 1, 1);
       const uint32_t bop = sbase + QSmem::bop;
-      // MMA 2 of tile i - 1 is issued after MMA 1 of tile i
-      for (int i = 0; ok && i <= nT; ++i) {
+      // Without RoPE, phi(Q) = ReLU(Q) is in place after the transform, so both
+      // MMAs of a tile go at once and the epilogue may then write dQ over the
+      // dnum box. With RoPE, MMA 2 of tile i - 1 (after the warpgroup has
+      // rotated Q in place) is issued after MMA 1 of tile i.
+      for (int i = 0; kRope == kNoRope && ok && i < nT; ++i) {
+        const int s = i % kBStages;
+        if (!(ok = mbar_wait(&ready_t[s], (i / kBStages) & 1, abort_flag, err, kErrWait))) break;
+        tc_fence_after();
+        const uint32_t st = sbase + QSmem::stages + s * kBTile;
+#pragma unroll
+        for (int hh = 0; hh < kPair; ++hh)
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            mma_bf16(tmem + 64 * s + hh * 32,
+                     smem_desc_sw128(st + kBBox + hh * 64 + kk * 32, 16, 1024),
+                     smem_desc_sw128(bop + hh * 64 + kk * 32, 16, 1024), id_t, kk);
+#pragma unroll
+        for (int kk = 0; kk < kBT / 16; ++kk)
+          mma_bf16(tmem + kColDS, smem_desc_sw128(st + kk * 2048, kBBox, 1024),
+                   smem_desc_sw128(st + kBBox + kk * 2048, kBBox, 1024), id_s,
+                   (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&t_full[s]);
+      }
+      for (int i = 0; kRope != kNoRope && ok && i <= nT; ++i) {
         if (i < nT) {
           const int s = i % kBStages;
           if (!(ok = mbar_wait(&ready_t[s], (i / kBStages) & 1, abort_flag, err, kErrWait))) break;
@@ -391,7 +414,23 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         }
         const float dden = -dot * inv[hh];
         my_dden[row * kPair + hh] = dden;
-        if (row_ok && h0 + hh < p.H) {
+        if (kRope == kNoRope) {
+          // both MMAs are done: dQ goes over the dnum box, stored with TMA
+          // (rows and heads beyond the tensor are clipped by the store)
+          const float* zz = zs + hh * kD;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int c = hh * 4 + c4;
+            float x[8];
+            unpack8(ld_shared_v4(st + sw128_offset(row, c)), x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int d = c4 * 8 + e;
+              x[e] = x[e] > 0.0f ? fmaf(dden, zz[d], t[d]) : 0.0f;
+            }
+            st_shared_v4(st + kBBox + sw128_offset(row, c), pack8(x));
+          }
+        } else if (row_ok && h0 + hh < p.H) {
           const float* zz = zs + hh * kD;
           __nv_bfloat16* dst = a.dQ + ((static_cast<size_t>(b) * p.N + n) * p.H + h0 + hh) * kD;
 #pragma unroll
@@ -409,6 +448,7 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         }
       }
       tc_fence_before();
+      if (kRope == kNoRope) fence_proxy_async_smem();  // dQ in shared memory, for the store
       named_bar_sync(kBarW0 + wg, 128);
 
       // ---- dz over the tile's rows (fixed order per thread)
@@ -425,6 +465,16 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       }
       named_bar_sync(kBarW0 + wg, 128);
 
+      if (kRope == kNoRope) {
+        // the stage is done with: store dQ, then hand it back to the TMA warp
+        if (wt == 0) {
+          tma_store_3d(&tm_dq, smem + QSmem::stages + s * kBTile + kBBox, h0 * 32, n0, b);
+          bulk_commit();
+          bulk_wait_read<0>();
+          mbar_arrive(&empty[s]);
+        }
+        continue;
+      }
       // ---- rewrite ReLU(Q) -> phi(Q) for MMA 2
       if (kRope != kNoRope) {
 #pragma unroll
@@ -440,6 +490,7 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       mbar_arrive(&ready_s[s]);
     }
 
+    if (kRope == kNoRope && wt == 0) bulk_wait<0>();
     // ---- partial (dS, dz) of this split
     alive = !bar_any(kBarAll, kBMath, !alive || *abort_flag);
     float* scratch = reinterpret_cast<float*>(smem + QSmem::stages);  // [kBMath][8] after the MMAs
@@ -774,10 +825,11 @@ cudaError_t launch_pdl(Kernel kern, dim3 grid, int smem, cudaStream_t s, const A
 cudaError_t launch_backward_q_tc(const Problem& p, const void* Q, const void* dO, const float* S,
                                  const float* z, void* dQ, float* partials, unsigned* counters,
                                  const StateOut& out, cudaStream_t s) {
-  CUtensorMap mq, mg;
+  CUtensorMap mq, mg, mdq;
   cudaError_t e;
   if ((e = make_map(&mq, Q, p, kBT)) != cudaSuccess) return e;
   if ((e = make_map(&mg, dO, p, kBT)) != cudaSuccess) return e;
+  if ((e = make_map(&mdq, dQ, p, kBT)) != cudaSuccess) return e;
   const int mode = rope_mode(rope_table_for(p));
   auto kern = mode == kNoRope ? bwd_q_tc<kNoRope>
                               : (mode == kRopeTable ? bwd_q_tc<kRopeTable> : bwd_q_tc<kRopeOnTheFly>);
@@ -800,7 +852,7 @@ cudaError_t launch_backward_q_tc(const Problem& p, const void* Q, const void* dO
   pb.chunk = ((p.N + splits - 1) / splits + kBT - 1) / kBT * kBT;
   pb.splits = (p.N + pb.chunk - 1) / pb.chunk;
   const dim3 grid(pb.splits, pairs, p.B);
-  e = launch_pdl(kern, grid, kQSmemBytes, s, mq, mg, pb, a);
+  e = launch_pdl(kern, grid, kQSmemBytes, s, mq, mg, mdq, pb, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
