@@ -16,11 +16,15 @@
 // 128-token tile of a head pair (one 64-dim TMA box per tensor),
 //   transform  Q -> ReLU(Q) and dO -> dnum (bf16) in place in shared memory;
 //   MMA 1      t = dnum S^T per head (M = 128 tokens, N = 32, K = 32) into TMEM;
-//   epilogue   dden, dQ (stored straight from registers), dz on CUDA cores;
+//   epilogue   dden, dQ, dz on CUDA cores;
 //   rewrite    ReLU(Q) -> phi(Q) in place (RoPE only);
 //   MMA 2      dS += phi(Q)^T dnum (the reduce's MN-major form, M = 128 with
 //              the upper 64 rows unused, N = 64, K = 16 tokens; the two 32x32
 //              diagonal blocks are the heads' dS).
+// Without RoPE phi(Q) = ReLU(Q) is ready after the transform, so MMA 1 and
+// MMA 2 are issued together; dQ then goes over the dnum box in shared memory
+// and out with one TMA store. With RoPE, MMA 2 waits for the rewrite and dQ
+// is stored from registers.
 // The split partials of (dS, dz) are combined by the last CTA of each head
 // pair in split order, as in the state reduce: deterministic.
 //

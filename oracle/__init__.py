@@ -30,3 +30,4 @@ from .linear_attention import (  # noqa: F401
     causal_bruteforce,
 )
 from .temporal_conv import temporal_conv  # noqa: F401,E402
+from .qkv_state import bf16_round, qkv_projection, qkv_state, key_value_heads  # noqa: F401,E402

@@ -496,3 +496,102 @@ def test_temporal_conv_cache_carries_the_previous_block():
     whole, _ = orc.temporal_conv(x, w, b)
     np.testing.assert_allclose(y1[:, 4] + w[:, 2] * x[:, 5], whole[:, 4], rtol=1e-13, atol=1e-13)
     np.testing.assert_allclose(y2, whole[:, 5:], rtol=1e-13, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# QKV projection fused with the state reduce
+
+
+def test_bf16_round_ties_to_even_and_matches_torch():
+    """bf16 keeps 8 significant bits: 257 lies halfway between 256 and 258 and
+    goes to the even 256; 259 goes to 260; 1 + 3 * 2^-8 goes to 1 + 2^-6. On
+    float32-representable values the rounding equals torch's own conversion."""
+    import torch
+    got = orc.bf16_round(np.array([257.0, 259.0, 1 + 3 * 2.0 ** -8, -257.0, 0.0, 1 + 2.0 ** -8]))
+    assert got.tolist() == [256.0, 260.0, 1 + 2.0 ** -6, -256.0, 0.0, 1.0]
+    x = np.random.default_rng(5).standard_normal(20000).astype(np.float32).astype(np.float64)
+    x *= np.exp2(np.random.default_rng(6).integers(-20, 20, x.shape))
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(orc.bf16_round(x), ref)
+
+
+def _qkv_bruteforce(X, W, bias, H, theta):
+    """Pure-Python loops over tokens, heads, dims and input channels."""
+    B, N, C = X.shape
+    hd = H * D
+    S = np.zeros((B, H, D, D))
+    z = np.zeros((B, H, D))
+    Q = np.zeros((B, N, H, D))
+    for b in range(B):
+        for n in range(N):
+            row = [sum(X[b, n, c] * W[j, c] for c in range(C)) + (bias[j] if bias is not None else 0.0)
+                   for j in range(3 * hd)]
+            row = [float(orc.bf16_round(np.array(v))) for v in row]
+            for h in range(H):
+                q = row[h * D:(h + 1) * D]
+                k = row[hd + h * D:hd + (h + 1) * D]
+                v = row[2 * hd + h * D:2 * hd + (h + 1) * D]
+                kp = [max(t, 0.0) for t in k]
+                phi = list(kp)
+                if theta is not None:
+                    for i in range(D // 2):
+                        c, s = math.cos(theta[n, i]), math.sin(theta[n, i])
+                        phi[2 * i] = kp[2 * i] * c - kp[2 * i + 1] * s
+                        phi[2 * i + 1] = kp[2 * i] * s + kp[2 * i + 1] * c
+                Q[b, n, h] = q
+                for d in range(D):
+                    z[b, h, d] += kp[d]
+                    for e in range(D):
+                        S[b, h, d, e] += phi[d] * v[e]
+    return Q, S, z
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_qkv_state_equals_loops_over_the_projection(rope):
+    """Small integers keep every product and sum exact in float64, and some
+    projected values need rounding (|y| > 256), so the loops and the oracle
+    must agree exactly: row blocks (q, k, v), head slices, bias, rounding,
+    ReLU and the state's orientation S[d][e] = sum phi(k)_d v_e."""
+    rng = np.random.default_rng(17)
+    B, N, C, H = 2, 3, 16, 2
+    X = rng.integers(-12, 13, (B, N, C)).astype(np.float64)
+    W = rng.integers(-9, 10, (3 * H * D, C)).astype(np.float64)
+    bias = rng.integers(-3, 4, 3 * H * D).astype(np.float64)
+    theta = orc.rope_angles(1, 1, N, 2) if rope else None
+    Q, S, z = orc.qkv_state(X, W, bias, H, theta)
+    Qr, Sr, zr = _qkv_bruteforce(X, W, bias, H, theta)
+    Y = X @ W.T + bias
+    assert ((np.abs(Y) > 256) & (Y % 2 != 0)).sum() > 10  # the rounding step is exercised
+    assert np.array_equal(Q, Qr) and np.array_equal(z, zr)
+    assert np.allclose(S, Sr, rtol=1e-12, atol=1e-9)
+    if not rope:
+        assert np.array_equal(S, Sr)
+
+
+def test_qkv_state_with_selection_weights_is_the_state_reduce_of_the_inputs():
+    """W that copies input channels into the key and value slots (a 0/1
+    selection matrix) gives k, v = the selected inputs, so the fused state is
+    the plain state reduce of those inputs (bf16 inputs round to themselves)."""
+    rng = np.random.default_rng(3)
+    B, N, H = 1, 50, 3
+    C = 2 * H * D
+    X = orc.bf16_round(rng.standard_normal((B, N, C)))
+    W = np.zeros((3 * H * D, C))
+    W[H * D:, :] = np.eye(C)
+    Q, S, z = orc.qkv_state(X, W, None, H)
+    K = X[..., :H * D].reshape(B, N, H, D)
+    V = X[..., H * D:].reshape(B, N, H, D)
+    S2, z2 = orc.state_reduce(K, V)
+    assert np.array_equal(S, S2) and np.array_equal(z, z2)
+    assert (Q == 0).all()
+
+
+def test_key_value_heads_matches_the_full_projection():
+    rng = np.random.default_rng(9)
+    B, N, C, H = 1, 40, 24, 5
+    X = orc.bf16_round(rng.standard_normal((B, N, C)))
+    W = orc.bf16_round(rng.standard_normal((3 * H * D, C)) / np.sqrt(C))
+    b = rng.standard_normal(3 * H * D) * 0.1
+    _, k, v = orc.qkv_projection(X, W, b, H)
+    k2, v2 = orc.key_value_heads(X, W, b, H, [1, 4])
+    assert np.array_equal(k2, k[:, :, [1, 4]]) and np.array_equal(v2, v[:, :, [1, 4]])
