@@ -27,7 +27,6 @@ from __future__ import annotations
 import argparse
 import ctypes
 import datetime
-import glob
 import hashlib
 import json
 import math
@@ -49,14 +48,18 @@ METRIC_BWD = "linear-attn backward tokens/s per layer at 1 B200; achieved HBM GB
 METRIC_CAUSAL = ("token-causal linear-attn tokens/s per layer at 1 B200; "
                  "achieved HBM GB/s vs peak")
 METRIC_TCONV = "temporal-conv tokens/s per layer at 1 B200; achieved HBM GB/s vs peak"
+METRIC_QKV = ("QKV projection + state reduce tokens/s per layer at 1 B200; "
+              "achieved TFLOP/s vs bf16 peak")
 METRICS = {"layer": METRIC, "backward": METRIC_BWD, "causal": METRIC_CAUSAL,
-           "tconv": METRIC_TCONV}
+           "tconv": METRIC_TCONV, "qkv": METRIC_QKV}
 # Channels of the temporal convolution: the FFN width of Sana-1.6B, which
 # SANA-Video starts from (width 2240, FFN 5600).
 FFN_WIDTH = 5600
 OP_CONFIG = {"layer": {}, "backward": {"op": "backward (dQ, dK, dV, dS, dz)"},
              "causal": {"op": "token-causal (query n sees keys 0..n), no carry"},
-             "tconv": {"op": "temporal depth-wise conv 3x1x1 + shortcut", "channels": FFN_WIDTH}}
+             "tconv": {"op": "temporal depth-wise conv 3x1x1 + shortcut", "channels": FFN_WIDTH},
+             "qkv": {"op": "QKV projection (bf16 GEMM, bias) fused with the state reduce; "
+                           "Q out, K and V never leave the chip"}}
 DEFAULT_WORKLOAD = "sana1.6b_1024px"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
@@ -117,12 +120,37 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
 
 
-def sources_sha():
+# Sources of each timed call's kernels: the kernel files and the device
+# headers they include. A committed DRAM-traffic figure holds while these
+# files are unchanged.
+_DEVICE_HEADERS = ("la_common.cuh", "la_sm100.cuh", "la_tc_common.cuh")
+KERNEL_SOURCES = {
+    "attention_layer": ("la_tc.cu",) + _DEVICE_HEADERS,
+    "attention_backward": ("la_backward_tc.cu",) + _DEVICE_HEADERS,
+    "causal_attention": ("la_tc.cu", "la_causal_tc.cu") + _DEVICE_HEADERS,
+    "temporal_conv": ("la_conv.cu",) + _DEVICE_HEADERS,
+    "qkv_state": ("la_qkv_tc.cu",) + _DEVICE_HEADERS,
+}
+
+
+def tensor_peaks():
+    """Measured dense bf16 GEMM throughput (TFLOP/s): burst and sustained."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return ({"burst": float(m["bf16_tflops"]), "sustained": float(m["bf16_tflops_sustained"])},
+                "measured (MEASURED_PEAKS.json bf16_tflops_sustained; the call is timed inside "
+                "a seconds-long loop of back-to-back calls)")
+    except Exception:
+        return {"burst": 1590.0, "sustained": 1400.0}, "fallback 1.59 / 1.4 PFLOP/s"
+
+
+def sources_sha(kernel):
     h = hashlib.sha256()
-    pat = os.path.join(ROOT, "linear_attention_diffusion_b200", "csrc", "*")
-    for fn in sorted(glob.glob(pat)):
-        with open(fn, "rb") as f:
-            h.update(os.path.basename(fn).encode())
+    for name in sorted(KERNEL_SOURCES[kernel]):
+        with open(os.path.join(ROOT, "linear_attention_diffusion_b200", "csrc", name), "rb") as f:
+            h.update(name.encode())
             h.update(f.read())
     return h.hexdigest()[:16]
 
@@ -133,7 +161,9 @@ def profiled_traffic(workload, kernel):
     path = os.path.join(ROOT, "profiles", f"traffic_{workload}.txt")
     if not os.path.exists(path):
         return None
-    sha = sources_sha()
+    if kernel not in KERNEL_SOURCES:
+        return None
+    sha = sources_sha(kernel)
     for line in open(path):
         if line.startswith("#") or "=" not in line:
             continue
@@ -548,6 +578,125 @@ def run_tconv(args, w, rank, world, local_rank):
             "per_set_bytes": per_set, "cache_bytes": 0 if cache is None else 2 * per_set // w.T}
 
 
+def run_qkv(args, w, rank, world, local_rank):
+    """The QKV projection fused with the state reduce, at the model's hidden
+    width, with the unfused path (three cuBLAS projections through torch, then
+    la_state_reduce) timed beside it for comparison."""
+    import torch
+    import torch.nn.functional as F
+    import linear_attention_diffusion_b200 as la
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(str(getattr(props, "uuid", "") or ""))
+    stream = torch.cuda.Stream(dev)
+    lib = la._lib
+    sp = stream.cuda_stream
+    C = wl.hidden_width(w)
+    HD = w.H * D
+    X0, Wt, bias = wl.make_projection(w, C, seed=rank_seed(rank) + 30)
+    per_set = X0.numel() * X0.element_size()
+    n_sets = max(2, -(-2 * L2_BYTES // per_set))
+    xs = [X0.to(dev)] + [wl.make_projection(w, C, seed=rank_seed(rank) + 30 + 10 * i)[0].to(dev)
+                         for i in range(1, n_sets)]
+    Wd, bd = Wt.to(dev), bias.to(dev)
+    Q = torch.empty((w.B, w.N, w.H, D), dtype=torch.bfloat16, device=dev)
+    S = torch.empty((w.B, w.H, D, D), device=dev)
+    z = torch.empty((w.B, w.H, D), device=dev)
+    shape = la.make_shape(w.B, w.N, w.H, D, "bf16", w.rope, w.T, w.Hh, w.W, 0, w.rope_base,
+                          w.eps)
+    ws_n = max(256, la.la_qkv_workspace_bytes(shape, C))
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
+    status = []
+
+    def step(i, evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        status.append(lib.la_qkv_state(ctypes.byref(shape), C, xs[i % n_sets].data_ptr(),
+                                       Wd.data_ptr(), bd.data_ptr(), Q.data_ptr(), S.data_ptr(),
+                                       z.data_ptr(), ws.data_ptr(), ws_n, sp))
+        if evs is not None:
+            evs[1].record(stream)
+
+    def check_status():
+        bad = [v for v in status if v != 0]
+        status.clear()
+        if bad:
+            raise RuntimeError(f"library call failed: {la.la_status_string(bad[0])} "
+                               f"{la.la_last_error()}")
+
+    ms_max, seg_us, chunk, t0, t1 = time_steps(args, step, stream, dev, world, n_sets, False,
+                                               check_status)
+    clocks = sampler.summary(t0, t1)
+
+    # the unfused path on the same inputs: projections, then the state reduce
+    Wq, Wk, Wv = (Wd[j * HD:(j + 1) * HD] for j in range(3))
+    bq, bk, bv = (bd[j * HD:(j + 1) * HD] for j in range(3))
+    Ku = torch.empty((w.B, w.N, HD), dtype=torch.bfloat16, device=dev)
+    Vu = torch.empty_like(Ku)
+    Qu = torch.empty_like(Ku)
+    lws = la.workspace(shape, dev)
+
+    def unfused(i, evs=None):
+        x = xs[i % n_sets]
+        if evs is not None:
+            evs[0].record(stream)
+        x2 = x.view(-1, C)
+        torch.addmm(bq, x2, Wq.t(), out=Qu.view(-1, HD))
+        torch.addmm(bk, x2, Wk.t(), out=Ku.view(-1, HD))
+        torch.addmm(bv, x2, Wv.t(), out=Vu.view(-1, HD))
+        la.la_state_reduce(shape, Ku, Vu, S, z, lws, sp)
+        if evs is not None:
+            evs[1].record(stream)
+
+    ums, _, _, _, _ = time_steps(args, unfused, stream, dev, world, n_sets, False, lambda: None)
+    e2e = None
+    if args.e2e_steps > 0:
+        steps = max(1, min(args.steps, args.e2e_steps))
+        hx = X0.pin_memory()
+        hq = torch.empty((w.B, w.N, w.H, D), dtype=torch.bfloat16).pin_memory()
+        hs = torch.empty((w.B, w.H, D, D)).pin_memory()
+        hz = torch.empty((w.B, w.H, D)).pin_memory()
+
+        def call(p, ins, outs, st):
+            la.la_qkv_state(shape, C, ins[0], Wd, bd, outs[0], outs[1], outs[2], ws, st)
+
+        ms = e2e_pipelined(dev, stream, [hx], [hq, hs, hz], call, 1, steps)
+        e2e = {"ms_per_step": ms, "tokens_per_step": w.B * w.N, "steps": steps,
+               "h2d_bytes_per_step": per_set,
+               "d2h_bytes_per_step": (hq.numel() * 2 + hs.numel() * 4 + hz.numel() * 4),
+               "copies": "pipelined: copy-in, calls and copy-out on three streams, two buffer sets"}
+    sampler.stop()
+    flops = 2.0 * w.B * w.N * C * 3 * HD
+    return {"ms": ms_max, "seg_us": seg_us, "kernel_names": ("qkv_state",), "e2e": e2e,
+            "clocks": clocks, "launches_per_step": 2, "n_sets": n_sets, "chunk": chunk,
+            "per_set_bytes": per_set, "flops": flops, "unfused_ms": ums / args.steps,
+            "C": C}
+
+
+def oracle_sample_qkv(w, seconds):
+    """The float64 fused projection + state on a token subset, scaled to N."""
+    import oracle as orc
+    C = wl.hidden_width(w)
+    X, Wt, b = wl.make_projection(w, C, seed=30)
+    th_all = orc.rope_angles(w.T, w.Hh, w.W, 0, w.rope_base) if w.rope else None
+    n_sub = min(w.N, 256)
+    Xs = X[:1, :n_sub]
+    th = None if th_all is None else th_all[:n_sub]
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        orc.qkv_state(Xs, Wt, b, w.H, th)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    per_call = el / reps * (w.B * w.N) / n_sub
+    desc = (f"oracle qkv_state on {n_sub} of {w.B * w.N} tokens (C = {C}), {reps} calls in "
+            f"{el:.1f} s, scaled to {w.B * w.N} tokens")
+    return w.B * w.N / per_call, desc, cpu_cores_used(), per_call
+
+
 def oracle_sample_tconv(w, seconds):
     """The float64 temporal convolution on a channel subset, scaled to FFN_WIDTH."""
     import oracle as orc
@@ -717,10 +866,11 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--soak", type=float, default=1.0)
-    ap.add_argument("--op", choices=["layer", "backward", "causal", "tconv"], default="layer")
+    ap.add_argument("--op", choices=["layer", "backward", "causal", "tconv", "qkv"],
+                    default="layer")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
-    if args.op in ("backward", "causal") and w.block_causal:
+    if args.op in ("backward", "causal", "qkv") and w.block_causal:
         ap.error(f"--op {args.op} covers the non-causal workloads")
     if args.op == "tconv" and not w.rope:
         ap.error("--op tconv needs a video workload (sanavideo_480p, longsana_block_causal)")
@@ -731,6 +881,8 @@ def main():
             per_step_us *= 10
         elif args.op == "tconv":
             per_step_us = 200
+        elif args.op == "qkv":
+            per_step_us *= 8
         args.steps = max(10, int(0.5e6 / per_step_us))
     args.warmup = max(args.warmup, 3)
 
@@ -746,7 +898,8 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
-    r = (run_tconv if args.op == "tconv" else run_la)(args, w, rank, world, local_rank)
+    r = {"tconv": run_tconv, "qkv": run_qkv}.get(args.op, run_la)(args, w, rank, world,
+                                                                  local_rank)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank != 0:
@@ -775,6 +928,8 @@ def main():
                           "note": "update=0 call, event graph; avg over all 60 calls"}}
         dom = name
         traffic = None
+    elif args.op == "qkv":
+        kernels, dom, traffic = {}, None, None
     else:
         kernels = {}
         for nm, us in zip(r["kernel_names"], r["seg_us"]):
@@ -784,8 +939,26 @@ def main():
                            "launches": r["launches_per_step"], "event_graph_us": us}
         dom = max(kernels, key=lambda k: kernels[k]["avg_us"])
         traffic = profiled_traffic(w.name, dom)
-    kd = kernels[dom]
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(kd["gbs"], 1),
+    kd = kernels.get(dom)
+    if args.op == "qkv":
+        # a dense contraction: tensor-bound against the measured bf16 GEMM peak
+        tf_peak, tf_src = tensor_peaks()
+        dur_us = ms_step * 1e3
+        tflops = r["flops"] / (dur_us * 1e-6) / 1e12
+        roofline = {"bound": "tensor", "kernel": "qkv_state", "achieved": round(tflops, 1),
+                    "peak": tf_peak["sustained"], "unit": "TFLOP/s",
+                    "frac": round(tflops / tf_peak["sustained"], 4),
+                    "frac_of_burst": round(tflops / tf_peak["burst"], 4),
+                    "traffic": profiled_traffic(w.name, "qkv_state"),
+                    "algorithmic_flops": r["flops"], "avg_launch_us": round(dur_us, 3),
+                    "event_graph_us": round(r["seg_us"][0], 3), "launches_per_call": 2,
+                    "peak_source": tf_src,
+                    "unfused_us": round(r["unfused_ms"] * 1e3, 3),
+                    "unfused_note": ("the same result through three cuBLAS projections "
+                                     "(torch.addmm with bias) writing Q, K, V, then "
+                                     "la_state_reduce reading K and V back")}
+    else:
+      roofline = {"bound": "hbm", "kernel": dom, "achieved": round(kd["gbs"], 1),
                 "peak": peak, "unit": "GB/s", "frac": round(kd["gbs"] / peak, 4),
                 "traffic": traffic, "algorithmic_bytes": kd["algorithmic_bytes"],
                 "avg_launch_us": round(kd["avg_us"], 3), "peak_source": peak_src,
@@ -806,6 +979,7 @@ def main():
         "api": ("la_attention_backward" if args.op == "backward" else
                 "la_causal_attention" if args.op == "causal" else
                 "la_temporal_conv" if args.op == "tconv" else
+                "la_qkv_state" if args.op == "qkv" else
                 "la_block_causal_step" if w.block_causal else "la_attention")}
     out = {"metric": METRICS[args.op], "value": value, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -816,8 +990,9 @@ def main():
            "roofline": roofline, "e2e": e2e,
            "gpu_launches": r["launches_per_step"] * args.steps,
            "clocks": r["clocks"], "graph_chunk_steps": r["chunk"], "soak_s": args.soak}
-    if world == 1 and args.cpu_seconds > 0 and args.op == "tconv":
-        tps, desc, cores, _ = oracle_sample_tconv(w, args.cpu_seconds)
+    if world == 1 and args.cpu_seconds > 0 and args.op in ("tconv", "qkv"):
+        sampler_fn = oracle_sample_tconv if args.op == "tconv" else oracle_sample_qkv
+        tps, desc, cores, _ = sampler_fn(w, args.cpu_seconds)
         out["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores,
                                "kind": "oracle", "sample": desc}
     elif world == 1 and args.cpu_seconds > 0:
@@ -833,8 +1008,9 @@ def main_reference(args, w, rank, world):
         return
     budget = 150.0  # seconds for warm-up + timed steps together
     per = budget / (args.steps + args.warmup)
-    if args.op == "tconv":
-        tps, desc, cores, per_call = oracle_sample_tconv(w, min(per * args.steps, 60.0))
+    if args.op in ("tconv", "qkv"):
+        sampler_fn = oracle_sample_tconv if args.op == "tconv" else oracle_sample_qkv
+        tps, desc, cores, per_call = sampler_fn(w, min(per * args.steps, 60.0))
         out = {"impl": "reference", "metric": METRICS[args.op], "value": tps, "unit": "tokens/s",
                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                "ms_per_step": per_call * 1e3, "higher_is_better": True, "scaling": "weak",
