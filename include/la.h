@@ -217,6 +217,34 @@ la_status la_temporal_conv(const la_conv_shape* shape, const void* x,
                            const float* w, const float* bias, const void* f_in,
                            void* f_out, void* y, la_stream stream);
 
+/* Bytes of workspace la_qkv_state needs for `shape` and hidden width C.
+ * Returns 0 iff the request is invalid or unsupported. Pure host function. */
+size_t la_qkv_workspace_bytes(const la_shape* shape, int C);
+
+/* QKV projection fused with the state reduce (Sana, section Infra: the
+ * deployment GEMM of the QKV projection also forms ReLU(K)^T V, so the keys
+ * and values never go to memory). For every token n of batch element b:
+ *   [q_n, k_n, v_n] = bf16(W x_n + bias)    (float32 sum, one rounding each)
+ * and then, exactly as la_state_reduce over those k and v:
+ *   S[b,h] = sum_n phi(k_n)^T v_n,  z[b,h] = sum_n ReLU(k_n).
+ * X: [B,N,C] bf16 token features (device, read). W: [3*H*D, C] bf16 (device,
+ * read): rows [0, H*D) give the queries, [H*D, 2*H*D) the keys, [2*H*D,
+ * 3*H*D) the values; head h owns rows [D*h, D*h + D) of each part. bias:
+ * [3*H*D] bf16 in the same order, or NULL for none. Q: [B,N,H,D] bf16
+ * (device, written): the queries. S [B,H,D,D], z [B,H,D] float32 (device,
+ * written). shape->io_dtype must be LA_IO_BF16; rope, T, Hh, W and t_offset
+ * select the feature map as for la_state_reduce (eps is not used). C: the
+ * hidden width, a multiple of 8 in [8, 2^20]. ws: device workspace of at
+ * least la_qkv_workspace_bytes(shape, C) bytes; it needs no zero fill.
+ * Two launches: a persistent tensor-core GEMM that writes Q and one partial
+ * state per run of key/value tiles, then a combine that sums each head's
+ * partials in an order fixed by (B, N, H, C), so every bit of S and z is
+ * reproducible. N == 0 gives S = 0, z = 0. Q, S and z must not overlap each
+ * other, the inputs or the workspace. */
+la_status la_qkv_state(const la_shape* shape, int C, const void* X,
+                       const void* W, const void* bias, void* Q, float* S,
+                       float* z, void* ws, size_t ws_bytes, la_stream stream);
+
 /* Reset of the KV cache at the start of a video (SANA-Video section 4: the
  * cache starts empty): S[B,H,D,D] = 0, z[B,H,D] = 0 on `stream`. */
 la_status la_state_reset(float* S, float* z, int B, int H, int D,

@@ -82,6 +82,10 @@ _lib.la_causal_attention.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _vp, _i,
 _lib.la_causal_attention.restype = _i
 _lib.la_temporal_conv.argtypes = [ctypes.POINTER(LaConvShape), _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.la_temporal_conv.restype = _i
+_lib.la_qkv_workspace_bytes.argtypes = [_shape_p, _i]
+_lib.la_qkv_workspace_bytes.restype = _sz
+_lib.la_qkv_state.argtypes = [_shape_p, _i] + [_vp] * 7 + [_sz, _vp]
+_lib.la_qkv_state.restype = _i
 _lib.la_state_reset.argtypes = [_vp, _vp, _i, _i, _i, _vp]
 _lib.la_state_reset.restype = _i
 _lib.la_status_string.argtypes = [_i]
@@ -198,6 +202,17 @@ def la_temporal_conv(shape: LaConvShape, x, w, bias, f_in, f_out, y, stream=None
                                  _ptr(f_out), _ptr(y), _stream(stream)), "la_temporal_conv")
 
 
+def la_qkv_workspace_bytes(shape: LaShape, C: int) -> int:
+    return int(_lib.la_qkv_workspace_bytes(ctypes.byref(shape), int(C)))
+
+
+def la_qkv_state(shape: LaShape, C: int, X, W, bias, Q, S, z, ws, stream=None) -> None:
+    """QKV projection fused with the state reduce (see include/la.h)."""
+    _check(_lib.la_qkv_state(ctypes.byref(shape), int(C), _ptr(X), _ptr(W), _ptr(bias), _ptr(Q),
+                             _ptr(S), _ptr(z), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "la_qkv_state")
+
+
 def la_state_reset(S, z, B: int, H: int, D: int = HEAD_DIM, stream=None) -> None:
     _check(_lib.la_state_reset(_ptr(S), _ptr(z), int(B), int(H), int(D), _stream(stream)),
            "la_state_reset")
@@ -300,3 +315,26 @@ def temporal_conv(x, w, bias=None, f_in=None, want_cache: bool = False, stream=N
     f_out = torch.empty((B, Hh, W, C), dtype=x.dtype, device=x.device) if want_cache else None
     la_temporal_conv(shape, x, w, bias, f_in, f_out, y, stream)
     return (y, f_out) if want_cache else y
+
+
+def qkv_state(X, W, bias=None, rope_grid=None, t_offset: int = 0, rope_base: float = 10000.0,
+              stream=None):
+    """Q [B, N, H, 32], S, z of the fused QKV projection + state reduce for
+    X [B, N, C] and W [3 H 32, C] bf16 CUDA tensors."""
+    import torch
+    B, N, C = X.shape
+    H = W.shape[0] // (3 * HEAD_DIM)
+    if rope_grid is None:
+        shape = make_shape(B, N, H, HEAD_DIM, "bf16", False)
+    else:
+        T, Hh, Wd = rope_grid
+        shape = make_shape(B, N, H, HEAD_DIM, "bf16", True, T, Hh, Wd, t_offset, rope_base)
+    Q = torch.empty((B, N, H, HEAD_DIM), dtype=torch.bfloat16, device=X.device)
+    S = torch.empty((B, H, HEAD_DIM, HEAD_DIM), dtype=torch.float32, device=X.device)
+    z = torch.empty((B, H, HEAD_DIM), dtype=torch.float32, device=X.device)
+    n = la_qkv_workspace_bytes(shape, C)
+    if n == 0:
+        raise LaError(LA_ERR_INVALID_ARG, "la_qkv_workspace_bytes")
+    ws = torch.empty(n, dtype=torch.uint8, device=X.device)
+    la_qkv_state(shape, C, X, W, bias, Q, S, z, ws, stream)
+    return Q, S, z

@@ -489,6 +489,76 @@ la_status la_temporal_conv(const la_conv_shape* shape, const void* x, const floa
   return LA_OK;
 }
 
+// Hidden width of la_qkv_state: at least 8, a multiple of 8 (rows of X and W
+// are 16-byte aligned for TMA), and small enough for 32-bit tile arithmetic.
+static la_status check_qkv(const la_shape* shape, int C, Problem& p) {
+  LA_TRY(make_problem(shape, p));
+  if (p.io != LA_IO_BF16)
+    return fail(LA_ERR_UNSUPPORTED, "la_qkv_state takes bf16 tensors only (io_dtype=%d)", p.io);
+  if (C < 8 || C % 8 != 0 || C > (1 << 20))
+    return fail(LA_ERR_UNSUPPORTED, "hidden width C=%d (a multiple of 8 in [8, 2^20])", C);
+  const long long tiles = 1LL * p.B * ((p.N + 127) / 128) * ((p.H + 3) / 4 + (p.H * kD + 255) / 256);
+  if (tiles >= (1LL << 30)) return fail(LA_ERR_UNSUPPORTED, "projection too large");
+  return LA_OK;
+}
+
+size_t la_qkv_workspace_bytes(const la_shape* shape, int C) {
+  Problem p;
+  if (check_qkv(shape, C, p) != LA_OK) return 0;
+  const size_t n = align256(qkv_workspace_floats(p.B, p.N, p.H, C) * sizeof(float));
+  return n == 0 ? 256 : n;
+}
+
+la_status la_qkv_state(const la_shape* shape, int C, const void* X, const void* W,
+                       const void* bias, void* Q, float* S, float* z, void* ws, size_t ws_bytes,
+                       la_stream stream) {
+  Problem p;
+  LA_TRY(check_qkv(shape, C, p));
+  const bool any_state = p.B > 0 && p.H > 0;
+  const bool any = any_state && p.N > 0;
+  LA_TRY(check_ptr(X, "X", any));
+  LA_TRY(check_ptr(W, "W", any));
+  LA_TRY(check_ptr(bias, "bias", any && bias != nullptr));
+  LA_TRY(check_ptr(Q, "Q", any));
+  LA_TRY(check_ptr(S, "S", any_state));
+  LA_TRY(check_ptr(z, "z", any_state));
+  const size_t hd = static_cast<size_t>(p.H) * kD;
+  const size_t nx = static_cast<size_t>(p.B) * p.N * C * 2, nw = 3 * hd * C * 2, nb = 3 * hd * 2;
+  const size_t nq = static_cast<size_t>(p.B) * p.N * hd * 2;
+  const size_t need = any ? la_qkv_workspace_bytes(shape, C) : 0;
+  if (any) {
+    if (ws == nullptr) return fail(LA_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", need);
+    if (!aligned16(ws)) return fail(LA_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    if (ws_bytes < need)
+      return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", ws_bytes, need);
+  }
+  const size_t ns = s_bytes(p), nz = z_bytes(p);
+  const void* ins[4] = {X, W, bias, ws};
+  const size_t in_n[4] = {nx, nw, bias != nullptr ? nb : 0, need};
+  void* outs[3] = {Q, S, z};
+  const size_t out_n[3] = {any ? nq : 0, ns, nz};
+  for (int a = 0; a < 3; ++a) {
+    for (int b = 0; b < 4; ++b)
+      if (overlap(outs[a], out_n[a], ins[b], in_n[b]))
+        return fail(LA_ERR_INVALID_ARG, "Q, S and z must not overlap X, W, bias or the workspace");
+    for (int b = a + 1; b < 3; ++b)
+      if (overlap(outs[a], out_n[a], outs[b], out_n[b]))
+        return fail(LA_ERR_INVALID_ARG, "Q, S and z must not overlap each other");
+  }
+  if (!any_state) return LA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (p.N == 0) {  // no tokens: the state of an empty sequence
+    cudaError_t e = cudaMemsetAsync(S, 0, ns, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(z, 0, nz, st);
+    if (e != cudaSuccess) return cuda_fail(e, "la_qkv_state (empty sequence)");
+    return LA_OK;
+  }
+  const cudaError_t e =
+      launch_qkv_state(p, C, X, W, bias, Q, S, z, static_cast<float*>(ws), st);
+  if (e != cudaSuccess) return cuda_fail(e, "la_qkv_state");
+  return LA_OK;
+}
+
 la_status la_state_reset(float* S, float* z, int B, int H, int D, la_stream stream) {
   if (B < 0 || H < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d", B, H);
   if (D != kD) return fail(LA_ERR_UNSUPPORTED, "head width D=%d (only 32 is built)", D);
@@ -535,13 +605,14 @@ la_status la_wait_selftest(unsigned limit_us, la_stream stream) {
 
 la_status la_device_error(unsigned* code, int reset) {
   if (code == nullptr) return fail(LA_ERR_INVALID_ARG, "code is NULL");
-  unsigned fwd = 0, bwd = 0, conv = 0, causal = 0;
+  unsigned fwd = 0, bwd = 0, conv = 0, causal = 0, qkv = 0;
   cudaError_t e = read_device_error(&fwd, reset != 0);
   if (e == cudaSuccess) e = read_device_error_bwd(&bwd, reset != 0);
   if (e == cudaSuccess) e = read_device_error_conv(&conv, reset != 0);
   if (e == cudaSuccess) e = read_device_error_causal(&causal, reset != 0);
+  if (e == cudaSuccess) e = read_device_error_qkv(&qkv, reset != 0);
   if (e != cudaSuccess) return cuda_fail(e, "la_device_error");
-  *code = fwd | bwd | conv | causal;
+  *code = fwd | bwd | conv | causal | qkv;
   return LA_OK;
 }
 

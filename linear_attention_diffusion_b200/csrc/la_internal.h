@@ -135,6 +135,15 @@ cudaError_t launch_wait_selftest(unsigned limit_us, cudaStream_t s);
 cudaError_t read_device_error_bwd(unsigned* code, bool reset);
 cudaError_t read_device_error_conv(unsigned* code, bool reset);  // la_conv.cu
 cudaError_t read_device_error_causal(unsigned* code, bool reset);  // la_causal_tc.cu
+cudaError_t read_device_error_qkv(unsigned* code, bool reset);     // la_qkv_tc.cu
+// QKV projection fused with the state reduce (la_qkv_tc.cu): a persistent
+// tcgen05 GEMM that writes Q and one partial state per run of key/value
+// tiles into `part` (qkv_workspace_floats floats), then a combine kernel that
+// sums the partials in a fixed order into S and z. bf16 only, N > 0.
+size_t qkv_workspace_floats(int B, int N, int H, int C);
+cudaError_t launch_qkv_state(const Problem& p, int C, const void* X, const void* W,
+                             const void* bias, void* Q, float* S, float* z, float* part,
+                             cudaStream_t s);
 
 // Host-side helpers of the C-ABI layer (la_api.cu).
 namespace detail {

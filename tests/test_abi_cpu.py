@@ -136,3 +136,34 @@ def test_wait_selftest_rejects_limits_out_of_range():
     for bad in (0, 10_000_001):  # refused on the host, before any launch
         with pytest.raises(la.LaError):
             la.la_wait_selftest(bad, stream=0)
+
+
+def test_qkv_state_host_checks():
+    ref = ctypes.byref
+    s = la.make_shape(2, 300, 6)
+    C = 192
+    n = la.la_qkv_workspace_bytes(s, C)
+    assert n > 0 and n % 256 == 0 and la.la_qkv_workspace_bytes(s, C) == n
+    assert la.la_qkv_workspace_bytes(s, 100) == 0          # C not a multiple of 8
+    assert la.la_qkv_workspace_bytes(s, 0) == 0
+    assert la.la_qkv_workspace_bytes(la.make_shape(2, 300, 6, io_dtype="f32"), C) == 0
+    assert la.la_qkv_workspace_bytes(la.make_shape(2, 300, 6, D=64), C) == 0
+    big = 1 << 32
+    X, W, Q, S, z, ws = (FAKE + i * big for i in range(6))
+    args = lambda **kw: [kw.get(k, v) for k, v in
+                         (("X", X), ("W", W), ("b", None), ("Q", Q), ("S", S), ("z", z),
+                          ("ws", ws), ("n", n))]
+    call = lambda shape=s, c=C, **kw: _call("la_qkv_state", ref(shape), c, *args(**kw), None)
+    assert call(c=100) == la.LA_ERR_UNSUPPORTED
+    assert call(shape=la.make_shape(2, 300, 6, io_dtype="f32")) == la.LA_ERR_UNSUPPORTED
+    assert call(X=None) == la.LA_ERR_INVALID_ARG and "X" in la.la_last_error()
+    assert call(W=FAKE + 8) == la.LA_ERR_INVALID_ARG and "aligned" in la.la_last_error()
+    assert call(ws=None) == la.LA_ERR_WORKSPACE
+    assert call(n=n - 256) == la.LA_ERR_WORKSPACE
+    assert call(Q=X + 64) == la.LA_ERR_INVALID_ARG and "overlap" in la.la_last_error()
+    assert call(z=S + 16) == la.LA_ERR_INVALID_ARG and "overlap" in la.la_last_error()
+    r = la.make_shape(1, 24, 2, rope=True, T=2, Hh=3, W=5)  # N != T*Hh*W
+    assert call(shape=r) == la.LA_ERR_INVALID_ARG
+    # nothing to do: no pointer needed
+    assert _call("la_qkv_state", ref(la.make_shape(0, 300, 6)), C, None, None, None, None, None,
+                 None, None, 0, None) == la.LA_OK

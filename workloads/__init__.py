@@ -127,3 +127,29 @@ def make_tensor(shape: Tuple[int, ...], seed: int, dtype=torch.bfloat16) -> torc
 def t_offset_of_block(w: Workload, m: int) -> int:
     """Global frame index of block m's first latent frame."""
     return int(m) * w.T
+
+
+def hidden_width(w: Workload) -> int:
+    """Model width of the DiT whose attention layer ``w`` describes: heads x
+    head width (2240 for Sana-1.6B's 70 heads, 1152 for Sana-0.6B's 36)."""
+    return int(w.H) * int(w.D)
+
+
+def make_projection(w: Workload, C: int, seed: int = 0) -> Tuple[torch.Tensor, torch.Tensor,
+                                                                  torch.Tensor]:
+    """Token features and a random-init QKV projection, all bf16 CPU tensors.
+
+    X [B, N, C] ~ N(0, 1); W [3 H D, C] ~ N(0, 1/C), so that each projected
+    feature is about N(0, 1) like the attention inputs above; bias [3 H D] ~
+    N(0, 0.1^2). Rows of W (and entries of the bias): all query features, then
+    all key features, then all value features; head h owns rows
+    [D h, D h + D) of each. Seeds ``seed + 0/1/2``. There are no trained
+    weights: only the shapes and scales follow the model."""
+    hd = w.H * w.D
+    x = make_tensor((w.B, w.N, C), seed)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) + 1)
+    wt = (torch.randn((3 * hd, C), generator=g, dtype=torch.float32) / float(C) ** 0.5)
+    g.manual_seed(int(seed) + 2)
+    b = torch.randn((3 * hd,), generator=g, dtype=torch.float32) * 0.1
+    return x, wt.to(torch.bfloat16), b.to(torch.bfloat16)
