@@ -13,32 +13,41 @@
 // Generation with Block Linear Diffusion Transformer", section 2.2). Only the
 // queries leave the operation.
 //
-// One persistent CTA per SM walks a contiguous range of output tiles of
-// 128 tokens x 256 columns (M = 128, N = 256, K = 64 per stage, both operands
-// K-major straight from 128-byte-swizzled TMA tiles; the accumulator is 256
-// TMEM columns). A column tile is either 256 query features, written to Q,
-// or the 128 key and 128 value features of a group of four heads. For a
-// key/value tile the epilogue rounds k and v to bf16, applies ReLU (and RoPE)
-// to k, sums ReLU(k) over the tile's tokens on CUDA cores, and writes phi(k)
-// and v to a shared-memory staging buffer in two rounds of 64 tokens; each
-// round is one more MMA, phi(K)^T V (M = 128 key dims x N = 128 value dims,
-// K = 64 tokens, both MN-major), accumulated in TMEM over the CTA's
-// consecutive tiles of the same head group (a "run"). The four 32 x 32
-// diagonal blocks of that accumulator are the heads' states. At the end of a
-// run they go to a partial slot; a second kernel sums each head's slots in a
-// fixed order, so S and z are bitwise reproducible.
+// The GEMM runs on CTA pairs (clusters of two, one per SM pair): an output
+// tile is 256 tokens x 256 features, one tcgen05.mma.cta_group::2 per 16
+// channels (M = 256, N = 256), both operands K-major from 128-byte-swizzled
+// TMA tiles. CTA r of the pair loads its own 128 token rows of X and the
+// r-th 128 of the tile's 256 rows of W, so each SM brings in 32 KB per 64
+// channels for 2 x 128 x 256 x 64 multiply-adds (a single-CTA 128 x 256 tile
+// needs 48 KB for half of that). Each CTA's tensor memory holds its 128
+// tokens x 256 features; two accumulators alternate, so the epilogue of one
+// tile overlaps the main loop of the next.
+//
+// A column tile is either 256 query features, written to Q, or the 128 key
+// and 128 value features of a group of four heads. For a key/value tile the
+// epilogue rounds k and v to bf16, applies ReLU (and RoPE) to k, sums ReLU(k)
+// over the tokens (warp transpose-sums), stages phi(k) and v in shared memory
+// and accumulates the four heads' phi(K)^T V on CUDA cores in float32 (every
+// thread a 4 x 4 block of one head's 32 x 32 state, tokens in order), over
+// the pair's consecutive tiles of the same head group (a "run"). At the end
+// of a run each CTA writes its partial (S, z) to a slot of the workspace; a
+// second kernel sums every head's slots in a fixed order, so S and z are
+// bitwise reproducible.
 //
 // Tile order: token tiles are cut into chunks of L tiles; chunk by chunk, all
 // column tiles of the chunk, each over the chunk's tokens. With L = tiles per
-// CTA, the CTAs running at any moment read few distinct token rows of X, so
-// X comes from HBM about once and W stays in L2.
+// pair, the pairs running at any moment read few distinct token rows of X,
+// so X comes from HBM about once and W stays in L2.
 //
-// Warp roles (320 threads): warps 0-7 epilogue (warp w reads TMEM lanes
-// 32 (w % 4) .. + 31, i.e. token rows; warps 0-3 the first 128 columns,
-// 4-7 the last 128), warp 8 TMA producer, warp 9 TMEM allocation and the MMA
-// issuer (one thread). Every wait is bounded; a wait that gives up raises the
-// CTA's abort flag and the device error word, and the CTA drains its copies
-// and MMAs before it frees tensor memory.
+// Warp roles (320 threads per CTA): warps 0-7 epilogue (warp w reads TMEM
+// lanes 32 (w % 4) .. + 31, i.e. token rows; warps 0-3 the first 128
+// columns, 4-7 the last 128), warp 8 TMA producer (both CTAs), warp 9 TMEM
+// allocation and, in the pair's first CTA, the MMA issuer (one thread).
+// Every wait is bounded; a wait that gives up raises the CTA's abort flag and
+// the device error word, and the CTA drains its copies and MMAs before it
+// frees tensor memory. The pair meets at cluster barriers after set-up and
+// before exit, so neither CTA leaves while the other may still touch its
+// shared memory. No load is multicast.
 #include <algorithm>
 
 #include "la_tc_common.cuh"
@@ -53,51 +62,53 @@ namespace {
 using namespace sm100;
 
 constexpr int kQkvEpiWarps = 8;
-constexpr int kQkvThreads = (kQkvEpiWarps + 2) * 32;  // 320
+constexpr int kEpiThreads = kQkvEpiWarps * 32;        // 256
+constexpr int kQkvThreads = kEpiThreads + 64;         // + TMA warp + MMA warp
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
-constexpr int kTok = 128;                  // tokens per tile (MMA M)
-constexpr int kCols = 256;                 // output columns per tile (MMA N)
-constexpr int kKBlk = 64;                  // hidden channels per stage
-constexpr int kQStages = 4;
+constexpr int kTokCta = 128;               // tokens per CTA per tile (TMEM lanes)
+constexpr int kTokPair = 2 * kTokCta;      // tokens per tile (MMA M, across the pair)
+constexpr int kCols = 256;                 // output features per tile (MMA N)
+constexpr int kKBlk = 64;                  // channels per stage
+constexpr int kQStages = 5;
 constexpr int kBoxBytes = 128 * 128;       // [128 rows][64 bf16], 128-byte swizzle
-constexpr int kQStageBytes = 3 * kBoxBytes;  // X box + two W boxes (256 rows)
-constexpr int kHalfTok = 64;               // tokens per state round
-constexpr int kStgBox = kHalfTok * 128;    // [64 tokens][64 dims] bf16
-constexpr int kStgBytes = 4 * kStgBox;     // phi(K) dims 0-63, 64-127; V the same
-constexpr int kTmemState = 256;            // state accumulators at columns 256 and 384
-constexpr int kQkvTmemCols = 512;
-// One partial slot: the state of 4 heads (4 x 32 x 32), then the key sums of
-// every TMEM lane quadrant ([4 quadrants][4 heads][32]); the quadrant sums are
-// added in the combine, in quadrant order.
+constexpr int kQStageBytes = 2 * kBoxBytes;  // this CTA's X rows + its 128 rows of W
+constexpr int kStgRow = 256;               // staging row: 128 bf16 features of a token
+constexpr int kStgHalf = kTokCta * kStgRow;  // phi(K) or V of the CTA's 128 tokens
+constexpr int kAccCols = 256;
+constexpr int kQkvTmemCols = 2 * kAccCols;
+constexpr int kBarEpi = 1;                 // named barrier of the epilogue warps
+// One partial slot (per CTA of a pair): the state of 4 heads (4 x 32 x 32),
+// then the key sums of every TMEM lane quadrant ([4 quadrants][4 heads][32]).
 constexpr int kPartS = 4 * kD * kD;
 constexpr int kPartFloats = kPartS + 4 * 4 * kD;
 
 struct QSmem {  // byte offsets from the 1024-aligned base
   static constexpr int stages = 0;
   static constexpr int stg = stages + kQStages * kQStageBytes;
-  static constexpr int bars = stg + kStgBytes;
-  // full[S] empty[S] acc_full acc_empty stg_full stg_empty[2] state_full[2] mma_done
-  static constexpr int nbars = 2 * kQStages + 8;
+  static constexpr int bars = stg + 2 * kStgHalf;
+  // full[S] empty[S] acc_full[2] acc_empty[2] mma_done
+  static constexpr int nbars = 2 * kQStages + 5;
   static constexpr int misc = bars + nbars * 8;  // tmem base, abort flag
   static constexpr int bytes = misc + 16;
 };
 constexpr int kQSmemBytes = QSmem::bytes + 1024;
 static_assert(kQSmemBytes <= 232448, "dynamic shared memory of one CTA");
 
-// The static schedule, a function of (B, N, H, C) only.
+// The static schedule, a function of (B, N, H, C) only. "Units" are CTA
+// pairs; a tile is 256 tokens of one batch element x one column tile.
 struct QkvSched {
   int B, N, H, C, HD;
-  int NT;     // token tiles per batch element
+  int NT;     // token tiles (of 256) per batch element
   int G;      // head groups of 4 (key/value column tiles)
   int QC;     // query column tiles of 256
   int CT;     // column tiles: G key/value, then QC query
   int KB;     // K-blocks of 64 channels
   int L;      // token tiles per chunk
   int NK;     // chunks per batch element
-  int J;      // partial slots per (batch, group, chunk)
+  int J;      // partial slots per (batch, group, chunk), per CTA of a pair
   int total;  // tiles
-  int ctas, q, r;  // total = q * ctas + r; CTA c owns [c q + min(c, r), ...)
+  int pairs, q, r;  // total = q * pairs + r; pair c owns [c q + min(c, r), ...)
 };
 
 __host__ __device__ inline int sched_begin(const QkvSched& s, int c) {
@@ -124,8 +135,8 @@ struct Tile {
   int col;    // g or the query column tile
   int k;      // chunk
   int run0;   // kv: first tile of the run's (b, k, g) block
-  int first;  // kv: first tile of its run in this CTA
-  int last;   // kv: last tile of its run in this CTA
+  int first;  // kv: first tile of its run in this pair
+  int last;   // kv: last tile of its run in this pair
 };
 
 __device__ __forceinline__ Tile decode(const QkvSched& s, int i, int i_begin, int i_end) {
@@ -170,6 +181,98 @@ __device__ __forceinline__ float warp_colsum(float (&x)[32], int lane) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// Byte offset of 16-byte chunk c (0..15) of token row r in a staging half:
+// rows of 256 bytes, chunks XOR-swizzled by the row so that 8 consecutive
+// rows writing the same chunk hit 8 different bank groups.
+__device__ __forceinline__ uint32_t stg_offset(int r, int c) {
+  return static_cast<uint32_t>(r * kStgRow + ((c ^ (r & 15)) << 4));
+}
+
+// ---------------------------------------------------------- CTA-pair PTX
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// All threads of both CTAs of the cluster.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::
+          : "memory");
+}
+
+// Shared-memory address, in the cluster window, of the variable at the same
+// offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+// 3D tiled load into this CTA's shared memory whose completion is counted on
+// an mbarrier of either CTA of the pair (no multicast).
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m,
+                                                 uint32_t bar_cluster, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// TMEM allocation shared by the pair: the same warp of both CTAs, the same
+// destination offset.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A[smem, 128 rows per CTA] * B[smem, 128 of N per
+// CTA]; bf16 inputs, fp32 accumulation; issued by one thread of CTA 0.
+__device__ __forceinline__ void mma_pair_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on the mbarrier at this offset in both CTAs of the pair when
+// the pair MMAs this thread issued so far have completed.
+__device__ __forceinline__ void mma_pair_commit_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+// ... on this CTA's mbarrier only.
+__device__ __forceinline__ void mma_pair_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
 template <int kRope>
 __global__ void __launch_bounds__(kQkvThreads, 1)
 qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
@@ -178,45 +281,41 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + QSmem::bars);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + QSmem::bars);  // CTA 0's count both
   uint64_t* empty = full + kQStages;
-  uint64_t* acc_full = empty + kQStages;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* stg_full = acc_empty + 1;
-  uint64_t* stg_empty = stg_full + 1;   // [2]: round 0, round 1
-  uint64_t* state_full = stg_empty + 2;  // [2]: run parity
-  uint64_t* mma_done = state_full + 2;
+  uint64_t* acc_full = empty + kQStages;  // [2]
+  uint64_t* acc_empty = acc_full + 2;     // [2], CTA 0's count both CTAs' epilogues
+  uint64_t* mma_done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + QSmem::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + QSmem::misc + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int cta = blockIdx.x;
-  const int i_begin = sched_begin(sc, cta), i_end = sched_begin(sc, cta + 1);
+  const uint32_t rank = cluster_rank();
+  const int pair = blockIdx.x >> 1;
+  const int i_begin = sched_begin(sc, pair), i_end = sched_begin(sc, pair + 1);
 
   if (tid == 0) {
     for (int s = 0; s < kQStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kQkvEpiWarps * 32);
-    mbar_init(stg_full, 4 * 32);  // the four warps of one round's token rows
-    mbar_init(&stg_empty[0], 1);
-    mbar_init(&stg_empty[1], 1);
-    mbar_init(&state_full[0], 1);
-    mbar_init(&state_full[1], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 2 * kQkvEpiWarps);  // one arrival per epilogue warp of the pair
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kWarpMma) {
-    tmem_alloc(tmem_slot, kQkvTmemCols);
-    tmem_relinquish();
-    tc_fence_before();
-  }
   if (warp == kWarpTma && lane == 0) {
     prefetch_tmap(&tm_x);
     prefetch_tmap(&tm_w);
+  }
+  cluster_sync_all();  // both CTAs' barriers are initialised before any remote use
+  if (warp == kWarpMma) {
+    tmem_alloc_pair(tmem_slot, kQkvTmemCols);
+    tmem_relinquish_pair();
+    tc_fence_before();
   }
   __syncthreads();
   tc_fence_after();
@@ -235,123 +334,69 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
       bool ok = true;
       for (int i = i_begin; ok && i < i_end; ++i) {
         const Tile t = decode(sc, i, i_begin, i_end);
-        const int y = t.nt * kTok;
-        // key/value tile: the group's 128 key rows and 128 value rows of W;
-        // query tile: 256 consecutive query rows. Rows past H*32 of a section
-        // read as zero.
-        const int wy0 = t.kv ? t.col * 128 : t.col * kCols;
-        const int wy1 = t.kv ? t.col * 128 : t.col * kCols + 128;
-        const int wz0 = t.kv ? 1 : 0, wz1 = t.kv ? 2 : 0;
+        const int y = t.nt * kTokPair + static_cast<int>(rank) * kTokCta;
+        // this CTA's 128 rows of the tile's 256 rows of W: the group's keys
+        // (CTA 0) or values (CTA 1), or half of 256 query rows. Rows past
+        // H*32 of a section read as zero, as do tokens past N and channels
+        // past C.
+        const int wy = t.kv ? t.col * 128 : t.col * kCols + static_cast<int>(rank) * 128;
+        const int wz = t.kv ? 1 + static_cast<int>(rank) : 0;
         for (int kb = 0; kb < sc.KB; ++kb, ++pos) {
           const int s = pos % kQStages;
           if (!(ok = mbar_wait(&empty[s], ((pos / kQStages) & 1) ^ 1, abort_flag, &g_qkv_error,
                                kErrWait)))
             break;
-          mbar_arrive_expect_tx(&full[s], kQStageBytes);
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * kQStageBytes);
+          const uint32_t bar = map_rank(smem_u32(&full[s]), 0);
           uint8_t* st = smem + QSmem::stages + s * kQStageBytes;
           const int x = kb * kKBlk;
-          tma_load_3d(st, &tm_x, &full[s], x, y, t.b);
-          tma_load_3d(st + kBoxBytes, &tm_w, &full[s], x, wy0, wz0);
-          tma_load_3d(st + 2 * kBoxBytes, &tm_w, &full[s], x, wy1, wz1);
+          tma_load_3d_pair(st, &tm_x, bar, x, y, t.b);
+          tma_load_3d_pair(st + kBoxBytes, &tm_w, bar, x, wy, wz);
         }
       }
-      // every load issued must have landed before the CTA exits
-      for (int qq = max(0, pos - kQStages); qq < pos; ++qq)
-        mbar_drain(&full[qq % kQStages], (qq / kQStages) & 1, &g_qkv_error, kErrWait);
+      // every load issued must have landed before the CTA frees its memory:
+      // CTA 0's full barriers count both CTAs' bytes; CTA 1's loads have
+      // landed once CTA 0's MMAs released the stages
+      for (int qq = max(0, pos - kQStages); qq < pos; ++qq) {
+        if (rank == 0)
+          mbar_drain(&full[qq % kQStages], (qq / kQStages) & 1, &g_qkv_error, kErrWait);
+        else
+          mbar_drain(&empty[qq % kQStages], (qq / kQStages) & 1, &g_qkv_error, kErrWait);
+      }
     }
   } else if (warp == kWarpMma) {
-    // ---------------------------------------------------------------- MMA
-    if (lane == 0) {
-      const uint32_t id_gemm = idesc_bf16_f32(kTok, kCols, 0, 0);
-      const uint32_t id_state = idesc_bf16_f32(128, 128, 1, 1);
-      const uint32_t stg = sbase + QSmem::stg;
-      int pending = 0;  // state rounds whose accumulator tile has been committed
-      int u = 0;        // state rounds issued so far
-      int svc_i = i_begin, svc_r = 0, run = -1;
-      bool have = false;
-      Tile svc{};
-      // Issue the next state round if its staging is written. Rounds are
-      // issued in tile order, between the GEMM's K-blocks.
-      auto service = [&]() -> bool {
-        if (pending == 0 || !mbar_try_wait(stg_full, u & 1)) return false;
-        if (!have) {
-          while (svc_i < i_end) {
-            svc = decode(sc, svc_i, i_begin, i_end);
-            if (svc.kv) break;
-            ++svc_i;
-          }
-          have = true;
-          if (svc.first) ++run;
-        }
-        tc_fence_after();
-        const uint32_t acc = tmem + kTmemState + (run & 1) * 128;
-#pragma unroll
-        for (int kk = 0; kk < kHalfTok / 16; ++kk) {
-          // 16 tokens = two 8-row groups; LBO = the second 64-dim box
-          const uint64_t ad = smem_desc_sw128(stg + kk * 2048, kStgBox, 1024);
-          const uint64_t bd = smem_desc_sw128(stg + 2 * kStgBox + kk * 2048, kStgBox, 1024);
-          mma_bf16(acc, ad, bd, id_state, (svc.first && svc_r == 0 && kk == 0) ? 0u : 1u);
-        }
-        mma_commit(&stg_empty[svc_r]);
-        if (svc_r == 1) {
-          if (svc.last) mma_commit(&state_full[run & 1]);
-          have = false;
-          ++svc_i;
-          svc_r = 0;
-        } else {
-          svc_r = 1;
-        }
-        ++u;
-        --pending;
-        return true;
-      };
-      // Bounded wait for a barrier phase (or, with bar == nullptr, for every
-      // pending state round) that keeps issuing state rounds meanwhile: the
-      // epilogue's next accumulator read may be waiting for one.
-      auto wait_svc = [&](uint64_t* bar, uint32_t parity) -> bool {
-        uint64_t t0 = globaltimer_ns();
-        while (true) {
-          if (bar != nullptr ? mbar_try_wait(bar, parity) : pending == 0) return true;
-          if (service()) {
-            t0 = globaltimer_ns();
-            continue;
-          }
-          if (*abort_flag) return false;
-          if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            atomicOr(&g_qkv_error, kErrWait);
-            return false;
-          }
-        }
-      };
+    // ----------------------------------------------------- MMA (CTA 0 only)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kTokPair, kCols, 0, 0);
       int pos = 0;
       bool ok = true;
       for (int i = i_begin; ok && i < i_end; ++i) {
-        const int tl = i - i_begin;
-        const bool kv = decode(sc, i, i_begin, i_end).kv;
-        // the epilogue has read the previous tile's accumulator
-        if (!(ok = wait_svc(acc_empty, (tl & 1) ^ 1))) break;
+        const int tl = i - i_begin, buf = tl & 1;
+        // both CTAs' epilogues have read this accumulator's previous tile
+        if (!(ok = mbar_wait(&acc_empty[buf], ((tl >> 1) & 1) ^ 1, abort_flag, &g_qkv_error,
+                             kErrWait)))
+          break;
         tc_fence_after();
+        const uint32_t acc = tmem + buf * kAccCols;
         for (int kb = 0; kb < sc.KB; ++kb, ++pos) {
           const int s = pos % kQStages;
-          if (!(ok = wait_svc(&full[s], (pos / kQStages) & 1))) break;
+          if (!(ok = mbar_wait(&full[s], (pos / kQStages) & 1, abort_flag, &g_qkv_error,
+                               kErrWait)))
+            break;
           tc_fence_after();
           const uint32_t st = sbase + QSmem::stages + s * kQStageBytes;
 #pragma unroll
           for (int kk = 0; kk < kKBlk / 16; ++kk) {
             const uint64_t ad = smem_desc_sw128(st + kk * 32, 16, 1024);
             const uint64_t bd = smem_desc_sw128(st + kBoxBytes + kk * 32, 16, 1024);
-            mma_bf16(tmem, ad, bd, id_gemm, (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_pair_bf16(acc, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&empty[s]);
-          service();
+          mma_pair_commit_both(&empty[s]);  // both CTAs' stages are free again
         }
         if (!ok) break;
-        mma_commit(acc_full);
-        if (kv) pending += 2;
+        mma_pair_commit_both(&acc_full[buf]);
       }
-      if (ok) wait_svc(nullptr, 0);
-      mma_commit(mma_done);
+      mma_pair_commit(mma_done);
       mbar_drain(mma_done, 0, &g_qkv_error, kErrWait);
     }
   } else {
@@ -359,19 +404,22 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
     const int quad = warp & 3;       // TMEM lane quadrant: token rows 32 quad ..
     const int hf = warp >> 2;        // 0: columns 0-127 (keys), 1: 128-255 (values)
     const int row = quad * 32 + lane;
-    const int rnd = quad >> 1;       // state round of this row
-    const int srow = row - rnd * kHalfTok;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t stg = sbase + QSmem::stg + (hf ? 2 * kStgBox : 0);
+    const uint32_t stg = sbase + QSmem::stg + (hf ? kStgHalf : 0);
+    const uint32_t stg_k = sbase + QSmem::stg, stg_v = stg_k + kStgHalf;
+    // the state block this thread accumulates: head sh, rows sd.., columns se..
+    const int sh = tid >> 6, sd = ((tid & 63) >> 3) * 4, se = (tid & 7) * 4;
+    float sacc[4][4] = {};
     float zacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    int kv_seen = 0, run = -1;
+    const uint32_t acc_empty_0[2] = {map_rank(smem_u32(&acc_empty[0]), 0),
+                                     map_rank(smem_u32(&acc_empty[1]), 0)};
     for (int i = i_begin; i < i_end; ++i) {
       const Tile t = decode(sc, i, i_begin, i_end);
-      const int tl = i - i_begin;
-      bool ok = mbar_wait(acc_full, tl & 1, abort_flag, &g_qkv_error, kErrWait);
+      const int tl = i - i_begin, buf = tl & 1;
+      bool ok = mbar_wait(&acc_full[buf], (tl >> 1) & 1, abort_flag, &g_qkv_error, kErrWait);
       if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.ld is warp-collective
       tc_fence_after();
-      const int n = t.nt * kTok + row;
+      const int n = t.nt * kTokPair + static_cast<int>(rank) * kTokCta + row;
       const bool valid = n < sc.N;
       // first feature (row of W, entry of the bias) of this warp's 128 columns
       const int f0 = t.kv ? (1 + hf) * sc.HD + t.col * 128 : t.col * kCols + hf * 128;
@@ -380,7 +428,7 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         float v[32];
-        tmem_ld_32x32b_x32(tmem + lane_base + hf * 128 + ch * 32, v);
+        tmem_ld_32x32b_x32(tmem + lane_base + buf * kAccCols + hf * 128 + ch * 32, v);
         const int f = f0 + ch * 32;
         if (f < f_end) {  // H*32 is a multiple of 32: a chunk is all in or all out
           if (bias != nullptr) {
@@ -403,8 +451,11 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
           for (int e = 0; e < 16; ++e) pk[ch * 16 + e] = 0u;
         }
       }
+      // the accumulator may take the tile after next (CTA 0's barrier counts
+      // one arrival per epilogue warp of the pair)
       tc_fence_before();
-      mbar_arrive(acc_empty);  // the accumulator may take the next tile
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(acc_empty_0[buf]);
 
       if (!t.kv) {
         // ---- query tile: the row's features straight to Q
@@ -424,7 +475,6 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
       }
 
       // ---- key/value tile
-      if (t.first) ++run;
       if (!valid) {
 #pragma unroll
         for (int e = 0; e < 64; ++e) pk[e] = 0u;
@@ -464,78 +514,96 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
           }
         }
       }
-      // staging: wait until the previous round's MMA has read it. Each round
-      // has its own barrier, which completes once per key/value tile: round 0
-      // waits for round 1 of the previous tile, round 1 for round 0 of this
-      // one. (With one barrier for both rounds a writer could be two phases
-      // ahead of it, which a parity wait cannot tell from the phase it wants.)
-      ok = rnd == 0 ? mbar_wait(&stg_empty[1], (kv_seen & 1) ^ 1, abort_flag, &g_qkv_error,
-                                kErrWait)
-                    : mbar_wait(&stg_empty[0], kv_seen & 1, abort_flag, &g_qkv_error, kErrWait);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      // staging: phi(k) (warps 0-3) and v (warps 4-7) of the CTA's 128
+      // tokens, once every thread has finished the previous tile's product
+      named_bar_sync(kBarEpi, kEpiThreads);
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch)
+      for (int c = 0; c < 16; ++c)
+        st_shared_v4(stg + stg_offset(row, c),
+                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
+      named_bar_sync(kBarEpi, kEpiThreads);
+      // S[sh][sd + a][se + c] += sum over the tile's tokens, in token order
+      {
+        const int ck = (sh * 32 + sd) >> 3, bk = ((sh * 32 + sd) & 7) * 2;  // chunk, byte
+        const int cv = (sh * 32 + se) >> 3, bv = ((sh * 32 + se) & 7) * 2;
+#pragma unroll 4
+        for (int r = 0; r < kTokCta; ++r) {
+          uint32_t k0, k1, v0, v1;
+          asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
+                       : "=r"(k0), "=r"(k1)
+                       : "r"(stg_k + stg_offset(r, ck) + bk));
+          asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
+                       : "=r"(v0), "=r"(v1)
+                       : "r"(stg_v + stg_offset(r, cv) + bv));
+          const float kx[4] = {bf16_lo(k0), bf16_hi(k0), bf16_lo(k1), bf16_hi(k1)};
+          const float2 v01 = make_float2(bf16_lo(v0), bf16_hi(v0));
+          const float2 v23 = make_float2(bf16_lo(v1), bf16_hi(v1));
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          st_shared_v4(stg + (ch >> 1) * kStgBox + sw128_offset(srow, (ch & 1) * 4 + k),
-                       make_uint4(pk[ch * 16 + 4 * k], pk[ch * 16 + 4 * k + 1],
-                                  pk[ch * 16 + 4 * k + 2], pk[ch * 16 + 4 * k + 3]));
-      fence_proxy_async_smem();
-      mbar_arrive(stg_full);
-      ++kv_seen;
+          for (int a = 0; a < 4; ++a) {
+            const float2 ka = make_float2(kx[a], kx[a]);
+            float2 lo = make_float2(sacc[a][0], sacc[a][1]);
+            float2 hi = make_float2(sacc[a][2], sacc[a][3]);
+            lo = __ffma2_rn(ka, v01, lo);
+            hi = __ffma2_rn(ka, v23, hi);
+            sacc[a][0] = lo.x;
+            sacc[a][1] = lo.y;
+            sacc[a][2] = hi.x;
+            sacc[a][3] = hi.y;
+          }
+        }
+      }
 
-      if (t.last && hf == 0) {
-        // ---- end of a run: head `quad`'s state block and this quadrant's
-        // key sums go to the run's partial slot
-        const int a = run & 1;
-        ok = mbar_wait(&state_full[a], (run >> 1) & 1, abort_flag, &g_qkv_error, kErrWait);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        tc_fence_after();
-        float s[32];
-        tmem_ld_32x32b_x32(tmem + lane_base + kTmemState + a * 128 + quad * 32, s);
-        tc_fence_before();
-        const int g = t.col;
-        const int slot = cta - sched_owner(sc, t.run0);
-        float* dst = part + ((static_cast<size_t>(t.b * sc.G + g) * sc.NK + t.k) * sc.J + slot) *
-                                kPartFloats;
-        float* ds = dst + quad * kD * kD + lane * kD;
+      if (t.last) {
+        // ---- end of a run: this CTA's partial (S, z) of the run
+        const int slot = pair - sched_owner(sc, t.run0);
+        float* dst = part + (((static_cast<size_t>(t.b * sc.G + t.col) * sc.NK + t.k) * sc.J +
+                              slot) * 2 + rank) * kPartFloats;
+        float* ds = dst + sh * kD * kD + sd * kD + se;
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(ds + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
+        for (int a = 0; a < 4; ++a) {
+          *reinterpret_cast<float4*>(ds + a * kD) =
+              make_float4(sacc[a][0], sacc[a][1], sacc[a][2], sacc[a][3]);
+          sacc[a][0] = sacc[a][1] = sacc[a][2] = sacc[a][3] = 0.0f;
+        }
+        if (hf == 0) {
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          dst[kPartS + quad * 4 * kD + ch * kD + lane] = zacc[ch];
-          zacc[ch] = 0.0f;
+          for (int ch = 0; ch < 4; ++ch) {
+            dst[kPartS + quad * 4 * kD + ch * kD + lane] = zacc[ch];
+            zacc[ch] = 0.0f;
+          }
         }
       }
     }
   }
 
+  // neither CTA leaves while the other may still use its shared memory or
+  // the pair's tensor memory
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();  // the cluster barrier is .aligned: whole warps
+  cluster_sync_all();
   if (warp == kWarpMma) {
     tc_fence_after();
-    tmem_dealloc(tmem, kQkvTmemCols);
+    tmem_dealloc_pair(tmem, kQkvTmemCols);
   }
 }
 
 // Sum of the partial slots of one (batch, head group) in a fixed order:
-// chunk, then slot, then (for z) TMEM lane quadrant.
+// chunk, slot, CTA of the pair, then (for z) TMEM lane quadrant.
 __global__ void __launch_bounds__(256)
 qkv_combine(const QkvSched sc, const float* __restrict__ part, float* __restrict__ S,
             float* __restrict__ z) {
   pdl_wait();
   const int bg = blockIdx.x;
   const int b = bg / sc.G, g = bg - b * sc.G;
-  const float* base = part + static_cast<size_t>(bg) * sc.NK * sc.J * kPartFloats;
+  const float* base = part + static_cast<size_t>(bg) * sc.NK * sc.J * 2 * kPartFloats;
   for (int v = threadIdx.x; v < (kPartS + 4 * kD) / 4; v += blockDim.x) {
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     for (int k = 0; k < sc.NK; ++k) {
       const int len = chunk_len(sc, k);
       const int run0 = chunk_begin(sc, b, k) + g * len;
       const int nslots = sched_owner(sc, run0 + len - 1) - sched_owner(sc, run0) + 1;
-      for (int j = 0; j < nslots; ++j) {
-        const float* src = base + (static_cast<size_t>(k) * sc.J + j) * kPartFloats;
+      for (int j = 0; j < 2 * nslots; ++j) {  // slot-major, then the CTA of the pair
+        const float* src = base + (static_cast<size_t>(k) * sc.J * 2 + j) * kPartFloats;
         if (v < kPartS / 4) {
           const float4 t = __ldcg(reinterpret_cast<const float4*>(src) + v);
           acc.x += t.x;
@@ -579,16 +647,16 @@ QkvSched make_sched(int B, int N, int H, int C) {
   s.H = H;
   s.C = C;
   s.HD = H * kD;
-  s.NT = (N + kTok - 1) / kTok;
+  s.NT = (N + kTokPair - 1) / kTokPair;
   s.G = (H + 3) / 4;
   s.QC = (s.HD + kCols - 1) / kCols;
   s.CT = s.G + s.QC;
   s.KB = (C + kKBlk - 1) / kKBlk;
   const long long total = 1LL * B * s.NT * s.CT;
   s.total = static_cast<int>(total);
-  s.ctas = static_cast<int>(std::min<long long>(kNumSMs, std::max<long long>(1, total)));
-  s.q = std::max(1, s.total / s.ctas);
-  s.r = s.total - s.q * s.ctas;
+  s.pairs = static_cast<int>(std::min<long long>(kNumSMs / 2, std::max<long long>(1, total)));
+  s.q = std::max(1, s.total / s.pairs);
+  s.r = s.total - s.q * s.pairs;
   s.L = std::max(1, std::min(s.NT, s.q));
   s.NK = (s.NT + s.L - 1) / s.L;
   s.J = std::min(s.L, (s.L - 1) / s.q + 2);
@@ -619,7 +687,7 @@ using QkvKernel = void (*)(CUtensorMap, CUtensorMap, QkvSched, Rope, const __nv_
 size_t qkv_workspace_floats(int B, int N, int H, int C) {
   if (N <= 0 || B <= 0 || H <= 0) return 0;
   const QkvSched s = make_sched(B, N, H, C);
-  return static_cast<size_t>(B) * s.G * s.NK * s.J * kPartFloats;
+  return static_cast<size_t>(B) * s.G * s.NK * s.J * 2 * kPartFloats;
 }
 
 cudaError_t launch_qkv_state(const Problem& p, int C, const void* X, const void* W,
@@ -635,16 +703,20 @@ cudaError_t launch_qkv_state(const Problem& p, int C, const void* X, const void*
   if ((e = ensure_smem_attr(mode == kNoRope ? 0 : 1, reinterpret_cast<const void*>(kern),
                             kQSmemBytes)) != cudaSuccess)
     return e;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(sc.ctas, 1, 1);
+  cfg.gridDim = dim3(2 * sc.pairs, 1, 1);
   cfg.blockDim = dim3(kQkvThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(kQSmemBytes);
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, kern, mx, mw, sc, p.rope,
                          static_cast<const __nv_bfloat16*>(bias), static_cast<__nv_bfloat16*>(Q),
                          part);
