@@ -70,6 +70,8 @@ constexpr int kTokCta = 128;               // tokens per CTA per tile (TMEM lane
 constexpr int kTokPair = 2 * kTokCta;      // tokens per tile (MMA M, across the pair)
 constexpr int kCols = 256;                 // output features per tile (MMA N)
 constexpr int kKBlk = 64;                  // channels per stage
+// TMA stages (6 stages, with the state staging cut into two rounds to make
+// room, measured the same: the loop is not short of loads in flight).
 constexpr int kQStages = 5;
 constexpr int kBoxBytes = 128 * 128;       // [128 rows][64 bf16], 128-byte swizzle
 constexpr int kQStageBytes = 2 * kBoxBytes;  // this CTA's X rows + its 128 rows of W
@@ -588,53 +590,59 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
 }
 
 // Sum of the partial slots of one (batch, head group) in a fixed order:
-// chunk, slot, CTA of the pair, then (for z) TMEM lane quadrant.
-__global__ void __launch_bounds__(256)
+// chunk, slot, CTA of the pair, then (for z) TMEM lane quadrant. One thread
+// per float4 of the result; a chunk's (at most 2 x 2) partials are loaded
+// together, then added in that order.
+constexpr int kCombineThreads = 128;
+constexpr int kResultVec = (kPartS + 4 * kD) / 4;  // 1024 float4 of S, 32 of z
+
+__global__ void __launch_bounds__(kCombineThreads)
 qkv_combine(const QkvSched sc, const float* __restrict__ part, float* __restrict__ S,
             float* __restrict__ z) {
   pdl_wait();
   const int bg = blockIdx.x;
   const int b = bg / sc.G, g = bg - b * sc.G;
-  const float* base = part + static_cast<size_t>(bg) * sc.NK * sc.J * 2 * kPartFloats;
-  for (int v = threadIdx.x; v < (kPartS + 4 * kD) / 4; v += blockDim.x) {
-    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    for (int k = 0; k < sc.NK; ++k) {
-      const int len = chunk_len(sc, k);
-      const int run0 = chunk_begin(sc, b, k) + g * len;
-      const int nslots = sched_owner(sc, run0 + len - 1) - sched_owner(sc, run0) + 1;
-      for (int j = 0; j < 2 * nslots; ++j) {  // slot-major, then the CTA of the pair
-        const float* src = base + (static_cast<size_t>(k) * sc.J * 2 + j) * kPartFloats;
-        if (v < kPartS / 4) {
-          const float4 t = __ldcg(reinterpret_cast<const float4*>(src) + v);
-          acc.x += t.x;
-          acc.y += t.y;
-          acc.z += t.z;
-          acc.w += t.w;
-        } else {
+  const int v = blockIdx.y * kCombineThreads + threadIdx.x;
+  if (v >= kResultVec) return;
+  const bool is_s = v < kPartS / 4;
+  constexpr int kVecPerPart = kPartFloats / 4;
+  const float4* base =
+      reinterpret_cast<const float4*>(part) + static_cast<size_t>(bg) * sc.NK * sc.J * 2 * kVecPerPart;
+  float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int k = 0; k < sc.NK; ++k) {
+    const int len = chunk_len(sc, k);
+    const int run0 = chunk_begin(sc, b, k) + g * len;
+    const int cnt = 2 * (sched_owner(sc, run0 + len - 1) - sched_owner(sc, run0) + 1);  // <= 4
+    const float4* src = base + static_cast<size_t>(k) * sc.J * 2 * kVecPerPart;
+    float4 t[4][4];
 #pragma unroll
-          for (int qd = 0; qd < 4; ++qd) {
-            const float4 t = __ldcg(reinterpret_cast<const float4*>(src + kPartS + qd * 4 * kD) +
-                                    (v - kPartS / 4));
-            acc.x += t.x;
-            acc.y += t.y;
-            acc.z += t.z;
-            acc.w += t.w;
-          }
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int qd = 0; qd < 4; ++qd)
+        if (j < cnt && (!is_s || qd == 0))
+          t[j][qd] = __ldcg(src + j * kVecPerPart +
+                            (is_s ? v : kPartS / 4 + qd * kD + (v - kPartS / 4)));
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int qd = 0; qd < 4; ++qd)
+        if (j < cnt && (!is_s || qd == 0)) {
+          acc.x += t[j][qd].x;
+          acc.y += t[j][qd].y;
+          acc.z += t[j][qd].z;
+          acc.w += t[j][qd].w;
         }
-      }
-    }
-    if (v < kPartS / 4) {
-      const int hh = v / (kD * kD / 4), h = 4 * g + hh;
-      if (h < sc.H)
-        *reinterpret_cast<float4*>(S + (static_cast<size_t>(b) * sc.H + h) * kD * kD +
-                                   (v - hh * (kD * kD / 4)) * 4) = acc;
-    } else {
-      const int w = v - kPartS / 4;  // head w / 8, dims 4 (w % 8) ..
-      const int hh = w >> 3, h = 4 * g + hh;
-      if (h < sc.H)
-        *reinterpret_cast<float4*>(z + (static_cast<size_t>(b) * sc.H + h) * kD + (w & 7) * 4) =
-            acc;
-    }
+  }
+  if (is_s) {
+    const int hh = v / (kD * kD / 4), h = 4 * g + hh;
+    if (h < sc.H)
+      *reinterpret_cast<float4*>(S + (static_cast<size_t>(b) * sc.H + h) * kD * kD +
+                                 (v - hh * (kD * kD / 4)) * 4) = acc;
+  } else {
+    const int w = v - kPartS / 4;  // head w / 8, dims 4 (w % 8) ..
+    const int hh = w >> 3, h = 4 * g + hh;
+    if (h < sc.H)
+      *reinterpret_cast<float4*>(z + (static_cast<size_t>(b) * sc.H + h) * kD + (w & 7) * 4) = acc;
   }
 }
 
@@ -659,7 +667,7 @@ QkvSched make_sched(int B, int N, int H, int C) {
   s.r = s.total - s.q * s.pairs;
   s.L = std::max(1, std::min(s.NT, s.q));
   s.NK = (s.NT + s.L - 1) / s.L;
-  s.J = std::min(s.L, (s.L - 1) / s.q + 2);
+  s.J = std::min(s.L, (s.L - 1) / s.q + 2);  // L <= q, so J <= 2: a run spans <= 2 pairs
   return s;
 }
 
@@ -722,8 +730,8 @@ cudaError_t launch_qkv_state(const Problem& p, int C, const void* X, const void*
                          part);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg2 = {};
-  cfg2.gridDim = dim3(p.B * sc.G, 1, 1);
-  cfg2.blockDim = dim3(256, 1, 1);
+  cfg2.gridDim = dim3(p.B * sc.G, (kResultVec + kCombineThreads - 1) / kCombineThreads, 1);
+  cfg2.blockDim = dim3(kCombineThreads, 1, 1);
   cfg2.stream = s;
   cfg2.attrs = attr;
   cfg2.numAttrs = 1;
