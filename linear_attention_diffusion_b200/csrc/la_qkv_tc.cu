@@ -27,8 +27,9 @@
 // and 128 value features of a group of four heads. For a key/value tile the
 // epilogue rounds k and v to bf16, applies ReLU (and RoPE) to k, sums ReLU(k)
 // over the tokens (warp transpose-sums), stages phi(k) and v in shared memory
-// and accumulates the four heads' phi(K)^T V on CUDA cores in float32 (every
-// thread a 4 x 4 block of one head's 32 x 32 state, tokens in order), over
+// and accumulates the four heads' phi(K)^T V with warp-level mma.sync
+// (bf16 operands read with ldmatrix, fp32 accumulators in registers; every
+// warp 16 rows of one head's 32 x 32 state, tokens in a fixed order), over
 // the pair's consecutive tiles of the same head group (a "run"). At the end
 // of a run each CTA writes its partial (S, z) to a slot of the workspace; a
 // second kernel sums every head's slots in a fixed order, so S and z are
@@ -188,6 +189,26 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 // rows writing the same chunk hit 8 different bank groups.
 __device__ __forceinline__ uint32_t stg_offset(int r, int c) {
   return static_cast<uint32_t>(r * kStgRow + ((c ^ (r & 15)) << 4));
+}
+
+// Four 8x8 bf16 matrices from shared memory, each transposed on the way
+// (thread i gives the address of row i % 8 of matrix i / 8).
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                              uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// d (16 x 8, fp32) += a (16 x 16, bf16) * b (16 x 8, bf16): a warp-wide MMA
+// for the small state product of the epilogue.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // ---------------------------------------------------------- CTA-pair PTX
@@ -409,8 +430,11 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t stg = sbase + QSmem::stg + (hf ? kStgHalf : 0);
     const uint32_t stg_k = sbase + QSmem::stg, stg_v = stg_k + kStgHalf;
-    // the state block this thread accumulates: head sh, rows sd.., columns se..
-    const int sh = tid >> 6, sd = ((tid & 63) >> 3) * 4, se = (tid & 7) * 4;
+    // the state block this warp accumulates: head sh, rows 16 smb .. + 15,
+    // all 32 columns (four 16 x 8 MMA accumulators); g, t4: the lane's place
+    // in an accumulator fragment
+    const int sh = warp >> 1, smb = warp & 1;
+    const int g = lane >> 2, t4 = lane & 3;
     float sacc[4][4] = {};
     float zacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     const uint32_t acc_empty_0[2] = {map_rank(smem_u32(&acc_empty[0]), 0),
@@ -418,32 +442,41 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
     for (int i = i_begin; i < i_end; ++i) {
       const Tile t = decode(sc, i, i_begin, i_end);
       const int tl = i - i_begin, buf = tl & 1;
-      bool ok = mbar_wait(&acc_full[buf], (tl >> 1) & 1, abort_flag, &g_qkv_error, kErrWait);
-      if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.ld is warp-collective
-      tc_fence_after();
       const int n = t.nt * kTokPair + static_cast<int>(rank) * kTokCta + row;
       const bool valid = n < sc.N;
       // first feature (row of W, entry of the bias) of this warp's 128 columns
       const int f0 = t.kv ? (1 + hf) * sc.HD + t.col * 128 : t.col * kCols + hf * 128;
       const int f_end = t.kv ? (2 + hf) * sc.HD : sc.HD;
+      // the bias of chunk ch (32 features as 16 bf16 pairs), loaded two chunks
+      // ahead; the first two before the accumulator wait, so that their
+      // latency hides behind it
+      uint4 bq[2][4];
+      auto load_bias = [&](int ch, uint4(&dst)[4]) {
+        const int f = f0 + ch * 32;
+        const bool have = bias != nullptr && f < f_end;
+        const uint4* bp = reinterpret_cast<const uint4*>(bias + (have ? f : 0));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) dst[k] = have ? __ldg(bp + k) : make_uint4(0u, 0u, 0u, 0u);
+      };
+      load_bias(0, bq[0]);
+      load_bias(1, bq[1]);
+      bool ok = mbar_wait(&acc_full[buf], (tl >> 1) & 1, abort_flag, &g_qkv_error, kErrWait);
+      if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.ld is warp-collective
+      tc_fence_after();
       uint32_t pk[64];  // the row's 128 features: bf16(acc + bias), in pairs
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         float v[32];
         tmem_ld_32x32b_x32(tmem + lane_base + buf * kAccCols + hf * 128 + ch * 32, v);
-        const int f = f0 + ch * 32;
-        if (f < f_end) {  // H*32 is a multiple of 32: a chunk is all in or all out
-          if (bias != nullptr) {
-            const uint4* bp = reinterpret_cast<const uint4*>(bias + f);
+        if (f0 + ch * 32 < f_end) {  // H*32 is a multiple of 32: a chunk is all in or all out
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint4 w4 = __ldg(bp + k);
-              const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t w[4] = {bq[ch & 1][k].x, bq[ch & 1][k].y, bq[ch & 1][k].z,
+                                   bq[ch & 1][k].w};
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                v[8 * k + 2 * e] += bf16_lo(w[e]);
-                v[8 * k + 2 * e + 1] += bf16_hi(w[e]);
-              }
+            for (int e = 0; e < 4; ++e) {
+              v[8 * k + 2 * e] += bf16_lo(w[e]);
+              v[8 * k + 2 * e + 1] += bf16_hi(w[e]);
             }
           }
 #pragma unroll
@@ -452,6 +485,7 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[ch * 16 + e] = 0u;
         }
+        if (ch + 2 < 4) load_bias(ch + 2, bq[ch & 1]);
       }
       // the accumulator may take the tile after next (CTA 0's barrier counts
       // one arrival per epilogue warp of the pair)
@@ -524,34 +558,26 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
         st_shared_v4(stg + stg_offset(row, c),
                      make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
       named_bar_sync(kBarEpi, kEpiThreads);
-      // S[sh][sd + a][se + c] += sum over the tile's tokens, in token order
+      // S[sh][16 smb + m][e] += sum over the tile's tokens of phi(k)[m] v[e]:
+      // 8 steps of 16 tokens, A = phi(K)^T and B = V straight from the
+      // staging rows (ldmatrix with transpose), fixed order
       {
-        const int ck = (sh * 32 + sd) >> 3, bk = ((sh * 32 + sd) & 7) * 2;  // chunk, byte
-        const int cv = (sh * 32 + se) >> 3, bv = ((sh * 32 + se) & 7) * 2;
-#pragma unroll 4
-        for (int r = 0; r < kTokCta; ++r) {
-          uint32_t k0, k1, v0, v1;
-          asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
-                       : "=r"(k0), "=r"(k1)
-                       : "r"(stg_k + stg_offset(r, ck) + bk));
-          asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
-                       : "=r"(v0), "=r"(v1)
-                       : "r"(stg_v + stg_offset(r, cv) + bv));
-          const float kx[4] = {bf16_lo(k0), bf16_hi(k0), bf16_lo(k1), bf16_hi(k1)};
-          const float2 v01 = make_float2(bf16_lo(v0), bf16_hi(v0));
-          const float2 v23 = make_float2(bf16_lo(v1), bf16_hi(v1));
+        const int j = lane >> 3, q = lane & 7;
+        const int a_dim = sh * 32 + smb * 16 + ((j & 1) << 3);  // A: matrix j = (m half, k half)
+        const int a_row = ((j >> 1) << 3) + q;
+        const int b_row = ((j & 1) << 3) + q;                    // B: matrix j = (k half, n block)
 #pragma unroll
-          for (int a = 0; a < 4; ++a) {
-            const float2 ka = make_float2(kx[a], kx[a]);
-            float2 lo = make_float2(sacc[a][0], sacc[a][1]);
-            float2 hi = make_float2(sacc[a][2], sacc[a][3]);
-            lo = __ffma2_rn(ka, v01, lo);
-            hi = __ffma2_rn(ka, v23, hi);
-            sacc[a][0] = lo.x;
-            sacc[a][1] = lo.y;
-            sacc[a][2] = hi.x;
-            sacc[a][3] = hi.y;
-          }
+        for (int kb = 0; kb < kTokCta / 16; ++kb) {
+          uint32_t a0, a1, a2, a3, b0, b1, b2, b3, b4, b5, b6, b7;
+          ldsm_x4_trans(stg_k + stg_offset(kb * 16 + a_row, a_dim >> 3), a0, a1, a2, a3);
+          ldsm_x4_trans(stg_v + stg_offset(kb * 16 + b_row, (sh * 32 + ((j >> 1) << 3)) >> 3), b0,
+                        b1, b2, b3);
+          ldsm_x4_trans(stg_v + stg_offset(kb * 16 + b_row, (sh * 32 + 16 + ((j >> 1) << 3)) >> 3),
+                        b4, b5, b6, b7);
+          mma_16816(sacc[0], a0, a1, a2, a3, b0, b1);
+          mma_16816(sacc[1], a0, a1, a2, a3, b2, b3);
+          mma_16816(sacc[2], a0, a1, a2, a3, b4, b5);
+          mma_16816(sacc[3], a0, a1, a2, a3, b6, b7);
         }
       }
 
@@ -560,12 +586,13 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
         const int slot = pair - sched_owner(sc, t.run0);
         float* dst = part + (((static_cast<size_t>(t.b * sc.G + t.col) * sc.NK + t.k) * sc.J +
                               slot) * 2 + rank) * kPartFloats;
-        float* ds = dst + sh * kD * kD + sd * kD + se;
+        // accumulator nb: rows 16 smb + g (+ 8), columns 8 nb + 2 t4 (+ 1)
+        float* ds = dst + sh * kD * kD + (smb * 16 + g) * kD + 2 * t4;
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          *reinterpret_cast<float4*>(ds + a * kD) =
-              make_float4(sacc[a][0], sacc[a][1], sacc[a][2], sacc[a][3]);
-          sacc[a][0] = sacc[a][1] = sacc[a][2] = sacc[a][3] = 0.0f;
+        for (int nb = 0; nb < 4; ++nb) {
+          *reinterpret_cast<float2*>(ds + nb * 8) = make_float2(sacc[nb][0], sacc[nb][1]);
+          *reinterpret_cast<float2*>(ds + 8 * kD + nb * 8) = make_float2(sacc[nb][2], sacc[nb][3]);
+          sacc[nb][0] = sacc[nb][1] = sacc[nb][2] = sacc[nb][3] = 0.0f;
         }
         if (hf == 0) {
 #pragma unroll
