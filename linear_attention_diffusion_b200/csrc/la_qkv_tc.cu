@@ -211,6 +211,18 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// cos and sin of pos * inv_freq for the key feature map: the angle is formed
+// and reduced to [-pi, pi] in double (exact enough for any position), then
+// evaluated with the hardware approximations, whose absolute error on
+// [-pi, pi] (about 2^-21) is far below the bf16 rounding of phi(k) that
+// follows.
+__device__ __forceinline__ void rope_cs_fast(int pos, double inv_freq, float& c, float& s) {
+  const double kTwoPi = 6.283185307179586476925286766559;
+  const double a = static_cast<double>(pos) * inv_freq;
+  const float r = static_cast<float>(a - kTwoPi * rint(a * (1.0 / kTwoPi)));
+  __sincosf(r, &s, &c);
+}
+
 // ---------------------------------------------------------- CTA-pair PTX
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -460,103 +472,89 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
       };
       load_bias(0, bq[0]);
       load_bias(1, bq[1]);
+      // RoPE angles of this token (the same for every head), once per tile
+      float2 cs[16];
+      if (kRope != kNoRope && t.kv && hf == 0) {
+        const TokPos tp = token_pos(rope, valid ? n : 0);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int ax = pair_axis(j);
+          const int pp = ax == 0 ? rope.t_offset + tp.t : (ax == 1 ? tp.h : tp.w);
+          rope_cs_fast(pp, rope.inv_freq[j], cs[j].x, cs[j].y);
+        }
+      }
       bool ok = mbar_wait(&acc_full[buf], (tl >> 1) & 1, abort_flag, &g_qkv_error, kErrWait);
       if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.ld is warp-collective
       tc_fence_after();
-      uint32_t pk[64];  // the row's 128 features: bf16(acc + bias), in pairs
+      // key/value tile: the staging is free once every thread has finished
+      // the previous tile's product
+      if (t.kv) named_bar_sync(kBarEpi, kEpiThreads);
+      __nv_bfloat16* qdst = Q + (static_cast<size_t>(t.b) * sc.N + (valid ? n : 0)) * sc.HD + f0;
+      // the row's 128 features in four chunks of 32: bf16(acc + bias), then
+      // straight to Q, or (keys) ReLU, key sums, RoPE, and to the staging
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         float v[32];
         tmem_ld_32x32b_x32(tmem + lane_base + buf * kAccCols + hf * 128 + ch * 32, v);
-        if (f0 + ch * 32 < f_end) {  // H*32 is a multiple of 32: a chunk is all in or all out
+        uint32_t w[16];  // 32 features as bf16 pairs
+        const bool in = f0 + ch * 32 < f_end;  // H*32 is a multiple of 32
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t w[4] = {bq[ch & 1][k].x, bq[ch & 1][k].y, bq[ch & 1][k].z,
-                                   bq[ch & 1][k].w};
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t bw[4] = {bq[ch & 1][k].x, bq[ch & 1][k].y, bq[ch & 1][k].z,
+                                  bq[ch & 1][k].w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              v[8 * k + 2 * e] += bf16_lo(w[e]);
-              v[8 * k + 2 * e + 1] += bf16_hi(w[e]);
+          for (int e = 0; e < 4; ++e) {
+            v[8 * k + 2 * e] += bf16_lo(bw[e]);
+            v[8 * k + 2 * e + 1] += bf16_hi(bw[e]);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = in && (valid || !t.kv) ? pack_bf16x2(v[2 * e], v[2 * e + 1]) : 0u;
+        if (ch + 2 < 4) load_bias(ch + 2, bq[ch & 1]);
+        if (!t.kv) {
+          if (valid && in) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              *reinterpret_cast<uint4*>(qdst + ch * 32 + 8 * k) =
+                  make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          }
+          continue;
+        }
+        if (hf == 0) {
+          // keys of head ch: ReLU (exact on bf16), the key sum of the
+          // unrotated ReLU(k), then phi(k) = R(t, h, w) ReLU(k)
+          float x[32];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            w[e] = relu_bf16x2(w[e]);
+            x[2 * e] = bf16_lo(w[e]);
+            x[2 * e + 1] = bf16_hi(w[e]);
+          }
+          zacc[ch] += warp_colsum(x, lane);
+          if (kRope != kNoRope && valid) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float x0 = bf16_lo(w[j]), x1 = bf16_hi(w[j]);
+              const float2 tt = __fmul2_rn(make_float2(x1, x1), make_float2(-cs[j].y, cs[j].x));
+              const float2 yy = __ffma2_rn(make_float2(x0, x0), cs[j], tt);
+              w[j] = pack_bf16x2(yy.x, yy.y);
             }
           }
-#pragma unroll
-          for (int e = 0; e < 16; ++e) pk[ch * 16 + e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) pk[ch * 16 + e] = 0u;
         }
-        if (ch + 2 < 4) load_bias(ch + 2, bq[ch & 1]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          st_shared_v4(stg + stg_offset(row, ch * 4 + k),
+                       make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]));
       }
       // the accumulator may take the tile after next (CTA 0's barrier counts
       // one arrival per epilogue warp of the pair)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(acc_empty_0[buf]);
+      if (!t.kv) continue;
 
-      if (!t.kv) {
-        // ---- query tile: the row's features straight to Q
-        if (valid) {
-          __nv_bfloat16* dst = Q + (static_cast<size_t>(t.b) * sc.N + n) * sc.HD + f0;
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            if (f0 + ch * 32 >= sc.HD) break;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              *reinterpret_cast<uint4*>(dst + ch * 32 + 8 * k) =
-                  make_uint4(pk[ch * 16 + 4 * k], pk[ch * 16 + 4 * k + 1],
-                             pk[ch * 16 + 4 * k + 2], pk[ch * 16 + 4 * k + 3]);
-          }
-        }
-        continue;
-      }
-
-      // ---- key/value tile
-      if (!valid) {
-#pragma unroll
-        for (int e = 0; e < 64; ++e) pk[e] = 0u;
-      }
-      if (hf == 0) {
-        // keys: ReLU (exact on bf16), key sums of the unrotated ReLU(k)
-#pragma unroll
-        for (int e = 0; e < 64; ++e) pk[e] = relu_bf16x2(pk[e]);
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          float x[32];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            x[2 * e] = bf16_lo(pk[ch * 16 + e]);
-            x[2 * e + 1] = bf16_hi(pk[ch * 16 + e]);
-          }
-          zacc[ch] += warp_colsum(x, lane);
-        }
-        if (kRope != kNoRope && valid) {
-          // phi(k) = R(t, h, w) ReLU(k): pair j of every head turns by the
-          // token's position on the pair's axis times inv_freq[j]
-          const TokPos tp = token_pos(rope, n);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int ax = pair_axis(j);
-            const int pp = ax == 0 ? rope.t_offset + tp.t : (ax == 1 ? tp.h : tp.w);
-            float2 r;
-            rope_cos_sin(pp, rope.inv_freq[j], r.x, r.y);
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {  // the same angle for every head
-              const uint32_t w = pk[ch * 16 + j];
-              const float x0 = bf16_lo(w), x1 = bf16_hi(w);
-              const float2 tt = __fmul2_rn(make_float2(x1, x1), make_float2(-r.y, r.x));
-              const float2 yy = __ffma2_rn(make_float2(x0, x0), r, tt);
-              pk[ch * 16 + j] = pack_bf16x2(yy.x, yy.y);
-            }
-          }
-        }
-      }
-      // staging: phi(k) (warps 0-3) and v (warps 4-7) of the CTA's 128
-      // tokens, once every thread has finished the previous tile's product
-      named_bar_sync(kBarEpi, kEpiThreads);
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        st_shared_v4(stg + stg_offset(row, c),
-                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
+      // ---- key/value tile: the staged rows are complete
       named_bar_sync(kBarEpi, kEpiThreads);
       // S[sh][16 smb + m][e] += sum over the tile's tokens of phi(k)[m] v[e]:
       // 8 steps of 16 tokens, A = phi(K)^T and B = V straight from the

@@ -205,3 +205,32 @@ def test_qkv_state_empty_sequence(cuda_device):
     la.la_qkv_state(shape, C, X, W, None, Q, S, z, None)
     torch.cuda.synchronize()
     assert (S == 0).all() and (z == 0).all()
+
+
+def test_qkv_state_video_rope_full_size_sampled(cuda_device):
+    """SANA-Video 480p grid (21 x 30 x 52 tokens, 3D RoPE on the keys, C = 2240):
+    Q at sampled tokens, S and z of sampled heads over every token."""
+    w = wl.WORKLOADS["sanavideo_480p"]
+    C = wl.hidden_width(w)
+    X, W, b = wl.make_projection(w, C, seed=31)
+    Q, S, z = _run(X, W, b, rope_grid=(w.T, w.Hh, w.W))
+    hd = w.H * D
+    rng = np.random.default_rng(6)
+    toks = np.sort(rng.choice(w.N, size=32, replace=False))
+    toks[-1] = w.N - 1
+    y, mag = _project(X[:, toks], W, b, np.arange(hd))
+    r, E = _step_and_near(y, mag)
+    _check_q(Q[:, toks], r.reshape(w.B, len(toks), w.H, D), E.reshape(w.B, len(toks), w.H, D),
+             "480p sampled tokens")
+    heads = [1, 38, 69]
+    theta = orc.rope_angles(w.T, w.Hh, w.W, 0)
+    k_o, v_o = orc.key_value_heads(X, W, b, w.H, heads)
+    rows_k = np.concatenate([np.arange(hd + D * h, hd + D * h + D) for h in heads])
+    yk, mk = _project(X, W, b, rows_k)
+    yv, mv = _project(X, W, b, rows_k + hd)
+    rk, Ek = _step_and_near(yk, mk)
+    rv, Ev = _step_and_near(yv, mv)
+    shp = (w.B, w.N, len(heads), D)
+    assert np.array_equal(rk.reshape(shp), k_o) and np.array_equal(rv.reshape(shp), v_o)
+    _check_state(S, z, k_o, v_o, Ek.reshape(shp), Ev.reshape(shp), theta, True,
+                 "480p sampled heads", heads=heads)
