@@ -866,6 +866,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--soak", type=float, default=1.0)
+    ap.add_argument("--ref-budget", type=float, default=150.0,
+                    help="seconds of oracle work for --impl reference (warm-up and steps)")
     ap.add_argument("--op", choices=["layer", "backward", "causal", "tconv", "qkv"],
                     default="layer")
     args = ap.parse_args()
@@ -1006,7 +1008,7 @@ def main_reference(args, w, rank, world):
     """The float64 oracle, timed as it stands on the host's cores."""
     if rank != 0:
         return
-    budget = 150.0  # seconds for warm-up + timed steps together
+    budget = float(getattr(args, "ref_budget", 150.0))  # seconds: warm-up + timed steps
     per = budget / (args.steps + args.warmup)
     if args.op in ("tconv", "qkv"):
         sampler_fn = oracle_sample_tconv if args.op == "tconv" else oracle_sample_qkv

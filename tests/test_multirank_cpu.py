@@ -65,3 +65,21 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     w = bench.wl.WORKLOADS["sana0.6b_512px"]
     bench.main_reference(args, w, rank=1, world=2)
     assert capsys.readouterr().out == ""
+
+
+@pytest.mark.parametrize("op", ["layer", "qkv"])
+def test_reference_arm_prints_one_contract_line(capsys, op):
+    import argparse
+    import json
+    args = argparse.Namespace(steps=1, warmup=3, op=op, ref_budget=2.0)
+    w = bench.wl.WORKLOADS["sana0.6b_512px"]
+    bench.main_reference(args, w, rank=0, world=1)
+    lines = capsys.readouterr().out.strip().splitlines()
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["metric"] == bench.METRICS[op]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
