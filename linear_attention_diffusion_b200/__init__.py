@@ -323,7 +323,11 @@ def qkv_state(X, W, bias=None, rope_grid=None, t_offset: int = 0, rope_base: flo
     X [B, N, C] and W [3 H 32, C] bf16 CUDA tensors."""
     import torch
     B, N, C = X.shape
+    if W.dim() != 2 or W.shape[1] != C or W.shape[0] % (3 * HEAD_DIM) != 0:
+        raise ValueError(f"W must be [3*H*{HEAD_DIM}, C={C}], got {tuple(W.shape)}")
     H = W.shape[0] // (3 * HEAD_DIM)
+    if bias is not None and tuple(bias.shape) != (W.shape[0],):
+        raise ValueError(f"bias must be [{W.shape[0]}], got {tuple(bias.shape)}")
     if rope_grid is None:
         shape = make_shape(B, N, H, HEAD_DIM, "bf16", False)
     else:

@@ -167,3 +167,15 @@ def test_qkv_state_host_checks():
     # nothing to do: no pointer needed
     assert _call("la_qkv_state", ref(la.make_shape(0, 300, 6)), C, None, None, None, None, None,
                  None, None, 0, None) == la.LA_OK
+
+
+def test_qkv_state_wrapper_checks_shapes():
+    import torch
+    X = torch.zeros((1, 4, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        la.qkv_state(X, torch.zeros((95, 64), dtype=torch.bfloat16))   # rows not 3*H*32
+    with pytest.raises(ValueError):
+        la.qkv_state(X, torch.zeros((96, 32), dtype=torch.bfloat16))   # C mismatch
+    with pytest.raises(ValueError):
+        la.qkv_state(X, torch.zeros((96, 64), dtype=torch.bfloat16),
+                     torch.zeros((95,), dtype=torch.bfloat16))
