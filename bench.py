@@ -2,12 +2,15 @@
 """Benchmark of one ReLU linear-attention layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl la|reference]
-                    [--workload NAME] [--op layer|backward|causal|tconv]
+                    [--workload NAME] [--op layer|reduce|apply|backward|causal|tconv|qkv]
 
 A step is one pass of the layer's hot path over one batch of synthetic input:
 the state reduce (S = sum phi(K)^T V, z = sum ReLU(K)) and the apply
-(O = phi(Q) S / (ReLU(Q).z + eps)) of the default workload, or a whole
-block-causal video (reset, 12 blocks x 5 calls) for the LongSANA workload.
+(O = phi(Q) S / (ReLU(Q).z + eps)) of the default workload (the SANA-Video
+480p layer, the largest single-layer call), or a whole block-causal video
+(reset, 12 blocks x 5 calls) for the LongSANA workload. With --op reduce or
+--op apply a step is one of the two halves alone (la_state_reduce, la_apply),
+each its own kernel launch.
 With --op backward a step is the layer's backward instead (dQ, dK, dV and the
 state gradients from Q, K, V, the state and dO); with --op causal it is
 token-causal attention over the workload's tokens (query n sees keys 0..n).
@@ -50,17 +53,22 @@ METRIC_CAUSAL = ("token-causal linear-attn tokens/s per layer at 1 B200; "
 METRIC_TCONV = "temporal-conv tokens/s per layer at 1 B200; achieved HBM GB/s vs peak"
 METRIC_QKV = ("QKV projection + state reduce tokens/s per layer at 1 B200; "
               "achieved TFLOP/s vs bf16 peak")
+METRIC_REDUCE = "linear-attn state-reduce tokens/s per layer at 1 B200; achieved HBM GB/s vs peak"
+METRIC_APPLY = "linear-attn apply tokens/s per layer at 1 B200; achieved HBM GB/s vs peak"
 METRICS = {"layer": METRIC, "backward": METRIC_BWD, "causal": METRIC_CAUSAL,
-           "tconv": METRIC_TCONV, "qkv": METRIC_QKV}
+           "tconv": METRIC_TCONV, "qkv": METRIC_QKV, "reduce": METRIC_REDUCE,
+           "apply": METRIC_APPLY}
 # Channels of the temporal convolution: the FFN width of Sana-1.6B, which
 # SANA-Video starts from (width 2240, FFN 5600).
 FFN_WIDTH = 5600
 OP_CONFIG = {"layer": {}, "backward": {"op": "backward (dQ, dK, dV, dS, dz)"},
+             "reduce": {"op": "state reduce alone (S = sum phi(K)^T V, z = sum ReLU(K))"},
+             "apply": {"op": "apply alone (O = phi(Q) S / (ReLU(Q).z + eps))"},
              "causal": {"op": "token-causal (query n sees keys 0..n), no carry"},
              "tconv": {"op": "temporal depth-wise conv 3x1x1 + shortcut", "channels": FFN_WIDTH},
              "qkv": {"op": "QKV projection (bf16 GEMM, bias) fused with the state reduce; "
                            "Q out, K and V never leave the chip"}}
-DEFAULT_WORKLOAD = "sana1.6b_1024px"
+DEFAULT_WORKLOAD = "sanavideo_480p"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 D = 32
@@ -105,7 +113,10 @@ def layer_bytes(w, io_bytes=2):
     state = w.B * w.H * (D * D + D) * 4
     # backward: read Q, K, V, dO and (S, z); write dQ, dK, dV and (dS, dz).
     # causal: the minimum, Q, K, V read once and O written once.
+    # reduce: read K, V, write the state; apply: read Q and the state, write O.
     return {"attention_layer": 4 * th * D * io_bytes + state,
+            "state_reduce": 2 * th * D * io_bytes + state,
+            "apply": 2 * th * D * io_bytes + state,
             "attention_backward": 7 * th * D * io_bytes + 2 * state,
             "causal_attention": 4 * th * D * io_bytes}
 
@@ -126,6 +137,8 @@ def peaks():
 _DEVICE_HEADERS = ("la_common.cuh", "la_sm100.cuh", "la_tc_common.cuh")
 KERNEL_SOURCES = {
     "attention_layer": ("la_tc.cu",) + _DEVICE_HEADERS,
+    "state_reduce": ("la_tc.cu",) + _DEVICE_HEADERS,
+    "apply": ("la_tc.cu",) + _DEVICE_HEADERS,
     "attention_backward": ("la_backward_tc.cu",) + _DEVICE_HEADERS,
     "causal_attention": ("la_tc.cu", "la_causal_tc.cu") + _DEVICE_HEADERS,
     "temporal_conv": ("la_conv.cu",) + _DEVICE_HEADERS,
@@ -253,10 +266,15 @@ def oracle_sample(w, seconds, max_reps=None, op="layer"):
     import oracle as orc
 
     dOa = wl.make_tensor((w.B, w.N, w.H, w.D), 3) if op == "backward" else None
+    states = {}  # apply: the state of the sampled heads, reduced once, untimed
 
     def run(h_sub, Q, K, V, th):
         if op == "backward":
             orc.backward(Q, K, V, dOa[:, :, :h_sub], w.eps, th)
+        elif op == "reduce":
+            orc.state_reduce(K, V, th)
+        elif op == "apply":
+            orc.apply(Q, *states[h_sub], w.eps, th)
         elif op == "causal":
             orc.causal_attention(Q, K, V, w.eps, th)
         elif w.block_causal:
@@ -269,11 +287,15 @@ def oracle_sample(w, seconds, max_reps=None, op="layer"):
     th = orc.rope_angles(w.T, w.Hh, w.W, 0, w.rope_base) if w.rope else None
     Qa, Ka, Va = wl.make_qkv(w, 0)
     h_sub = min(w.H, 2)
+    if op == "apply":
+        states[h_sub] = orc.state_reduce(Ka[:, :, :h_sub], Va[:, :, :h_sub], th)
     t = time.perf_counter()
     run(h_sub, Qa[:, :, :h_sub], Ka[:, :, :h_sub], Va[:, :, :h_sub], th)
     per_head = (time.perf_counter() - t) / h_sub
     h_sub = max(1, min(w.H, int((seconds / 3) / max(per_head, 1e-9))))
     Q, K, V = (x[:, :, :h_sub].contiguous() for x in (Qa, Ka, Va))
+    if op == "apply":
+        states[h_sub] = orc.state_reduce(K, V, th)
     reps, t0 = 0, time.perf_counter()
     while True:
         run(h_sub, Q, K, V, th)
@@ -290,7 +312,8 @@ def oracle_sample(w, seconds, max_reps=None, op="layer"):
                 f"{reps} calls in {el:.1f} s, scaled to {w.H} heads x {calls} calls per video")
     else:
         tokens_per_s = w.B * w.N / full_call
-        what = {"backward": "backward", "causal": "causal_attention"}.get(op, "attention")
+        what = {"backward": "backward", "causal": "causal_attention", "reduce": "state_reduce",
+                "apply": "apply"}.get(op, "attention")
         desc = (f"oracle {what} on {h_sub} of {w.H} heads (B={w.B}, N={w.N}), {reps} calls "
                 f"in {el:.1f} s, scaled to {w.H} heads")
     return tokens_per_s, desc, cpu_cores_used(), per_call, h_sub
@@ -398,6 +421,9 @@ def run_la(args, w, rank, world, local_rank):
     bwd = args.op == "backward"
     per_set = (4 if bwd else 3) * w.B * w.N * w.H * D * 2
     n_sets = max(1, min(8, math.ceil(2 * L2_BYTES / per_set)))
+    if args.op in ("reduce", "apply"):
+        # a step touches two of the set's tensors: rotate over at least two sets
+        n_sets = max(2, min(8, math.ceil(2 * L2_BYTES / (per_set * 2 // 3))))
     if w.block_causal:
         n_sets = 5  # one set per call of a block; each set is far above L2
     sets = []
@@ -435,7 +461,26 @@ def run_la(args, w, rank, world, local_rank):
     shapes = [ctypes.byref(s) for s in keep]
     status = []
 
-    if args.op == "causal":
+    if args.op in ("reduce", "apply"):
+        launches_per_step = 1
+        if args.op == "apply":
+            # the state the apply reads: the reduce of the first set (untimed)
+            q0, k0, v0, _ = ptrs[0]
+            status.append(lib.la_state_reduce(shapes[0], k0, v0, S_p, z_p, ws_p, ws_n, sp))
+            torch.cuda.synchronize(dev)
+
+        def step(i, evs=None):
+            q, k, v, o = ptrs[i % n_sets]
+            if evs is not None:
+                evs[0].record(stream)
+            if args.op == "reduce":
+                status.append(lib.la_state_reduce(shapes[0], k, v, S_p, z_p, ws_p, ws_n, sp))
+            else:
+                status.append(lib.la_apply(shapes[0], q, S_p, z_p, o, sp))
+            if evs is not None:
+                evs[1].record(stream)
+        kernel_names = ("state_reduce" if args.op == "reduce" else "apply",)
+    elif args.op == "causal":
         launches_per_step = 2  # split states, then the causal pass
 
         def step(i, evs=None):
@@ -508,6 +553,8 @@ def run_la(args, w, rank, world, local_rank):
         e2e = run_e2e_backward(args, w, dev, stream, la, rank)
     elif args.op == "causal":
         e2e = run_e2e(args, w, dev, stream, la, rank, causal=True)
+    elif args.op in ("reduce", "apply"):
+        e2e = run_e2e_half(args, w, dev, stream, la, rank, args.op)
     else:
         e2e = run_e2e(args, w, dev, stream, la, rank)
     clocks = sampler.summary(t0, t1)
@@ -767,6 +814,41 @@ def e2e_pipelined(dev, compute, host_in, host_out, call, passes_per_step, steps)
     return start.elapsed_time(end) / steps
 
 
+def run_e2e_half(args, w, dev, stream, la, rank, op):
+    """The reduce or the apply alone through la_state_reduce / la_apply: the
+    reduce copies K, V in and S, z out; the apply copies Q, S, z in and O out
+    (pipelined over three streams, e2e_pipelined)."""
+    import torch
+    steps = max(1, min(args.steps, args.e2e_steps))
+    q, k, v = wl.make_qkv(w, 1000 * rank + 7)
+    shape = la.make_shape(w.B, w.N, w.H, D, "bf16", w.rope, w.T, w.Hh, w.W, 0, w.rope_base,
+                          w.eps)
+    ws = la.workspace(shape, dev)
+    S = torch.zeros((w.B, w.H, D, D), device=dev)
+    z = torch.zeros((w.B, w.H, D), device=dev)
+    la.la_state_reduce(shape, k.to(dev), v.to(dev), S, z, ws, stream)
+    torch.cuda.synchronize(dev)
+    hS, hz = S.cpu().pin_memory(), z.cpu().pin_memory()
+    if op == "reduce":
+        hin = [x.pin_memory() for x in (k, v)]
+        hout = [torch.empty_like(hS).pin_memory(), torch.empty_like(hz).pin_memory()]
+
+        def call(p, ins, outs, st):
+            la.la_state_reduce(shape, ins[0], ins[1], outs[0], outs[1], ws, st)
+    else:
+        hin = [q.pin_memory(), hS, hz]
+        hout = [torch.empty_like(hin[0]).pin_memory()]
+
+        def call(p, ins, outs, st):
+            la.la_apply(shape, ins[0], ins[1], ins[2], outs[0], st)
+
+    ms = e2e_pipelined(dev, stream, hin, hout, call, 1, steps)
+    nb = lambda ts: sum(t.numel() * t.element_size() for t in ts)
+    return {"ms_per_step": ms, "tokens_per_step": w.B * w.N, "steps": steps,
+            "h2d_bytes_per_step": nb(hin), "d2h_bytes_per_step": nb(hout),
+            "copies": "pipelined: copy-in, calls and copy-out on three streams, two buffer sets"}
+
+
 def run_e2e(args, w, dev, stream, la, rank, causal=False):
     """Same metric through la_attention / la_block_causal_step /
     la_causal_attention, every call copying its Q, K, V in from pinned host
@@ -868,11 +950,12 @@ def main():
     ap.add_argument("--soak", type=float, default=1.0)
     ap.add_argument("--ref-budget", type=float, default=150.0,
                     help="seconds of oracle work for --impl reference (warm-up and steps)")
-    ap.add_argument("--op", choices=["layer", "backward", "causal", "tconv", "qkv"],
+    ap.add_argument("--op", choices=["layer", "reduce", "apply", "backward", "causal", "tconv",
+                                     "qkv"],
                     default="layer")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
-    if args.op in ("backward", "causal", "qkv") and w.block_causal:
+    if args.op in ("backward", "causal", "qkv", "reduce", "apply") and w.block_causal:
         ap.error(f"--op {args.op} covers the non-causal workloads")
     if args.op == "tconv" and not w.rope:
         ap.error("--op tconv needs a video workload (sanavideo_480p, longsana_block_causal)")
@@ -979,6 +1062,8 @@ def main():
         "d2h_bytes_per_step": e["d2h_bytes_per_step"], "steps": e["steps"],
         "ms_per_step": round(e["ms_per_step"], 4), "copies": e.get("copies"),
         "api": ("la_attention_backward" if args.op == "backward" else
+                "la_state_reduce" if args.op == "reduce" else
+                "la_apply" if args.op == "apply" else
                 "la_causal_attention" if args.op == "causal" else
                 "la_temporal_conv" if args.op == "tconv" else
                 "la_qkv_state" if args.op == "qkv" else
@@ -1033,10 +1118,15 @@ def main_reference(args, w, rank, world):
     Q, K, V = (x[:, :, :h_sub].contiguous() for x in wl.make_qkv(w, 0))
     bwd = args.op == "backward"
     dO = wl.make_tensor((w.B, w.N, w.H, w.D), 3)[:, :, :h_sub].contiguous() if bwd else None
+    S0, z0 = orc.state_reduce(K, V, th) if args.op == "apply" else (None, None)
 
     def call():
         if bwd:
             orc.backward(Q, K, V, dO, w.eps, th)
+        elif args.op == "reduce":
+            orc.state_reduce(K, V, th)
+        elif args.op == "apply":
+            orc.apply(Q, S0, z0, w.eps, th)
         elif args.op == "causal":
             orc.causal_attention(Q, K, V, w.eps, th)
         elif w.block_causal:
@@ -1062,7 +1152,8 @@ def main_reference(args, w, rank, world):
     else:
         value = w.B * w.N / full_call
         ms_step = full_call * 1e3
-        what = {"backward": "backward", "causal": "causal_attention"}.get(args.op, "attention")
+        what = {"backward": "backward", "causal": "causal_attention", "reduce": "state_reduce",
+                "apply": "apply"}.get(args.op, "attention")
         sample = f"each step: oracle {what} on {h_sub} of {w.H} heads; scaled to {w.H} heads"
     out = {"impl": "reference", "metric": METRICS[args.op], "value": value, "unit": "tokens/s",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,

@@ -39,7 +39,12 @@
  *     e) and z is float32 [B, H, D].
  *   - Memory: every tensor pointer is a DEVICE pointer owned by the caller,
  *     16-byte aligned. The library allocates nothing and keeps no state
- *     between calls. Scratch memory ("workspace") is passed in by the
+ *     between calls, with one exception: la_state_reduce_static keeps its
+ *     scratch in a fixed 8 MiB device array that the library holds on every
+ *     GPU it is loaded on (plus a host-side cache of that array's address per
+ *     device and context); its calls on one GPU share the array and must be
+ *     ordered when they could overlap. Scratch memory ("workspace") for
+ *     every other entry point is passed in by the
  *     caller; its size comes from la_workspace_bytes(). A workspace must be
  *     zero-filled once before its first use (cudaMemsetAsync(ws, 0, bytes));
  *     every call leaves it zero-filled where it matters again, so it is
@@ -186,7 +191,9 @@ la_status la_attention_backward(const la_shape* shape, const void* Q,
  * for la_attention (same size). Two launches: the state reduce leaves each
  * token split's partial state in the workspace; the causal kernel starts
  * each split from the carry plus the earlier splits (summed in split order)
- * and walks its tokens in chunks of 32 on CUDA cores. Deterministic. */
+ * and walks its tokens chunk by chunk: 128-token chunks on the tensor cores
+ * (tcgen05) for bf16 I/O without RoPE, 32-token chunks on CUDA cores with
+ * RoPE or float32 I/O. Deterministic. */
 la_status la_causal_attention(const la_shape* shape, const void* Q,
                               const void* K, const void* V, float* S_carry,
                               float* z_carry, void* O, int update, void* ws,
@@ -266,8 +273,10 @@ la_status la_state_reset(float* S, float* z, int B, int H, int D,
  * counters it needs (cudaMemsetAsync on `stream`) before the kernel.
  * All calls on one GPU share the array: calls whose kernels may overlap on
  * the GPU (different streams or host threads) race and must be ordered.
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
+ * The array's device address is looked up (cudaGetSymbolAddress) by the
+ * first call in each CUDA context, with that context's device current, and
+ * cached under the context's unique id, so a context created again after
+ * cudaDeviceReset gets a fresh lookup; make the first call on each device
  * before any stream capture. */
 la_status la_state_reduce_static(const la_shape* shape, const void* K,
                                  const void* V, float* S, float* z,

@@ -15,42 +15,94 @@
 // share it. Calls whose kernels may run at the same time on one GPU (other
 // streams, other host threads) race on the array and must be ordered by the
 // caller.
-#include <mutex>
+#include <cuda.h>
 
 #include "la_internal.h"
+#include "la_scratch_cache.h"
 
 namespace la {
 namespace {
 
-// 8 MiB: enough for B*H*splits*(32*32+32) floats of every workload this
-// library targets (at most 4.7 MB: 70 heads x 16 splits, or 4 x 70 heads x
-// 4 splits) plus the counters.
+// 8 MiB. The scratch of a shape is a 256-aligned block of B*H arrival
+// counters followed by B*H*splits partial states of (32*32 + 32) floats. The
+// split rule gives one split per head group whenever B*ceil(H/4) > 74, and
+// more splits only for smaller shapes (B*H <= 296), so a shape fits exactly
+// when B*H <= 1984. The bench workloads need 2.4 MB: 70 heads x 8 splits for
+// the 4K and video layers (B = 1), 4 x 70 heads x 2 splits for the 1024px
+// layer.
 constexpr size_t kStaticScratchBytes = size_t(8) << 20;
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+SymbolAddressCache<kMaxDevices> g_scratch_cache;
 
-// Device address of g_static_scratch on the current device, looked up once per
-// device. In host code the array's name only stands for the symbol; the
-// address a kernel may use comes from cudaGetSymbolAddress.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+std::once_flag g_ctx_fn_once;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+bool load_ctx_functions() {
+  std::call_once(g_ctx_fn_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(fn);
+  });
+  return g_ctx_get_current != nullptr && g_ctx_get_id != nullptr;
+}
+
+// Unique id of the context current on this thread; 0 when there is none yet.
+cudaError_t current_context_id(unsigned long long* id) {
+  *id = 0;
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
+  if (ctx == nullptr) return cudaSuccess;
+  return g_ctx_get_id(ctx, id) == CUDA_SUCCESS ? cudaSuccess : cudaErrorUnknown;
+}
+
+// Device address of g_static_scratch in the current device's context. In
+// host code the array's name only stands for the symbol; the address a kernel
+// may use comes from cudaGetSymbolAddress, called with the device current.
+// The result is cached per device and keyed on the context id, so a context
+// that was destroyed and created again (its module reloaded, the array
+// possibly elsewhere) gets a fresh lookup instead of a stale address.
 la_status scratch_address(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return detail::cuda_fail(e, "la_state_reduce_static: cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices)
     return detail::fail(LA_ERR_UNSUPPORTED, "la_state_reduce_static: device %d", dev);
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (!load_ctx_functions())
+    return detail::fail(LA_ERR_CUDA, "la_state_reduce_static: cuCtxGetCurrent / cuCtxGetId "
+                                     "not available from the driver");
+  unsigned long long ctx_id = 0;
+  if ((e = current_context_id(&ctx_id)) != cudaSuccess)
+    return detail::cuda_fail(e, "la_state_reduce_static: current context");
+  if (ctx_id == 0) {
+    // No context is current on this thread yet: the symbol lookup creates
+    // the device's primary context and makes it current; key on that one.
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_static_scratch);
-    if (e != cudaSuccess || ptr == nullptr)
-      return detail::cuda_fail(e, "la_state_reduce_static: cudaGetSymbolAddress");
-    g_scratch_addr[dev] = ptr;
+    if (e != cudaSuccess) return detail::cuda_fail(e, "la_state_reduce_static: cudaGetSymbolAddress");
+    if ((e = current_context_id(&ctx_id)) != cudaSuccess || ctx_id == 0)
+      return detail::cuda_fail(e == cudaSuccess ? cudaErrorDeviceUninitialized : e,
+                               "la_state_reduce_static: current context");
   }
-  *out = g_scratch_addr[dev];
+  cudaError_t lookup = cudaSuccess;
+  const int rc = g_scratch_cache.get(dev, ctx_id, [&lookup](void** addr) {
+    lookup = cudaGetSymbolAddress(addr, g_static_scratch);
+    return (lookup == cudaSuccess && *addr != nullptr) ? 0 : 1;
+  }, out);
+  if (rc != 0)
+    return detail::cuda_fail(lookup == cudaSuccess ? cudaErrorInvalidSymbol : lookup,
+                             "la_state_reduce_static: cudaGetSymbolAddress");
   return LA_OK;
 }
 

@@ -9,6 +9,11 @@ It checks the new entry point, called through the C ABI, against
 la_state_reduce with a workspace, on two calls in a row (the second call
 reuses the array the first one left behind), within the tolerance the parity
 tests use, and checks that an oversized shape is refused before any launch.
+The static-scratch result is also checked against the float64 oracle's state,
+with the bound of the parity tests, so the comparison is not only CUDA against
+CUDA. Small ragged shapes (tokens and heads that fill no whole tile or head
+group), float32 I/O (the CUDA-core reduce) and the empty sequence go through
+the same array and are compared bitwise with the workspace path.
 """
 import ctypes
 
@@ -62,10 +67,37 @@ def test_static_scratch_matches_workspace_reduce_twice(cuda_device, name, rope):
                       A, tol_s, what=f"{name} call {call}")
         # same kernel, same split order: the two are in fact identical
         assert torch.equal(S_st, S_ws) and torch.equal(z_st, z_ws)
+        # and the static-scratch state against the float64 oracle
+        S_ref, z_ref = orc.state_reduce(K, V, th)
+        P.check_state(S_st.cpu(), z_st.cpu(), S_ref, z_ref, A, tol_s,
+                      what=f"{name} call {call} vs oracle")
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+@pytest.mark.parametrize("B,N,H", [(2, 300, 5), (1, 1, 1), (2, 0, 3)])
+def test_static_scratch_small_shapes_bitwise_twice(cuda_device, io, B, N, H):
+    dtype = torch.bfloat16 if io == "bf16" else torch.float32
+    w_shape = (B, N, H, D)
+    for call, seed in enumerate((21, 22)):  # two calls in a row, different inputs
+        K = wl.make_tensor(w_shape, seed, dtype)
+        V = wl.make_tensor(w_shape, seed + 1, dtype)
+        Kd, Vd = P.to_dev(K, V)
+        shape = la.shape_for(Kd)
+        S_ws, z_ws = _reduce_with_workspace(shape, Kd, Vd)
+        S_st, z_st = _reduce_static(shape, Kd, Vd)
+        torch.cuda.synchronize()
+        assert torch.equal(S_st, S_ws) and torch.equal(z_st, z_ws), f"{io} {B}x{N}x{H} call {call}"
+        S_ref, z_ref = orc.state_reduce(K, V, None)
+        tol_s, _ = P.tolerances(io, False)
+        P.check_state(S_st.cpu(), z_st.cpu(), S_ref, z_ref, P.magnitude_state(K, V, None), tol_s,
+                      what=f"{io} {B}x{N}x{H} call {call} vs oracle")
 
 
 def test_static_scratch_refuses_oversized_shapes(cuda_device):
-    # 64 splits x 4096 heads of partial states do not fit the 8 MiB array.
+    # B*H = 4096 heads get one split each (B*ceil(H/4) = 1024 head groups is
+    # more than a wave), so the scratch is 4096 partial states of 4224 bytes
+    # plus the counters, 17.3 MB: more than the 8 MiB array (which holds any
+    # shape with B*H <= 1984).
     shape = la.make_shape(16, 1 << 16, 256)
     st = la._lib.la_state_reduce_static(ctypes.byref(shape), 1 << 20, 1 << 20, 1 << 36,
                                         1 << 37, None)
