@@ -44,40 +44,83 @@ using namespace sm100;
 
 // ============================================================ the kernel
 
-// One kernel template serves three launches: the state reduce alone, the
+// One kernel template serves four launches: the state reduce alone, the
 // apply alone, and the fused layer (reduce, a per-head-group hand-off, then
-// apply). All share one TMA stage ring: a ring position p uses stage p % 5
-// with phase parity (p / 5) & 1, whichever operation the tile belongs to.
-enum Phases : int { kReduceOnly = 1, kApplyOnly = 2, kFusedLayer = 3 };
+// apply) in two forms: the head group's CTAs as one thread-block cluster that
+// hands the split partials over through distributed shared memory
+// (kClusterLayer), or a cooperative grid that hands them over through global
+// memory (kFusedLayer). All share one TMA stage ring of kNS stages (six; five
+// in the cluster layer): a ring position p uses stage p % kNS with phase
+// parity (p / kNS) & 1, whichever operation the tile belongs to.
+enum Phases : int { kReduceOnly = 1, kApplyOnly = 2, kFusedLayer = 3, kClusterLayer = 7 };
+
+// Largest cluster of the cluster layer: the portable limit.
+constexpr int kMaxCluster = 8;
 
 constexpr int kMath = 512;                   // 16 math warps (warps 2..17)
 constexpr int kThreadsTc = 64 + kMath;       // + TMA warp + MMA warp
-constexpr int kApWG = kMath / 128;           // apply: 4 warpgroups, one tile each in turn
-constexpr int kStages = 5;
+constexpr int kApWG = kMath / 128;           // apply: at most 4 warpgroups, one tile each in turn
 constexpr int kStageBytes = 32768;
 constexpr int kRedT = 64;                    // reduce: tokens per stage (K and V, 4 heads)
 constexpr int kRedBox = kRedT * 128;         // [64 tokens][64 dims] bf16
 constexpr int kApT = 128;                    // apply: tokens per tile (Q, 4 heads)
 constexpr int kApBox = kApT * 128;           // [128 tokens][64 dims] bf16
-constexpr int kTmemCols = 512;               // reduce: cols [0,128); apply: kApWG x 128
+constexpr int kTmemCols = 512;               // reduce: cols [0,128); apply: one block per warpgroup
+
+// The apply with and without RoPE. Without RoPE the denominators ReLU(q).z
+// come from the tensor core too (an MMA against z, split into two bf16
+// parts), so the transform of a Q tile is ReLU alone; the warpgroup's TMEM
+// block then holds 4 x 32 numerator and 16 denominator columns, and three
+// warpgroups fit the 512 columns. With RoPE the numerator needs the rotated
+// phi(q) and the denominator the unrotated ReLU(q): the denominators are
+// formed on the CUDA cores during the transform, and four warpgroups take
+// tiles.
+template <int kRope>
+struct ApplyCfg {
+  static constexpr bool kDenMma = kRope == kNoRope;
+  static constexpr int kWG = kDenMma ? 3 : 4;            // warpgroups taking tiles
+  static constexpr int kCols = kDenMma ? 160 : 128;      // TMEM columns per warpgroup
+  static constexpr int kDenCol = 128;                    // first denominator column
+};
 
 // named barriers: 0 = whole CTA, 1 = all math threads, 2.. = apply warpgroups
 constexpr int kBarMath = 1;
 constexpr int kBarWG0 = 2;
 
-struct Smem {  // byte offsets from the 1024-aligned base
+// Shared-memory layout (byte offsets from the 1024-aligned base) for kNS
+// stages of the ring; the RoPE table only with RoPE, the denominator operand
+// only without, the partial-state buffer only in the cluster layer.
+template <int kNS, bool kWithPart, bool kWithRope>
+struct SmemLayout {
   static constexpr int stages = 0;
-  static constexpr int zred = stages + kStages * kStageBytes;  // [512][8] f32; then S scratch
-  static constexpr int bop = zred + kMath * 8 * 4;             // [2 pairs][32 rows][128 B]
-  static constexpr int zs = bop + 2 * 32 * 128;                // [4][32] f32
-  static constexpr int rope = zs + kGroupHeads * kD * 4;       // float2[kRopeTableMax]
-  static constexpr int bars = rope + kRopeTableMax * 8;
-  // full[5] empty[5] ready_a[5] ready_b[5] t_full[4] t_empty[4] acc_full mma_done b_ready
-  static constexpr int nbars = 4 * kStages + 2 * kApWG + 3;
+  // [16 warps][16] f32 key sums of the reduce; then the state S [4][32][32]
+  // f32 that the apply uses
+  static constexpr int zred = stages + kNS * kStageBytes;
+  static constexpr int bop = zred + kGroupHeads * kD * kD * 4;  // [2 pairs][32 rows][128 B]
+  // the apply's denominator operand: [2 boxes][16 rows][128 B] bf16, rows
+  // 0-3 the heads' z (upper bf16 part), rows 4-7 the remainders
+  static constexpr int zop = bop + 2 * 32 * 128;
+  static constexpr int zs = zop + (kWithRope ? 0 : 2 * 16 * 128);  // [4][32] f32
+  static constexpr int rope = zs + kGroupHeads * kD * 4;          // float2[kRopeTableMax]
+  // cluster layer: this CTA's partial state, [4 heads][32*32 + 32] f32
+  static constexpr int part = rope + (kWithRope ? kRopeTableMax * 8 : 0);
+  static constexpr int bars = part + (kWithPart ? kGroupHeads * kStateFloats * 4 : 0);
+  // full[kNS] empty[kNS] ready_a[kNS] ready_b[kNS] o_full[kNS] t_full[4]
+  // t_empty[4] acc_full mma_done b_ready part_full done s_full
+  static constexpr int nbars = 5 * kNS + 2 * kApWG + 6;
   static constexpr int misc = bars + nbars * 8;                // tmem base, abort, last flag
   static constexpr int bytes = misc + 16;
 };
-constexpr int kSmemBytes = Smem::bytes + 1024;
+
+// Six stages of the ring in every launch but the cluster layer, whose
+// partial-state buffer leaves room for five.
+template <int kRope, int kPh>
+struct LayerCfg {
+  static constexpr int kNS = kPh == kClusterLayer ? 5 : 6;
+  using Smem = SmemLayout<kNS, kPh == kClusterLayer, kRope != kNoRope>;
+  static constexpr int kSmemBytes = Smem::bytes + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+};
 
 struct LayerArgs {
   float* partials;     // [B*H][splits][kStateFloats]
@@ -98,18 +141,28 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
          const Problem p, const RopeTable rt, const LayerArgs a) {
   constexpr bool kRed = (kPh & kReduceOnly) != 0;
   constexpr bool kApp = (kPh & kApplyOnly) != 0;
+  constexpr bool kCl = kPh == kClusterLayer;
+  constexpr int kNS = LayerCfg<kRope, kPh>::kNS;
+  using Smem = typename LayerCfg<kRope, kPh>::Smem;
+  using AC = ApplyCfg<kRope>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Smem::bars);
-  uint64_t* empty = full + kStages;
-  uint64_t* ready_a = empty + kStages;  // reduce stage transformed: 512 arrivals
-  uint64_t* ready_b = ready_a + kStages; // apply tile transformed: 128 arrivals
-  uint64_t* t_full = ready_b + kStages;  // [kApWG]
+  uint64_t* empty = full + kNS;
+  uint64_t* ready_a = empty + kNS;  // reduce stage transformed: 512 arrivals
+  uint64_t* ready_b = ready_a + kNS; // apply tile transformed: 128 arrivals
+  uint64_t* o_full = ready_b + kNS;  // apply tile's O in the stage: 1 arrival
+  uint64_t* t_full = o_full + kNS;   // [kApWG]
   uint64_t* t_empty = t_full + kApWG;   // [kApWG]
   uint64_t* acc_full = t_empty + kApWG;
   uint64_t* mma_done = acc_full + 1;
   uint64_t* b_ready = mma_done + 1;
+  // cluster layer: every CTA's partial is in its shared memory / every CTA
+  // is done reading this one's memory and the carry
+  uint64_t* part_full = b_ready + 1;
+  uint64_t* done = part_full + 1;
+  uint64_t* s_full = done + 1;  // apply only: the state (S, z) copied in
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc + 4);
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + Smem::misc + 8);
@@ -131,11 +184,12 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
   const int nB = kApp ? max(0, min(ntiles_all, tile_begin + a.tiles_per_cta) - tile_begin) : 0;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kNS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&ready_a[s], kMath);
       mbar_init(&ready_b[s], 128);
+      mbar_init(&o_full[s], 1);
     }
     for (int w = 0; w < kApWG; ++w) {
       mbar_init(&t_full[w], 1);
@@ -144,6 +198,11 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
     mbar_init(b_ready, 1);
+    mbar_init(s_full, 1);
+    if (kCl) {  // one arrival from each CTA of the cluster
+      mbar_init(part_full, gridDim.x);
+      mbar_init(done, gridDim.x);
+    }
     *abort_flag = 0;
     *last_flag = 0;
     fence_mbar_init();
@@ -165,6 +224,9 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
   }
   if (kRope == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kMath);
   __syncthreads();
+  // cluster layer: every CTA's barriers are initialised before any other CTA
+  // may arrive on them
+  if (kCl) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(smem);
@@ -183,8 +245,8 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       int pos = 0;
       bool ok = true;
       for (int i = 0; ok && i < nA; ++i, ++pos) {
-        const int s = pos % kStages;
-        if (!(ok = mbar_wait(&empty[s], ((pos / kStages) & 1) ^ 1, abort_flag, &g_tc_error,
+        const int s = pos % kNS;
+        if (!(ok = mbar_wait(&empty[s], ((pos / kNS) & 1) ^ 1, abort_flag, &g_tc_error,
                              kErrWait)))
           break;
         mbar_arrive_expect_tx(&full[s], kStageBytes);
@@ -195,20 +257,69 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
         tma_load_3d(st + 2 * kRedBox, &tm_v, &full[s], h0 * 32, y, b);
         tma_load_3d(st + 3 * kRedBox, &tm_v, &full[s], h0 * 32 + 64, y, b);
       }
+      // Q tiles. A stage last used by an apply tile is handed back by this
+      // thread: once that tile's O is in the stage (o_full), it stores it
+      // with TMA, waits until the store has read the stage, releases the
+      // stage (empty: the warpgroups' phase guard waits on it) and reloads
+      // it. The warpgroups never wait for their stores.
+      auto store_tile = [&](int q) -> bool {  // q: apply tile index
+        const int qs = (nA + q) % kNS;
+        if (!mbar_wait(&o_full[qs], (q / kNS) & 1, abort_flag, &g_tc_error, kErrWait))
+          return false;
+        uint8_t* tile = smem + Smem::stages + qs * kStageBytes;
+        const int n0 = (tile_begin + q) * kApT;
+        tma_store_3d(&tm_o, tile, h0 * 32, n0, b);
+        tma_store_3d(&tm_o, tile + kApBox, h0 * 32 + 64, n0, b);
+        bulk_commit();
+        bulk_wait_read<0>();
+        mbar_arrive(&empty[qs]);
+        return true;
+      };
+      // apply only: the state (S, z) of the group's heads, one bulk copy
+      // each, issued ahead of the Q tiles so that it does not queue behind
+      // them; when Q may be read before the previous grid completes, after
+      // the first ring of Q tiles and the wait for that grid
+      const int sheads = kApp ? max(0, min(kGroupHeads, p.H - h0)) : 0;
+      bool state_issued = kPh != kApplyOnly;
+      auto issue_state = [&]() {
+        mbar_arrive_expect_tx(s_full, sheads * (kD * kD + kD) * 4);
+        if (sheads > 0) {
+          bulk_load(smem + Smem::zred, a.S_in + cidx * kD * kD, sheads * kD * kD * 4, s_full);
+          bulk_load(smem + Smem::zs, a.z_in + cidx * kD, sheads * kD * 4, s_full);
+        }
+        state_issued = true;
+      };
+      if (!state_issued && !early_q) issue_state();
+      int stored = 0;  // apply tiles whose O has been stored
       for (int i = 0; ok && i < nB; ++i, ++pos) {
-        const int s = pos % kStages;
-        if (!(ok = mbar_wait(&empty[s], ((pos / kStages) & 1) ^ 1, abort_flag, &g_tc_error,
-                             kErrWait)))
+        const int s = pos % kNS;
+        if (i >= kNS) {  // the stage's previous tile was apply tile i - kNS
+          if (!(ok = store_tile(i - kNS))) break;
+          ++stored;
+        } else if (!(ok = mbar_wait(&empty[s], ((pos / kNS) & 1) ^ 1, abort_flag, &g_tc_error,
+                                    kErrWait))) {
           break;
+        }
         mbar_arrive_expect_tx(&full[s], kStageBytes);
         uint8_t* st = smem + Smem::stages + s * kStageBytes;
         const int y = (tile_begin + i) * kApT;
         tma_load_3d(st, &tm_q, &full[s], h0 * 32, y, b);
         tma_load_3d(st + kApBox, &tm_q, &full[s], h0 * 32 + 64, y, b);
+        if (!state_issued && i + 1 == min(kNS, nB)) {
+          pdl_wait();
+          issue_state();
+        }
       }
-      // drain: every load issued must have landed before the CTA exits
-      for (int q = max(0, pos - kStages); q < pos; ++q)
-        mbar_drain(&full[q % kStages], (q / kStages) & 1, &g_tc_error, kErrWait);
+      if (!state_issued) {  // (only when the loop stopped early)
+        pdl_wait();
+        issue_state();
+      }
+      for (int q = stored; ok && q < nB; ++q) ok = store_tile(q);
+      // drain: every load issued must have landed, and every store completed,
+      // before the CTA exits
+      for (int q = max(0, pos - kNS); q < pos; ++q)
+        mbar_drain(&full[q % kNS], (q / kNS) & 1, &g_tc_error, kErrWait);
+      bulk_wait<0>();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
@@ -217,8 +328,8 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       bool ok = true;
       const uint32_t id_red = idesc_bf16_f32(128, 128, 1, 1);
       for (int i = 0; i < nA; ++i, ++pos) {
-        const int s = pos % kStages;
-        if (!(ok = mbar_wait(&ready_a[s], (i / kStages) & 1, abort_flag, &g_tc_error, kErrWait)))
+        const int s = pos % kNS;
+        if (!(ok = mbar_wait(&ready_a[s], (i / kNS) & 1, abort_flag, &g_tc_error, kErrWait)))
           break;
         tc_fence_after();
         const uint32_t st = sbase + Smem::stages + s * kStageBytes;
@@ -234,17 +345,20 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       if (kRed) mma_commit(acc_full);
       if (ok && kApp && nB > 0) ok = mbar_wait(b_ready, 0, abort_flag, &g_tc_error, kErrWait);
       const uint32_t id_ap = idesc_bf16_f32(128, 32, 0, 0);
+      const uint32_t id_den = idesc_bf16_f32(128, 16, 0, 0);
       const uint32_t bop = sbase + Smem::bop;
+      const uint32_t zop = sbase + Smem::zop;
       for (int j = 0; ok && j < nB; ++j, ++pos) {
-        const int s = pos % kStages;
-        const int w = j % kApWG;
-        if (!(ok = mbar_wait(&ready_b[s], (j / kStages) & 1, abort_flag, &g_tc_error, kErrWait)))
+        const int s = pos % kNS;
+        const int w = j % AC::kWG;
+        if (!(ok = mbar_wait(&ready_b[s], (j / kNS) & 1, abort_flag, &g_tc_error, kErrWait)))
           break;
-        if (!(ok = mbar_wait(&t_empty[w], ((j / kApWG) & 1) ^ 1, abort_flag, &g_tc_error,
+        if (!(ok = mbar_wait(&t_empty[w], ((j / AC::kWG) & 1) ^ 1, abort_flag, &g_tc_error,
                              kErrWait)))
           break;
         tc_fence_after();
         const uint32_t st = sbase + Smem::stages + s * kStageBytes;
+        const uint32_t acc = tmem + w * AC::kCols;
 #pragma unroll
         for (int hh = 0; hh < kGroupHeads; ++hh) {
           const uint32_t koff = (hh & 1) * 64;
@@ -252,7 +366,16 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
           for (int kk = 0; kk < 2; ++kk) {
             const uint64_t ad = smem_desc_sw128(st + (hh >> 1) * kApBox + koff + kk * 32, 16, 1024);
             const uint64_t bd = smem_desc_sw128(bop + (hh >> 1) * 4096 + koff + kk * 32, 16, 1024);
-            mma_bf16(tmem + w * 128 + hh * 32, ad, bd, id_ap, kk);
+            mma_bf16(acc + hh * 32, ad, bd, id_ap, kk);
+          }
+        }
+        if (AC::kDenMma) {
+          // the denominators: ReLU(Q) (all 128 dims) times the z operand
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t ad = smem_desc_sw128(st + (kk >> 2) * kApBox + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(zop + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
+            mma_bf16(acc + AC::kDenCol, ad, bd, id_den, kk > 0 ? 1u : 0u);
           }
         }
         mma_commit(&t_full[w]);
@@ -265,74 +388,98 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
     const int mt = tid - 64;
     bool alive = true;
     if (kRed) {
-      // feature map of K, key sum: thread mt owns 16-byte chunk column c of
-      // rows rg and rg + 32 of every stage
-      const int c = mt & 15, rg = mt >> 4;
-      const int box = c >> 3, cc = c & 7;
-      const int dpos = (cc & 3) * 8;  // first dim of the chunk inside its head
-      float2 zacc[4] = {};
+      // feature map of K, key sum. Math warp wi owns, in every 64-token
+      // stage, the rows 32 (wi >> 3) + lane of head (wi >> 1) & 3 of the
+      // group, dims [16 half, 16 half + 16) with half = wi & 1: two 16-byte
+      // chunks of one row per thread, so a warp reads 32 rows of one chunk
+      // column (conflict-free under the 128-byte swizzle) and which RoPE
+      // pairs a thread rotates is fixed per warp.
+      const int wi = mt >> 5;
+      const int half = wi & 1, hq = (wi >> 1) & 3;
+      const int rg = (wi >> 3) * 32 + lane;
+      const int cc0 = (hq & 1) * 4 + half * 2;  // first of the two chunks in the 128-byte row
+      float2 zacc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) zacc[e] = make_float2(0.0f, 0.0f);
       TokPos tp = {0, 0, 0};
       if (kRope != kNoRope) tp = token_pos(p.rope, n_begin + rg);
-      const int j0 = dpos / 2;
-      int sel[4], off[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        sel[q] = pair_axis(j0 + q);
-        off[q] = pair_off(j0 + q);
-      }
       for (int i = 0; i < nA; ++i) {
-        const int s = i % kStages;
-        if (!mbar_wait(&full[s], (i / kStages) & 1, abort_flag, &g_tc_error, kErrWait)) {
+        const int s = i % kNS;
+        if (!mbar_wait(&full[s], (i / kNS) & 1, abort_flag, &g_tc_error, kErrWait)) {
           alive = false;
           break;
         }
-        const uint32_t kb = sbase + Smem::stages + s * kStageBytes + box * kRedBox;
-        const int y0 = n_begin + i * kRedT;
+        const uint32_t kb = sbase + Smem::stages + s * kStageBytes + (hq >> 1) * kRedBox;
+        const uint32_t a0 = kb + sw128_offset(rg, cc0), a1 = kb + sw128_offset(rg, cc0 + 1);
+        uint4 u0 = ld_shared_v4(a0), u1 = ld_shared_v4(a1);
+        u0.x = relu_bf16x2(u0.x);
+        u0.y = relu_bf16x2(u0.y);
+        u0.z = relu_bf16x2(u0.z);
+        u0.w = relu_bf16x2(u0.w);
+        u1.x = relu_bf16x2(u1.x);
+        u1.y = relu_bf16x2(u1.y);
+        u1.z = relu_bf16x2(u1.z);
+        u1.w = relu_bf16x2(u1.w);
+        float x[16];
+        {
+          float xa[8], xb[8];
+          unpack8(u0, xa);
+          unpack8(u1, xb);
 #pragma unroll
-        for (int k = 0; k < kRedT / 32; ++k) {
-          const int r = rg + 32 * k;
-          const uint32_t addr = kb + sw128_offset(r, cc);
-          uint4 u = ld_shared_v4(addr);
-          u.x = relu_bf16x2(u.x);
-          u.y = relu_bf16x2(u.y);
-          u.z = relu_bf16x2(u.z);
-          u.w = relu_bf16x2(u.w);
-          float x[8];
-          unpack8(u, x);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            zacc[e] = __fadd2_rn(zacc[e], make_float2(x[2 * e], x[2 * e + 1]));
-          if (kRope != kNoRope) {
-            if (y0 + r < p.N) {
-              const RopeBases rb = rope_bases(p.rope, tp);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                float2 cs;
-                if (kRope == kRopeTable) {
-                  cs = rope_tab[(sel[q] == 0 ? rb.t : (sel[q] == 1 ? rb.h : rb.w)) + off[q]];
-                } else {
-                  const int pos = sel[q] == 0 ? p.rope.t_offset + tp.t : (sel[q] == 1 ? tp.h : tp.w);
-                  rope_cos_sin(pos, p.rope.inv_freq[j0 + q], cs.x, cs.y);
-                }
-                const float2 t = __fmul2_rn(make_float2(x[2 * q + 1], x[2 * q + 1]),
-                                            make_float2(-cs.y, cs.x));
-                const float2 y = __ffma2_rn(make_float2(x[2 * q], x[2 * q]), cs, t);
-                x[2 * q] = y.x;
-                x[2 * q + 1] = y.y;
-              }
-              u = pack8(x);
-            }
-            token_pos_advance(p.rope, tp, 32);
+          for (int e = 0; e < 8; ++e) {
+            x[e] = xa[e];
+            x[8 + e] = xb[e];
           }
-          st_shared_v4(addr, u);
         }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          zacc[e] = __fadd2_rn(zacc[e], make_float2(x[2 * e], x[2 * e + 1]));
+        if (kRope != kNoRope) {
+          if (n_begin + i * kRedT + rg < p.N) {
+            float2 cs[8];
+            if (kRope == kRopeTable) {
+              const RopeBases rb = rope_bases(p.rope, tp);
+              if (half == 0) rope_table8<0>(rope_tab, rb, cs);
+              else rope_table8<1>(rope_tab, rb, cs);
+            } else {
+              if (half == 0) rope_fly8<0>(p.rope, tp, cs);
+              else rope_fly8<1>(p.rope, tp, cs);
+            }
+            rotate8(x, cs);
+            float xa[8], xb[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              xa[e] = x[e];
+              xb[e] = x[8 + e];
+            }
+            u0 = pack8(xa);
+            u1 = pack8(xb);
+          }
+          token_pos_advance(p.rope, tp, kRedT);
+        }
+        st_shared_v4(a0, u0);
+        st_shared_v4(a1, u1);
         fence_proxy_async_smem();
         mbar_arrive(&ready_a[s]);
       }
+      {
+        // the warp's 16 key sums over its 32 rows (fixed butterfly order);
+        // lane 0 leaves them in zred[wi][16]
+        float zv[16];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        zred[mt * 8 + 2 * e] = zacc[e].x;
-        zred[mt * 8 + 2 * e + 1] = zacc[e].y;
+        for (int e = 0; e < 8; ++e) {
+          zv[2 * e] = zacc[e].x;
+          zv[2 * e + 1] = zacc[e].y;
+        }
+#pragma unroll
+        for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) zv[e] += __shfl_xor_sync(0xffffffffu, zv[e], w);
+        if (lane == 0) {
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<float4*>(zred + wi * 16 + e) = make_float4(zv[e], zv[e + 1], zv[e + 2], zv[e + 3]);
+        }
       }
       alive = !bar_any(kBarMath, kMath, !alive || *abort_flag);
       // state of the four heads: the 32x32 diagonal blocks of the accumulator
@@ -349,27 +496,82 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
           for (int e = 0; e < 32; ++e) v[e] = 0.0f;
         }
         const int h = h0 + q;
-        if (h < p.H) {
-          float* dst = a.partials + ((cidx + q) * p.splits + blockIdx.x) * kStateFloats + lane * kD;
+        if (kCl || h < p.H) {
+          float* dst = kCl ? reinterpret_cast<float*>(smem + Smem::part) + q * kStateFloats + lane * kD
+                           : a.partials + ((cidx + q) * p.splits + blockIdx.x) * kStateFloats + lane * kD;
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4*>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
         }
       }
       if (mt < 128) {
-        // key sum of dim mt of the group: 32 row groups, in order
+        // key sum of dim mt of the group: the two row groups' warp sums, in order
         const int q = mt >> 5, d = mt & 31;
-        const int col = mt >> 3, e = mt & 7;  // chunk column and element holding this dim
-        float sum = 0.0f;
-        for (int r = 0; r < kMath / 16; ++r) sum += zred[(r * 16 + col) * 8 + e];
-        if (h0 + q < p.H)
+        const int wq = q * 2 + (d >> 4);  // warp (of row group 0) holding this dim
+        const float sum = zred[wq * 16 + (d & 15)] + zred[(8 + wq) * 16 + (d & 15)];
+        if (kCl)
+          reinterpret_cast<float*>(smem + Smem::part)[q * kStateFloats + kD * kD + d] = sum;
+        else if (h0 + q < p.H)
           a.partials[((cidx + q) * p.splits + blockIdx.x) * kStateFloats + kD * kD + d] = sum;
       }
       tc_fence_before();
     }
 
     float* sbuf = zred;  // [4][32][32] f32: the state for the apply, free once the reduce is done
-    if (kRed) {
+    if (kCl) {
+      // ---- hand-off inside the cluster (the head group's token splits, one
+      // CTA each; cluster rank = split index). Once every CTA's partial is in
+      // its shared memory, every CTA sums all of them in split order, plus the
+      // carry, straight into its own shared memory (the loads of all splits
+      // are issued before the sum): the sums are those of the reduce-only
+      // launch's combine, bit for bit. The state is written out at the end,
+      // once no CTA reads the carry any more (it may be updated in place).
+      named_bar_sync(kBarMath, kMath);  // this CTA's partial is in Smem::part
+      const uint32_t ncta = gridDim.x;
+      if (mt == 0) {
+        fence_acq_rel_cluster();
+        for (uint32_t r = 0; r < ncta; ++r) mbar_arrive_remote(mapa_shared(smem_u32(part_full), r));
+      }
+      bool ok = alive && mbar_wait_cluster(part_full, 0, abort_flag, &g_tc_error, kErrWait);
+      constexpr int kVec = kStateFloats / 4;  // float4 per head
+      const int heads = min(kGroupHeads, p.H - h0);
+      const uint32_t part_s = sbase + Smem::part;
+      if (ok) {
+        for (int v = mt; v < kGroupHeads * kVec; v += kMath) {
+          float4 t[kMaxCluster];
+#pragma unroll
+          for (int r = 0; r < kMaxCluster; ++r)
+            if (r < static_cast<int>(ncta)) t[r] = ld_cluster_v4(mapa_shared(part_s + v * 16, r));
+          float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+          for (int r = 0; r < kMaxCluster; ++r)
+            if (r < static_cast<int>(ncta)) {
+              acc.x += t[r].x;
+              acc.y += t[r].y;
+              acc.z += t[r].z;
+              acc.w += t[r].w;
+            }
+          const int hh = v / kVec, i = (v - hh * kVec) * 4;
+          const bool is_s = i < kD * kD;
+          if (hh < heads) {
+            const size_t bh = cidx + hh;
+            const float* c = is_s ? a.out.carry_S : a.out.carry_z;
+            if (c != nullptr) {
+              const float4 cv = *reinterpret_cast<const float4*>(
+                  c + (is_s ? bh * kD * kD + i : bh * kD + (i - kD * kD)));
+              acc = make_float4(cv.x + acc.x, cv.y + acc.y, cv.z + acc.z, cv.w + acc.w);
+            }
+          }
+          *reinterpret_cast<float4*>(is_s ? sbuf + hh * kD * kD + i : zs + hh * kD + (i - kD * kD)) =
+              acc;
+        }
+      }
+      alive = !bar_any(kBarMath, kMath, !ok || *abort_flag);
+      // no more reads of other CTAs' shared memory, nor of the carry
+      if (mt == 0)
+        for (uint32_t r = 0; r < ncta; ++r) mbar_arrive_remote(mapa_shared(smem_u32(done), r));
+    }
+    if (kRed && !kCl) {
       // ---- second phase of the reduce. The named barrier orders each math
       // thread's partial stores before the release fence of the arriving
       // thread.
@@ -420,18 +622,13 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       // pair j holds S[h][0..31][e] of heads 2j and 2j+1 in bf16 (K-major,
       // 128-byte swizzle); S goes through shared memory with 16-byte loads
       if (kPh == kApplyOnly) {  // the fused layer has it in shared memory already
-        for (int idx = mt; idx < kGroupHeads * kD * kD / 4; idx += kMath) {
-          const int hh = idx >> 8, h = h0 + hh;
-          float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          if (h < p.H)
-            v = __ldcg(reinterpret_cast<const float4*>(a.S_in + (cidx + hh) * kD * kD) + (idx & 255));
-          *reinterpret_cast<float4*>(sbuf + idx * 4) = v;
-        }
-        if (mt < kGroupHeads * kD) {
-          const int h = h0 + mt / kD;
-          zs[mt] = h < p.H ? __ldcg(a.z_in + cidx * kD + mt) : 0.0f;
-        }
-        named_bar_sync(kBarMath, kMath);
+        // the TMA warp copies the group's heads in; heads beyond H are zero
+        const int heads = min(kGroupHeads, p.H - h0);
+        for (int idx = heads * kD * kD / 4 + mt; idx < kGroupHeads * kD * kD / 4; idx += kMath)
+          *reinterpret_cast<float4*>(sbuf + idx * 4) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (mt >= heads * kD && mt < kGroupHeads * kD) zs[mt] = 0.0f;
+        const bool got = mbar_wait(s_full, 0, abort_flag, &g_tc_error, kErrWait);
+        if (bar_any(kBarMath, kMath, !got || *abort_flag)) alive = false;
       }
       {
         const int idx = mt;  // 2 pairs x 32 rows x 8 chunks = 512 = kMath
@@ -442,43 +639,63 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
         for (int k = 0; k < 8; ++k) x[k] = sbuf[hh * kD * kD + (d0 + k) * kD + e];
         st_shared_v4(sbase + Smem::bop + j * 4096 + sw128_offset(e, c), pack8(x));
       }
+      if (AC::kDenMma && mt < 256) {
+        // the denominator operand (K-major, 2 boxes x 16 rows x 128 B): row
+        // hh < 4 holds bf16(z) of head hh in the head's 32 dims, row 4 + hh
+        // the remainder z - bf16(z), rounded to bf16; everything else is 0,
+        // so column hh + 4 t of the MMA's result is ReLU(q) . (part t of z)
+        const int box = mt >> 7, r = (mt >> 3) & 15, c = mt & 7;
+        const int hh = 2 * box + (c >> 2), d0 = (c & 3) * 8;
+        float x[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float zv = zs[hh * kD + d0 + k];
+          const float hi = __bfloat162float(__float2bfloat16_rn(zv));
+          x[k] = (r & 3) != hh || r >= 8 ? 0.0f : (r < 4 ? hi : zv - hi);
+        }
+        st_shared_v4(sbase + Smem::zop + box * 2048 + sw128_offset(r, c), pack8(x));
+      }
       fence_proxy_async_smem();
       named_bar_sync(kBarMath, kMath);
       if (mt == 0) mbar_arrive(b_ready);
-      // ---- apply: warpgroup wg owns tiles wg, wg + 4, ...; thread = token row
+      // ---- apply: warpgroup wg < AC::kWG owns tiles wg, wg + kWG, ...;
+      // thread = token row
       const int wg = (warp - 2) >> 2;
       const int quad = warp & 3;
       const int row = quad * 32 + lane;
       const bool leader = (warp == 2 + 4 * wg) && lane == 0;
-      for (int j = wg; j < nB; j += kApWG) {
+      for (int j = wg; wg < AC::kWG && j < nB; j += AC::kWG) {
         const int pos = nA + j;
-        const int s = pos % kStages;
-        // The stage's previous apply tile (pos - kStages) belonged to another
+        const int s = pos % kNS;
+        // The stage's previous apply tile (pos - kNS) belonged to another
         // warpgroup. A parity wait cannot tell phase k from k + 2, so wait for
         // that tile's release first: then the full phase awaited next is
         // unambiguous. (Every earlier release precedes the load of this
         // warpgroup's previous tile, which it has already consumed.)
         bool ok = true;
-        if (pos - kStages >= nA)
-          ok = mbar_wait(&empty[s], ((pos - kStages) / kStages) & 1, abort_flag, &g_tc_error,
+        if (pos - kNS >= nA)
+          ok = mbar_wait(&empty[s], ((pos - kNS) / kNS) & 1, abort_flag, &g_tc_error,
                          kErrWait);
-        ok = ok && mbar_wait(&full[s], (pos / kStages) & 1, abort_flag, &g_tc_error, kErrWait);
+        ok = ok && mbar_wait(&full[s], (pos / kNS) & 1, abort_flag, &g_tc_error, kErrWait);
         if (bar_any(kBarWG0 + wg, 128, !ok || *abort_flag)) break;
         const int n0 = (tile_begin + j) * kApT;
         const int n = n0 + row;
         float2 cs[16];
         if (kRope != kNoRope) {
           const TokPos tp = token_pos(p.rope, min(n, p.N - 1));
-          const RopeBases rb = rope_bases(p.rope, tp);
+          float2 c0[8], c1[8];
+          if (kRope == kRopeTable) {
+            const RopeBases rb = rope_bases(p.rope, tp);
+            rope_table8<0>(rope_tab, rb, c0);
+            rope_table8<1>(rope_tab, rb, c1);
+          } else {
+            rope_fly8<0>(p.rope, tp, c0);
+            rope_fly8<1>(p.rope, tp, c1);
+          }
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int ax = pair_axis(jj);
-            if (kRope == kRopeTable) {
-              cs[jj] = rope_tab[(ax == 0 ? rb.t : (ax == 1 ? rb.h : rb.w)) + pair_off(jj)];
-            } else {
-              const int pp = ax == 0 ? p.rope.t_offset + tp.t : (ax == 1 ? tp.h : tp.w);
-              rope_cos_sin(pp, p.rope.inv_freq[jj], cs[jj].x, cs[jj].y);
-            }
+          for (int jj = 0; jj < 8; ++jj) {
+            cs[jj] = c0[jj];
+            cs[8 + jj] = c1[jj];
           }
         }
         float den[kGroupHeads] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -492,6 +709,10 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
           u.y = relu_bf16x2(u.y);
           u.z = relu_bf16x2(u.z);
           u.w = relu_bf16x2(u.w);
+          if (AC::kDenMma) {  // ReLU is the whole transform
+            st_shared_v4(addr, u);
+            continue;
+          }
           float x[8];
           unpack8(u, x);
           const float4 za = *reinterpret_cast<const float4*>(zs + hh * kD + d0);
@@ -522,15 +743,21 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
         mbar_arrive(&ready_b[s]);
 
         // epilogue: O = num / den over the tile in shared memory (the MMA has
-        // read it), stored with TMA; the stage returns once the store read it
-        ok = mbar_wait(&t_full[wg], (j / kApWG) & 1, abort_flag, &g_tc_error, kErrWait);
+        // read it); the TMA warp stores it and hands the stage back
+        ok = mbar_wait(&t_full[wg], (j / AC::kWG) & 1, abort_flag, &g_tc_error, kErrWait);
         tc_fence_after();
         if (bar_any(kBarWG0 + wg, 128, !ok || *abort_flag)) break;
+        const uint32_t acc = tmem + (static_cast<uint32_t>(quad * 32) << 16) + wg * AC::kCols;
+        if (AC::kDenMma) {
+          float dv[8];
+          tmem_ld_32x32b_x8(acc + AC::kDenCol, dv);
+#pragma unroll
+          for (int hh = 0; hh < kGroupHeads; ++hh) den[hh] = dv[hh] + dv[4 + hh];
+        }
 #pragma unroll
         for (int hh = 0; hh < kGroupHeads; ++hh) {
           float v[32];
-          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + wg * 128 + hh * 32,
-                             v);
+          tmem_ld_32x32b_x32(acc + hh * 32, v);
           const float inv = 1.0f / (den[hh] + p.eps);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -545,15 +772,46 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
         named_bar_sync(kBarWG0 + wg, 128);
         if (leader) {
           mbar_arrive(&t_empty[wg]);
-          uint8_t* tile = smem + Smem::stages + s * kStageBytes;
-          tma_store_3d(&tm_o, tile, h0 * 32, n0, b);
-          tma_store_3d(&tm_o, tile + kApBox, h0 * 32 + 64, n0, b);
-          bulk_commit();
-          bulk_wait_read<0>();      // the store has read the stage
-          mbar_arrive(&empty[s]);   // hand the stage back to the TMA warp
+          mbar_arrive(&o_full[s]);  // the TMA warp stores the tile
         }
       }
-      if (leader) bulk_wait<0>();
+    }
+    if (kCl) {
+      // The CTA's shared memory must outlive the other CTAs' reads of it, and
+      // the carry may be overwritten only once every CTA has read it: wait
+      // until every CTA of the cluster is done (not stopped by an abort: the
+      // other CTAs read this one's memory regardless), then write slice
+      // `rank` of the combined state out.
+      if (mt == 0 && !mbar_try_wait_acq_cluster(done, 0)) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait_acq_cluster(done, 0)) {
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_tc_error, kErrWait);
+            *abort_flag = 1;
+            break;
+          }
+        }
+      }
+      named_bar_sync(kBarMath, kMath);
+      if (alive && !*abort_flag) {
+        constexpr int kVec = kStateFloats / 4;
+        const int heads = min(kGroupHeads, p.H - h0);
+        const int nv = heads * kVec;
+        const int per = (nv + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+        const int v_lo = static_cast<int>(cluster_ctarank()) * per;
+        for (int v = v_lo + mt; v < min(nv, v_lo + per); v += kMath) {
+          const int hh = v / kVec, i = (v - hh * kVec) * 4;
+          const bool is_s = i < kD * kD;
+          const size_t bh = cidx + hh;
+          const size_t o = is_s ? bh * kD * kD + i : bh * kD + (i - kD * kD);
+          const float4 val = *reinterpret_cast<const float4*>(
+              is_s ? sbuf + hh * kD * kD + i : zs + hh * kD + (i - kD * kD));
+          float* d1 = is_s ? a.out.out1_S : a.out.out1_z;
+          float* d2 = is_s ? a.out.out2_S : a.out.out2_z;
+          if (d1 != nullptr) *reinterpret_cast<float4*>(d1 + o) = val;
+          if (d2 != nullptr) *reinterpret_cast<float4*>(d2 + o) = val;
+        }
+      }
     }
     if (kPh == kFusedLayer) {
       // every CTA has read the carry and the partials once all have reached
@@ -612,19 +870,42 @@ __global__ void __launch_bounds__(32) wait_selftest(unsigned long long limit_ns)
 
 // ============================================================== host side
 
+// Dynamic shared memory of layer_tc<mode, kPh>.
+template <int kPh>
+int layer_smem_bytes(int mode) {
+  return mode == kNoRope ? LayerCfg<kNoRope, kPh>::kSmemBytes
+                         : (mode == kRopeTable ? LayerCfg<kRopeTable, kPh>::kSmemBytes
+                                               : LayerCfg<kRopeOnTheFly, kPh>::kSmemBytes);
+}
+
 // Launch of layer_tc with programmatic dependent launch (the prologue may
-// overlap the previous kernel in the stream) and, for the fused layer, as a
-// cooperative launch (its CTAs wait on each other, so all must be resident).
+// overlap the previous kernel in the stream); for the fused layer either as a
+// cooperative launch (its CTAs wait on each other, so all must be resident) or
+// with clusters of `cluster_x` CTAs along x (each cluster is co-scheduled).
 cudaError_t launch_layer(void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, Problem,
                                       RopeTable, LayerArgs),
-                         dim3 grid, cudaStream_t s, bool cooperative, const CUtensorMap& mk,
+                         int smem_bytes, dim3 grid, cudaStream_t s, bool cooperative,
+                         const CUtensorMap& mk,
                          const CUtensorMap& mv, const CUtensorMap& mq, const CUtensorMap& mo,
-                         const Problem& p, const RopeTable& rt, const LayerArgs& a) {
+                         const Problem& p, const RopeTable& rt, const LayerArgs& a,
+                         int cluster_x = 0) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreadsTc, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(kSmemBytes);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
   cfg.stream = s;
+  if (cluster_x > 0) {
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, mk, mv, mq, mo, p, rt, a);
+  }
   // A cooperative launch that the runtime refuses with the programmatic
   // attribute is retried without it (the kernel's griddepcontrol
   // instructions are then no-ops); the outcome is remembered.
@@ -657,6 +938,43 @@ cudaError_t launch_layer(void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUt
 using LayerKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, Problem,
                              RopeTable, LayerArgs);
 
+// Whether every cluster of the cluster layer's grid (splits CTAs each, one
+// per SM) can be resident at once, asked once per (RoPE mode, splits, device).
+// Clusters must fit inside one GPC, so this can be less than the SM count
+// divided by the cluster size.
+int g_cluster_fit[3][kMaxCluster + 1][kMaxDev];  // 0 unknown, else co-resident clusters (-1 none)
+std::mutex g_cluster_mu;
+
+bool cluster_layer_fits(const Problem& p, int mode, LayerKernel kern) {
+  if (p.splits < 1 || p.splits > kMaxCluster) return false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
+  const long long clusters = static_cast<long long>((p.H + kGroupHeads - 1) / kGroupHeads) * p.B;
+  std::lock_guard<std::mutex> lk(g_cluster_mu);
+  int& known = g_cluster_fit[mode][p.splits][dev];
+  if (known == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.splits, 1, 1);
+    cfg.blockDim = dim3(kThreadsTc, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(layer_smem_bytes<kClusterLayer>(mode));
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(p.splits);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    known = n > 0 ? n : -1;  // cached: the number of co-resident clusters
+  }
+  return known > 0 && clusters <= known;
+}
+
 template <int kPh>
 LayerKernel pick_kernel(int mode) {
   return mode == kNoRope ? layer_tc<kNoRope, kPh>
@@ -681,14 +999,15 @@ cudaError_t launch_reduce_tc(const Problem& p, const void* K, const void* V, flo
   const RopeTable rt = rope_table_for(p);
   const int mode = rope_mode(rt);
   LayerKernel kern = pick_kernel<kReduceOnly>(mode);
-  if ((e = ensure_smem_attr(mode, reinterpret_cast<const void*>(kern), kSmemBytes)) != cudaSuccess)
+  const int kBytes = layer_smem_bytes<kReduceOnly>(mode);
+  if ((e = ensure_smem_attr(mode, reinterpret_cast<const void*>(kern), kBytes)) != cudaSuccess)
     return e;
   LayerArgs a = {};
   a.partials = partials;
   a.arrive = counters;
   a.out = out;
   const dim3 grid(p.splits, (p.H + kGroupHeads - 1) / kGroupHeads, p.B);
-  e = launch_layer(kern, grid, s, false, mk, mv, mk, mk, p, rt, a);
+  e = launch_layer(kern, kBytes, grid, s, false, mk, mv, mk, mk, p, rt, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -702,7 +1021,8 @@ cudaError_t launch_apply_tc(const Problem& p, const void* Q, const float* S, con
   const RopeTable rt = rope_table_for(p);
   const int mode = rope_mode(rt);
   LayerKernel kern = pick_kernel<kApplyOnly>(mode);
-  if ((e = ensure_smem_attr(3 + mode, reinterpret_cast<const void*>(kern), kSmemBytes)) !=
+  const int kBytes = layer_smem_bytes<kApplyOnly>(mode);
+  if ((e = ensure_smem_attr(3 + mode, reinterpret_cast<const void*>(kern), kBytes)) !=
       cudaSuccess)
     return e;
   const int groups = (p.H + kGroupHeads - 1) / kGroupHeads;
@@ -721,7 +1041,7 @@ cudaError_t launch_apply_tc(const Problem& p, const void* Q, const float* S, con
   // started reading only after everything before it had completed.
   a.q_before_wait = after_own_reduce ? 1 : 0;
   const dim3 grid(ctas, groups, p.B);
-  e = launch_layer(kern, grid, s, false, mq, mq, mq, mo, p, rt, a);
+  e = launch_layer(kern, kBytes, grid, s, false, mq, mq, mq, mo, p, rt, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -751,8 +1071,24 @@ cudaError_t launch_layer_tc(const Problem& p, const void* Q, const void* K, cons
   if ((e = make_map(&mo, O, p, kApT)) != cudaSuccess) return e;
   const RopeTable rt = rope_table_for(p);
   const int mode = rope_mode(rt);
+  LayerKernel kern_cl = pick_kernel<kClusterLayer>(mode);
+  const int kBytesCl = layer_smem_bytes<kClusterLayer>(mode);
+  if ((e = ensure_smem_attr(9 + mode, reinterpret_cast<const void*>(kern_cl), kBytesCl)) !=
+      cudaSuccess)
+    return e;
+  const dim3 grid(p.splits, (p.H + kGroupHeads - 1) / kGroupHeads, p.B);
+  if (cluster_layer_fits(p, mode, kern_cl)) {
+    // the head group's splits as one cluster: the hand-off stays on chip
+    LayerArgs a = {};
+    a.out = out;
+    a.tiles_per_cta = apply_tiles_per_cta(p, p.splits);
+    e = launch_layer(kern_cl, kBytesCl, grid, s, false, mk, mv, mq, mo, p, rt, a, p.splits);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   LayerKernel kern = pick_kernel<kFusedLayer>(mode);
-  if ((e = ensure_smem_attr(6 + mode, reinterpret_cast<const void*>(kern), kSmemBytes)) !=
+  const int kBytes = layer_smem_bytes<kFusedLayer>(mode);
+  if ((e = ensure_smem_attr(6 + mode, reinterpret_cast<const void*>(kern), kBytes)) !=
       cudaSuccess)
     return e;
   const size_t bh = static_cast<size_t>(p.B) * p.H;
@@ -765,8 +1101,7 @@ cudaError_t launch_layer_tc(const Problem& p, const void* Q, const void* K, cons
   a.S_in = out.out1_S;
   a.z_in = out.out1_z;
   a.tiles_per_cta = apply_tiles_per_cta(p, p.splits);
-  const dim3 grid(p.splits, (p.H + kGroupHeads - 1) / kGroupHeads, p.B);
-  e = launch_layer(kern, grid, s, true, mk, mv, mq, mo, p, rt, a);
+  e = launch_layer(kern, kBytes, grid, s, true, mk, mv, mq, mo, p, rt, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -19,16 +19,18 @@ namespace {
 using namespace sm100;
 
 constexpr int kGroupHeads = 4;
-constexpr int kRopeTableMax = 1536;  // float2 entries of the per-CTA RoPE table
+constexpr int kRopeTableMax = 768;  // float2 entries of the per-CTA RoPE table
 
 enum : unsigned { kErrWait = 1u };
 
 // ------------------------------------------------------------------ RoPE
 
 // Per-CTA table of (cos, sin) for every position of the block: T frames x 4
-// pairs (time), then Hh x 6 pairs (height), then W x 6 pairs (width). Angles
-// are formed and reduced to [-pi, pi] in double, then evaluated in float. When
-// the table does not fit in shared memory the angles are evaluated per token
+// pairs (time), then Hh rows of 6 pairs (height) and W rows of 6 pairs
+// (width), each of these rows padded to 8 entries so that every row starts on
+// a 16-byte boundary and two pairs load as one 16-byte vector. Angles are
+// formed and reduced to [-pi, pi] in double, then evaluated in float. When the
+// table does not fit in shared memory the angles are evaluated per token
 // instead.
 struct RopeTable {
   int enabled;
@@ -36,7 +38,7 @@ struct RopeTable {
 };
 
 __host__ __device__ inline int rope_table_entries(const Rope& r) {
-  return 4 * r.T + 6 * r.Hh + 6 * r.W;
+  return 4 * r.T + 8 * r.Hh + 8 * r.W;
 }
 
 __device__ void build_rope_table(const Rope& r, float2* tab, int tid, int nthreads) {
@@ -46,14 +48,18 @@ __device__ void build_rope_table(const Rope& r, float2* tab, int tid, int nthrea
     if (i < 4 * r.T) {
       pos = r.t_offset + i / 4;
       j = i % 4;
-    } else if (i < 4 * r.T + 6 * r.Hh) {
+    } else if (i < 4 * r.T + 8 * r.Hh) {
       const int k = i - 4 * r.T;
-      pos = k / 6;
-      j = 4 + k % 6;
+      pos = k / 8;
+      j = k % 8 < 6 ? 4 + k % 8 : -1;
     } else {
-      const int k = i - 4 * r.T - 6 * r.Hh;
-      pos = k / 6;
-      j = 10 + k % 6;
+      const int k = i - 4 * r.T - 8 * r.Hh;
+      pos = k / 8;
+      j = k % 8 < 6 ? 10 + k % 8 : -1;
+    }
+    if (j < 0) {  // padding
+      tab[i] = make_float2(0.0f, 0.0f);
+      continue;
     }
     float cs, sn;
     rope_cos_sin(pos, r.inv_freq[j], cs, sn);
@@ -95,7 +101,56 @@ struct RopeBases {
   int t, h, w;
 };
 __device__ __forceinline__ RopeBases rope_bases(const Rope& r, const TokPos& tp) {
-  return {tp.t * 4, 4 * r.T + tp.h * 6, 4 * r.T + 6 * r.Hh + tp.w * 6};
+  return {tp.t * 4, 4 * r.T + tp.h * 8, 4 * r.T + 8 * r.Hh + tp.w * 8};
+}
+
+// (cos, sin) of the 8 pairs [8 kHalf, 8 kHalf + 8) of one token (16 dims of a
+// head): from the table, four 16-byte loads (every row base is even).
+template <int kHalf>
+__device__ __forceinline__ void rope_table8(const float2* tab, const RopeBases& rb,
+                                            float2 (&cs)[8]) {
+  const float4* t4 = reinterpret_cast<const float4*>(tab);
+  float4 v[4];
+  if (kHalf == 0) {  // pairs 0-3: time; 4-7: height 0-3
+    v[0] = t4[rb.t / 2];
+    v[1] = t4[rb.t / 2 + 1];
+    v[2] = t4[rb.h / 2];
+    v[3] = t4[rb.h / 2 + 1];
+  } else {           // pairs 8-9: height 4-5; 10-15: width 0-5
+    v[0] = t4[rb.h / 2 + 2];
+    v[1] = t4[rb.w / 2];
+    v[2] = t4[rb.w / 2 + 1];
+    v[3] = t4[rb.w / 2 + 2];
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    cs[2 * k] = make_float2(v[k].x, v[k].y);
+    cs[2 * k + 1] = make_float2(v[k].z, v[k].w);
+  }
+}
+
+// The same 8 pairs evaluated from the token's position (no table).
+template <int kHalf>
+__device__ __forceinline__ void rope_fly8(const Rope& r, const TokPos& tp, float2 (&cs)[8]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int j = 8 * kHalf + q;
+    const int ax = j < 4 ? 0 : (j < 10 ? 1 : 2);
+    const int pos = ax == 0 ? r.t_offset + tp.t : (ax == 1 ? tp.h : tp.w);
+    rope_cos_sin(pos, r.inv_freq[j], cs[q].x, cs[q].y);
+  }
+}
+
+// Rotate 8 interleaved pairs of x by (cos, sin): (x0, x1) -> (x0 c - x1 s, x0 s + x1 c).
+__device__ __forceinline__ void rotate8(float (&x)[16], const float2 (&cs)[8]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float2 t = __fmul2_rn(make_float2(x[2 * q + 1], x[2 * q + 1]),
+                                make_float2(-cs[q].y, cs[q].x));
+    const float2 y = __ffma2_rn(make_float2(x[2 * q], x[2 * q]), cs[q], t);
+    x[2 * q] = y.x;
+    x[2 * q + 1] = y.y;
+  }
 }
 
 // Barrier over `threads` threads of named barrier `id` that also ORs `pred`
