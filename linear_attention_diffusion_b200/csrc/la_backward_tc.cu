@@ -74,10 +74,12 @@ struct QSmem {  // query side, byte offsets from the 1024-aligned base
   static constexpr int bop = stages + kBStages * kBTile;    // S as B operand: [32 rows][128 B]
   static constexpr int zs = bop + 4096;                     // [2][32] f32
   static constexpr int dden = zs + 256;                     // [3][128 rows][2] f32
-  static constexpr int rope = dden + kBWG * kBT * kPair * 4;  // float2[kRopeTableMax]
+  static constexpr int sraw = dden + kBWG * kBT * kPair * 4;  // S of the pair as copied: [2][32][32] f32
+  static constexpr int rope = sraw + kPair * kD * kD * 4;     // float2[kRopeTableMax]
   static constexpr int bars = rope + kRopeTableMax * 8;
-  // full[6] empty[6] ready_t[6] ready_s[6] t_full[6] acc_full mma_done b_ready
-  static constexpr int nbars = 5 * kBStages + 3;
+  // full[6] empty[6] ready_t[6] ready_s[6] t_full[6] o_full[6] s2_done[6]
+  // acc_full mma_done b_ready s_full
+  static constexpr int nbars = 7 * kBStages + 4;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int bytes = misc + 16;
 };
@@ -177,9 +179,12 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   uint64_t* ready_t = empty + kBStages;   // tile transformed (128 arrivals)
   uint64_t* ready_s = ready_t + kBStages; // phi(Q) in place, dz done (128 arrivals)
   uint64_t* t_full = ready_s + kBStages;  // t of the stage's tile is in TMEM
-  uint64_t* acc_full = t_full + kBStages;
+  uint64_t* o_full = t_full + kBStages;   // dQ of the stage's tile in its dO box
+  uint64_t* s2_done = o_full + kBStages;  // RoPE: MMA 2 of the stage's tile done
+  uint64_t* acc_full = s2_done + kBStages;
   uint64_t* mma_done = acc_full + 1;
   uint64_t* b_ready = mma_done + 1;
+  uint64_t* s_full = b_ready + 1;         // S and z of the pair copied in
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + QSmem::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + QSmem::misc + 4);
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + QSmem::misc + 8);
@@ -203,10 +208,13 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       mbar_init(&ready_t[s], 128);
       mbar_init(&ready_s[s], 128);
       mbar_init(&t_full[s], 1);
+      mbar_init(&o_full[s], 1);
+      mbar_init(&s2_done[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
     mbar_init(b_ready, 1);
+    mbar_init(s_full, 1);
     *abort_flag = 0;
     *last_flag = 0;
     fence_mbar_init();
@@ -232,18 +240,41 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   if (warp == 0) {
     // ------------------------------------------------------------ TMA loads
     if (lane == 0) {
+      // S and z of the pair first, ahead of the tiles in the memory queues
+      const int heads = min(kPair, p.H - h0);
+      mbar_arrive_expect_tx(s_full, heads * (kD * kD + kD) * 4);
+      bulk_load(smem + QSmem::sraw, a.S + cidx * kD * kD, heads * kD * kD * 4, s_full);
+      bulk_load(smem + QSmem::zs, a.z + cidx * kD, heads * kD * 4, s_full);
+      // The warpgroups leave dQ in the tile's dO box (o_full) once both MMAs
+      // have read the stage, and this thread stores it with TMA before it
+      // reloads the stage.
+      auto store_dq = [&](int k) -> bool {
+        const int ks = k % kBStages;
+        if (!mbar_wait(&o_full[ks], (k / kBStages) & 1, abort_flag, err, kErrWait)) return false;
+        tma_store_3d(&tm_dq, smem + QSmem::stages + ks * kBTile + kBBox, h0 * 32, n_begin + k * kBT, b);
+        bulk_commit();
+        bulk_wait_read<0>();
+        return true;
+      };
       int i = 0;
+      bool ok = true;
       for (; i < nT; ++i) {
         const int s = i % kBStages;
-        if (!mbar_wait(&empty[s], ((i / kBStages) & 1) ^ 1, abort_flag, err, kErrWait)) break;
+        if (i >= kBStages) {
+          if (!(ok = store_dq(i - kBStages))) break;
+        } else if (!mbar_wait(&empty[s], ((i / kBStages) & 1) ^ 1, abort_flag, err, kErrWait)) {
+          break;
+        }
         mbar_arrive_expect_tx(&full[s], kBTile);
         uint8_t* st = smem + QSmem::stages + s * kBTile;
         const int y = n_begin + i * kBT;
         tma_load_3d(st, &tm_q, &full[s], h0 * 32, y, b);
         tma_load_3d(st + kBBox, &tm_g, &full[s], h0 * 32, y, b);
       }
+      for (int k = max(0, i - kBStages); ok && k < i; ++k) ok = store_dq(k);
       for (int q = max(0, i - kBStages); q < i; ++q)
         mbar_drain(&full[q % kBStages], (q / kBStages) & 1, err, kErrWait);
+      bulk_wait<0>();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
@@ -306,7 +337,7 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
             const uint64_t bd = smem_desc_sw128(st + kBBox + kk * 2048, kBBox, 1024);
             mma_bf16(tmem + kColDS, ad, bd, id_s, (k > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&empty[s]);
+          mma_commit(&s2_done[s]);  // the warpgroup then writes dQ over the dnum box
         }
       }
       mma_commit(acc_full);
@@ -321,9 +352,22 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     const int row = quad * 32 + lane;     // token row of the tile (thread = row)
     bool alive = true;
 
-    // S as the B operand of MMA 1 (rows d, K = e), z of the two heads
-    build_bop(sbase + QSmem::bop, a.S, cidx, h0, p.H, false, mt, kBMath);
-    if (mt < kPair * kD) zs[mt] = h0 + mt / kD < p.H ? __ldcg(a.z + cidx * kD + mt) : 0.0f;
+    // S as the B operand of MMA 1 (rows d, K = e), z of the two heads: the
+    // TMA warp has copied the pair's S and z in (a missing head is zero)
+    {
+      const int heads = min(kPair, p.H - h0);
+      if (mt >= heads * kD && mt < kPair * kD) zs[mt] = 0.0f;
+      if (!mbar_wait(s_full, 0, abort_flag, err, kErrWait)) alive = false;
+      const float* sr = reinterpret_cast<const float*>(smem + QSmem::sraw);
+      for (int idx = mt; idx < 32 * 8; idx += kBMath) {
+        const int r = idx >> 3, c = idx & 7;
+        const int hh = c >> 2, k0 = (c & 3) * 8;
+        float x[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] = hh < heads ? sr[hh * kD * kD + r * kD + k0 + k] : 0.0f;
+        st_shared_v4(sbase + QSmem::bop + sw128_offset(r, c), pack8(x));
+      }
+    }
     fence_proxy_async_smem();
     named_bar_sync(kBarAll, kBMath);
     if (mt == 0) mbar_arrive(b_ready);
@@ -390,7 +434,7 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         alive = false;
         break;
       }
-      const bool row_ok = n < n_end;
+      uint4 dq[kPair][4];  // RoPE: this row's dQ until MMA 2 has read the stage
 #pragma unroll
       for (int hh = 0; hh < kPair; ++hh) {
         float t[32];
@@ -434,9 +478,9 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
             }
             st_shared_v4(st + kBBox + sw128_offset(row, c), pack8(x));
           }
-        } else if (row_ok && h0 + hh < p.H) {
+        } else {
+          // MMA 2 still reads the dnum box: dQ waits in registers
           const float* zz = zs + hh * kD;
-          __nv_bfloat16* dst = a.dQ + ((static_cast<size_t>(b) * p.N + n) * p.H + h0 + hh) * kD;
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
             const int c = hh * 4 + c4;
@@ -447,7 +491,7 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
               const int d = c4 * 8 + e;
               x[e] = x[e] > 0.0f ? fmaf(dden, zz[d], t[d]) : 0.0f;
             }
-            *reinterpret_cast<uint4*>(dst + c4 * 8) = pack8(x);
+            dq[hh][c4] = pack8(x);
           }
         }
       }
@@ -470,13 +514,8 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       named_bar_sync(kBarW0 + wg, 128);
 
       if (kRope == kNoRope) {
-        // the stage is done with: store dQ, then hand it back to the TMA warp
-        if (wt == 0) {
-          tma_store_3d(&tm_dq, smem + QSmem::stages + s * kBTile + kBBox, h0 * 32, n0, b);
-          bulk_commit();
-          bulk_wait_read<0>();
-          mbar_arrive(&empty[s]);
-        }
+        // the stage is done with: the TMA warp stores dQ and reloads it
+        if (wt == 0) mbar_arrive(&o_full[s]);
         continue;
       }
       // ---- rewrite ReLU(Q) -> phi(Q) for MMA 2
@@ -492,9 +531,23 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       }
       fence_proxy_async_smem();
       mbar_arrive(&ready_s[s]);
+      // ---- once MMA 2 has read the stage, dQ goes over the dnum box and the
+      // TMA warp stores it (rows and heads beyond the tensor are clipped)
+      ok = mbar_wait(&s2_done[s], par, abort_flag, err, kErrWait);
+      if (bar_any(kBarW0 + wg, 128, !ok || *abort_flag)) {
+        alive = false;
+        break;
+      }
+#pragma unroll
+      for (int hh = 0; hh < kPair; ++hh)
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+          st_shared_v4(st + kBBox + sw128_offset(row, hh * 4 + c4), dq[hh][c4]);
+      fence_proxy_async_smem();
+      named_bar_sync(kBarW0 + wg, 128);
+      if (wt == 0) mbar_arrive(&o_full[s]);
     }
 
-    if (kRope == kNoRope && wt == 0) bulk_wait<0>();
     // ---- partial (dS, dz) of this split
     alive = !bar_any(kBarAll, kBMath, !alive || *abort_flag);
     float* scratch = reinterpret_cast<float*>(smem + QSmem::stages);  // [kBMath][8] after the MMAs

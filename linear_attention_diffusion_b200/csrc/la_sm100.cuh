@@ -176,6 +176,13 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Orders this thread's view of global memory (e.g. what an acquire made
+// visible) before its later async-proxy accesses of global memory (bulk
+// copies reading data that other CTAs wrote with ordinary stores).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Acquire load / release store of a flag in global memory, GPU scope.
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* ptr) {
   unsigned v;

@@ -595,7 +595,51 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
         // (+ carry) and writes the state
         const bool wanted = a.out.out1_S != nullptr || a.out.out1_z != nullptr ||
                             a.out.out2_S != nullptr || a.out.out2_z != nullptr;
-        if (last && alive && wanted) combine_from_global<kMath>(p, b, h0, mt, a.partials, a.out);
+        const int heads = min(kGroupHeads, p.H - h0);
+        const uint32_t pbytes =
+            static_cast<uint32_t>(heads) * static_cast<uint32_t>(p.splits) * kStateFloats * 4u;
+        if (last && alive && wanted && pbytes <= static_cast<uint32_t>(kNS) * kStageBytes) {
+          // The group's partials are contiguous in the workspace: one bulk
+          // copy brings them all into the idle stage ring (every load has
+          // landed and every MMA has read its stage), then each thread sums
+          // its columns over the splits from shared memory.
+          if (mt == 0) {
+            fence_proxy_async_global();  // after the acquire above
+            mbar_arrive_expect_tx(s_full, pbytes);
+            bulk_load(smem + Smem::stages, a.partials + cidx * p.splits * kStateFloats, pbytes,
+                      s_full);
+          }
+          if (mbar_wait(s_full, 0, abort_flag, &g_tc_error, kErrWait)) {
+            const float* ps = reinterpret_cast<const float*>(smem + Smem::stages);
+            constexpr int kVec = kStateFloats / 4;
+            for (int v = mt; v < heads * kVec; v += kMath) {
+              const int hh = v / kVec, i = (v - hh * kVec) * 4;
+              float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+              for (int s2 = 0; s2 < p.splits; ++s2) {
+                const float4 t = *reinterpret_cast<const float4*>(
+                    ps + (static_cast<size_t>(hh) * p.splits + s2) * kStateFloats + i);
+                acc.x += t.x;
+                acc.y += t.y;
+                acc.z += t.z;
+                acc.w += t.w;
+              }
+              const bool is_s = i < kD * kD;
+              const size_t bh = cidx + hh;
+              const size_t o = is_s ? bh * kD * kD + i : bh * kD + (i - kD * kD);
+              const float* c = is_s ? a.out.carry_S : a.out.carry_z;
+              if (c != nullptr) {
+                const float4 cv = *reinterpret_cast<const float4*>(c + o);
+                acc = make_float4(cv.x + acc.x, cv.y + acc.y, cv.z + acc.z, cv.w + acc.w);
+              }
+              float* d1 = is_s ? a.out.out1_S : a.out.out1_z;
+              float* d2 = is_s ? a.out.out2_S : a.out.out2_z;
+              if (d1 != nullptr) *reinterpret_cast<float4*>(d1 + o) = acc;
+              if (d2 != nullptr) *reinterpret_cast<float4*>(d2 + o) = acc;
+            }
+          }
+        } else if (last && alive && wanted) {
+          combine_from_global<kMath>(p, b, h0, mt, a.partials, a.out);
+        }
         named_bar_sync(kBarMath, kMath);
         if (mt == 0 && last) a.arrive[cidx] = 0u;  // ready for the next call
       } else {
