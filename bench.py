@@ -137,11 +137,12 @@ def peaks():
 _DEVICE_HEADERS = ("la_common.cuh", "la_sm100.cuh", "la_tc_common.cuh")
 KERNEL_SOURCES = {
     "attention_layer": ("la_tc.cu",) + _DEVICE_HEADERS,
+    "la_block_causal_step": ("la_tc.cu",) + _DEVICE_HEADERS,
     "state_reduce": ("la_tc.cu",) + _DEVICE_HEADERS,
     "apply": ("la_tc.cu",) + _DEVICE_HEADERS,
     "attention_backward": ("la_backward_tc.cu",) + _DEVICE_HEADERS,
     "causal_attention": ("la_tc.cu", "la_causal_tc.cu") + _DEVICE_HEADERS,
-    "temporal_conv": ("la_conv.cu",) + _DEVICE_HEADERS,
+    "temporal_conv": ("la_conv.cu", "la_common.cuh", "la_sm100.cuh"),
     "qkv_state": ("la_qkv_tc.cu",) + _DEVICE_HEADERS,
 }
 
@@ -1012,7 +1013,7 @@ def main():
                           "event_graph_us": r["seg_us"][0],
                           "note": "update=0 call, event graph; avg over all 60 calls"}}
         dom = name
-        traffic = None
+        traffic = profiled_traffic(w.name, name)
     elif args.op == "qkv":
         kernels, dom, traffic = {}, None, None
     else:
