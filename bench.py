@@ -141,7 +141,7 @@ KERNEL_SOURCES = {
     "state_reduce": ("la_tc.cu",) + _DEVICE_HEADERS,
     "apply": ("la_tc.cu",) + _DEVICE_HEADERS,
     "attention_backward": ("la_backward_tc.cu",) + _DEVICE_HEADERS,
-    "causal_attention": ("la_tc.cu", "la_causal_tc.cu") + _DEVICE_HEADERS,
+    "causal_attention": ("la_tc.cu", "la_causal_chunk.cu") + _DEVICE_HEADERS,
     "temporal_conv": ("la_conv.cu", "la_common.cuh", "la_sm100.cuh"),
     "qkv_state": ("la_qkv_tc.cu",) + _DEVICE_HEADERS,
 }
@@ -454,7 +454,7 @@ def run_la(args, w, rank, world, local_rank):
                              w.rope_base, w.eps)
 
     shape0 = shape_at(0)
-    ws = la.workspace(shape0, dev)
+    ws = la.workspace(shape0, dev, causal=args.op == "causal")
     ws_p, ws_n = ws.data_ptr(), ws.numel()
     S_p, z_p = S.data_ptr(), z.data_ptr()
     ptrs = [tuple(t.data_ptr() for t in s) for s in sets]
@@ -866,7 +866,7 @@ def run_e2e(args, w, dev, stream, la, rank, causal=False):
     z = torch.zeros((w.B, w.H, D), device=dev)
     shapes = [la.make_shape(w.B, w.N, w.H, D, "bf16", w.rope, w.T, w.Hh, w.W, m * w.T,
                             w.rope_base, w.eps) for m in range(max(1, w.M))]
-    ws = la.workspace(shapes[0], dev)
+    ws = la.workspace(shapes[0], dev, causal=causal)
     per = w.steps + 1
 
     def call(p, ins, outs, st):

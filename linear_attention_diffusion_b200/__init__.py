@@ -66,6 +66,8 @@ _shape_p = ctypes.POINTER(LaShape)
 
 _lib.la_workspace_bytes.argtypes = [_shape_p]
 _lib.la_workspace_bytes.restype = _sz
+_lib.la_causal_workspace_bytes.argtypes = [_shape_p]
+_lib.la_causal_workspace_bytes.restype = _sz
 _lib.la_state_reduce.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.la_state_reduce.restype = _i
 _lib.la_state_reduce_static.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp]
@@ -141,6 +143,10 @@ def _check(status: int, func: str) -> None:
 
 def la_workspace_bytes(shape: LaShape) -> int:
     return int(_lib.la_workspace_bytes(ctypes.byref(shape)))
+
+
+def la_causal_workspace_bytes(shape: LaShape) -> int:
+    return int(_lib.la_causal_workspace_bytes(ctypes.byref(shape)))
 
 
 def la_state_reduce(shape: LaShape, K, V, S, z, ws, stream=None) -> None:
@@ -259,10 +265,11 @@ def shape_for(Q, eps: float = 1e-6, rope_grid=None, t_offset: int = 0,
     return make_shape(B, N, H, D, io, True, T, Hh, W, t_offset, rope_base, eps)
 
 
-def workspace(shape: LaShape, device="cuda"):
-    """A zero-filled workspace of la_workspace_bytes(shape) bytes."""
+def workspace(shape: LaShape, device="cuda", causal: bool = False):
+    """A zero-filled workspace of la_workspace_bytes(shape) bytes
+    (la_causal_workspace_bytes(shape) with causal=True)."""
     import torch
-    n = la_workspace_bytes(shape)
+    n = la_causal_workspace_bytes(shape) if causal else la_workspace_bytes(shape)
     if n == 0:
         raise LaError(LA_ERR_INVALID_ARG, "la_workspace_bytes")
     return torch.zeros(n, dtype=torch.uint8, device=device)
@@ -302,7 +309,7 @@ def causal_attention(Q, K, V, S_carry=None, z_carry=None, update: int = 0, eps: 
     import torch
     O = torch.empty_like(Q)
     la_causal_attention(shape, Q, K, V, S_carry, z_carry, O, update,
-                        workspace(shape, Q.device), stream)
+                        workspace(shape, Q.device, causal=True), stream)
     return O
 
 

@@ -1,5 +1,6 @@
 // C-ABI layer: argument checks on the host, workspace layout, and the order
 // of the kernel launches for each entry point of include/la.h.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -134,6 +135,14 @@ la_status check_ws(const Problem& p, const void* ws, size_t ws_bytes) {
   return LA_OK;
 }
 
+// Workspace of la_causal_attention: the chunk states of the chunked
+// tensor-core path (bf16 without RoPE), else the ordinary layout.
+size_t causal_workspace_bytes(const Problem& p) {
+  const size_t base = workspace_layout(p).total;
+  if (!causal_chunk_supported(p)) return base;
+  return std::max(base, align256(causal_chunk_state_bytes(p)));
+}
+
 // State reduce of (K, V) into `out`, using the workspace's partials and
 // counters.
 la_status run_reduce(const Problem& p, const void* K, const void* V, char* ws,
@@ -193,6 +202,12 @@ using namespace la;
 using namespace la::detail;
 
 extern "C" {
+
+size_t la_causal_workspace_bytes(const la_shape* shape) {
+  Problem p;
+  if (make_problem(shape, p) != LA_OK) return 0;
+  return causal_workspace_bytes(p);
+}
 
 size_t la_workspace_bytes(const la_shape* shape) {
   Problem p;
@@ -410,7 +425,14 @@ la_status la_causal_attention(const la_shape* shape, const void* Q, const void* 
   LA_TRY(check_ptr(O, "O", any_input));
   LA_TRY(check_ptr(S_carry, "S_carry", any_state && S_carry != nullptr));
   LA_TRY(check_ptr(z_carry, "z_carry", any_state && z_carry != nullptr));
-  LA_TRY(check_ws(p, ws, ws_bytes));
+  {
+    const size_t need = causal_workspace_bytes(p);
+    if (ws == nullptr) return fail(LA_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", need);
+    if (!aligned16(ws)) return fail(LA_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    if (ws_bytes < need)
+      return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed (la_causal_workspace_bytes)",
+                  ws_bytes, need);
+  }
   const size_t nb = io_bytes(p);
   if (overlap(O, nb, Q, nb) || overlap(O, nb, K, nb) || overlap(O, nb, V, nb) ||
       overlap(O, nb, ws, ws_bytes) || overlap(O, nb, S_carry, s_bytes(p)) ||
@@ -421,6 +443,13 @@ la_status la_causal_attention(const la_shape* shape, const void* Q, const void* 
   if (!any_state) return LA_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
+  if (causal_chunk_supported(p)) {
+    // bf16 without RoPE: every chunk's state, their prefix, then the chunks
+    const cudaError_t e = launch_causal_chunks(p, Q, K, V, reinterpret_cast<float*>(w), S_carry,
+                                               z_carry, update, O, st);
+    if (e != cudaSuccess) return cuda_fail(e, "causal attention");
+    return LA_OK;
+  }
   const WsLayout L = workspace_layout(p);
   // the splits' partial states only: no combine
   LA_TRY(run_reduce(p, K, V, w, StateOut{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr},
@@ -610,6 +639,9 @@ la_status la_device_error(unsigned* code, int reset) {
   if (e == cudaSuccess) e = read_device_error_bwd(&bwd, reset != 0);
   if (e == cudaSuccess) e = read_device_error_conv(&conv, reset != 0);
   if (e == cudaSuccess) e = read_device_error_causal(&causal, reset != 0);
+  unsigned chunked = 0;
+  if (e == cudaSuccess) e = read_device_error_causal_chunk(&chunked, reset != 0);
+  causal |= chunked;
   if (e == cudaSuccess) e = read_device_error_qkv(&qkv, reset != 0);
   if (e != cudaSuccess) return cuda_fail(e, "la_device_error");
   *code = fwd | bwd | conv | causal | qkv;

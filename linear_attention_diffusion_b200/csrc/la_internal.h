@@ -114,7 +114,21 @@ cudaError_t launch_backward_kv_simt(const Problem& p, const void* K, const void*
 cudaError_t launch_causal(const Problem& p, const void* Q, const void* K, const void* V,
                           const float* partials, float* S_carry, float* z_carry, int update,
                           unsigned* counters, void* O, cudaStream_t s);
-// The tensor-core version (la_causal_tc.cu): bf16 I/O without RoPE.
+// The chunked tensor-core version (la_causal_chunk.cu, bf16 I/O without
+// RoPE): the state reduce writes every 128-token chunk's own state into
+// `states` (causal_chunk_state_bytes), a prefix kernel turns them into each
+// chunk's exclusive prefix (carry included; update = 1 folds the sequence into
+// the carry), and the output kernel computes every chunk independently.
+bool causal_chunk_supported(const Problem& p);
+size_t causal_chunk_state_bytes(const Problem& p);
+cudaError_t launch_chunk_states_tc(const Problem& p, const void* K, const void* V, float* states,
+                                   int nchunks, cudaStream_t s);
+cudaError_t launch_causal_chunks(const Problem& p, const void* Q, const void* K, const void* V,
+                                 float* states, float* S_carry, float* z_carry, int update,
+                                 void* O, cudaStream_t s);
+cudaError_t read_device_error_causal_chunk(unsigned* code, bool reset);
+// The earlier tensor-core version (la_causal_tc.cu): bf16 I/O without RoPE,
+// a running state carried from chunk to chunk.
 bool causal_tc_supported(const Problem& p);
 cudaError_t launch_causal_tc(const Problem& p, const void* Q, const void* K, const void* V,
                              const float* partials, float* S_carry, float* z_carry, int update,

@@ -49,10 +49,14 @@ using namespace sm100;
 // apply) in two forms: the head group's CTAs as one thread-block cluster that
 // hands the split partials over through distributed shared memory
 // (kClusterLayer), or a cooperative grid that hands them over through global
-// memory (kFusedLayer). All share one TMA stage ring of kNS stages (six; five
+// memory (kFusedLayer). A fifth launch, kChunkStates (bf16 without RoPE),
+// is the reduce that writes the state of every 128-token chunk instead of
+// one partial per split: the first step of token-causal attention. All share
+// one TMA stage ring of kNS stages (six; five
 // in the cluster layer): a ring position p uses stage p % kNS with phase
 // parity (p / kNS) & 1, whichever operation the tile belongs to.
-enum Phases : int { kReduceOnly = 1, kApplyOnly = 2, kFusedLayer = 3, kClusterLayer = 7 };
+enum Phases : int { kReduceOnly = 1, kApplyOnly = 2, kFusedLayer = 3, kClusterLayer = 7,
+                    kChunkStates = 9 };
 
 // Largest cluster of the cluster layer: the portable limit.
 constexpr int kMaxCluster = 8;
@@ -132,6 +136,8 @@ struct LayerArgs {
   const float* z_in;
   int tiles_per_cta;   // apply: 128-token tiles per CTA
   int q_before_wait;   // apply only: Q may be read before the previous grid completes
+  float* chunk_states; // kChunkStates: [B*H][nchunks][kStateFloats], chunk c's own (S, z)
+  int nchunks;         // kChunkStates: ceil(N / 128)
 };
 
 template <int kRope, int kPh>
@@ -142,6 +148,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
   constexpr bool kRed = (kPh & kReduceOnly) != 0;
   constexpr bool kApp = (kPh & kApplyOnly) != 0;
   constexpr bool kCl = kPh == kClusterLayer;
+  constexpr bool kCh = kPh == kChunkStates;
   constexpr int kNS = LayerCfg<kRope, kPh>::kNS;
   using Smem = typename LayerCfg<kRope, kPh>::Smem;
   using AC = ApplyCfg<kRope>;
@@ -193,7 +200,9 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
     }
     for (int w = 0; w < kApWG; ++w) {
       mbar_init(&t_full[w], 1);
-      mbar_init(&t_empty[w], 1);
+      // kChunkStates uses t_full/t_empty[0..1] for its two chunk accumulators;
+      // t_empty then counts the four epilogue warps
+      mbar_init(&t_empty[w], kCh ? 4 : 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
@@ -223,6 +232,13 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
     }
   }
   if (kRope == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kMath);
+  if (kCh && tid >= 64 && tid < 64 + 256) {
+    // a 4 KB tile of bf16 ones: the B operand whose product with phi(K)^T is
+    // the key sum of every dim
+    st_shared_v4(smem_u32(smem + Smem::zop) + (tid - 64) * 16,
+                 make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u));
+    fence_proxy_async_smem();
+  }
   __syncthreads();
   // cluster layer: every CTA's barriers are initialised before any other CTA
   // may arrive on them
@@ -327,20 +343,33 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       int pos = 0;
       bool ok = true;
       const uint32_t id_red = idesc_bf16_f32(128, 128, 1, 1);
+      const uint32_t id_z = idesc_bf16_f32(128, 16, 1, 1);
+      const uint64_t ones_d = smem_desc_sw128(sbase + Smem::zop, 2048, 1024);
       for (int i = 0; i < nA; ++i, ++pos) {
         const int s = pos % kNS;
+        // kChunkStates: chunk c = stages 2c, 2c + 1 accumulates in TMEM block
+        // c & 1 (state in 128 columns, key sums in the next 16), afresh
+        const int c = i >> 1, cb = c & 1;
+        const bool first = (i & 1) == 0;
+        if (kCh && first &&
+            !(ok = mbar_wait(&t_empty[cb], ((c >> 1) & 1) ^ 1, abort_flag, &g_tc_error, kErrWait)))
+          break;
         if (!(ok = mbar_wait(&ready_a[s], (i / kNS) & 1, abort_flag, &g_tc_error, kErrWait)))
           break;
         tc_fence_after();
         const uint32_t st = sbase + Smem::stages + s * kStageBytes;
+        const uint32_t acc = kCh ? tmem + cb * 160 : tmem;
 #pragma unroll
         for (int kk = 0; kk < kRedT / 16; ++kk) {
           // 16 tokens = two 8-row groups of 128 bytes; LBO = the second 64-dim box
           const uint64_t ad = smem_desc_sw128(st + kk * 2048, kRedBox, 1024);
           const uint64_t bd = smem_desc_sw128(st + 2 * kRedBox + kk * 2048, kRedBox, 1024);
-          mma_bf16(tmem, ad, bd, id_red, (i > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t accum = kCh ? ((first && kk == 0) ? 0u : 1u) : ((i > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16(acc, ad, bd, id_red, accum);
+          if (kCh) mma_bf16(acc + 128, ad, ones_d, id_z, accum);  // key sums
         }
         mma_commit(&empty[s]);
+        if (kCh && (!first || i == nA - 1)) mma_commit(&t_full[cb]);
       }
       if (kRed) mma_commit(acc_full);
       if (ok && kApp && nB > 0) ok = mbar_wait(b_ready, 0, abort_flag, &g_tc_error, kErrWait);
@@ -403,6 +432,34 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       for (int e = 0; e < 8; ++e) zacc[e] = make_float2(0.0f, 0.0f);
       TokPos tp = {0, 0, 0};
       if (kRope != kNoRope) tp = token_pos(p.rope, n_begin + rg);
+      // kChunkStates: warps 2..5 (TMEM lane quadrant q = head q of the group)
+      // copy each finished chunk's (S, z) from TMEM to the chunk-state buffer,
+      // one stage after the chunk's last stage so its MMAs are done by then
+      const int nch = (nA + 1) / 2;
+      int next_chunk = 0;
+      auto chunk_epilogue = [&](int c) {
+        const int q = warp & 3, cb = c & 1;
+        bool got = mbar_wait(&t_full[cb], (c >> 1) & 1, abort_flag, &g_tc_error, kErrWait);
+        got = __all_sync(0xffffffffu, got);  // tcgen05.ld is warp-collective
+        float v[32], zv[8];
+        if (got) {
+          tc_fence_after();
+          const uint32_t base = tmem + (static_cast<uint32_t>(32 * q) << 16) + cb * 160;
+          tmem_ld_32x32b_x32(base + 32 * q, v);
+          tmem_ld_32x32b_x8(base + 128, zv);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&t_empty[cb]);
+        if (got && h0 + q < p.H) {
+          float* dst = a.chunk_states +
+                       ((cidx + q) * a.nchunks + n_begin / kTileTokens + c) * kStateFloats;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + lane * kD + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          dst[kD * kD + lane] = zv[0];
+        }
+      };
       for (int i = 0; i < nA; ++i) {
         const int s = i % kNS;
         if (!mbar_wait(&full[s], (i / kNS) & 1, abort_flag, &g_tc_error, kErrWait)) {
@@ -461,7 +518,18 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
         st_shared_v4(a1, u1);
         fence_proxy_async_smem();
         mbar_arrive(&ready_a[s]);
+        if (kCh && warp >= 2 && warp < 6) {
+          // chunk c ends at stage min(2c + 1, nA - 1)
+          while (next_chunk < nch && min(2 * next_chunk + 1, nA - 1) <= i - 1)
+            chunk_epilogue(next_chunk++);
+        }
       }
+      if (kCh) {
+        if (warp >= 2 && warp < 6 && alive)
+          while (next_chunk < nch) chunk_epilogue(next_chunk++);
+        alive = !bar_any(kBarMath, kMath, !alive || *abort_flag);
+      }
+      if (!kCh) {
       {
         // the warp's 16 key sums over its 32 rows (fixed butterfly order);
         // lane 0 leaves them in zred[wi][16]
@@ -514,6 +582,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
         else if (h0 + q < p.H)
           a.partials[((cidx + q) * p.splits + blockIdx.x) * kStateFloats + kD * kD + d] = sum;
       }
+      }  // !kCh
       tc_fence_before();
     }
 
@@ -571,7 +640,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       if (mt == 0)
         for (uint32_t r = 0; r < ncta; ++r) mbar_arrive_remote(mapa_shared(smem_u32(done), r));
     }
-    if (kRed && !kCl) {
+    if (kRed && !kCl && !kCh) {
       // ---- second phase of the reduce. The named barrier orders each math
       // thread's partial stores before the release fence of the arriving
       // thread.
@@ -1050,6 +1119,27 @@ cudaError_t launch_reduce_tc(const Problem& p, const void* K, const void* V, flo
   a.partials = partials;
   a.arrive = counters;
   a.out = out;
+  const dim3 grid(p.splits, (p.H + kGroupHeads - 1) / kGroupHeads, p.B);
+  e = launch_layer(kern, kBytes, grid, s, false, mk, mv, mk, mk, p, rt, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_states_tc(const Problem& p, const void* K, const void* V, float* states,
+                                   int nchunks, cudaStream_t s) {
+  if (p.io != LA_IO_BF16 || p.rope.enabled || p.N <= 0) return cudaErrorNotSupported;
+  CUtensorMap mk, mv;
+  cudaError_t e;
+  if ((e = make_map(&mk, K, p, kRedT)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, V, p, kRedT)) != cudaSuccess) return e;
+  const RopeTable rt = rope_table_for(p);
+  LayerKernel kern = layer_tc<kNoRope, kChunkStates>;
+  const int kBytes = LayerCfg<kNoRope, kChunkStates>::kSmemBytes;
+  if ((e = ensure_smem_attr(12, reinterpret_cast<const void*>(kern), kBytes)) != cudaSuccess)
+    return e;
+  LayerArgs a = {};
+  a.chunk_states = states;
+  a.nchunks = nchunks;
   const dim3 grid(p.splits, (p.H + kGroupHeads - 1) / kGroupHeads, p.B);
   e = launch_layer(kern, kBytes, grid, s, false, mk, mv, mk, mk, p, rt, a);
   if (e != cudaSuccess) return e;

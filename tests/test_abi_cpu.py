@@ -179,3 +179,29 @@ def test_qkv_state_wrapper_checks_shapes():
     with pytest.raises(ValueError):
         la.qkv_state(X, torch.zeros((96, 64), dtype=torch.bfloat16),
                      torch.zeros((95,), dtype=torch.bfloat16))
+
+
+def test_causal_workspace_bytes():
+    # bf16 without RoPE: room for every 128-token chunk's state (4224 bytes a
+    # head), never less than the ordinary workspace
+    s = la.make_shape(1, 16384, 70)
+    n = la.la_causal_workspace_bytes(s)
+    assert n >= la.la_workspace_bytes(s)
+    assert n >= 70 * (16384 // 128) * 4224
+    assert la.la_causal_workspace_bytes(la.make_shape(2, 300, 5)) >= 2 * 5 * 3 * 4224
+    # RoPE or float32 I/O use the ordinary workspace
+    r = la.make_shape(1, 8, 3, rope=True, T=2, Hh=2, W=2)
+    assert la.la_causal_workspace_bytes(r) == la.la_workspace_bytes(r)
+    f = la.make_shape(1, 300, 3, io_dtype="f32")
+    assert la.la_causal_workspace_bytes(f) == la.la_workspace_bytes(f)
+    assert la.la_causal_workspace_bytes(la.make_shape(1, 16, 70, D=64)) == 0
+
+
+def test_causal_attention_refuses_a_short_workspace():
+    s = la.make_shape(1, 16384, 4)
+    short = la.la_workspace_bytes(s)  # enough for la_attention, not for the chunk states
+    assert short < la.la_causal_workspace_bytes(s)
+    st = la._lib.la_causal_attention(ctypes.byref(s), FAKE, FAKE, FAKE, None, None, FAKE + (1 << 30),
+                                     0, FAKE + (2 << 30), short, None)
+    assert st == la.LA_ERR_WORKSPACE
+    assert "la_causal_workspace_bytes" in la.la_last_error()
