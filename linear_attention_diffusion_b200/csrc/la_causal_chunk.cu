@@ -26,10 +26,13 @@
 //   into the same TMEM columns as two bf16 parts (the rounded value and the
 //   rounded remainder: about 16 bits of each weight), 32 columns per block
 //   of 32 keys (16 of each part);
-//   O_h = P_hi V + P_lo V                 A from TMEM, B = V (MN-major, N = 64)
+//   O_h = P_hi V_h + P_lo V_h              A from TMEM, B = V_h (MN-major, N = 32)
 //       + phi(Q_h) (S_hi + S_lo)           S of the prefix in two bf16 parts
-// and the warpgroup divides by the denominator and writes O over the Q box,
-// which the TMA warp stores. Every wait is bounded.
+// and the warpgroup divides by the denominator and writes O over its head's
+// half of the Q box, which the TMA warp stores once both halves are in. The
+// two heads run as separate pipelines (their own barriers; the MMA warp issues
+// P_0(c), P.V_1(c - 1), P_1(c), P.V_0(c), ...), so the tensor core works on one
+// head while the other head's warpgroup masks. Every wait is bounded.
 #include <algorithm>
 
 #include "la_tc_common.cuh"
@@ -43,15 +46,18 @@ namespace {
 
 constexpr int kXT = 128;                    // tokens per chunk
 constexpr int kXBox = kXT * 128;            // [128 tokens][64 dims] bf16 = 16 KB
+constexpr int kXVBox = kXT * 64;            // [128 tokens][32 dims] bf16 = 8 KB
 constexpr int kXStages = 3;
 constexpr int kXMath = 256;                 // two warpgroups, one per head
 constexpr int kXThreads = 64 + kXMath;
 constexpr int kXTmemCols = 512;
-constexpr int kBarBothX = 1;                // named barrier over both warpgroups
+constexpr int kBarHeadX = 1;                // named barriers kBarHeadX + h: one warpgroup
 
-// Stage layout: Q, K, V boxes, then the S operand of the chunk's prefix in two
-// bf16 parts ([hi, lo][32 rows e][128 B]: head h in bytes [64h, 64h + 64) of
-// a row), then the prefix state as copied ([2 heads][32*32 + 32] f32).
+// Stage layout: Q and K boxes (both heads, 128-byte swizzle), V as one box
+// per head ([128 tokens][32 dims], 64-byte swizzle, so that each head's P.V
+// has N = 32), then the S operand of the chunk's prefix in two bf16 parts
+// ([hi, lo][32 rows e][128 B]: head h in bytes [64h, 64h + 64) of a row),
+// then the prefix state as copied ([2 heads][32*32 + 32] f32).
 struct XStage {
   static constexpr int q = 0;
   static constexpr int k = q + kXBox;
@@ -62,15 +68,14 @@ struct XStage {
   static constexpr int stride = (bytes + 1023) / 1024 * 1024;
 };
 
-// TMEM columns: P of head h at 128 h; O of head h at kColO + 64 h (N = 64
-// over both heads' V columns; head h's numerator is its columns 32 h ..).
+// TMEM columns: P of head h at 128 h; O of head h at kColO + 32 h.
 constexpr uint32_t kColO = 256;
 
 struct XSmem {
   static constexpr int stages = 0;
   static constexpr int bars = stages + kXStages * XStage::stride;
-  // full[3] ready[3] bop_ready[3] o_done[3] p_full pm_ready[2] o_full[2] mma_done
-  static constexpr int nbars = 4 * kXStages + 6;
+  // full[3] ready[3][2] o_done[3] p_full[2] pm_ready[2] o_full[2] mma_done
+  static constexpr int nbars = 4 * kXStages + 7;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int bytes = misc + 16;
 };
@@ -109,6 +114,38 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 32 lanes x 32 consecutive fp32 columns without the wait (tmem_ld_wait
+// completes every load issued before it).
+__device__ __forceinline__ void tmem_ld_32x32b_x32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 64-byte swizzle, MN-major operand of 32
+// elements along MN (one swizzle atom, tile base 512-aligned): sbo is the
+// distance between 8-row K groups (8 x 64 B).
+__device__ __forceinline__ uint64_t smem_desc_sw64_mn32(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFF) >> 4);
+  d |= static_cast<uint64_t>((kXVBox >> 4) & 0x3FFF) << 16;  // between MN atoms (one here)
+  d |= static_cast<uint64_t>((512 >> 4) & 0x3FFF) << 32;
+  d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
+  d |= static_cast<uint64_t>(4) << 61;  // 64-byte swizzle
+  return d;
+}
+
 __global__ void __launch_bounds__(kXThreads, 1)
 causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -117,12 +154,11 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + XSmem::bars);
-  uint64_t* ready = full + kXStages;        // Q and K of the chunk ReLU'd (256 arrivals)
-  uint64_t* bop_ready = ready + kXStages;   // the prefix's S operand built (256)
-  uint64_t* o_done = bop_ready + kXStages;  // O written over the Q box (256)
-  uint64_t* p_full = o_done + kXStages;     // P of both heads in TMEM (1)
-  uint64_t* pm_ready = p_full + 1;          // [head] P masked, in two parts, in TMEM (128)
-  uint64_t* o_full = pm_ready + 2;          // [head] O in TMEM (1)
+  uint64_t* ready = full + kXStages;          // [stage][head] Q, K ReLU'd, S operand built (128)
+  uint64_t* o_done = ready + 2 * kXStages;    // [stage] O written over the Q box (256)
+  uint64_t* p_full = o_done + kXStages;       // [head] P in TMEM (1)
+  uint64_t* pm_ready = p_full + 2;            // [head] P masked, in two parts, in TMEM (128)
+  uint64_t* o_full = pm_ready + 2;            // [head] O in TMEM (1)
   uint64_t* mma_done = o_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + XSmem::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + XSmem::misc + 4);
@@ -139,15 +175,15 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (tid == 0) {
     for (int i = 0; i < kXStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&ready[i], kXMath);
-      mbar_init(&bop_ready[i], kXMath);
+      mbar_init(&ready[2 * i], 128);
+      mbar_init(&ready[2 * i + 1], 128);
       mbar_init(&o_done[i], kXMath);
     }
-    mbar_init(p_full, 1);
-    mbar_init(&pm_ready[0], 128);
-    mbar_init(&pm_ready[1], 128);
-    mbar_init(&o_full[0], 1);
-    mbar_init(&o_full[1], 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&p_full[h], 1);
+      mbar_init(&pm_ready[h], 128);
+      mbar_init(&o_full[h], 1);
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -195,6 +231,7 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tma_load_3d(st + XStage::q, &tm_q, &full[s], h0 * 32, y, b);
         tma_load_3d(st + XStage::k, &tm_k, &full[s], h0 * 32, y, b);
         tma_load_3d(st + XStage::v, &tm_v, &full[s], h0 * 32, y, b);
+        tma_load_3d(st + XStage::v + kXVBox, &tm_v, &full[s], h0 * 32 + 32, y, b);
         for (int hh = 0; hh < heads; ++hh)
           bulk_load(st + XStage::state + hh * kStateFloats * 4,
                     a.prefix + ((cidx + hh) * a.nchunks + c_begin + c) * kStateFloats,
@@ -209,50 +246,64 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // ------------------------------------------------------------ MMA
     if (lane == 0) {
       const uint32_t id_p = idesc_bf16_f32(128, 128, 0, 0);
-      const uint32_t id_pv = idesc_bf16_f32(128, 64, 0, 1);
+      const uint32_t id_pv = idesc_bf16_f32(128, 32, 0, 1);
       const uint32_t id_qs = idesc_bf16_f32(128, 32, 0, 0);
-      bool ok = true;
-      for (int c = 0; ok && c < nC; ++c) {
+      auto stage_addr = [&](int c) { return sbase + XSmem::stages + (c % kXStages) * XStage::stride; };
+      // The issue path is kept short (one tcgen05.mma costs tens of cycles to
+      // issue, about as long as a small MMA runs): a stage's descriptors are
+      // built once, and each MMA adds a constant offset (in 16-byte units) to
+      // the start-address field, which cannot carry out of its 14 bits below
+      // 256 KB.
+      //
+      // P_h = phi(Q_h) phi(K_h)^T of chunk c. It overwrites the P columns that
+      // head h's P.V of chunk c - 1 read; those were issued earlier by this
+      // thread and run in order.
+      auto issue_p = [&](int c, int h) -> bool {
         const int s = c % kXStages;
-        const uint32_t par = (c / kXStages) & 1;
-        const uint32_t st = sbase + XSmem::stages + s * XStage::stride;
-        const uint32_t qb = st + XStage::q, kb = st + XStage::k, vb = st + XStage::v;
-        const uint32_t bop = st + XStage::bop;
-        if (!(ok = mbar_wait(&ready[s], par, abort_flag, err, kErrWait))) break;
-        // P of chunk c overwrites the P columns the previous chunk's P.V MMAs
-        // read; those were issued earlier by this thread and run in order
+        if (!mbar_wait(&ready[2 * s + h], (c / kXStages) & 1, abort_flag, err, kErrWait)) return false;
         tc_fence_after();
+        const uint32_t st = stage_addr(c);
+        const uint64_t dq = smem_desc_sw128(st + XStage::q, 16, 1024);
+        const uint64_t dk = smem_desc_sw128(st + XStage::k, 16, 1024);
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+        for (int kk = 0; kk < 2; ++kk)
+          mma_bf16(tmem + 128 * h, dq + (h * 64 + kk * 32) / 16, dk + (h * 64 + kk * 32) / 16, id_p, kk);
+        mma_commit(&p_full[h]);
+        return true;
+      };
+      // O_h = P_hi V_h + P_lo V_h (A from TMEM: keys 16 kk .. of block kk / 2)
+      //     + phi(Q_h) (S_hi + S_lo) of the prefix
+      auto issue_pv = [&](int c, int h) -> bool {
+        if (!mbar_wait(&pm_ready[h], c & 1, abort_flag, err, kErrWait)) return false;
+        tc_fence_after();
+        const uint32_t st = stage_addr(c);
+        const uint64_t dv = smem_desc_sw64_mn32(st + XStage::v + h * kXVBox);
+        const uint64_t dq = smem_desc_sw128(st + XStage::q, 16, 1024);
+        const uint64_t db = smem_desc_sw128(st + XStage::bop, 16, 1024);
+        const uint32_t d = tmem + kColO + 32 * h;
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+          for (int kk = 0; kk < kXT / 16; ++kk)
+            mma_bf16_tmem_a(d, tmem + 128 * h + 32 * (kk >> 1) + 16 * part + 8 * (kk & 1),
+                            dv + kk * 1024 / 16, id_pv, (part > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            mma_bf16(tmem + 128 * h, smem_desc_sw128(qb + h * 64 + kk * 32, 16, 1024),
-                     smem_desc_sw128(kb + h * 64 + kk * 32, 16, 1024), id_p, kk);
-        mma_commit(p_full);
-        for (int h = 0; ok && h < 2; ++h) {
-          // O_h = P_hi V + P_lo V (A from TMEM: keys 16 kk .. of block kk / 2)
-          if (!(ok = mbar_wait(&pm_ready[h], c & 1, abort_flag, err, kErrWait))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int part = 0; part < 2; ++part)
-#pragma unroll
-            for (int kk = 0; kk < kXT / 16; ++kk)
-              mma_bf16_tmem_a(tmem + kColO + 64 * h,
-                              tmem + 128 * h + 32 * (kk >> 1) + 16 * part + 8 * (kk & 1),
-                              smem_desc_sw128(vb + kk * 2048, kXBox, 1024), id_pv,
-                              (part > 0 || kk > 0) ? 1u : 0u);
-          // + phi(Q_h) S of the prefix, S = S_hi + S_lo
-          if (h == 0 && !(ok = mbar_wait(&bop_ready[s], par, abort_flag, err, kErrWait))) break;
-#pragma unroll
-          for (int part = 0; part < 2; ++part)
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk)
-              mma_bf16(tmem + kColO + 64 * h + 32 * h,
-                       smem_desc_sw128(qb + h * 64 + kk * 32, 16, 1024),
-                       smem_desc_sw128(bop + part * 4096 + h * 64 + kk * 32, 16, 1024), id_qs, 1u);
-          mma_commit(&o_full[h]);
-        }
+            mma_bf16(d, dq + (h * 64 + kk * 32) / 16, db + (part * 4096 + h * 64 + kk * 32) / 16,
+                     id_qs, 1u);
+        mma_commit(&o_full[h]);
+        return true;
+      };
+      bool ok = true;
+      for (int c = 0; ok && c < nC; ++c) {
+        ok = issue_p(c, 0);
+        if (ok && c > 0) ok = issue_pv(c - 1, 1);
+        if (ok) ok = issue_p(c, 1);
+        if (ok) ok = issue_pv(c, 0);
       }
+      if (ok && nC > 0) issue_pv(nC - 1, 1);
       mma_commit(mma_done);
       mbar_drain(mma_done, 0, err, kErrWait);
     }
@@ -275,11 +326,11 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // ReLU of this head's Q and K columns of chunk c in place, then the
     // prefix's S as the B operand: row e holds S[0..31][e] of this head in two
     // bf16 parts (thread wt: row e = wt / 4, dims 8 (wt % 4) ..). False when
-    // a wait gave up (decided by both warpgroups together).
+    // a wait gave up (decided by the warpgroup together).
     auto prepare = [&](int c) -> bool {
       const int s = c % kXStages;
       const bool ok = mbar_wait(&full[s], (c / kXStages) & 1, abort_flag, err, kErrWait);
-      if (bar_any(kBarBothX, kXMath, !ok || *abort_flag)) return false;
+      if (bar_any(kBarHeadX + h, 128, !ok || *abort_flag)) return false;
       const uint32_t st = stage_of(c);
       const uint32_t qb = st + XStage::q, kb = st + XStage::k;
 #pragma unroll
@@ -293,8 +344,6 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         w.x = relu_bf16x2(w.x); w.y = relu_bf16x2(w.y); w.z = relu_bf16x2(w.z); w.w = relu_bf16x2(w.w);
         st_shared_v4(ak, w);
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&ready[s]);
       {
         const float* pre = prefix_of(c);
         const int e = wt >> 2, c4 = wt & 3;
@@ -311,7 +360,7 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         st_shared_v4(bop + 4096 + sw128_offset(e, h * 4 + c4), pack8(lo));
       }
       fence_proxy_async_smem();
-      mbar_arrive(&bop_ready[s]);
+      mbar_arrive(&ready[2 * s + h]);
       return true;
     };
 
@@ -322,27 +371,44 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float* pre = prefix_of(c);
 
       // ---- P: mask j <= i, row sums, two bf16 parts back into TMEM
-      bool ok = mbar_wait(p_full, c & 1, abort_flag, err, kErrWait);
+      bool ok = mbar_wait(&p_full[h], c & 1, abort_flag, err, kErrWait);
       tc_fence_after();
-      if (bar_any(kBarBothX, kXMath, !ok || *abort_flag)) break;
+      if (bar_any(kBarHeadX + h, 128, !ok || *abort_flag)) break;
+      // key block q of this warp's rows (32 quad .. 32 quad + 31): below the
+      // diagonal block every key is kept, above it none (zeros, no load); the
+      // loads of blocks (0, 1) and of (2, 3) are issued together
       float psum = 0.0f;
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        float v[32];
-        tmem_ld_32x32b_x32(tmem + lq + 128 * h + 32 * q, v);
-        uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int j = q * 32 + 2 * e;
-          const float x0 = j <= row ? v[2 * e] : 0.0f;
-          const float x1 = j + 1 <= row ? v[2 * e + 1] : 0.0f;
-          psum += x0 + x1;
-          hi[e] = pack_bf16x2(x0, x1);
-          const float h0f = __uint_as_float(hi[e] << 16), h1f = __uint_as_float(hi[e] & 0xffff0000u);
-          lo[e] = pack_bf16x2(x0 - h0f, x1 - h1f);
+      for (int q2 = 0; q2 < 4; q2 += 2) {
+        uint32_t r[2][32];
+        if (q2 <= quad) {
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+            if (q2 + t <= quad) tmem_ld_32x32b_x32_nowait(tmem + lq + 128 * h + 32 * (q2 + t), r[t]);
+          tmem_ld_wait();
         }
-        tmem_st_32x32b_x16(tmem + lq + 128 * h + 32 * q, hi);
-        tmem_st_32x32b_x16(tmem + lq + 128 * h + 32 * q + 16, lo);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int q = q2 + t;
+          uint32_t hi[16], lo[16];
+          if (q > quad) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
+          } else {
+            const int lim = q < quad ? 32 : lane + 1;  // keys of the block this row keeps
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float x0 = 2 * e < lim ? __uint_as_float(r[t][2 * e]) : 0.0f;
+              const float x1 = 2 * e + 1 < lim ? __uint_as_float(r[t][2 * e + 1]) : 0.0f;
+              psum += x0 + x1;
+              hi[e] = pack_bf16x2(x0, x1);
+              const float h0f = __uint_as_float(hi[e] << 16), h1f = __uint_as_float(hi[e] & 0xffff0000u);
+              lo[e] = pack_bf16x2(x0 - h0f, x1 - h1f);
+            }
+          }
+          tmem_st_32x32b_x16(tmem + lq + 128 * h + 32 * q, hi);
+          tmem_st_32x32b_x16(tmem + lq + 128 * h + 32 * q + 16, lo);
+        }
       }
       tmem_st_wait();
       tc_fence_before();
@@ -363,10 +429,10 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // ---- O = numerator / den over this head's columns of the Q box
       ok = mbar_wait(&o_full[h], c & 1, abort_flag, err, kErrWait);
       tc_fence_after();
-      if (bar_any(kBarBothX, kXMath, !ok || *abort_flag)) break;
+      if (bar_any(kBarHeadX + h, 128, !ok || *abort_flag)) break;
       {
         float v[32];
-        tmem_ld_32x32b_x32(tmem + lq + kColO + 64 * h + 32 * h, v);
+        tmem_ld_32x32b_x32(tmem + lq + kColO + 32 * h, v);
         const float inv = 1.0f / den;
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
@@ -390,44 +456,81 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   }
 }
 
-// Exclusive prefix over the chunks, per head and float4 column, in chunk
-// order: chunk c's state becomes carry + the sum of the chunks before it.
-// update: the carry becomes carry + the sum of all chunks.
-__global__ void __launch_bounds__(256)
-chunk_prefix(float* states, int bh_count, int nchunks, float* S_carry, float* z_carry, int update) {
+// Exclusive prefix over the chunks, per head and float4 column: chunk c's
+// state becomes carry + the sum of the chunks before it (update: the carry
+// becomes carry + the sum of all chunks). The chunk axis is cut into `segs`
+// segments (a power of two, so that a segment holds about kPrefBatch chunks);
+// a block covers 256 / segs consecutive float4 columns, each warp's lanes
+// consecutive columns of one segment. Each thread sums its segment, the block
+// exchanges the segment totals in shared memory, and each thread writes
+// carry + the earlier segments' totals + the earlier chunks of its own
+// segment. The sum order is fixed by the shape.
+constexpr int kPrefThreads = 256, kPrefMaxSeg = 16, kPrefBatch = 8;
+
+int prefix_segments(int nchunks) {
+  int segs = 1;
+  while (segs < kPrefMaxSeg && segs * kPrefBatch < nchunks) segs *= 2;
+  return segs;
+}
+
+__global__ void __launch_bounds__(kPrefThreads, 4)
+chunk_prefix(float* states, int bh_count, int nchunks, int segs, float* S_carry, float* z_carry,
+             int update) {
   constexpr int kVec = kStateFloats / 4;
-  const long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  constexpr int kStride = kStateFloats / 4;  // float4 between consecutive chunks
+  __shared__ float4 seg_total[kPrefThreads];
+  const int cpb = kPrefThreads / segs;
+  const int col = threadIdx.x % cpb, seg = threadIdx.x / cpb;
+  const long long g = static_cast<long long>(blockIdx.x) * cpb + col;
   pdl_wait();
   if (threadIdx.x == 0) pdl_trigger();
-  if (g >= static_cast<long long>(bh_count) * kVec) return;
-  const int bh = static_cast<int>(g / kVec), i = static_cast<int>(g % kVec) * 4;
+  const bool live = g < static_cast<long long>(bh_count) * kVec;
+  const int bh = live ? static_cast<int>(g / kVec) : 0;
+  const int i = live ? static_cast<int>(g % kVec) * 4 : 0;
   const bool is_s = i < kD * kD;
-  float* carry = S_carry == nullptr ? nullptr
-                                    : (is_s ? S_carry + static_cast<size_t>(bh) * kD * kD + i
-                                            : z_carry + static_cast<size_t>(bh) * kD + (i - kD * kD));
-  float4 acc = carry != nullptr ? *reinterpret_cast<const float4*>(carry)
-                                : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  float4* col = reinterpret_cast<float4*>(states + static_cast<size_t>(bh) * nchunks * kStateFloats + i);
-  constexpr int kStride = kStateFloats / 4;  // float4 between consecutive chunks
-  // 16 chunks' loads in flight at a time (the chain of adds is in chunk order)
-  constexpr int kBatch = 16;
-  int c = 0;
-  for (; c + kBatch <= nchunks; c += kBatch) {
-    float4 d[kBatch];
+  float* carry = !live || S_carry == nullptr
+                     ? nullptr
+                     : (is_s ? S_carry + static_cast<size_t>(bh) * kD * kD + i
+                             : z_carry + static_cast<size_t>(bh) * kD + (i - kD * kD));
+  float4* colp = reinterpret_cast<float4*>(states + static_cast<size_t>(bh) * nchunks * kStateFloats + i);
+  const int len = (nchunks + segs - 1) / segs;
+  const int c0 = min(nchunks, seg * len), c1 = live ? min(nchunks, c0 + len) : c0;
+  auto add4 = [](float4 x, float4 y) { return make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w); };
+  const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+
+  // the segment's sum (kept in registers when the segment is one batch)
+  float4 d[kPrefBatch];
+  float4 sum = zero;
+  for (int c = c0; c < c1; c += kPrefBatch) {
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) d[k] = __ldcg(col + static_cast<size_t>(c + k) * kStride);
+    for (int k = 0; k < kPrefBatch; ++k)
+      d[k] = c + k < c1 ? __ldcg(colp + static_cast<size_t>(c + k) * kStride) : zero;
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      __stcg(col + static_cast<size_t>(c + k) * kStride, acc);
-      acc = make_float4(acc.x + d[k].x, acc.y + d[k].y, acc.z + d[k].z, acc.w + d[k].w);
+    for (int k = 0; k < kPrefBatch; ++k) sum = add4(sum, d[k]);
+  }
+  seg_total[threadIdx.x] = sum;
+  __syncthreads();
+  float4 acc = carry != nullptr ? *reinterpret_cast<const float4*>(carry) : zero;
+  for (int t = 0; t < seg; ++t) acc = add4(acc, seg_total[t * cpb + col]);
+
+  // the exclusive prefixes of the segment's chunks (a second read only when
+  // the segment is longer than one batch)
+  const bool one_batch = c1 - c0 <= kPrefBatch;
+  for (int c = c0; c < c1; c += kPrefBatch) {
+    if (!one_batch) {
+#pragma unroll
+      for (int k = 0; k < kPrefBatch; ++k)
+        d[k] = c + k < c1 ? __ldcg(colp + static_cast<size_t>(c + k) * kStride) : zero;
     }
+#pragma unroll
+    for (int k = 0; k < kPrefBatch; ++k)
+      if (c + k < c1) {
+        __stcg(colp + static_cast<size_t>(c + k) * kStride, acc);
+        acc = add4(acc, d[k]);
+      }
   }
-  for (; c < nchunks; ++c) {
-    const float4 d = __ldcg(col + static_cast<size_t>(c) * kStride);
-    __stcg(col + static_cast<size_t>(c) * kStride, acc);
-    acc = make_float4(acc.x + d.x, acc.y + d.y, acc.z + d.z, acc.w + d.w);
-  }
-  if (update && carry != nullptr) *reinterpret_cast<float4*>(carry) = acc;
+  // the last segment ends on the sum of everything (an empty one adds nothing)
+  if (update && carry != nullptr && seg == segs - 1) *reinterpret_cast<float4*>(carry) = acc;
 }
 
 cudaError_t launch_pdl_x(const void* fn, void** args, dim3 grid, dim3 block, int smem,
@@ -443,6 +546,24 @@ cudaError_t launch_pdl_x(const void* fn, void** args, dim3 grid, dim3 block, int
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+// V as [B][N][H*32] bf16 with a box of one head: 32 dims x 128 tokens x 1,
+// 64-byte swizzle.
+cudaError_t make_map_head(CUtensorMap* m, const void* base, const Problem& p) {
+  cudaError_t e = get_encoder();
+  if (e != cudaSuccess) return e;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p.H) * kD, static_cast<cuuint64_t>(p.N),
+                              static_cast<cuuint64_t>(p.B)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p.H) * kD * 2,
+                                 static_cast<cuuint64_t>(p.N) * p.H * kD * 2};
+  const cuuint32_t box[3] = {kD, static_cast<cuuint32_t>(kXT), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -472,17 +593,20 @@ cudaError_t launch_causal_chunks(const Problem& p, const void* Q, const void* K,
     float* sc = S_carry;
     float* zc = z_carry;
     int up = update;
-    void* args[] = {&st, &bh, &nc, &sc, &zc, &up};
-    const long long threads = static_cast<long long>(bh) * (kStateFloats / 4);
-    const dim3 grid(static_cast<unsigned>((threads + 255) / 256));
-    e = launch_pdl_x(reinterpret_cast<const void*>(chunk_prefix), args, grid, dim3(256), 0, s);
+    int segs = prefix_segments(nchunks);
+    void* args[] = {&st, &bh, &nc, &segs, &sc, &zc, &up};
+    const long long cols = static_cast<long long>(bh) * (kStateFloats / 4);
+    const int cpb = kPrefThreads / segs;
+    const dim3 grid(static_cast<unsigned>((cols + cpb - 1) / cpb));
+    e = launch_pdl_x(reinterpret_cast<const void*>(chunk_prefix), args, grid, dim3(kPrefThreads),
+                     0, s);
     if (e != cudaSuccess) return e;
   }
   // (3) every chunk on its own
   CUtensorMap mq, mk, mv, mo;
   if ((e = make_map(&mq, Q, p, kXT)) != cudaSuccess) return e;
   if ((e = make_map(&mk, K, p, kXT)) != cudaSuccess) return e;
-  if ((e = make_map(&mv, V, p, kXT)) != cudaSuccess) return e;
+  if ((e = make_map_head(&mv, V, p)) != cudaSuccess) return e;
   if ((e = make_map(&mo, O, p, kXT)) != cudaSuccess) return e;
   if ((e = ensure_smem_attr(0, reinterpret_cast<const void*>(causal_chunk_tc), kXSmemBytes)) !=
       cudaSuccess)
