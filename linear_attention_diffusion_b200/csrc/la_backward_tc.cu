@@ -282,7 +282,7 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       bool ok = nT == 0 || mbar_wait(b_ready, 0, abort_flag, err, kErrWait);
       const uint32_t id_t = idesc_bf16_f32(128, 32, 0, 0);
       const uint32_t id_s = idesc_bf16_f32(128, 64, 1, 1);
-      const uint32_t bop = sbase + QSmem::bop;
+      const uint64_t bop0 = smem_desc_sw128(sbase + QSmem::bop, 16, 1024);
       // Without RoPE, phi(Q) = ReLU(Q) is in place after the transform, so both
       // MMAs of a tile go at once and the epilogue may then write dQ over the
       // dnum box. With RoPE, MMA 2 of tile i - 1 (after the warpgroup has
@@ -292,17 +292,18 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         if (!(ok = mbar_wait(&ready_t[s], (i / kBStages) & 1, abort_flag, err, kErrWait))) break;
         tc_fence_after();
         const uint32_t st = sbase + QSmem::stages + s * kBTile;
+        const uint64_t g0 = smem_desc_sw128(st + kBBox, 16, 1024);
 #pragma unroll
         for (int hh = 0; hh < kPair; ++hh)
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            mma_bf16(tmem + 64 * s + hh * 32,
-                     smem_desc_sw128(st + kBBox + hh * 64 + kk * 32, 16, 1024),
-                     smem_desc_sw128(bop + hh * 64 + kk * 32, 16, 1024), id_t, kk);
+            mma_bf16(tmem + 64 * s + hh * 32, desc_at(g0, hh * 64 + kk * 32),
+                     desc_at(bop0, hh * 64 + kk * 32), id_t, kk);
+        const uint64_t a0 = smem_desc_sw128(st, kBBox, 1024);
+        const uint64_t b0 = smem_desc_sw128(st + kBBox, kBBox, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBT / 16; ++kk)
-          mma_bf16(tmem + kColDS, smem_desc_sw128(st + kk * 2048, kBBox, 1024),
-                   smem_desc_sw128(st + kBBox + kk * 2048, kBBox, 1024), id_s,
+          mma_bf16(tmem + kColDS, desc_at(a0, kk * 2048), desc_at(b0, kk * 2048), id_s,
                    (i > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&t_full[s]);
       }
@@ -311,13 +312,13 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           const int s = i % kBStages;
           if (!(ok = mbar_wait(&ready_t[s], (i / kBStages) & 1, abort_flag, err, kErrWait))) break;
           tc_fence_after();
-          const uint32_t st = sbase + QSmem::stages + s * kBTile;
+          const uint64_t g0 = smem_desc_sw128(sbase + QSmem::stages + s * kBTile + kBBox, 16, 1024);
 #pragma unroll
           for (int hh = 0; hh < kPair; ++hh) {
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
-              const uint64_t ad = smem_desc_sw128(st + kBBox + hh * 64 + kk * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(bop + hh * 64 + kk * 32, 16, 1024);
+              const uint64_t ad = desc_at(g0, hh * 64 + kk * 32);
+              const uint64_t bd = desc_at(bop0, hh * 64 + kk * 32);
               mma_bf16(tmem + 64 * s + hh * 32, ad, bd, id_t, kk);
             }
           }
@@ -329,12 +330,14 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           if (!(ok = mbar_wait(&ready_s[s], (k / kBStages) & 1, abort_flag, err, kErrWait))) break;
           tc_fence_after();
           const uint32_t st = sbase + QSmem::stages + s * kBTile;
+          // A: phi(Q) as M = 128 dims; its second 64-dim atom (LBO) is the
+          // dO box, whose rows of the product are not used
+          const uint64_t a0 = smem_desc_sw128(st, kBBox, 1024);
+          const uint64_t b0 = smem_desc_sw128(st + kBBox, kBBox, 1024);
 #pragma unroll
           for (int kk = 0; kk < kBT / 16; ++kk) {
-            // A: phi(Q) as M = 128 dims; its second 64-dim atom (LBO) is the
-            // dO box, whose rows of the product are not used
-            const uint64_t ad = smem_desc_sw128(st + kk * 2048, kBBox, 1024);
-            const uint64_t bd = smem_desc_sw128(st + kBBox + kk * 2048, kBBox, 1024);
+            const uint64_t ad = desc_at(a0, kk * 2048);
+            const uint64_t bd = desc_at(b0, kk * 2048);
             mma_bf16(tmem + kColDS, ad, bd, id_s, (k > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&s2_done[s]);  // the warpgroup then writes dQ over the dnum box
@@ -696,7 +699,8 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     if (lane == 0) {
       bool ok = nT == 0 || mbar_wait(b_ready, 0, abort_flag, err, kErrWait);
       const uint32_t id = idesc_bf16_f32(128, 32, 0, 0);
-      const uint32_t bop1 = sbase + KVSmem::bop1, bop2 = sbase + KVSmem::bop2;
+      const uint64_t bop1d = smem_desc_sw128(sbase + KVSmem::bop1, 16, 1024);
+      const uint64_t bop2d = smem_desc_sw128(sbase + KVSmem::bop2, 16, 1024);
       // t_empty[s] completes twice per tile (MMA 1's and MMA 2's results
       // read), so the waits alternate parity 1 (before MMA 1) and 0 (before
       // MMA 2). MMA 2 of tile i - 1 is issued after MMA 1 of tile i.
@@ -706,14 +710,14 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
           if (!(ok = mbar_wait(&ready[s], (i / kBStages) & 1, abort_flag, err, kErrWait))) break;
           if (!(ok = mbar_wait(&t_empty[s], 1, abort_flag, err, kErrWait))) break;
           tc_fence_after();
-          const uint32_t st = sbase + KVSmem::stages + s * kBTile;
+          const uint64_t v0 = smem_desc_sw128(sbase + KVSmem::stages + s * kBTile + kBBox, 16, 1024);
 #pragma unroll
           for (int hh = 0; hh < kPair; ++hh) {
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
               // dphi(K)[n][d] = sum_e V[n][e] dS[d][e]
-              const uint64_t av = smem_desc_sw128(st + kBBox + hh * 64 + kk * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(bop1 + hh * 64 + kk * 32, 16, 1024);
+              const uint64_t av = desc_at(v0, hh * 64 + kk * 32);
+              const uint64_t bd = desc_at(bop1d, hh * 64 + kk * 32);
               mma_bf16(tmem + s * 64 + hh * 32, av, bd, id, kk);
             }
           }
@@ -724,14 +728,14 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
           const int s = k % kBStages;
           if (!(ok = mbar_wait(&t_empty[s], 0, abort_flag, err, kErrWait))) break;
           tc_fence_after();
-          const uint32_t st = sbase + KVSmem::stages + s * kBTile;
+          const uint64_t k0 = smem_desc_sw128(sbase + KVSmem::stages + s * kBTile, 16, 1024);
 #pragma unroll
           for (int hh = 0; hh < kPair; ++hh) {
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
               // dV[n][e] = sum_d phi(K)[n][d] dS[d][e]
-              const uint64_t ak = smem_desc_sw128(st + hh * 64 + kk * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(bop2 + hh * 64 + kk * 32, 16, 1024);
+              const uint64_t ak = desc_at(k0, hh * 64 + kk * 32);
+              const uint64_t bd = desc_at(bop2d, hh * 64 + kk * 32);
               mma_bf16(tmem + s * 64 + hh * 32, ak, bd, id, kk);
             }
           }

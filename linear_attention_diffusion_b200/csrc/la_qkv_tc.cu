@@ -420,10 +420,12 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
             break;
           tc_fence_after();
           const uint32_t st = sbase + QSmem::stages + s * kQStageBytes;
+          const uint64_t a0 = smem_desc_sw128(st, 16, 1024);
+          const uint64_t b0 = smem_desc_sw128(st + kBoxBytes, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < kKBlk / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(st + kk * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(st + kBoxBytes + kk * 32, 16, 1024);
+            const uint64_t ad = desc_at(a0, kk * 32);
+            const uint64_t bd = desc_at(b0, kk * 32);
             mma_pair_bf16(acc, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
           }
           mma_pair_commit_both(&empty[s]);  // both CTAs' stages are free again

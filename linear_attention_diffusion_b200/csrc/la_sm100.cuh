@@ -349,6 +349,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// The descriptor of the operand `bytes` past the one `d` describes: the
+// start-address field holds the address in 16-byte units, and shared-memory
+// addresses stay below 256 KB, so the add cannot carry out of the field. One
+// descriptor per tile plus constant offsets keeps the MMA issue path short
+// (a tcgen05.mma costs tens of cycles to issue; the arithmetic around it
+// should not add more).
+__device__ __forceinline__ uint64_t desc_at(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
 // Instruction descriptor of kind::f16: bf16 A and B, fp32 D, M x N, with the
 // major-ness (0 = K-major, 1 = MN-major) of A and B.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major,

@@ -359,11 +359,13 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
         tc_fence_after();
         const uint32_t st = sbase + Smem::stages + s * kStageBytes;
         const uint32_t acc = kCh ? tmem + cb * 160 : tmem;
+        // 16 tokens = two 8-row groups of 128 bytes; LBO = the second 64-dim box
+        const uint64_t a0 = smem_desc_sw128(st, kRedBox, 1024);
+        const uint64_t b0 = smem_desc_sw128(st + 2 * kRedBox, kRedBox, 1024);
 #pragma unroll
         for (int kk = 0; kk < kRedT / 16; ++kk) {
-          // 16 tokens = two 8-row groups of 128 bytes; LBO = the second 64-dim box
-          const uint64_t ad = smem_desc_sw128(st + kk * 2048, kRedBox, 1024);
-          const uint64_t bd = smem_desc_sw128(st + 2 * kRedBox + kk * 2048, kRedBox, 1024);
+          const uint64_t ad = desc_at(a0, kk * 2048);
+          const uint64_t bd = desc_at(b0, kk * 2048);
           const uint32_t accum = kCh ? ((first && kk == 0) ? 0u : 1u) : ((i > 0 || kk > 0) ? 1u : 0u);
           mma_bf16(acc, ad, bd, id_red, accum);
           if (kCh) mma_bf16(acc + 128, ad, ones_d, id_z, accum);  // key sums
@@ -375,8 +377,8 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
       if (ok && kApp && nB > 0) ok = mbar_wait(b_ready, 0, abort_flag, &g_tc_error, kErrWait);
       const uint32_t id_ap = idesc_bf16_f32(128, 32, 0, 0);
       const uint32_t id_den = idesc_bf16_f32(128, 16, 0, 0);
-      const uint32_t bop = sbase + Smem::bop;
-      const uint32_t zop = sbase + Smem::zop;
+      const uint64_t bop0 = smem_desc_sw128(sbase + Smem::bop, 16, 1024);
+      const uint64_t zop0 = smem_desc_sw128(sbase + Smem::zop, 16, 1024);
       for (int j = 0; ok && j < nB; ++j, ++pos) {
         const int s = pos % kNS;
         const int w = j % AC::kWG;
@@ -386,15 +388,15 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
                              kErrWait)))
           break;
         tc_fence_after();
-        const uint32_t st = sbase + Smem::stages + s * kStageBytes;
         const uint32_t acc = tmem + w * AC::kCols;
+        const uint64_t q0 = smem_desc_sw128(sbase + Smem::stages + s * kStageBytes, 16, 1024);
 #pragma unroll
         for (int hh = 0; hh < kGroupHeads; ++hh) {
           const uint32_t koff = (hh & 1) * 64;
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
-            const uint64_t ad = smem_desc_sw128(st + (hh >> 1) * kApBox + koff + kk * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(bop + (hh >> 1) * 4096 + koff + kk * 32, 16, 1024);
+            const uint64_t ad = desc_at(q0, (hh >> 1) * kApBox + koff + kk * 32);
+            const uint64_t bd = desc_at(bop0, (hh >> 1) * 4096 + koff + kk * 32);
             mma_bf16(acc + hh * 32, ad, bd, id_ap, kk);
           }
         }
@@ -402,8 +404,8 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
           // the denominators: ReLU(Q) (all 128 dims) times the z operand
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ad = smem_desc_sw128(st + (kk >> 2) * kApBox + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(zop + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
+            const uint64_t ad = desc_at(q0, (kk >> 2) * kApBox + (kk & 3) * 32);
+            const uint64_t bd = desc_at(zop0, (kk >> 2) * 2048 + (kk & 3) * 32);
             mma_bf16(acc + AC::kDenCol, ad, bd, id_den, kk > 0 ? 1u : 0u);
           }
         }
