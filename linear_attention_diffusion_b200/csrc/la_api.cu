@@ -457,9 +457,7 @@ la_status la_causal_attention(const la_shape* shape, const void* Q, const void* 
   const float* partials = reinterpret_cast<const float*>(w + L.partials);
   unsigned* counters = reinterpret_cast<unsigned*>(w + L.counters);
   const cudaError_t e =
-      causal_tc_supported(p)
-          ? launch_causal_tc(p, Q, K, V, partials, S_carry, z_carry, update, counters, O, st)
-          : launch_causal(p, Q, K, V, partials, S_carry, z_carry, update, counters, O, st);
+      launch_causal(p, Q, K, V, partials, S_carry, z_carry, update, counters, O, st);
   if (e != cudaSuccess) return cuda_fail(e, "causal attention");
   return LA_OK;
 }
@@ -638,10 +636,7 @@ la_status la_device_error(unsigned* code, int reset) {
   cudaError_t e = read_device_error(&fwd, reset != 0);
   if (e == cudaSuccess) e = read_device_error_bwd(&bwd, reset != 0);
   if (e == cudaSuccess) e = read_device_error_conv(&conv, reset != 0);
-  if (e == cudaSuccess) e = read_device_error_causal(&causal, reset != 0);
-  unsigned chunked = 0;
-  if (e == cudaSuccess) e = read_device_error_causal_chunk(&chunked, reset != 0);
-  causal |= chunked;
+  if (e == cudaSuccess) e = read_device_error_causal_chunk(&causal, reset != 0);
   if (e == cudaSuccess) e = read_device_error_qkv(&qkv, reset != 0);
   if (e != cudaSuccess) return cuda_fail(e, "la_device_error");
   *code = fwd | bwd | conv | causal | qkv;

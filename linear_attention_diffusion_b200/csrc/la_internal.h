@@ -127,12 +127,6 @@ cudaError_t launch_causal_chunks(const Problem& p, const void* Q, const void* K,
                                  float* states, float* S_carry, float* z_carry, int update,
                                  void* O, cudaStream_t s);
 cudaError_t read_device_error_causal_chunk(unsigned* code, bool reset);
-// The earlier tensor-core version (la_causal_tc.cu): bf16 I/O without RoPE,
-// a running state carried from chunk to chunk.
-bool causal_tc_supported(const Problem& p);
-cudaError_t launch_causal_tc(const Problem& p, const void* Q, const void* K, const void* V,
-                             const float* partials, float* S_carry, float* z_carry, int update,
-                             unsigned* counters, void* O, cudaStream_t s);
 // Temporal depth-wise convolution with the conv cache (la_conv.cu).
 struct ConvProblem {
   int B, T, HW, C;  // C a multiple of 8
@@ -148,7 +142,6 @@ cudaError_t read_device_error(unsigned* code, bool reset);
 cudaError_t launch_wait_selftest(unsigned limit_us, cudaStream_t s);
 cudaError_t read_device_error_bwd(unsigned* code, bool reset);
 cudaError_t read_device_error_conv(unsigned* code, bool reset);  // la_conv.cu
-cudaError_t read_device_error_causal(unsigned* code, bool reset);  // la_causal_tc.cu
 cudaError_t read_device_error_qkv(unsigned* code, bool reset);     // la_qkv_tc.cu
 // QKV projection fused with the state reduce (la_qkv_tc.cu): a persistent
 // tcgen05 GEMM that writes Q and one partial state per run of key/value
