@@ -456,6 +456,513 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   }
 }
 
+// ---------------------------------------------------------------------------
+// With RoPE. The numerator takes the rotated features, the denominator the
+// unrotated ones (SANA-Video, section 2.2):
+//   num_i = sum_{j <= i in chunk} (R_i phi(q_i) . R_j phi(k_j)) v_j + R_i phi(q_i) S_P
+//   den_i = ReLU(q_i) . (z_P + Z_i) + eps,   Z_i = sum_{j <= i in chunk} ReLU(k_j)
+// with S_P the prefix state of rotated keys and z_P that of plain key sums.
+// Z = L ReLU(K_h) is a tensor-core product with L the 128 x 128 lower
+// triangle of ones (kept in TMEM as an A operand). The rotated q and k enter
+// their products in two bf16 parts each (value and rounded remainder:
+// P = q_hi.k_hi + q_hi.k_lo + q_lo.k_hi, and likewise q.S), so the weights
+// keep about 16 bits as in the unrotated kernel.
+//
+// Stage layout (two stages): the Q box, overwritten with the rotated q's
+// high part; the low part; the K box, overwritten with the rotated k's high
+// part; its low part; plain ReLU(k) per head ([128][32] bf16, 64-byte
+// swizzle, the B operand of Z); V per head; the prefix S operand (hi, lo).
+// The prefix state itself is copied into one buffer shared by the stages.
+struct RStage {
+  static constexpr int q = 0;
+  static constexpr int qlo = q + kXBox;
+  static constexpr int k = qlo + kXBox;
+  static constexpr int klo = k + kXBox;
+  static constexpr int kp = klo + kXBox;     // 2 x 8 KB
+  static constexpr int v = kp + kXBox;       // 2 x 8 KB
+  static constexpr int bop = v + kXBox;      // 2 x 4 KB
+  static constexpr int bytes = bop + 2 * 4096;
+  static constexpr int stride = (bytes + 1023) / 1024 * 1024;
+};
+constexpr int kRStages = 2;
+
+struct RSmem {
+  static constexpr int stages = 0;
+  static constexpr int state = stages + kRStages * RStage::stride;  // [2 heads][1056] f32
+  static constexpr int rope = state + 2 * kStateFloats * 4;         // RoPE (cos, sin) table
+  static constexpr int bars = rope + kRopeTableMax * 8;
+  // full[2] ready[2][2] o_done[2] st_full st_empty p_full[2] pm_ready[2] o_full[2] mma_done
+  static constexpr int nbars = 2 * kRStages + 2 * kRStages + kRStages + 2 + 7;
+  static constexpr int misc = bars + nbars * 8;
+  static constexpr int bytes = misc + 16;
+};
+constexpr int kRSmemBytes = RSmem::bytes + 1024;
+static_assert(kRSmemBytes <= 232448, "shared memory per CTA");
+
+// TMEM columns of the RoPE kernel: P of head h at 128 h, O at 256 + 32 h, Z at
+// 320 + 32 h, L (bf16 pairs) at 384 .. 447.
+constexpr uint32_t kRColO = 256, kRColZ = 320, kRColL = 384;
+
+// Physical byte offset of 16-byte chunk c of row r in a 64-byte-swizzled tile
+// of 64-byte rows (512-aligned base).
+__device__ __forceinline__ uint32_t sw64_offset(uint32_t r, uint32_t c) {
+  return r * 64u + ((c ^ ((r >> 1) & 3u)) << 4);
+}
+
+// Every chunk's key sum z_c = sum over its tokens of ReLU(k), into the z slot
+// of the chunk-state buffer (the chunk-state reduce leaves it alone with
+// RoPE). Block (x, c, b): 32 consecutive 16-byte vectors of a token row (head
+// vec / 4, dims 8 (vec % 4) ..) over chunk c, eight warps taking 16 tokens
+// each; the eight partial sums are added in warp order.
+__global__ void __launch_bounds__(256)
+chunk_key_sums(const __nv_bfloat16* K, float* states, int N, int H, int nchunks) {
+  __shared__ float part[8][32][8];
+  const int lane = threadIdx.x & 31, slice = threadIdx.x >> 5;
+  const int vec = blockIdx.x * 32 + lane;
+  const int c = blockIdx.y, b = blockIdx.z;
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_trigger();
+  const bool live = vec < H * 4;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+  if (live) {
+    const int n0 = c * kXT + slice * 16;
+    uint4 u[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t)
+      u[t] = n0 + t < N ? __ldg(reinterpret_cast<const uint4*>(
+                              K + (static_cast<size_t>(b) * N + n0 + t) * H * kD + vec * 8))
+                        : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      float x[8];
+      unpack8(u[t], x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += fmaxf(x[e], 0.0f);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[slice][lane][e] = acc[e];
+  __syncthreads();
+  if (slice == 0 && live) {
+    float z[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) z[e] = part[0][lane][e];
+    for (int t = 1; t < 8; ++t)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) z[e] += part[t][lane][e];
+    float* dst = states + ((static_cast<size_t>(b) * H + vec / 4) * nchunks + c) * kStateFloats +
+                 kD * kD + (vec % 4) * 8;
+    *reinterpret_cast<float4*>(dst) = make_float4(z[0], z[1], z[2], z[3]);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(z[4], z[5], z[6], z[7]);
+  }
+}
+
+// causal_chunk_rope_tc: the same CTA shape, roles and head pipelines as
+// causal_chunk_tc. Per chunk and head, after the warpgroup has prepared the
+// stage (ReLU, rotation, the two parts, plain ReLU(k), the S operand):
+//   Z_h = L ReLU(K_h)                    M = 128, N = 32, K = 128 (A = L in TMEM)
+//   P_h = three products of the parts    M = N = 128, K = 32
+// then the mask and split of P as without RoPE, and
+//   O_h = P_hi V_h + P_lo V_h + (q_hi S_hi + q_hi S_lo + q_lo S_hi)
+// The warpgroup keeps ReLU(q) of its row (16 registers) from the preparation
+// to the denominator.
+template <int kRopeMode>
+__global__ void __launch_bounds__(kXThreads, 1)
+causal_chunk_rope_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                     const Problem p, const ChunkArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + RSmem::bars);
+  uint64_t* ready = full + kRStages;          // [stage][head] stage prepared (128)
+  uint64_t* o_done = ready + 2 * kRStages;    // [stage] O written over the Q box (256)
+  uint64_t* st_full = o_done + kRStages;      // the chunk's prefix state copied in (1)
+  uint64_t* st_empty = st_full + 1;           // the prefix state read (256)
+  uint64_t* p_full = st_empty + 1;            // [head] Z and P in TMEM (1)
+  uint64_t* pm_ready = p_full + 2;            // [head] P masked, in two parts (128)
+  uint64_t* o_full = pm_ready + 2;            // [head] O in TMEM (1)
+  uint64_t* mma_done = o_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + RSmem::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + RSmem::misc + 4);
+  float2* rope_tab = reinterpret_cast<float2*>(smem + RSmem::rope);
+  unsigned* err = &g_causal_chunk_error;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int pair = blockIdx.y, b = blockIdx.z;
+  const int h0 = pair * 2;
+  const size_t cidx = static_cast<size_t>(b) * p.H + h0;
+  const int c_begin = blockIdx.x * a.chunks_per_cta;
+  const int nC = max(0, min(a.nchunks, c_begin + a.chunks_per_cta) - c_begin);
+  const int heads = min(2, p.H - h0);
+
+  if (tid == 0) {
+    for (int i = 0; i < kRStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&ready[2 * i], 128);
+      mbar_init(&ready[2 * i + 1], 128);
+      mbar_init(&o_done[i], kXMath);
+    }
+    mbar_init(st_full, 1);
+    mbar_init(st_empty, kXMath);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&p_full[h], 1);
+      mbar_init(&pm_ready[h], 128);
+      mbar_init(&o_full[h], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kXTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_o);
+  }
+  if (kRopeMode == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kXMath);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sbase = smem_u32(smem);
+  if (tid >= 64 && tid < 64 + 128) {
+    // L into TMEM: row i holds keys j <= i as bf16 ones (pairs per column)
+    const int quad = warp & 3, row = quad * 32 + lane;
+    const uint32_t lq = static_cast<uint32_t>(quad * 32) << 16;
+#pragma unroll
+    for (int cb = 0; cb < 4; ++cb) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int j = 32 * cb + 2 * e;
+        pk[e] = (j <= row ? 0x3F80u : 0u) | (j + 1 <= row ? 0x3F800000u : 0u);
+      }
+      tmem_st_32x32b_x16(tmem + lq + kRColL + 16 * cb, pk);
+    }
+    tmem_st_wait();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  pdl_wait();
+  if (tid == 64) pdl_trigger();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0) {
+      auto stage_ptr = [&](int c) { return smem + RSmem::stages + (c % kRStages) * RStage::stride; };
+      auto store_o = [&](int c) -> bool {
+        if (!mbar_wait(&o_done[c % kRStages], (c / kRStages) & 1, abort_flag, err, kErrWait))
+          return false;
+        tma_store_3d(&tm_o, stage_ptr(c) + RStage::q, h0 * 32, (c_begin + c) * kXT, b);
+        bulk_commit();
+        bulk_wait_read<0>();
+        return true;
+      };
+      bool ok = true;
+      int c = 0;
+      for (; ok && c < nC; ++c) {
+        const int s = c % kRStages;
+        if (c >= kRStages && !(ok = store_o(c - kRStages))) break;
+        // the shared state buffer takes chunk c once chunk c - 1's has been read
+        if (c > 0 && !(ok = mbar_wait(st_empty, (c - 1) & 1, abort_flag, err, kErrWait))) break;
+        uint8_t* st = stage_ptr(c);
+        const int y = (c_begin + c) * kXT;
+        mbar_arrive_expect_tx(&full[s], 3 * kXBox);
+        tma_load_3d(st + RStage::q, &tm_q, &full[s], h0 * 32, y, b);
+        tma_load_3d(st + RStage::k, &tm_k, &full[s], h0 * 32, y, b);
+        tma_load_3d(st + RStage::v, &tm_v, &full[s], h0 * 32, y, b);
+        tma_load_3d(st + RStage::v + kXVBox, &tm_v, &full[s], h0 * 32 + 32, y, b);
+        mbar_arrive_expect_tx(st_full, heads * kStateFloats * 4);
+        for (int hh = 0; hh < heads; ++hh)
+          bulk_load(smem + RSmem::state + hh * kStateFloats * 4,
+                    a.prefix + ((cidx + hh) * a.nchunks + c_begin + c) * kStateFloats,
+                    kStateFloats * 4, st_full);
+      }
+      for (int k = max(0, c - kRStages); ok && k < c; ++k) ok = store_o(k);
+      for (int k = max(0, c - kRStages); k < c; ++k)
+        mbar_drain(&full[k % kRStages], (k / kRStages) & 1, err, kErrWait);
+      if (c > 0) mbar_drain(st_full, (c - 1) & 1, err, kErrWait);
+      bulk_wait<0>();
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      const uint32_t id_z = idesc_bf16_f32(128, 32, 0, 1);
+      const uint32_t id_p = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t id_pv = idesc_bf16_f32(128, 32, 0, 1);
+      const uint32_t id_qs = idesc_bf16_f32(128, 32, 0, 0);
+      auto stage_addr = [&](int c) { return sbase + RSmem::stages + (c % kRStages) * RStage::stride; };
+      auto issue_p = [&](int c, int h) -> bool {
+        const int s = c % kRStages;
+        if (!mbar_wait(&ready[2 * s + h], (c / kRStages) & 1, abort_flag, err, kErrWait)) return false;
+        tc_fence_after();
+        const uint32_t st = stage_addr(c);
+        // Z_h = L ReLU(K_h): keys 16 kk .. 16 kk + 15 are columns 8 kk .. of L
+        const uint64_t dkp = smem_desc_sw64_mn32(st + RStage::kp + h * kXVBox);
+#pragma unroll
+        for (int kk = 0; kk < kXT / 16; ++kk)
+          mma_bf16_tmem_a(tmem + kRColZ + 32 * h, tmem + kRColL + 8 * kk, desc_at(dkp, kk * 1024),
+                          id_z, kk > 0 ? 1u : 0u);
+        // P_h = q_hi.k_hi + q_hi.k_lo + q_lo.k_hi (P of chunk c - 1 was read
+        // by this thread's earlier P.V MMAs, which run first)
+        const uint64_t dq = smem_desc_sw128(st + RStage::q, 16, 1024);
+        const uint64_t dql = smem_desc_sw128(st + RStage::qlo, 16, 1024);
+        const uint64_t dk = smem_desc_sw128(st + RStage::k, 16, 1024);
+        const uint64_t dkl = smem_desc_sw128(st + RStage::klo, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+          mma_bf16(tmem + 128 * h, desc_at(dq, h * 64 + kk * 32), desc_at(dk, h * 64 + kk * 32), id_p,
+                   kk);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+          mma_bf16(tmem + 128 * h, desc_at(dq, h * 64 + kk * 32), desc_at(dkl, h * 64 + kk * 32),
+                   id_p, 1u);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+          mma_bf16(tmem + 128 * h, desc_at(dql, h * 64 + kk * 32), desc_at(dk, h * 64 + kk * 32),
+                   id_p, 1u);
+        mma_commit(&p_full[h]);
+        return true;
+      };
+      auto issue_pv = [&](int c, int h) -> bool {
+        if (!mbar_wait(&pm_ready[h], c & 1, abort_flag, err, kErrWait)) return false;
+        tc_fence_after();
+        const uint32_t st = stage_addr(c);
+        const uint64_t dv = smem_desc_sw64_mn32(st + RStage::v + h * kXVBox);
+        const uint32_t d = tmem + kRColO + 32 * h;
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+          for (int kk = 0; kk < kXT / 16; ++kk)
+            mma_bf16_tmem_a(d, tmem + 128 * h + 32 * (kk >> 1) + 16 * part + 8 * (kk & 1),
+                            desc_at(dv, kk * 1024), id_pv, (part > 0 || kk > 0) ? 1u : 0u);
+        const uint64_t dq = smem_desc_sw128(st + RStage::q, 16, 1024);
+        const uint64_t dql = smem_desc_sw128(st + RStage::qlo, 16, 1024);
+        const uint64_t db = smem_desc_sw128(st + RStage::bop, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint32_t off = h * 64 + kk * 32;
+          mma_bf16(d, desc_at(dq, off), desc_at(db, off), id_qs, 1u);
+          mma_bf16(d, desc_at(dq, off), desc_at(db, 4096 + off), id_qs, 1u);
+          mma_bf16(d, desc_at(dql, off), desc_at(db, off), id_qs, 1u);
+        }
+        mma_commit(&o_full[h]);
+        return true;
+      };
+      bool ok = true;
+      for (int c = 0; ok && c < nC; ++c) {
+        ok = issue_p(c, 0);
+        if (ok && c > 0) ok = issue_pv(c - 1, 1);
+        if (ok) ok = issue_p(c, 1);
+        if (ok) ok = issue_pv(c, 0);
+      }
+      if (ok && nC > 0) issue_pv(nC - 1, 1);
+      mma_commit(mma_done);
+      mbar_drain(mma_done, 0, err, kErrWait);
+    }
+  } else {
+    // ------------------------------------------------- math: one warpgroup per head
+    const int mt = tid - 64;
+    const int h = mt >> 7;
+    const int wt = mt & 127;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lq = static_cast<uint32_t>(quad * 32) << 16;
+    auto stage_of = [&](int c) { return sbase + RSmem::stages + (c % kRStages) * RStage::stride; };
+    const float* state_h = reinterpret_cast<const float*>(smem + RSmem::state) + h * kStateFloats;
+    uint32_t qp[16];    // ReLU(q) of this row, bf16 pairs: kept for the denominator
+    float dpre = 0.0f;  // ReLU(q) . z_P + eps
+    // Chunk c's stage for this head: ReLU of q and k; plain ReLU(k) for Z;
+    // q and k rotated by the row's token position and written back as two
+    // bf16 parts; ReLU(q) . z_P; the prefix's S operand. Rows past the end of
+    // the sequence are zeros (TMA fill) and are not rotated. False when a wait
+    // gave up (decided by the warpgroup together).
+    auto prepare = [&](int c) -> bool {
+      const int s = c % kRStages;
+      bool ok = mbar_wait(&full[s], (c / kRStages) & 1, abort_flag, err, kErrWait);
+      ok = ok && mbar_wait(st_full, c & 1, abort_flag, err, kErrWait);
+      if (bar_any(kBarHeadX + h, 128, !ok || *abort_flag)) return false;
+      const uint32_t st = stage_of(c);
+      float xq[2][16], xk[2][16];
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint4 u = ld_shared_v4(st + RStage::q + sw128_offset(row, h * 4 + c4));
+        u.x = relu_bf16x2(u.x); u.y = relu_bf16x2(u.y); u.z = relu_bf16x2(u.z); u.w = relu_bf16x2(u.w);
+        qp[4 * c4] = u.x; qp[4 * c4 + 1] = u.y; qp[4 * c4 + 2] = u.z; qp[4 * c4 + 3] = u.w;
+        float t[8];
+        unpack8(u, t);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) xq[c4 >> 1][(c4 & 1) * 8 + k] = t[k];
+        uint4 w = ld_shared_v4(st + RStage::k + sw128_offset(row, h * 4 + c4));
+        w.x = relu_bf16x2(w.x); w.y = relu_bf16x2(w.y); w.z = relu_bf16x2(w.z); w.w = relu_bf16x2(w.w);
+        st_shared_v4(st + RStage::kp + h * kXVBox + sw64_offset(row, c4), w);
+        unpack8(w, t);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) xk[c4 >> 1][(c4 & 1) * 8 + k] = t[k];
+      }
+      {
+        float dz = p.eps;
+#pragma unroll
+        for (int d = 0; d < kD; ++d)
+          dz = fmaf(xq[d >> 4][d & 15], h < heads ? state_h[kD * kD + d] : 0.0f, dz);
+        dpre = dz;
+      }
+      const int n = (c_begin + c) * kXT + row;
+      if (n < p.N) {
+        const TokPos tp = token_pos(p.rope, n);
+        float2 cs0[8], cs1[8];
+        if (kRopeMode == kRopeTable) {
+          const RopeBases rb = rope_bases(p.rope, tp);
+          rope_table8<0>(rope_tab, rb, cs0);
+          rope_table8<1>(rope_tab, rb, cs1);
+        } else {
+          rope_fly8<0>(p.rope, tp, cs0);
+          rope_fly8<1>(p.rope, tp, cs1);
+        }
+        rotate8(xq[0], cs0);
+        rotate8(xq[1], cs1);
+        rotate8(xk[0], cs0);
+        rotate8(xk[1], cs1);
+      }
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float x[8], hx[8], lo[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] = xq[c4 >> 1][(c4 & 1) * 8 + k];
+        uint4 hi = pack8(x);
+        unpack8(hi, hx);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) lo[k] = x[k] - hx[k];
+        st_shared_v4(st + RStage::q + sw128_offset(row, h * 4 + c4), hi);
+        st_shared_v4(st + RStage::qlo + sw128_offset(row, h * 4 + c4), pack8(lo));
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] = xk[c4 >> 1][(c4 & 1) * 8 + k];
+        hi = pack8(x);
+        unpack8(hi, hx);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) lo[k] = x[k] - hx[k];
+        st_shared_v4(st + RStage::k + sw128_offset(row, h * 4 + c4), hi);
+        st_shared_v4(st + RStage::klo + sw128_offset(row, h * 4 + c4), pack8(lo));
+      }
+      {
+        // the prefix's S as the B operand: row e holds S[0..31][e] of this
+        // head in two bf16 parts (thread wt: row e = wt / 4, dims 8 (wt % 4) ..)
+        const int e = wt >> 2, c4 = wt & 3;
+        float x[8], hx[8], lo[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] = h < heads ? state_h[(c4 * 8 + k) * kD + e] : 0.0f;
+        const uint4 hi = pack8(x);
+        unpack8(hi, hx);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) lo[k] = x[k] - hx[k];
+        st_shared_v4(st + RStage::bop + sw128_offset(e, h * 4 + c4), hi);
+        st_shared_v4(st + RStage::bop + 4096 + sw128_offset(e, h * 4 + c4), pack8(lo));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();  // this thread's TMEM reads of the previous chunk come first
+      mbar_arrive(&ready[2 * s + h]);
+      mbar_arrive(st_empty);
+      return true;
+    };
+
+    bool alive = nC == 0 || prepare(0);
+    for (int c = 0; alive && c < nC; ++c) {
+      const int s = c % kRStages;
+      const uint32_t qb = stage_of(c) + RStage::q;
+
+      // ---- P: mask j <= i, two bf16 parts back into TMEM
+      bool ok = mbar_wait(&p_full[h], c & 1, abort_flag, err, kErrWait);
+      tc_fence_after();
+      if (bar_any(kBarHeadX + h, 128, !ok || *abort_flag)) break;
+#pragma unroll
+      for (int q2 = 0; q2 < 4; q2 += 2) {
+        uint32_t r[2][32];
+        if (q2 <= quad) {
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+            if (q2 + t <= quad) tmem_ld_32x32b_x32_nowait(tmem + lq + 128 * h + 32 * (q2 + t), r[t]);
+          tmem_ld_wait();
+        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int q = q2 + t;
+          uint32_t hi[16], lo[16];
+          if (q > quad) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
+          } else {
+            const int lim = q < quad ? 32 : lane + 1;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float x0 = 2 * e < lim ? __uint_as_float(r[t][2 * e]) : 0.0f;
+              const float x1 = 2 * e + 1 < lim ? __uint_as_float(r[t][2 * e + 1]) : 0.0f;
+              hi[e] = pack_bf16x2(x0, x1);
+              const float h0f = __uint_as_float(hi[e] << 16), h1f = __uint_as_float(hi[e] & 0xffff0000u);
+              lo[e] = pack_bf16x2(x0 - h0f, x1 - h1f);
+            }
+          }
+          tmem_st_32x32b_x16(tmem + lq + 128 * h + 32 * q, hi);
+          tmem_st_32x32b_x16(tmem + lq + 128 * h + 32 * q + 16, lo);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&pm_ready[h]);
+
+      // ---- den = ReLU(q) . (z_P + Z_i) + eps
+      float den = dpre;
+      {
+        float zr[32];
+        tmem_ld_32x32b_x32(tmem + lq + kRColZ + 32 * h, zr);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float x[8];
+          unpack8(make_uint4(qp[4 * c4], qp[4 * c4 + 1], qp[4 * c4 + 2], qp[4 * c4 + 3]), x);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) den = fmaf(x[k], zr[c4 * 8 + k], den);
+        }
+      }
+
+      // ---- the next chunk, ahead of this chunk's output
+      if (c + 1 < nC && !prepare(c + 1)) break;
+
+      // ---- O = numerator / den over this head's columns of the Q box
+      ok = mbar_wait(&o_full[h], c & 1, abort_flag, err, kErrWait);
+      tc_fence_after();
+      if (bar_any(kBarHeadX + h, 128, !ok || *abort_flag)) break;
+      {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem + lq + kRColO + 32 * h, v);
+        const float inv = 1.0f / den;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float x[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) x[k] = v[c4 * 8 + k] * inv;
+          st_shared_v4(qb + sw128_offset(row, h * 4 + c4), pack8(x));
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      mbar_arrive(&o_done[s]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kXTmemCols);
+  }
+}
 // Exclusive prefix over the chunks, per head and float4 column: chunk c's
 // state becomes carry + the sum of the chunks before it (update: the carry
 // becomes carry + the sum of all chunks). The chunk axis is cut into `segs`
@@ -568,9 +1075,7 @@ cudaError_t make_map_head(CUtensorMap* m, const void* base, const Problem& p) {
 
 }  // namespace
 
-bool causal_chunk_supported(const Problem& p) {
-  return p.io == LA_IO_BF16 && p.N > 0 && !p.rope.enabled;
-}
+bool causal_chunk_supported(const Problem& p) { return p.io == LA_IO_BF16 && p.N > 0; }
 
 size_t causal_chunk_state_bytes(const Problem& p) {
   const size_t nchunks = static_cast<size_t>((p.N + kXT - 1) / kXT);
@@ -582,9 +1087,19 @@ cudaError_t launch_causal_chunks(const Problem& p, const void* Q, const void* K,
                                  void* O, cudaStream_t s) {
   if (!causal_chunk_supported(p)) return cudaErrorNotSupported;
   const int nchunks = (p.N + kXT - 1) / kXT;
-  // (1) every chunk's own state
+  // (1) every chunk's own state (with RoPE its key sums come from a second kernel)
   cudaError_t e = launch_chunk_states_tc(p, K, V, states, nchunks, s);
   if (e != cudaSuccess) return e;
+  if (p.rope.enabled) {
+    const __nv_bfloat16* kp = static_cast<const __nv_bfloat16*>(K);
+    float* st = states;
+    int n = p.N, hh = p.H, nc = nchunks;
+    void* args[] = {&kp, &st, &n, &hh, &nc};
+    const dim3 grid(static_cast<unsigned>((p.H * 4 + 31) / 32), static_cast<unsigned>(nchunks),
+                    static_cast<unsigned>(p.B));
+    e = launch_pdl_x(reinterpret_cast<const void*>(chunk_key_sums), args, grid, dim3(256), 0, s);
+    if (e != cudaSuccess) return e;
+  }
   // (2) the exclusive prefix over the chunks (and the carry update)
   {
     int bh = p.B * p.H;
@@ -608,9 +1123,13 @@ cudaError_t launch_causal_chunks(const Problem& p, const void* Q, const void* K,
   if ((e = make_map(&mk, K, p, kXT)) != cudaSuccess) return e;
   if ((e = make_map_head(&mv, V, p)) != cudaSuccess) return e;
   if ((e = make_map(&mo, O, p, kXT)) != cudaSuccess) return e;
-  if ((e = ensure_smem_attr(0, reinterpret_cast<const void*>(causal_chunk_tc), kXSmemBytes)) !=
-      cudaSuccess)
-    return e;
+  const RopeTable rt = rope_table_for(p);
+  const int mode = rope_mode(rt);
+  const void* kern = mode == kNoRope      ? reinterpret_cast<const void*>(causal_chunk_tc)
+                     : mode == kRopeTable ? reinterpret_cast<const void*>(causal_chunk_rope_tc<kRopeTable>)
+                                          : reinterpret_cast<const void*>(causal_chunk_rope_tc<kRopeOnTheFly>);
+  const int smem_bytes = mode == kNoRope ? kXSmemBytes : kRSmemBytes;
+  if ((e = ensure_smem_attr(mode, kern, smem_bytes)) != cudaSuccess) return e;
   const int pairs = (p.H + 1) / 2;
   const long long units = static_cast<long long>(pairs) * p.B;
   int ctas = static_cast<int>(std::max<long long>(1, kNumSMs / std::max<long long>(1, units)));
@@ -622,8 +1141,7 @@ cudaError_t launch_causal_chunks(const Problem& p, const void* Q, const void* K,
   ctas = (nchunks + a.chunks_per_cta - 1) / a.chunks_per_cta;
   Problem pc = p;
   void* args[] = {&mq, &mk, &mv, &mo, &pc, &a};
-  e = launch_pdl_x(reinterpret_cast<const void*>(causal_chunk_tc), args, dim3(ctas, pairs, p.B),
-                   dim3(kXThreads), kXSmemBytes, s);
+  e = launch_pdl_x(kern, args, dim3(ctas, pairs, p.B), dim3(kXThreads), smem_bytes, s);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -49,9 +49,11 @@ using namespace sm100;
 // apply) in two forms: the head group's CTAs as one thread-block cluster that
 // hands the split partials over through distributed shared memory
 // (kClusterLayer), or a cooperative grid that hands them over through global
-// memory (kFusedLayer). A fifth launch, kChunkStates (bf16 without RoPE),
-// is the reduce that writes the state of every 128-token chunk instead of
-// one partial per split: the first step of token-causal attention. All share
+// memory (kFusedLayer). A fifth launch, kChunkStates (bf16), is the reduce
+// that writes the state of every 128-token chunk instead of one partial per
+// split: the first step of token-causal attention (without RoPE it also writes
+// the chunk's key sum; with RoPE the keys it holds are rotated and another
+// kernel forms the key sums). All share
 // one TMA stage ring of kNS stages (six; five
 // in the cluster layer): a ring position p uses stage p % kNS with phase
 // parity (p / kNS) & 1, whichever operation the tile belongs to.
@@ -232,9 +234,10 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
     }
   }
   if (kRope == kRopeTable && tid >= 64) build_rope_table(p.rope, rope_tab, tid - 64, kMath);
-  if (kCh && tid >= 64 && tid < 64 + 256) {
+  if (kCh && kRope == kNoRope && tid >= 64 && tid < 64 + 256) {
     // a 4 KB tile of bf16 ones: the B operand whose product with phi(K)^T is
-    // the key sum of every dim
+    // the key sum of every dim (with RoPE the keys in shared memory are
+    // rotated, so the chunks' key sums are formed by another kernel)
     st_shared_v4(smem_u32(smem + Smem::zop) + (tid - 64) * 16,
                  make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u));
     fence_proxy_async_smem();
@@ -368,7 +371,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
           const uint64_t bd = desc_at(b0, kk * 2048);
           const uint32_t accum = kCh ? ((first && kk == 0) ? 0u : 1u) : ((i > 0 || kk > 0) ? 1u : 0u);
           mma_bf16(acc, ad, bd, id_red, accum);
-          if (kCh) mma_bf16(acc + 128, ad, ones_d, id_z, accum);  // key sums
+          if (kCh && kRope == kNoRope) mma_bf16(acc + 128, ad, ones_d, id_z, accum);  // key sums
         }
         mma_commit(&empty[s]);
         if (kCh && (!first || i == nA - 1)) mma_commit(&t_full[cb]);
@@ -448,7 +451,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
           tc_fence_after();
           const uint32_t base = tmem + (static_cast<uint32_t>(32 * q) << 16) + cb * 160;
           tmem_ld_32x32b_x32(base + 32 * q, v);
-          tmem_ld_32x32b_x8(base + 128, zv);
+          if (kRope == kNoRope) tmem_ld_32x32b_x8(base + 128, zv);
         }
         tc_fence_before();
         __syncwarp();
@@ -459,7 +462,7 @@ layer_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4*>(dst + lane * kD + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-          dst[kD * kD + lane] = zv[0];
+          if (kRope == kNoRope) dst[kD * kD + lane] = zv[0];
         }
       };
       for (int i = 0; i < nA; ++i) {
@@ -1129,15 +1132,20 @@ cudaError_t launch_reduce_tc(const Problem& p, const void* K, const void* V, flo
 
 cudaError_t launch_chunk_states_tc(const Problem& p, const void* K, const void* V, float* states,
                                    int nchunks, cudaStream_t s) {
-  if (p.io != LA_IO_BF16 || p.rope.enabled || p.N <= 0) return cudaErrorNotSupported;
+  if (p.io != LA_IO_BF16 || p.N <= 0) return cudaErrorNotSupported;
   CUtensorMap mk, mv;
   cudaError_t e;
   if ((e = make_map(&mk, K, p, kRedT)) != cudaSuccess) return e;
   if ((e = make_map(&mv, V, p, kRedT)) != cudaSuccess) return e;
   const RopeTable rt = rope_table_for(p);
-  LayerKernel kern = layer_tc<kNoRope, kChunkStates>;
-  const int kBytes = LayerCfg<kNoRope, kChunkStates>::kSmemBytes;
-  if ((e = ensure_smem_attr(12, reinterpret_cast<const void*>(kern), kBytes)) != cudaSuccess)
+  const int mode = rope_mode(rt);
+  LayerKernel kern = mode == kNoRope      ? layer_tc<kNoRope, kChunkStates>
+                     : mode == kRopeTable ? layer_tc<kRopeTable, kChunkStates>
+                                          : layer_tc<kRopeOnTheFly, kChunkStates>;
+  const int kBytes = mode == kNoRope      ? LayerCfg<kNoRope, kChunkStates>::kSmemBytes
+                     : mode == kRopeTable ? LayerCfg<kRopeTable, kChunkStates>::kSmemBytes
+                                          : LayerCfg<kRopeOnTheFly, kChunkStates>::kSmemBytes;
+  if ((e = ensure_smem_attr(12 + mode, reinterpret_cast<const void*>(kern), kBytes)) != cudaSuccess)
     return e;
   LayerArgs a = {};
   a.chunk_states = states;
