@@ -491,8 +491,8 @@ struct RSmem {
   static constexpr int state = stages + kRStages * RStage::stride;  // [2 heads][1056] f32
   static constexpr int rope = state + 2 * kStateFloats * 4;         // RoPE (cos, sin) table
   static constexpr int bars = rope + kRopeTableMax * 8;
-  // full[2] ready[2][2] o_done[2] st_full st_empty p_full[2] pm_ready[2] o_full[2] mma_done
-  static constexpr int nbars = 2 * kRStages + 2 * kRStages + kRStages + 2 + 7;
+  // full[2] ready[2][2] o_done[2] st_full st_empty p_full[2] pm_ready[2] o_full[2] mma_done[2]
+  static constexpr int nbars = 2 * kRStages + 2 * kRStages + kRStages + 2 + 8;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int bytes = misc + 16;
 };
@@ -528,12 +528,18 @@ chunk_key_sums(const __nv_bfloat16* K, float* states, int N, int H, int nchunks)
   for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
   if (live) {
     const int n0 = c * kXT + slice * 16;
+    const int cnt = min(16, N - n0);  // tokens of this slice inside the sequence
+    const size_t stride = static_cast<size_t>(H) * kD;
+    const uint4* src = reinterpret_cast<const uint4*>(
+        K + (static_cast<size_t>(b) * N + max(0, min(n0, N - 1))) * stride + vec * 8);
     uint4 u[16];
+    if (cnt == 16) {  // all 16 loads in flight
 #pragma unroll
-    for (int t = 0; t < 16; ++t)
-      u[t] = n0 + t < N ? __ldg(reinterpret_cast<const uint4*>(
-                              K + (static_cast<size_t>(b) * N + n0 + t) * H * kD + vec * 8))
-                        : make_uint4(0u, 0u, 0u, 0u);
+      for (int t = 0; t < 16; ++t) u[t] = __ldg(src + t * stride / 8);
+    } else {
+#pragma unroll
+      for (int t = 0; t < 16; ++t) u[t] = t < cnt ? __ldg(src + t * stride / 8) : make_uint4(0u, 0u, 0u, 0u);
+    }
 #pragma unroll
     for (int t = 0; t < 16; ++t) {
       float x[8];
@@ -559,8 +565,10 @@ chunk_key_sums(const __nv_bfloat16* K, float* states, int N, int H, int nchunks)
   }
 }
 
-// causal_chunk_rope_tc: the same CTA shape, roles and head pipelines as
-// causal_chunk_tc. Per chunk and head, after the warpgroup has prepared the
+// causal_chunk_rope_tc: the same CTA shape and head pipelines as
+// causal_chunk_tc, with one MMA-issuing warp per head (warp 1: head 0, warp
+// 10: head 1), so that neither head's products wait behind the other's in one
+// issue order. Per chunk and head, after the warpgroup has prepared the
 // stage (ReLU, rotation, the two parts, plain ReLU(k), the S operand):
 //   Z_h = L ReLU(K_h)                    M = 128, N = 32, K = 128 (A = L in TMEM)
 //   P_h = three products of the parts    M = N = 128, K = 32
@@ -568,8 +576,10 @@ chunk_key_sums(const __nv_bfloat16* K, float* states, int N, int H, int nchunks)
 //   O_h = P_hi V_h + P_lo V_h + (q_hi S_hi + q_hi S_lo + q_lo S_hi)
 // The warpgroup keeps ReLU(q) of its row (16 registers) from the preparation
 // to the denominator.
+constexpr int kRThreads = kXThreads + 32;
+
 template <int kRopeMode>
-__global__ void __launch_bounds__(kXThreads, 1)
+__global__ void __launch_bounds__(kRThreads, 1)
 causal_chunk_rope_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                      const Problem p, const ChunkArgs a) {
@@ -584,7 +594,7 @@ causal_chunk_rope_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   uint64_t* p_full = st_empty + 1;            // [head] Z and P in TMEM (1)
   uint64_t* pm_ready = p_full + 2;            // [head] P masked, in two parts (128)
   uint64_t* o_full = pm_ready + 2;            // [head] O in TMEM (1)
-  uint64_t* mma_done = o_full + 2;
+  uint64_t* mma_done = o_full + 2;           // [head] this head's MMAs drained (1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + RSmem::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + RSmem::misc + 4);
   float2* rope_tab = reinterpret_cast<float2*>(smem + RSmem::rope);
@@ -611,8 +621,8 @@ causal_chunk_rope_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       mbar_init(&p_full[h], 1);
       mbar_init(&pm_ready[h], 128);
       mbar_init(&o_full[h], 1);
+      mbar_init(&mma_done[h], 1);
     }
-    mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -692,9 +702,10 @@ causal_chunk_rope_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (c > 0) mbar_drain(st_full, (c - 1) & 1, err, kErrWait);
       bulk_wait<0>();
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA
+  } else if (warp == 1 || warp == kRThreads / 32 - 1) {
+    // ------------------------------------------------------------ MMA, one head per warp
     if (lane == 0) {
+      const int hm = warp == 1 ? 0 : 1;
       const uint32_t id_z = idesc_bf16_f32(128, 32, 0, 1);
       const uint32_t id_p = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t id_pv = idesc_bf16_f32(128, 32, 0, 1);
@@ -758,15 +769,13 @@ causal_chunk_rope_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         return true;
       };
       bool ok = true;
-      for (int c = 0; ok && c < nC; ++c) {
-        ok = issue_p(c, 0);
-        if (ok && c > 0) ok = issue_pv(c - 1, 1);
-        if (ok) ok = issue_p(c, 1);
-        if (ok) ok = issue_pv(c, 0);
+      if (hm == 0) {
+        for (int c = 0; ok && c < nC; ++c) ok = issue_p(c, 0) && issue_pv(c, 0);
+      } else {
+        for (int c = 0; ok && c < nC; ++c) ok = issue_p(c, 1) && issue_pv(c, 1);
       }
-      if (ok && nC > 0) issue_pv(nC - 1, 1);
-      mma_commit(mma_done);
-      mbar_drain(mma_done, 0, err, kErrWait);
+      mma_commit(&mma_done[hm]);
+      mbar_drain(&mma_done[hm], 0, err, kErrWait);
     }
   } else {
     // ------------------------------------------------- math: one warpgroup per head
@@ -1141,7 +1150,8 @@ cudaError_t launch_causal_chunks(const Problem& p, const void* Q, const void* K,
   ctas = (nchunks + a.chunks_per_cta - 1) / a.chunks_per_cta;
   Problem pc = p;
   void* args[] = {&mq, &mk, &mv, &mo, &pc, &a};
-  e = launch_pdl_x(kern, args, dim3(ctas, pairs, p.B), dim3(kXThreads), smem_bytes, s);
+  e = launch_pdl_x(kern, args, dim3(ctas, pairs, p.B), dim3(mode == kNoRope ? kXThreads : kRThreads),
+                   smem_bytes, s);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
