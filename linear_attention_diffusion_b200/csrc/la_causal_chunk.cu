@@ -18,8 +18,8 @@
 // current chunk's products and output complete.
 //
 // causal_chunk_tc: a CTA owns two heads (one 64-dim TMA box per tensor) of one
-// batch element and a range of chunks; 320 threads (TMA warp, MMA warp, one
-// warpgroup per head). Per chunk, with three stages of Q, K, V and the
+// batch element and a range of chunks; 352 threads (TMA warp, one warpgroup
+// per head, and one MMA-issuing warp per head: warps 1 and 10). Per chunk, with three stages of Q, K, V and the
 // chunk's prefix state in flight:
 //   P   = phi(Q_h) phi(K_h)^T            M = N = 128, K = 32   (TMEM)
 //   the head's warpgroup masks P to j <= i, sums its rows, and writes P back
@@ -30,9 +30,9 @@
 //       + phi(Q_h) (S_hi + S_lo)           S of the prefix in two bf16 parts
 // and the warpgroup divides by the denominator and writes O over its head's
 // half of the Q box, which the TMA warp stores once both halves are in. The
-// two heads run as separate pipelines (their own barriers; the MMA warp issues
-// P_0(c), P.V_1(c - 1), P_1(c), P.V_0(c), ...), so the tensor core works on one
-// head while the other head's warpgroup masks. Every wait is bounded.
+// two heads run as separate pipelines (their own barriers and MMA issuers:
+// a tcgen05.mma costs tens of cycles to issue, and one issuer would make each
+// head's products wait behind the other's). Every wait is bounded.
 #include <algorithm>
 
 #include "la_tc_common.cuh"
@@ -50,6 +50,7 @@ constexpr int kXVBox = kXT * 64;            // [128 tokens][32 dims] bf16 = 8 KB
 constexpr int kXStages = 3;
 constexpr int kXMath = 256;                 // two warpgroups, one per head
 constexpr int kXThreads = 64 + kXMath;
+constexpr int kRThreads = kXThreads + 32;   // + a second MMA-issuing warp (warp 10)
 constexpr int kXTmemCols = 512;
 constexpr int kBarHeadX = 1;                // named barriers kBarHeadX + h: one warpgroup
 
@@ -74,8 +75,8 @@ constexpr uint32_t kColO = 256;
 struct XSmem {
   static constexpr int stages = 0;
   static constexpr int bars = stages + kXStages * XStage::stride;
-  // full[3] ready[3][2] o_done[3] p_full[2] pm_ready[2] o_full[2] mma_done
-  static constexpr int nbars = 4 * kXStages + 7;
+  // full[3] ready[3][2] o_done[3] p_full[2] pm_ready[2] o_full[2] mma_done[2]
+  static constexpr int nbars = 4 * kXStages + 8;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int bytes = misc + 16;
 };
@@ -146,7 +147,7 @@ __device__ __forceinline__ uint64_t smem_desc_sw64_mn32(uint32_t saddr) {
   return d;
 }
 
-__global__ void __launch_bounds__(kXThreads, 1)
+__global__ void __launch_bounds__(kRThreads, 1)
 causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                 const Problem p, const ChunkArgs a) {
@@ -159,7 +160,7 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* p_full = o_done + kXStages;       // [head] P in TMEM (1)
   uint64_t* pm_ready = p_full + 2;            // [head] P masked, in two parts, in TMEM (128)
   uint64_t* o_full = pm_ready + 2;            // [head] O in TMEM (1)
-  uint64_t* mma_done = o_full + 2;
+  uint64_t* mma_done = o_full + 2;            // [head] this head's MMAs drained (1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + XSmem::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + XSmem::misc + 4);
   unsigned* err = &g_causal_chunk_error;
@@ -184,7 +185,8 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(&pm_ready[h], 128);
       mbar_init(&o_full[h], 1);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(&mma_done[0], 1);
+    mbar_init(&mma_done[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -242,9 +244,10 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_drain(&full[k % kXStages], (k / kXStages) & 1, err, kErrWait);
       bulk_wait<0>();
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA
+  } else if (warp == 1 || warp == kRThreads / 32 - 1) {
+    // ------------------------------------------------------------ MMA, one head per warp
     if (lane == 0) {
+      const int hm = warp == 1 ? 0 : 1;
       const uint32_t id_p = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t id_pv = idesc_bf16_f32(128, 32, 0, 1);
       const uint32_t id_qs = idesc_bf16_f32(128, 32, 0, 0);
@@ -297,15 +300,13 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         return true;
       };
       bool ok = true;
-      for (int c = 0; ok && c < nC; ++c) {
-        ok = issue_p(c, 0);
-        if (ok && c > 0) ok = issue_pv(c - 1, 1);
-        if (ok) ok = issue_p(c, 1);
-        if (ok) ok = issue_pv(c, 0);
+      if (hm == 0) {
+        for (int c = 0; ok && c < nC; ++c) ok = issue_p(c, 0) && issue_pv(c, 0);
+      } else {
+        for (int c = 0; ok && c < nC; ++c) ok = issue_p(c, 1) && issue_pv(c, 1);
       }
-      if (ok && nC > 0) issue_pv(nC - 1, 1);
-      mma_commit(mma_done);
-      mbar_drain(mma_done, 0, err, kErrWait);
+      mma_commit(&mma_done[hm]);
+      mbar_drain(&mma_done[hm], 0, err, kErrWait);
     }
   } else {
     // ------------------------------------------------- math: one warpgroup per head
@@ -565,10 +566,8 @@ chunk_key_sums(const __nv_bfloat16* K, float* states, int N, int H, int nchunks)
   }
 }
 
-// causal_chunk_rope_tc: the same CTA shape and head pipelines as
-// causal_chunk_tc, with one MMA-issuing warp per head (warp 1: head 0, warp
-// 10: head 1), so that neither head's products wait behind the other's in one
-// issue order. Per chunk and head, after the warpgroup has prepared the
+// causal_chunk_rope_tc: the same CTA shape, roles and head pipelines as
+// causal_chunk_tc. Per chunk and head, after the warpgroup has prepared the
 // stage (ReLU, rotation, the two parts, plain ReLU(k), the S operand):
 //   Z_h = L ReLU(K_h)                    M = 128, N = 32, K = 128 (A = L in TMEM)
 //   P_h = three products of the parts    M = N = 128, K = 32
@@ -576,8 +575,6 @@ chunk_key_sums(const __nv_bfloat16* K, float* states, int N, int H, int nchunks)
 //   O_h = P_hi V_h + P_lo V_h + (q_hi S_hi + q_hi S_lo + q_lo S_hi)
 // The warpgroup keeps ReLU(q) of its row (16 registers) from the preparation
 // to the denominator.
-constexpr int kRThreads = kXThreads + 32;
-
 template <int kRopeMode>
 __global__ void __launch_bounds__(kRThreads, 1)
 causal_chunk_rope_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -819,9 +816,16 @@ causal_chunk_rope_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       }
       {
         float dz = p.eps;
+        const float4* z4 = reinterpret_cast<const float4*>(state_h + kD * kD);
 #pragma unroll
-        for (int d = 0; d < kD; ++d)
-          dz = fmaf(xq[d >> 4][d & 15], h < heads ? state_h[kD * kD + d] : 0.0f, dz);
+        for (int d4 = 0; d4 < kD / 4; ++d4) {
+          const float4 z = h < heads ? z4[d4] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          const float* x = &xq[d4 >> 2][(d4 & 3) * 4];
+          dz = fmaf(x[0], z.x, dz);
+          dz = fmaf(x[1], z.y, dz);
+          dz = fmaf(x[2], z.z, dz);
+          dz = fmaf(x[3], z.w, dz);
+        }
         dpre = dz;
       }
       const int n = (c_begin + c) * kXT + row;
@@ -1150,8 +1154,7 @@ cudaError_t launch_causal_chunks(const Problem& p, const void* Q, const void* K,
   ctas = (nchunks + a.chunks_per_cta - 1) / a.chunks_per_cta;
   Problem pc = p;
   void* args[] = {&mq, &mk, &mv, &mo, &pc, &a};
-  e = launch_pdl_x(kern, args, dim3(ctas, pairs, p.B), dim3(mode == kNoRope ? kXThreads : kRThreads),
-                   smem_bytes, s);
+  e = launch_pdl_x(kern, args, dim3(ctas, pairs, p.B), dim3(kRThreads), smem_bytes, s);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
