@@ -87,6 +87,7 @@ struct ChunkArgs {
   const float* prefix;  // [B*H][nchunks][kStateFloats]: each chunk's exclusive prefix state
   int nchunks;          // ceil(N / 128)
   int chunks_per_cta;
+  int adv_w, adv_h, adv_t;  // RoPE: 128 tokens as a step of the (t, h, w) grid (w, h below W, Hh)
 };
 
 // D[tmem] (+)= A[tmem] * B[smem]: bf16 A read from tensor memory (K-major,
@@ -145,6 +146,65 @@ __device__ __forceinline__ uint64_t smem_desc_sw64_mn32(uint32_t saddr) {
   d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
   d |= static_cast<uint64_t>(4) << 61;  // 64-byte swizzle
   return d;
+}
+
+// Eight floats as two bf16 parts: hi = the values truncated to bf16 (their
+// upper 16 bits), lo = the exact remainders rounded to bf16; hi + lo keeps
+// about 16 bits of each value.
+__device__ __forceinline__ void split_bf16x8(const float* x, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t u0 = __float_as_uint(x[2 * k]), u1 = __float_as_uint(x[2 * k + 1]);
+    h[k] = __byte_perm(u0, u1, 0x7632);
+    l[k] = pack_bf16x2(x[2 * k] - __uint_as_float(u0 & 0xffff0000u),
+                       x[2 * k + 1] - __uint_as_float(u1 & 0xffff0000u));
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// The causal mask and split of one head's P in TMEM (warp of lane quadrant
+// `quad`: rows 32 quad + lane): key block q < quad is kept whole, the
+// diagonal block q = quad keeps keys j <= row, blocks q > quad become zeros
+// (not loaded); the loads of blocks (0, 1) and of (2, 3) are issued together.
+// Each block goes back as 16 columns of rounded bf16 pairs and 16 of the
+// rounded remainders. Returns the sum of the kept weights.
+__device__ __forceinline__ float mask_split_p(uint32_t taddr, int quad, int lane) {
+  float psum = 0.0f;
+#pragma unroll
+  for (int q2 = 0; q2 < 4; q2 += 2) {
+    uint32_t r[2][32];
+    if (q2 <= quad) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+        if (q2 + t <= quad) tmem_ld_32x32b_x32_nowait(taddr + 32 * (q2 + t), r[t]);
+      tmem_ld_wait();
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int q = q2 + t;
+      uint32_t hi[16], lo[16];
+      if (q > quad) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
+      } else {
+        const int lim = q < quad ? 32 : lane + 1;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float x0 = 2 * e < lim ? __uint_as_float(r[t][2 * e]) : 0.0f;
+          const float x1 = 2 * e + 1 < lim ? __uint_as_float(r[t][2 * e + 1]) : 0.0f;
+          psum += x0 + x1;
+          hi[e] = pack_bf16x2(x0, x1);
+          const float h0f = __uint_as_float(hi[e] << 16), h1f = __uint_as_float(hi[e] & 0xffff0000u);
+          lo[e] = pack_bf16x2(x0 - h0f, x1 - h1f);
+        }
+      }
+      tmem_st_32x32b_x16(taddr + 32 * q, hi);
+      tmem_st_32x32b_x16(taddr + 32 * q + 16, lo);
+    }
+  }
+  return psum;
 }
 
 __global__ void __launch_bounds__(kRThreads, 1)
@@ -326,7 +386,7 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     };
     // ReLU of this head's Q and K columns of chunk c in place, then the
     // prefix's S as the B operand: row e holds S[0..31][e] of this head in two
-    // bf16 parts (thread wt: row e = wt / 4, dims 8 (wt % 4) ..). False when
+    // bf16 parts (thread wt: row e = wt % 32, dims 8 (wt / 32) ..). False when
     // a wait gave up (decided by the warpgroup together).
     auto prepare = [&](int c) -> bool {
       const int s = c % kXStages;
@@ -347,18 +407,15 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       {
         const float* pre = prefix_of(c);
-        const int e = wt >> 2, c4 = wt & 3;
-        float x[8], lo[8];
+        const int e = wt & 31, c4 = wt >> 5;  // a warp reads 32 consecutive floats
+        float x[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) x[k] = h < heads ? pre[(c4 * 8 + k) * kD + e] : 0.0f;
-        const uint4 hi = pack8(x);
-        float hx[8];
-        unpack8(hi, hx);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) lo[k] = x[k] - hx[k];
+        uint4 hi, lo;
+        split_bf16x8(x, hi, lo);
         const uint32_t bop = st + XStage::bop;
         st_shared_v4(bop + sw128_offset(e, h * 4 + c4), hi);
-        st_shared_v4(bop + 4096 + sw128_offset(e, h * 4 + c4), pack8(lo));
+        st_shared_v4(bop + 4096 + sw128_offset(e, h * 4 + c4), lo);
       }
       fence_proxy_async_smem();
       mbar_arrive(&ready[2 * s + h]);
@@ -375,42 +432,7 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       bool ok = mbar_wait(&p_full[h], c & 1, abort_flag, err, kErrWait);
       tc_fence_after();
       if (bar_any(kBarHeadX + h, 128, !ok || *abort_flag)) break;
-      // key block q of this warp's rows (32 quad .. 32 quad + 31): below the
-      // diagonal block every key is kept, above it none (zeros, no load); the
-      // loads of blocks (0, 1) and of (2, 3) are issued together
-      float psum = 0.0f;
-#pragma unroll
-      for (int q2 = 0; q2 < 4; q2 += 2) {
-        uint32_t r[2][32];
-        if (q2 <= quad) {
-#pragma unroll
-          for (int t = 0; t < 2; ++t)
-            if (q2 + t <= quad) tmem_ld_32x32b_x32_nowait(tmem + lq + 128 * h + 32 * (q2 + t), r[t]);
-          tmem_ld_wait();
-        }
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const int q = q2 + t;
-          uint32_t hi[16], lo[16];
-          if (q > quad) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
-          } else {
-            const int lim = q < quad ? 32 : lane + 1;  // keys of the block this row keeps
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float x0 = 2 * e < lim ? __uint_as_float(r[t][2 * e]) : 0.0f;
-              const float x1 = 2 * e + 1 < lim ? __uint_as_float(r[t][2 * e + 1]) : 0.0f;
-              psum += x0 + x1;
-              hi[e] = pack_bf16x2(x0, x1);
-              const float h0f = __uint_as_float(hi[e] << 16), h1f = __uint_as_float(hi[e] & 0xffff0000u);
-              lo[e] = pack_bf16x2(x0 - h0f, x1 - h1f);
-            }
-          }
-          tmem_st_32x32b_x16(tmem + lq + 128 * h + 32 * q, hi);
-          tmem_st_32x32b_x16(tmem + lq + 128 * h + 32 * q + 16, lo);
-        }
-      }
+      const float psum = mask_split_p(tmem + lq + 128 * h, quad, lane);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&pm_ready[h]);
@@ -786,98 +808,117 @@ causal_chunk_rope_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const float* state_h = reinterpret_cast<const float*>(smem + RSmem::state) + h * kStateFloats;
     uint32_t qp[16];    // ReLU(q) of this row, bf16 pairs: kept for the denominator
     float dpre = 0.0f;  // ReLU(q) . z_P + eps
+    // grid position of this row's token in the next chunk to prepare, moved
+    // on by one chunk (128 tokens) per preparation without divisions
+    TokPos tp = token_pos(p.rope, min(c_begin * kXT + row, p.N - 1));
     // Chunk c's stage for this head: ReLU of q and k; plain ReLU(k) for Z;
     // q and k rotated by the row's token position and written back as two
-    // bf16 parts; ReLU(q) . z_P; the prefix's S operand. Rows past the end of
-    // the sequence are zeros (TMA fill) and are not rotated. False when a wait
+    // bf16 parts (the value truncated to bf16, and the remainder rounded);
+    // ReLU(q) . z_P; the prefix's S operand. Rows past the end of the
+    // sequence are zeros (TMA fill) and are not rotated. False when a wait
     // gave up (decided by the warpgroup together).
     auto prepare = [&](int c) -> bool {
       const int s = c % kRStages;
+      const int n = (c_begin + c) * kXT + row;
+      const TokPos tpc = tp;
+      tp.w += a.adv_w;
+      tp.h += a.adv_h;
+      tp.t += a.adv_t;
+      if (tp.w >= p.rope.W) {
+        tp.w -= p.rope.W;
+        ++tp.h;
+      }
+      if (tp.h >= p.rope.Hh) {
+        tp.h -= p.rope.Hh;
+        ++tp.t;
+      }
       bool ok = mbar_wait(&full[s], (c / kRStages) & 1, abort_flag, err, kErrWait);
       ok = ok && mbar_wait(st_full, c & 1, abort_flag, err, kErrWait);
       if (bar_any(kBarHeadX + h, 128, !ok || *abort_flag)) return false;
       const uint32_t st = stage_of(c);
-      float xq[2][16], xk[2][16];
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint4 u = ld_shared_v4(st + RStage::q + sw128_offset(row, h * 4 + c4));
-        u.x = relu_bf16x2(u.x); u.y = relu_bf16x2(u.y); u.z = relu_bf16x2(u.z); u.w = relu_bf16x2(u.w);
-        qp[4 * c4] = u.x; qp[4 * c4 + 1] = u.y; qp[4 * c4 + 2] = u.z; qp[4 * c4 + 3] = u.w;
-        float t[8];
-        unpack8(u, t);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) xq[c4 >> 1][(c4 & 1) * 8 + k] = t[k];
-        uint4 w = ld_shared_v4(st + RStage::k + sw128_offset(row, h * 4 + c4));
-        w.x = relu_bf16x2(w.x); w.y = relu_bf16x2(w.y); w.z = relu_bf16x2(w.z); w.w = relu_bf16x2(w.w);
-        st_shared_v4(st + RStage::kp + h * kXVBox + sw64_offset(row, c4), w);
-        unpack8(w, t);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) xk[c4 >> 1][(c4 & 1) * 8 + k] = t[k];
-      }
+      float2 cs0[8], cs1[8];  // (cos, sin) of the row's 16 pairs
+      // q: ReLU (kept for the denominator), ReLU(q) . z_P, rotation, two parts
       {
-        float dz = p.eps;
+        float x[2][16];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint4 u = ld_shared_v4(st + RStage::q + sw128_offset(row, h * 4 + c4));
+          u.x = relu_bf16x2(u.x); u.y = relu_bf16x2(u.y); u.z = relu_bf16x2(u.z); u.w = relu_bf16x2(u.w);
+          qp[4 * c4] = u.x; qp[4 * c4 + 1] = u.y; qp[4 * c4 + 2] = u.z; qp[4 * c4 + 3] = u.w;
+          float t[8];
+          unpack8(u, t);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) x[c4 >> 1][(c4 & 1) * 8 + k] = t[k];
+        }
+        float dz[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four partial sums
         const float4* z4 = reinterpret_cast<const float4*>(state_h + kD * kD);
 #pragma unroll
         for (int d4 = 0; d4 < kD / 4; ++d4) {
           const float4 z = h < heads ? z4[d4] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          const float* x = &xq[d4 >> 2][(d4 & 3) * 4];
-          dz = fmaf(x[0], z.x, dz);
-          dz = fmaf(x[1], z.y, dz);
-          dz = fmaf(x[2], z.z, dz);
-          dz = fmaf(x[3], z.w, dz);
+          const float* xv = &x[d4 >> 2][(d4 & 3) * 4];
+          dz[0] = fmaf(xv[0], z.x, dz[0]);
+          dz[1] = fmaf(xv[1], z.y, dz[1]);
+          dz[2] = fmaf(xv[2], z.z, dz[2]);
+          dz[3] = fmaf(xv[3], z.w, dz[3]);
         }
-        dpre = dz;
-      }
-      const int n = (c_begin + c) * kXT + row;
-      if (n < p.N) {
-        const TokPos tp = token_pos(p.rope, n);
-        float2 cs0[8], cs1[8];
-        if (kRopeMode == kRopeTable) {
-          const RopeBases rb = rope_bases(p.rope, tp);
-          rope_table8<0>(rope_tab, rb, cs0);
-          rope_table8<1>(rope_tab, rb, cs1);
-        } else {
-          rope_fly8<0>(p.rope, tp, cs0);
-          rope_fly8<1>(p.rope, tp, cs1);
+        dpre = ((dz[0] + dz[1]) + (dz[2] + dz[3])) + p.eps;
+        if (n < p.N) {
+          if (kRopeMode == kRopeTable) {
+            const RopeBases rbs = rope_bases(p.rope, tpc);
+            rope_table8<0>(rope_tab, rbs, cs0);
+            rope_table8<1>(rope_tab, rbs, cs1);
+          } else {
+            rope_fly8<0>(p.rope, tpc, cs0);
+            rope_fly8<1>(p.rope, tpc, cs1);
+          }
+          rotate8(x[0], cs0);
+          rotate8(x[1], cs1);
         }
-        rotate8(xq[0], cs0);
-        rotate8(xq[1], cs1);
-        rotate8(xk[0], cs0);
-        rotate8(xk[1], cs1);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint4 hi, lo;
+          split_bf16x8(&x[c4 >> 1][(c4 & 1) * 8], hi, lo);
+          st_shared_v4(st + RStage::q + sw128_offset(row, h * 4 + c4), hi);
+          st_shared_v4(st + RStage::qlo + sw128_offset(row, h * 4 + c4), lo);
+        }
       }
+      // k: ReLU (plain copy for Z), rotation, two parts
+      {
+        float x[2][16];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float x[8], hx[8], lo[8];
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint4 w = ld_shared_v4(st + RStage::k + sw128_offset(row, h * 4 + c4));
+          w.x = relu_bf16x2(w.x); w.y = relu_bf16x2(w.y); w.z = relu_bf16x2(w.z); w.w = relu_bf16x2(w.w);
+          st_shared_v4(st + RStage::kp + h * kXVBox + sw64_offset(row, c4), w);
+          float t[8];
+          unpack8(w, t);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) x[k] = xq[c4 >> 1][(c4 & 1) * 8 + k];
-        uint4 hi = pack8(x);
-        unpack8(hi, hx);
+          for (int k = 0; k < 8; ++k) x[c4 >> 1][(c4 & 1) * 8 + k] = t[k];
+        }
+        if (n < p.N) {
+          rotate8(x[0], cs0);
+          rotate8(x[1], cs1);
+        }
 #pragma unroll
-        for (int k = 0; k < 8; ++k) lo[k] = x[k] - hx[k];
-        st_shared_v4(st + RStage::q + sw128_offset(row, h * 4 + c4), hi);
-        st_shared_v4(st + RStage::qlo + sw128_offset(row, h * 4 + c4), pack8(lo));
-#pragma unroll
-        for (int k = 0; k < 8; ++k) x[k] = xk[c4 >> 1][(c4 & 1) * 8 + k];
-        hi = pack8(x);
-        unpack8(hi, hx);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) lo[k] = x[k] - hx[k];
-        st_shared_v4(st + RStage::k + sw128_offset(row, h * 4 + c4), hi);
-        st_shared_v4(st + RStage::klo + sw128_offset(row, h * 4 + c4), pack8(lo));
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint4 hi, lo;
+          split_bf16x8(&x[c4 >> 1][(c4 & 1) * 8], hi, lo);
+          st_shared_v4(st + RStage::k + sw128_offset(row, h * 4 + c4), hi);
+          st_shared_v4(st + RStage::klo + sw128_offset(row, h * 4 + c4), lo);
+        }
       }
       {
         // the prefix's S as the B operand: row e holds S[0..31][e] of this
-        // head in two bf16 parts (thread wt: row e = wt / 4, dims 8 (wt % 4) ..)
-        const int e = wt >> 2, c4 = wt & 3;
-        float x[8], hx[8], lo[8];
+        // head in two bf16 parts (thread wt: row e = wt % 32, dims 8 (wt / 32) ..;
+        // the state reads of a warp are then 32 consecutive floats)
+        const int e = wt & 31, c4 = wt >> 5;
+        float x[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) x[k] = h < heads ? state_h[(c4 * 8 + k) * kD + e] : 0.0f;
-        const uint4 hi = pack8(x);
-        unpack8(hi, hx);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) lo[k] = x[k] - hx[k];
+        uint4 hi, lo;
+        split_bf16x8(x, hi, lo);
         st_shared_v4(st + RStage::bop + sw128_offset(e, h * 4 + c4), hi);
-        st_shared_v4(st + RStage::bop + 4096 + sw128_offset(e, h * 4 + c4), pack8(lo));
+        st_shared_v4(st + RStage::bop + 4096 + sw128_offset(e, h * 4 + c4), lo);
       }
       fence_proxy_async_smem();
       tc_fence_before();  // this thread's TMEM reads of the previous chunk come first
@@ -895,37 +936,7 @@ causal_chunk_rope_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       bool ok = mbar_wait(&p_full[h], c & 1, abort_flag, err, kErrWait);
       tc_fence_after();
       if (bar_any(kBarHeadX + h, 128, !ok || *abort_flag)) break;
-#pragma unroll
-      for (int q2 = 0; q2 < 4; q2 += 2) {
-        uint32_t r[2][32];
-        if (q2 <= quad) {
-#pragma unroll
-          for (int t = 0; t < 2; ++t)
-            if (q2 + t <= quad) tmem_ld_32x32b_x32_nowait(tmem + lq + 128 * h + 32 * (q2 + t), r[t]);
-          tmem_ld_wait();
-        }
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const int q = q2 + t;
-          uint32_t hi[16], lo[16];
-          if (q > quad) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
-          } else {
-            const int lim = q < quad ? 32 : lane + 1;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float x0 = 2 * e < lim ? __uint_as_float(r[t][2 * e]) : 0.0f;
-              const float x1 = 2 * e + 1 < lim ? __uint_as_float(r[t][2 * e + 1]) : 0.0f;
-              hi[e] = pack_bf16x2(x0, x1);
-              const float h0f = __uint_as_float(hi[e] << 16), h1f = __uint_as_float(hi[e] & 0xffff0000u);
-              lo[e] = pack_bf16x2(x0 - h0f, x1 - h1f);
-            }
-          }
-          tmem_st_32x32b_x16(tmem + lq + 128 * h + 32 * q, hi);
-          tmem_st_32x32b_x16(tmem + lq + 128 * h + 32 * q + 16, lo);
-        }
-      }
+      mask_split_p(tmem + lq + 128 * h, quad, lane);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&pm_ready[h]);
@@ -1151,6 +1162,11 @@ cudaError_t launch_causal_chunks(const Problem& p, const void* Q, const void* K,
   a.prefix = states;
   a.nchunks = nchunks;
   a.chunks_per_cta = (nchunks + ctas - 1) / ctas;
+  if (p.rope.enabled) {
+    a.adv_w = kXT % p.rope.W;
+    a.adv_h = (kXT / p.rope.W) % p.rope.Hh;
+    a.adv_t = (kXT / p.rope.W) / p.rope.Hh;
+  }
   ctas = (nchunks + a.chunks_per_cta - 1) / a.chunks_per_cta;
   Problem pc = p;
   void* args[] = {&mq, &mk, &mv, &mo, &pc, &a};
