@@ -190,20 +190,22 @@ la_status la_attention_backward(const la_shape* shape, const void* Q,
  * O: [B,N,H,D] io_dtype (written); carry [B,H,D,D] / [B,H,D] float32. ws:
  * device workspace of at least la_causal_workspace_bytes(shape) bytes,
  * zero-filled once before its first use like the others.
- * bf16 I/O without RoPE: three launches on the tensor cores. The state reduce
- * writes every 128-token chunk's own state to the workspace, a prefix pass
- * turns each into its chunk's exclusive prefix (the carry plus the earlier
- * chunks, summed in chunk order; update = 1 also folds the sequence into the
- * carry), and the output kernel computes every chunk independently: the
- * masked chunk-local product plus the chunk's prefix.
- * RoPE or float32 I/O: two launches. The state reduce leaves each token
- * split's partial state in the workspace; a CUDA-core kernel starts each split
- * from the carry plus the earlier splits (summed in split order) and walks its
+ * bf16 I/O: three launches on the tensor cores (four with RoPE). The state
+ * reduce writes every 128-token chunk's own state to the workspace (with RoPE
+ * a second kernel adds the chunks' key sums of the unrotated ReLU(k)), a
+ * prefix pass turns each into its chunk's exclusive prefix (the carry plus
+ * the earlier chunks, summed in chunk order; update = 1 also folds the
+ * sequence into the carry), and the output kernel computes every chunk
+ * independently: the masked chunk-local product plus the chunk's prefix, the
+ * weights and the rotated features carried in two bf16 parts each.
+ * float32 I/O: two launches. The state reduce leaves each token split's
+ * partial state in the workspace; a CUDA-core kernel starts each split from
+ * the carry plus the earlier splits (summed in split order) and walks its
  * tokens in 32-token chunks. Deterministic either way. */
 /* Bytes of workspace la_causal_attention needs for `shape` (at least
- * la_workspace_bytes(shape); for bf16 without RoPE, room for the state of
- * every 128-token chunk: B*H*ceil(N/128)*4224 bytes). 0 iff the shape is
- * invalid. Pure host function. */
+ * la_workspace_bytes(shape); for bf16, room for the state of every 128-token
+ * chunk: B*H*ceil(N/128)*4224 bytes). 0 iff the shape is invalid. Pure host
+ * function. */
 size_t la_causal_workspace_bytes(const la_shape* shape);
 
 la_status la_causal_attention(const la_shape* shape, const void* Q,

@@ -444,7 +444,8 @@ la_status la_causal_attention(const la_shape* shape, const void* Q, const void* 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
   if (causal_chunk_supported(p)) {
-    // bf16 without RoPE: every chunk's state, their prefix, then the chunks
+    // bf16: every chunk's state (and with RoPE its key sums), their prefix,
+    // then the chunks
     const cudaError_t e = launch_causal_chunks(p, Q, K, V, reinterpret_cast<float*>(w), S_carry,
                                                z_carry, update, O, st);
     if (e != cudaSuccess) return cuda_fail(e, "causal attention");

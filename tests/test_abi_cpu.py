@@ -182,16 +182,16 @@ def test_qkv_state_wrapper_checks_shapes():
 
 
 def test_causal_workspace_bytes():
-    # bf16 without RoPE: room for every 128-token chunk's state (4224 bytes a
-    # head), never less than the ordinary workspace
+    # bf16, with or without RoPE: room for every 128-token chunk's state (4224
+    # bytes a head), never less than the ordinary workspace
     s = la.make_shape(1, 16384, 70)
     n = la.la_causal_workspace_bytes(s)
     assert n >= la.la_workspace_bytes(s)
     assert n >= 70 * (16384 // 128) * 4224
     assert la.la_causal_workspace_bytes(la.make_shape(2, 300, 5)) >= 2 * 5 * 3 * 4224
-    # RoPE or float32 I/O use the ordinary workspace
-    r = la.make_shape(1, 8, 3, rope=True, T=2, Hh=2, W=2)
-    assert la.la_causal_workspace_bytes(r) == la.la_workspace_bytes(r)
+    r = la.make_shape(1, 16384, 70, rope=True, T=16, Hh=32, W=32)
+    assert la.la_causal_workspace_bytes(r) == n
+    # float32 I/O uses the ordinary workspace
     f = la.make_shape(1, 300, 3, io_dtype="f32")
     assert la.la_causal_workspace_bytes(f) == la.la_workspace_bytes(f)
     assert la.la_causal_workspace_bytes(la.make_shape(1, 16, 70, D=64)) == 0
