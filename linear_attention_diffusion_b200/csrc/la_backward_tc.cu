@@ -394,37 +394,75 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       float2 cs[16];
       if (kRope != kNoRope) row_angles<kRope>(p, rope_tab, n, cs);
 
-      // ---- transform: ReLU(Q) in place, den, dnum = dO / den in place
+      // ---- transform: ReLU(Q) in place, den, dnum = dO / den in place.
+      // Without RoPE a head's eight shared-memory loads go first (a store
+      // orders every later access after it) and den is four partial sums;
+      // with RoPE (short of registers) one 16-byte chunk at a time.
       float inv[kPair];
+      if (kRope == kNoRope) {
 #pragma unroll
-      for (int hh = 0; hh < kPair; ++hh) {
-        float den = 0.0f;
+        for (int hh = 0; hh < kPair; ++hh) {
+          uint4 uq[4], ug[4];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int c = hh * 4 + c4;
-          const uint32_t addr = st + sw128_offset(row, c);
-          uint4 u = ld_shared_v4(addr);
-          u.x = relu_bf16x2(u.x);
-          u.y = relu_bf16x2(u.y);
-          u.z = relu_bf16x2(u.z);
-          u.w = relu_bf16x2(u.w);
-          float x[8];
-          unpack8(u, x);
-          const float* zz = zs + hh * kD + c4 * 8;
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uq[c4] = ld_shared_v4(st + sw128_offset(row, hh * 4 + c4));
+            ug[c4] = ld_shared_v4(st + kBBox + sw128_offset(row, hh * 4 + c4));
+          }
+          float dp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) den = fmaf(x[e], zz[e], den);
-          st_shared_v4(addr, u);
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uq[c4].x = relu_bf16x2(uq[c4].x);
+            uq[c4].y = relu_bf16x2(uq[c4].y);
+            uq[c4].z = relu_bf16x2(uq[c4].z);
+            uq[c4].w = relu_bf16x2(uq[c4].w);
+            float x[8];
+            unpack8(uq[c4], x);
+            const float* zz = zs + hh * kD + c4 * 8;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dp[e & 3] = fmaf(x[e], zz[e], dp[e & 3]);
+          }
+          inv[hh] = 1.0f / (((dp[0] + dp[1]) + (dp[2] + dp[3])) + p.eps);
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            st_shared_v4(st + sw128_offset(row, hh * 4 + c4), uq[c4]);
+            float x[8];
+            unpack8(ug[c4], x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] *= inv[hh];
+            st_shared_v4(st + kBBox + sw128_offset(row, hh * 4 + c4), pack8(x));
+          }
         }
-        inv[hh] = 1.0f / (den + p.eps);
+      } else {
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int c = hh * 4 + c4;
-          const uint32_t addr = st + kBBox + sw128_offset(row, c);
-          float x[8];
-          unpack8(ld_shared_v4(addr), x);
+        for (int hh = 0; hh < kPair; ++hh) {
+          float den = 0.0f;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] *= inv[hh];
-          st_shared_v4(addr, pack8(x));
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int c = hh * 4 + c4;
+            const uint32_t addr = st + sw128_offset(row, c);
+            uint4 u = ld_shared_v4(addr);
+            u.x = relu_bf16x2(u.x);
+            u.y = relu_bf16x2(u.y);
+            u.z = relu_bf16x2(u.z);
+            u.w = relu_bf16x2(u.w);
+            float x[8];
+            unpack8(u, x);
+            const float* zz = zs + hh * kD + c4 * 8;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) den = fmaf(x[e], zz[e], den);
+            st_shared_v4(addr, u);
+          }
+          inv[hh] = 1.0f / (den + p.eps);
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int c = hh * 4 + c4;
+            const uint32_t addr = st + kBBox + sw128_offset(row, c);
+            float x[8];
+            unpack8(ld_shared_v4(addr), x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] *= inv[hh];
+            st_shared_v4(addr, pack8(x));
+          }
         }
       }
       fence_proxy_async_smem();
@@ -453,15 +491,34 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
             for (int e = 0; e < 8; ++e) t[c4 * 8 + e] = y[e];
           }
         }
-        // ReLU(q) is read from shared memory twice rather than held in registers
-        float dot = 0.0f;
+        // ReLU(q) of the row: without RoPE the four loads go together and
+        // are kept for dQ; with RoPE (short of registers) one chunk at a time,
+        // read again below
+        uint4 uq[4];
+        if (kRope == kNoRope) {
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int c = hh * 4 + c4;
-          float x[8];
-          unpack8(ld_shared_v4(st + sw128_offset(row, c)), x);
+          for (int c4 = 0; c4 < 4; ++c4) uq[c4] = ld_shared_v4(st + sw128_offset(row, hh * 4 + c4));
+        }
+        float dot;
+        if (kRope == kNoRope) {
+          float dp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) dot = fmaf(x[e], t[c4 * 8 + e], dot);
+          for (int c4 = 0; c4 < 4; ++c4) {
+            float x[8];
+            unpack8(uq[c4], x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dp[e & 3] = fmaf(x[e], t[c4 * 8 + e], dp[e & 3]);
+          }
+          dot = (dp[0] + dp[1]) + (dp[2] + dp[3]);
+        } else {
+          dot = 0.0f;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            float x[8];
+            unpack8(ld_shared_v4(st + sw128_offset(row, hh * 4 + c4)), x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dot = fmaf(x[e], t[c4 * 8 + e], dot);
+          }
         }
         const float dden = -dot * inv[hh];
         my_dden[row * kPair + hh] = dden;
@@ -473,7 +530,7 @@ bwd_q_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           for (int c4 = 0; c4 < 4; ++c4) {
             const int c = hh * 4 + c4;
             float x[8];
-            unpack8(ld_shared_v4(st + sw128_offset(row, c)), x);
+            unpack8(uq[c4], x);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const int d = c4 * 8 + e;
@@ -770,24 +827,34 @@ bwd_kv_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
 
       // ---- transform: K -> phi(K) in place; keep the sign mask of K
       uint32_t mask[kPair] = {0u, 0u};
+      // without RoPE a head's four loads go first (a store orders every later
+      // access after it); with RoPE (short of registers) one chunk at a time
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t addr = st + sw128_offset(row, c);
-        uint4 v = ld_shared_v4(addr);
-        v.x = relu_bf16x2(v.x);
-        v.y = relu_bf16x2(v.y);
-        v.z = relu_bf16x2(v.z);
-        v.w = relu_bf16x2(v.w);
-        float x[8];
-        unpack8(v, x);
+      for (int hh = 0; hh < kPair; ++hh) {
+        uint4 kv[4];
+        if (kRope == kNoRope) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (x[e] > 0.0f) mask[c >> 2] |= 1u << ((c & 3) * 8 + e);
-        if (kRope != kNoRope) {
-          rotate_chunk<1>(cs, (c & 3) * 4, x);
-          v = pack8(x);
+          for (int c4 = 0; c4 < 4; ++c4) kv[c4] = ld_shared_v4(st + sw128_offset(row, hh * 4 + c4));
         }
-        st_shared_v4(addr, v);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int c = hh * 4 + c4;
+          uint4 v = kRope == kNoRope ? kv[c4] : ld_shared_v4(st + sw128_offset(row, c));
+          v.x = relu_bf16x2(v.x);
+          v.y = relu_bf16x2(v.y);
+          v.z = relu_bf16x2(v.z);
+          v.w = relu_bf16x2(v.w);
+          float x[8];
+          unpack8(v, x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if (x[e] > 0.0f) mask[hh] |= 1u << (c4 * 8 + e);
+          if (kRope != kNoRope) {
+            rotate_chunk<1>(cs, c4 * 4, x);
+            v = pack8(x);
+          }
+          st_shared_v4(st + sw128_offset(row, c), v);
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(&ready[s]);
