@@ -885,12 +885,9 @@ causal_chunk_rope_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       // k: ReLU (plain copy for Z), rotation, two parts
       {
         float x[2][16];
-        uint4 kw[4];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) kw[c4] = ld_shared_v4(st + RStage::k + sw128_offset(row, h * 4 + c4));
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
-          uint4 w = kw[c4];
+          uint4 w = ld_shared_v4(st + RStage::k + sw128_offset(row, h * 4 + c4));
           w.x = relu_bf16x2(w.x); w.y = relu_bf16x2(w.y); w.z = relu_bf16x2(w.z); w.w = relu_bf16x2(w.w);
           st_shared_v4(st + RStage::kp + h * kXVBox + sw64_offset(row, c4), w);
           float t[8];
