@@ -1,16 +1,18 @@
 // Token-causal linear attention on the tensor cores with independent chunks
-// (bf16 I/O, no RoPE): query n sees keys 0..n ("SANA-Video: Efficient Video
-// Generation with Block Linear Diffusion Transformer", section 2.3, with the
-// sum over earlier j read at token granularity).
+// (bf16 I/O): query n sees keys 0..n ("SANA-Video: Efficient Video Generation
+// with Block Linear Diffusion Transformer", section 2.3, with the sum over
+// earlier j read at token granularity).
 //
-// Three launches. (1) The state reduce in its chunk form (layer_tc, la_tc.cu)
-// writes every 128-token chunk's own state (dS_c, dz_c). (2) chunk_prefix
-// replaces them, per head and in chunk order, by the exclusive prefix
+// Three launches without RoPE, four with it. (1) The state reduce in its chunk
+// form (layer_tc, la_tc.cu) writes every 128-token chunk's own state (dS_c,
+// dz_c); with RoPE its keys are rotated, and chunk_key_sums forms dz_c from
+// the plain ReLU(k). (2) chunk_prefix replaces the states, per head and in
+// chunk order, by the exclusive prefix
 //   P_c = carry + sum_{c' < c} (dS_c', dz_c'),
 // and folds the whole sequence into the carry when asked. (3) causal_chunk_tc
-// computes every chunk on its own:
+// (or causal_chunk_rope_tc, further down) computes every chunk on its own:
 //   O_i = (sum_{j <= i in chunk} (phi(q_i).phi(k_j)) v_j + phi(q_i) S_P)
-//         / (sum_{j <= i in chunk} phi(q_i).phi(k_j) + phi(q_i).z_P + eps)
+//         / (sum_{j <= i in chunk} ReLU(q_i).ReLU(k_j) + ReLU(q_i).z_P + eps)
 // with (S_P, z_P) the chunk's prefix (without RoPE the denominator's
 // ReLU(q).ReLU(k) is the numerator's weight itself, so one matrix serves
 // both). No state travels from chunk to chunk inside the last launch, so a
@@ -19,8 +21,8 @@
 //
 // causal_chunk_tc: a CTA owns two heads (one 64-dim TMA box per tensor) of one
 // batch element and a range of chunks; 352 threads (TMA warp, one warpgroup
-// per head, and one MMA-issuing warp per head: warps 1 and 10). Per chunk, with three stages of Q, K, V and the
-// chunk's prefix state in flight:
+// per head, and one MMA-issuing warp per head: warps 1 and 10). Per chunk,
+// with three stages of Q, K, V and the chunk's prefix state in flight:
 //   P   = phi(Q_h) phi(K_h)^T            M = N = 128, K = 32   (TMEM)
 //   the head's warpgroup masks P to j <= i, sums its rows, and writes P back
 //   into the same TMEM columns as two bf16 parts (the rounded value and the
@@ -487,9 +489,9 @@ causal_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 // with S_P the prefix state of rotated keys and z_P that of plain key sums.
 // Z = L ReLU(K_h) is a tensor-core product with L the 128 x 128 lower
 // triangle of ones (kept in TMEM as an A operand). The rotated q and k enter
-// their products in two bf16 parts each (value and rounded remainder:
-// P = q_hi.k_hi + q_hi.k_lo + q_lo.k_hi, and likewise q.S), so the weights
-// keep about 16 bits as in the unrotated kernel.
+// their products in two bf16 parts each (the value truncated to bf16 and the
+// rounded remainder: P = q_hi.k_hi + q_hi.k_lo + q_lo.k_hi, and likewise
+// q.S), so the weights keep about 16 bits as in the unrotated kernel.
 //
 // Stage layout (two stages): the Q box, overwritten with the rotated q's
 // high part; the low part; the K box, overwritten with the rotated k's high
