@@ -49,6 +49,8 @@ SMALL = [
     (1, 1, 1, None, 0),
     (2, 4096, 7, (4, 32, 32), 11),  # several splits per head
     (1, 4096, 148, None, 0),        # many head groups
+    (1, 2048, 3, (32, 8, 8), 5),    # a 128-token chunk spans two frames
+    (2, 600, 2, (4, 150, 1), 0),    # W = 1: a chunk steps 128 rows at once
 ]
 
 
