@@ -109,19 +109,10 @@ struct QkvSched {
   int KB;     // K-blocks of 64 channels
   int L;      // token tiles per chunk
   int NK;     // chunks per batch element
-  int J;      // partial slots per (batch, group, chunk), per CTA of a pair
   int total;  // tiles
-  int pairs, q, r;  // total = q * pairs + r; pair c owns [c q + min(c, r), ...)
+  int units;  // runs: B * NK * CT
+  int pairs;  // CTA pairs; pair c takes runs c, c + pairs, c + 2 pairs, ...
 };
-
-__host__ __device__ inline int sched_begin(const QkvSched& s, int c) {
-  return c * s.q + (c < s.r ? c : s.r);
-}
-
-__host__ __device__ inline int sched_owner(const QkvSched& s, int i) {
-  const int big = s.r * (s.q + 1);
-  return i < big ? i / (s.q + 1) : s.r + (i - big) / s.q;
-}
 
 // First tile of chunk k of batch element b, and the chunk's length.
 __host__ __device__ inline int chunk_begin(const QkvSched& s, int b, int k) {
@@ -140,6 +131,37 @@ struct Tile {
   int run0;   // kv: first tile of the run's (b, k, g) block
   int first;  // kv: first tile of its run in this pair
   int last;   // kv: last tile of its run in this pair
+};
+
+// Run u (a column tile over the consecutive token tiles of one chunk): its
+// first tile and the end of its tiles.
+__host__ __device__ inline void run_span(const QkvSched& s, int u, int& i0, int& i1) {
+  const int b = u / (s.NK * s.CT);
+  const int rem = u - b * s.NK * s.CT;
+  const int k = rem / s.CT, ct = rem - k * s.CT;
+  const int len = chunk_len(s, k);
+  i0 = chunk_begin(s, b, k) + ct * len;
+  i1 = i0 + len;
+}
+
+// The tiles of one pair in order: its runs u = pair, pair + pairs, ...; at any
+// moment all pairs stand at about the same token tile of neighbouring chunks,
+// so each X tile is read from HBM about once and its other reads hit L2.
+struct PairTiles {
+  int u, i, beg, end, tl;  // run, tile, run's first tile and end, tiles done
+  __device__ PairTiles(const QkvSched& s, int pair) : u(pair), i(0), beg(0), end(0), tl(0) {
+    if (u < s.units) run_span(s, u, beg, end);
+    i = beg;
+  }
+  __device__ bool valid(const QkvSched& s) const { return u < s.units; }
+  __device__ void next(const QkvSched& s) {
+    ++tl;
+    if (++i == end) {
+      u += s.pairs;
+      if (u < s.units) run_span(s, u, beg, end);
+      i = beg;
+    }
+  }
 };
 
 __device__ __forceinline__ Tile decode(const QkvSched& s, int i, int i_begin, int i_end) {
@@ -327,7 +349,6 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_rank();
   const int pair = blockIdx.x >> 1;
-  const int i_begin = sched_begin(sc, pair), i_end = sched_begin(sc, pair + 1);
 
   if (tid == 0) {
     for (int s = 0; s < kQStages; ++s) {
@@ -367,8 +388,8 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
     if (lane == 0) {
       int pos = 0;
       bool ok = true;
-      for (int i = i_begin; ok && i < i_end; ++i) {
-        const Tile t = decode(sc, i, i_begin, i_end);
+      for (PairTiles it(sc, pair); ok && it.valid(sc); it.next(sc)) {
+        const Tile t = decode(sc, it.i, it.beg, it.end);
         const int y = t.nt * kTokPair + static_cast<int>(rank) * kTokCta;
         // this CTA's 128 rows of the tile's 256 rows of W: the group's keys
         // (CTA 0) or values (CTA 1), or half of 256 query rows. Rows past
@@ -405,8 +426,8 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
       const uint32_t idesc = idesc_bf16_f32(kTokPair, kCols, 0, 0);
       int pos = 0;
       bool ok = true;
-      for (int i = i_begin; ok && i < i_end; ++i) {
-        const int tl = i - i_begin, buf = tl & 1;
+      for (PairTiles it(sc, pair); ok && it.valid(sc); it.next(sc)) {
+        const int tl = it.tl, buf = tl & 1;
         // both CTAs' epilogues have read this accumulator's previous tile
         if (!(ok = mbar_wait(&acc_empty[buf], ((tl >> 1) & 1) ^ 1, abort_flag, &g_qkv_error,
                              kErrWait)))
@@ -453,9 +474,9 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
     float zacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     const uint32_t acc_empty_0[2] = {map_rank(smem_u32(&acc_empty[0]), 0),
                                      map_rank(smem_u32(&acc_empty[1]), 0)};
-    for (int i = i_begin; i < i_end; ++i) {
-      const Tile t = decode(sc, i, i_begin, i_end);
-      const int tl = i - i_begin, buf = tl & 1;
+    for (PairTiles it(sc, pair); it.valid(sc); it.next(sc)) {
+      const Tile t = decode(sc, it.i, it.beg, it.end);
+      const int tl = it.tl, buf = tl & 1;
       const int n = t.nt * kTokPair + static_cast<int>(rank) * kTokCta + row;
       const bool valid = n < sc.N;
       // first feature (row of W, entry of the bias) of this warp's 128 columns
@@ -583,9 +604,8 @@ qkv_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ C
 
       if (t.last) {
         // ---- end of a run: this CTA's partial (S, z) of the run
-        const int slot = pair - sched_owner(sc, t.run0);
-        float* dst = part + (((static_cast<size_t>(t.b * sc.G + t.col) * sc.NK + t.k) * sc.J +
-                              slot) * 2 + rank) * kPartFloats;
+        float* dst = part + ((static_cast<size_t>(t.b * sc.G + t.col) * sc.NK + t.k) * 2 + rank) *
+                                kPartFloats;
         // accumulator nb: rows 16 smb + g (+ 8), columns 8 nb + 2 t4 (+ 1)
         float* ds = dst + sh * kD * kD + (smb * 16 + g) * kD + 2 * t4;
 #pragma unroll
@@ -634,31 +654,33 @@ qkv_combine(const QkvSched sc, const float* __restrict__ part, float* __restrict
   const bool is_s = v < kPartS / 4;
   constexpr int kVecPerPart = kPartFloats / 4;
   const float4* base =
-      reinterpret_cast<const float4*>(part) + static_cast<size_t>(bg) * sc.NK * sc.J * 2 * kVecPerPart;
+      reinterpret_cast<const float4*>(part) + static_cast<size_t>(bg) * sc.NK * 2 * kVecPerPart;
   float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  for (int k = 0; k < sc.NK; ++k) {
-    const int len = chunk_len(sc, k);
-    const int run0 = chunk_begin(sc, b, k) + g * len;
-    const int cnt = 2 * (sched_owner(sc, run0 + len - 1) - sched_owner(sc, run0) + 1);  // <= 4
-    const float4* src = base + static_cast<size_t>(k) * sc.J * 2 * kVecPerPart;
-    float4 t[4][4];
+  // chunk by chunk, the two CTAs of the run's pair; a chunk's loads go together
+  constexpr int kBatchK = 2;
+  for (int k0 = 0; k0 < sc.NK; k0 += kBatchK) {
+    float4 t[kBatchK][2][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int kk = 0; kk < kBatchK; ++kk)
 #pragma unroll
-      for (int qd = 0; qd < 4; ++qd)
-        if (j < cnt && (!is_s || qd == 0))
-          t[j][qd] = __ldcg(src + j * kVecPerPart +
-                            (is_s ? v : kPartS / 4 + qd * kD + (v - kPartS / 4)));
+      for (int j = 0; j < 2; ++j)
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+        for (int qd = 0; qd < 4; ++qd)
+          if (k0 + kk < sc.NK && (!is_s || qd == 0))
+            t[kk][j][qd] = __ldcg(base + (static_cast<size_t>(k0 + kk) * 2 + j) * kVecPerPart +
+                                  (is_s ? v : kPartS / 4 + qd * kD + (v - kPartS / 4)));
 #pragma unroll
-      for (int qd = 0; qd < 4; ++qd)
-        if (j < cnt && (!is_s || qd == 0)) {
-          acc.x += t[j][qd].x;
-          acc.y += t[j][qd].y;
-          acc.z += t[j][qd].z;
-          acc.w += t[j][qd].w;
-        }
+    for (int kk = 0; kk < kBatchK; ++kk)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd)
+          if (k0 + kk < sc.NK && (!is_s || qd == 0)) {
+            acc.x += t[kk][j][qd].x;
+            acc.y += t[kk][j][qd].y;
+            acc.z += t[kk][j][qd].z;
+            acc.w += t[kk][j][qd].w;
+          }
   }
   if (is_s) {
     const int hh = v / (kD * kD / 4), h = 4 * g + hh;
@@ -689,12 +711,26 @@ QkvSched make_sched(int B, int N, int H, int C) {
   s.KB = (C + kKBlk - 1) / kKBlk;
   const long long total = 1LL * B * s.NT * s.CT;
   s.total = static_cast<int>(total);
-  s.pairs = static_cast<int>(std::min<long long>(kNumSMs / 2, std::max<long long>(1, total)));
-  s.q = std::max(1, s.total / s.pairs);
-  s.r = s.total - s.q * s.pairs;
-  s.L = std::max(1, std::min(s.NT, s.q));
+  // Runs of L token tiles; the pairs take the runs in turn. L is the longest
+  // run length whose load (the most tiles a pair gets) is within 3% of the
+  // best over all L (short runs mean more partial states to write and sum).
+  const int P = kNumSMs / 2;
+  auto load = [&](int L) {
+    const long long nk = (s.NT + L - 1) / L;
+    const long long units = 1LL * B * nk * s.CT;
+    return ((units + P - 1) / P) * L;  // tiles of the busiest pair (upper bound)
+  };
+  long long best = load(1);
+  for (int L = 2; L <= s.NT; ++L) best = std::min(best, load(L));
+  s.L = 1;
+  for (int L = s.NT; L >= 1; --L)
+    if (load(L) * 100 <= best * 103) {
+      s.L = L;
+      break;
+    }
   s.NK = (s.NT + s.L - 1) / s.L;
-  s.J = std::min(s.L, (s.L - 1) / s.q + 2);  // L <= q, so J <= 2: a run spans <= 2 pairs
+  s.units = B * s.NK * s.CT;
+  s.pairs = std::max(1, std::min(P, s.units));
   return s;
 }
 
@@ -722,7 +758,7 @@ using QkvKernel = void (*)(CUtensorMap, CUtensorMap, QkvSched, Rope, const __nv_
 size_t qkv_workspace_floats(int B, int N, int H, int C) {
   if (N <= 0 || B <= 0 || H <= 0) return 0;
   const QkvSched s = make_sched(B, N, H, C);
-  return static_cast<size_t>(B) * s.G * s.NK * s.J * 2 * kPartFloats;
+  return static_cast<size_t>(B) * s.G * s.NK * 2 * kPartFloats;
 }
 
 cudaError_t launch_qkv_state(const Problem& p, int C, const void* X, const void* W,
