@@ -35,10 +35,12 @@
 // second kernel sums every head's slots in a fixed order, so S and z are
 // bitwise reproducible.
 //
-// Tile order: token tiles are cut into chunks of L tiles; chunk by chunk, all
-// column tiles of the chunk, each over the chunk's tokens. With L = tiles per
-// pair, the pairs running at any moment read few distinct token rows of X,
-// so X comes from HBM about once and W stays in L2.
+// Tile order: token tiles are cut into chunks of L tiles; a run is one column
+// tile over the token tiles of one chunk, and pair c takes runs c, c + pairs,
+// c + 2 pairs, ... (L is chosen on the host so that the busiest pair's tile
+// count stays within 3% of the best). All pairs then stand at about the same
+// token tile of neighbouring chunks, so X comes from HBM about once and W
+// stays in L2.
 //
 // Warp roles (320 threads per CTA): warps 0-7 epilogue (warp w reads TMEM
 // lanes 32 (w % 4) .. + 31, i.e. token rows; warps 0-3 the first 128
