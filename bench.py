@@ -482,7 +482,9 @@ def run_la(args, w, rank, world, local_rank):
                 evs[1].record(stream)
         kernel_names = ("state_reduce" if args.op == "reduce" else "apply",)
     elif args.op == "causal":
-        launches_per_step = 2  # split states, then the causal pass
+        # bf16: every chunk's state (+ the chunks' key sums with RoPE), their
+        # prefix, then the chunks
+        launches_per_step = 4 if w.rope else 3
 
         def step(i, evs=None):
             q, k, v, o = ptrs[i % n_sets]
